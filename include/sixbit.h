@@ -1,0 +1,220 @@
+/*
+ * sixbit.h -- C ABI of the B200 (sm_100a) hot path of 6Bit-Diffusion.
+ *
+ * 6Bit-Diffusion (arXiv:2603.18742, as described by the write-up "6Bit-Diffusion: dynamic
+ * quantization ..." and the explainer "6Bit-Diffusion: Inference-Time Mixed-Precision
+ * Quantization for Video Diffusion Models") runs every linear layer of a video diffusion
+ * transformer in NVFP4 or INT8, chosen per layer and per denoising step from the previous step's
+ * input/output difference, rotates activations with a block Hadamard transform first, skips whole
+ * modules whose outputs barely change (Temporal Delta Cache, TDC), and computes in full precision
+ * when the input's outlier ratio is too large (Purified Delta Refresh, PDR).
+ *
+ * Conventions (apply to every entry point):
+ *  - Pointers are DEVICE pointers unless the parameter is marked "host". Structs passed by
+ *    pointer (sb_config, sb_rule, sb_weight, sb_fp4, sb_i8) are HOST structs whose pointer
+ *    fields are device pointers; sb_module_state and sb_stats live in DEVICE memory.
+ *  - The caller owns all memory. The library allocates no device memory and keeps no device
+ *    state between calls; scratch lives in the caller's workspace `ws` (sb_workspace_size).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; 0 = legacy default stream).
+ *    Calls that share a workspace must be ordered on one stream.
+ *  - Arguments are validated synchronously; on failure nothing is launched, the status is
+ *    returned and sb_last_error() describes it. Device-side faults of the method (a bounded wait
+ *    that gave up, non-finite input) set an error word inside `ws`; sb_check() reads and clears it.
+ *  - Every device pointer must be 16-byte aligned (SB_EALIGN otherwise).
+ *  - Shapes: activations are [M][K] row-major bf16 (M tokens, K channels); weights are [N][K]
+ *    row-major (row = output channel, the PyTorch Linear layout); outputs are [M][N].
+ *  - No C++ exception crosses this boundary.
+ */
+#ifndef SIXBIT_H
+#define SIXBIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sb_stream; /* identical to cudaStream_t */
+
+typedef enum {
+  SB_OK = 0,
+  SB_EINVAL = 1,        /* null pointer where one is required, bad enum value */
+  SB_ESHAPE = 2,        /* inconsistent or out-of-range sizes */
+  SB_EALIGN = 3,        /* a device pointer is not 16-byte aligned */
+  SB_EUNSUPPORTED = 4,  /* block not in {16,32,64,128,256}, K % block, K % 64, N % 32, K > 16384 */
+  SB_ECUDA = 5,         /* a CUDA runtime call failed (launch, attribute, tensor map) */
+  SB_ETIMEOUT = 6,      /* device: a bounded wait inside a kernel gave up (reported by sb_check) */
+  SB_ENONFINITE = 7     /* device: a pre-pass input held Inf/NaN (reported by sb_check) */
+} sb_status;
+
+/* Precision of one layer at one step ("write-up" section 一: NVFP4 is the fast, coarse format,
+ * INT8 the precise one; section 三: full precision when PDR fires; section 二: skip). */
+typedef enum { SB_NVFP4 = 0, SB_INT8 = 1, SB_BF16 = 2, SB_SKIP = 3 } sb_prec;
+
+enum { SB_OUT_BF16 = 0, SB_OUT_F32 = 1, SB_OUT_RAW = 2 };   /* sb_linear out_dtype */
+enum { SB_EPI_NONE = 0, SB_EPI_GELU_TANH = 1 };             /* sb_linear epilogue  */
+enum { SB_PREPASS_QUANT = 0, SB_PREPASS_STATS = 1 };        /* sb_prepass mode     */
+
+/* NVFP4 tensor: E2M1 codes packed two per byte along K (element 2i in the low nibble), one E4M3
+ * scale per 16 consecutive elements of a row stored in the tensor-core block-scale layout
+ * (sb_fp4_sf_bytes), one FP32 tensor scale s_g. value = e2m1 * e4m3 * s_g. */
+typedef struct {
+  uint8_t* codes;   /* [rows][cols/2] */
+  uint8_t* sf;      /* sb_fp4_sf_bytes(rows, cols) bytes; rows padded to 128 with zero scales */
+  float* gscale;    /* 1 float */
+  int64_t rows, cols;
+} sb_fp4;
+
+/* INT8 tensor, symmetric, one FP32 scale per row: value = code * scale[row]. */
+typedef struct {
+  int8_t* codes;    /* [rows][cols] */
+  float* scale;     /* [rows] */
+  int64_t rows, cols;
+} sb_i8;
+
+/* A prepared linear layer. w4 and w8 hold the Hadamard-rotated weight (rows rotated along K with
+ * the same block as the activations) quantized to NVFP4 (tensor scale) and INT8 (per output
+ * channel); w_bf16 is the original weight kept for the PDR full-precision path. */
+typedef struct {
+  const void* w_bf16;     /* [N][K] bf16, original */
+  const void* bias_bf16;  /* [N] bf16 or NULL */
+  sb_fp4 w4;
+  sb_i8 w8;
+  int64_t N, K;
+  int32_t block;
+} sb_weight;
+
+/* Per-layer linear rule ("write-up" section 一 and 六: a simple linear model of the previous
+ * step's difference predicts the need for precision): INT8 iff a * d_prev + b > tau. */
+typedef struct { double a, b, tau; } sb_rule;
+
+typedef struct {
+  double rho;         /* PDR outlier-ratio threshold (max|x| / mean|x|), e.g. 64 */
+  double tdc_thresh;  /* TDC accumulator threshold, e.g. 0.1 */
+  int32_t block;      /* Hadamard block B (16..256, power of two), default 128 */
+  int32_t force_prec; /* -1: decide; 0/1/2 force NVFP4/INT8/BF16 (benchmarks, tests) */
+} sb_config;
+
+/* Per-module decision state (device memory, 64 bytes). */
+typedef struct {
+  double prev_d;        /* d of the last computed step */
+  double acc;           /* accumulated delta since the last computed step */
+  double delta;         /* relative L1 change between the last two computed outputs */
+  int32_t have_d;       /* prev_d belongs to the step just before the current one */
+  int32_t n_out;        /* computed outputs so far */
+  int32_t last_skipped; /* the previous step was skipped */
+  int32_t skip;         /* decision of the current step (1 = reuse the cache) */
+  int32_t steps;        /* sb_tdc_step calls so far */
+  int32_t reserved[3];
+} sb_module_state;
+
+/* Pre-pass statistics (device memory, 96 bytes). Sums are the deterministic pairwise reductions
+ * (FP32 per row, FP64 across rows) so that every decision is reproducible bit for bit. */
+typedef struct {
+  double sum_abs;   /* sum |x| */
+  double sum_d2;    /* sum (x - x_ref)^2 (0 without x_ref) */
+  double sum_ref2;  /* sum x_ref^2 (0 without x_ref) */
+  double max_abs;   /* max |x| */
+  double amax_rot;  /* max |H x| over the tensor: the NVFP4 tensor amax */
+  double ratio;     /* PDR outlier ratio max|x| / (sum|x| / numel); +inf when sum|x| = 0 */
+  double d;         /* sqrt(sum_d2) / sqrt(sum_ref2) (relative input/output difference) */
+  double numel;
+  int32_t has_ref;  /* d is valid */
+  int32_t prec_in;  /* precision on entry */
+  int32_t prec_out; /* precision after PDR */
+  int32_t nonfinite;
+} sb_stats;
+
+const char* sb_version(void);
+
+/* Thread-local description of the last failed call of this thread ("" if none). */
+const char* sb_last_error(void);
+
+/* Bytes of workspace needed by calls with at most max_M rows (tokens or weight rows N) of at most
+ * max_K columns. `bytes` is a host pointer. */
+sb_status sb_workspace_size(int64_t max_M, int64_t max_K, size_t* bytes);
+
+/* Zero a workspace (counters and error word) before its first use. */
+sb_status sb_workspace_init(void* ws, size_t bytes, sb_stream stream);
+
+/* Bytes of the block-scale array of an NVFP4 tensor: ceil(rows/128)*128 * cols/16. */
+int64_t sb_fp4_sf_bytes(int64_t rows, int64_t cols);
+
+/* Reset a module state (n_out = 0, no difference, nothing accumulated). */
+sb_status sb_state_init(sb_module_state* state, sb_stream stream);
+
+/* Block Hadamard rotation only (utility and test hook): Y[m][k] = (H_B X[m][block(k)])[k] in FP32,
+ * H_B the unnormalised Sylvester matrix, butterfly stages h = 1, 2, ..., B/2 ascending.
+ * X bf16 [M][K], Y float [M][K]. ("write-up" section 一: block Hadamard transform.) */
+sb_status sb_rotate(const void* X, float* Y, int64_t M, int64_t K, int32_t block, sb_stream stream);
+
+/* Offline weight preparation (untimed): rotate each row of W [N][K] along K in blocks of
+ * `block`, write the INT8 copy (per-row scale) into w->w8 and the NVFP4 copy (tensor scale from
+ * the rotated amax) into w->w4. The caller sets w->w_bf16, w->bias_bf16 and the device buffers of
+ * w->w4 (codes N*K/2, sf sb_fp4_sf_bytes(N,K), gscale 1 float) and w->w8 (codes N*K, scale N);
+ * this call fills N, K and block. ("write-up" section 四: W4A6, weights pre-quantized.) */
+sb_status sb_prepare_weight(const void* W, const void* bias, int64_t N, int64_t K, int32_t block,
+                            sb_weight* w /* host */, void* ws, sb_stream stream);
+
+/* TDC check of one module for the current step ("write-up" section 二): the first two steps are
+ * computed; afterwards acc += delta and the module is skipped while acc <= cfg->tdc_thresh. A skip
+ * clears have_d (the next computed step is a restart). Writes state->skip. */
+sb_status sb_tdc_step(sb_module_state* state, const sb_config* cfg /* host */, sb_stream stream);
+
+/* Precision of one layer for the current step ("write-up" sections 一 and 三): SB_SKIP if the
+ * module is skipped; cfg->force_prec if >= 0; INT8 if no previous difference exists (first step or
+ * restart after skips); else INT8 iff rule->a * prev_d + rule->b > rule->tau, NVFP4 otherwise.
+ * Writes *prec (device int32). */
+sb_status sb_select_precision(const sb_module_state* state, const sb_rule* rule /* host */,
+                              const sb_config* cfg /* host */, int32_t* prec, sb_stream stream);
+
+/* Activation pre-pass of one layer input X [M][K] bf16 ("write-up" sections 一, 三, 四).
+ * One pass computes the statistics record *stats (PDR ratio on the raw X; d against X_ref when
+ * given) and, in SB_PREPASS_QUANT mode, the block-Hadamard-rotated quantized activations for the
+ * precision in *prec: INT8 into a8 (codes [M][K], per-token scales [M]) or NVFP4 into a4 (codes,
+ * block scales, tensor scale; a second streaming kernel, which needs the tensor amax first).
+ * In SB_PREPASS_QUANT mode PDR is applied: a quantized *prec becomes SB_BF16 when
+ * stats->ratio > cfg->rho (unless cfg->force_prec >= 0). *prec == SB_SKIP makes every kernel exit
+ * at once. SB_PREPASS_STATS computes the record only and leaves *prec unchanged (prec may be
+ * NULL). a4/a8 may be NULL in STATS mode; in QUANT mode both must be given (the precision is only
+ * known on the device). Requires M*K > 0, K % block == 0, K % 64 == 0, K <= 16384. */
+sb_status sb_prepass(const void* X, const void* X_ref, int64_t M, int64_t K,
+                     const sb_config* cfg /* host */, int32_t mode, int32_t* prec,
+                     const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */, sb_stats* stats,
+                     void* ws, sb_stream stream);
+
+/* Quantized linear layer Y = X W^T + bias ("write-up" section 四; tcgen05 tensor cores):
+ *   NVFP4: Y = acc * s_gx * s_gw / B + bias, acc = sum of block-scaled E2M1 products
+ *          (tcgen05.mma kind::mxf4nvf4, UE4M3 scales per 16);
+ *   INT8:  Y = acc * s_x[m] * s_w[n] / B + bias, acc exact int32 (kind::i8);
+ *   BF16:  Y = X W^T + bias on the raw X and original W (kind::f16), the PDR path.
+ * The kind is read from *prec on the device (SB_SKIP: nothing is written). 1/B undoes the
+ * unnormalised rotation of both operands. epilogue SB_EPI_GELU_TANH applies the tanh GELU.
+ * out_dtype: SB_OUT_BF16 / SB_OUT_F32 write the result; SB_OUT_RAW writes the raw accumulator
+ * (int32 for INT8, FP32 otherwise; test hook). X (bf16 [M][K]) may be NULL if the BF16 path is
+ * never taken; a4/a8 may be NULL if that precision is never taken (the kernel then reports
+ * SB_EINVAL through sb_check). Requires K % 128 == 0, N % 32 == 0. */
+sb_status sb_linear(const void* X, const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */,
+                    const int32_t* prec, const sb_weight* w /* host */, int32_t epilogue,
+                    int32_t out_dtype, void* Y, int64_t M, void* ws, sb_stream stream);
+
+/* TDC record after a computed step ("write-up" section 二; explainer section 3): y_new and
+ * y_cache are bf16 [M][C]; y_cache holds the last computed output. If at least one output was
+ * recorded before, delta = sum|y_new - y_cache| / sum|y_cache| (pairwise FP32 rows, FP64 across
+ * rows; +inf when sum|y_cache| = 0) is stored. Then n_out += 1, acc = 0, and d is taken from
+ * d_src (if non-NULL and d_src->has_ref) as prev_d with have_d = 1, else have_d = 0. With
+ * update_cache != 0 the same pass refreshes y_cache with y_new. Does nothing if state->skip. */
+sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C,
+                        const sb_stats* d_src, int32_t update_cache, sb_module_state* state,
+                        void* ws, sb_stream stream);
+
+/* Synchronise `stream`, read and clear the device error word of `ws`. Returns SB_OK,
+ * SB_ETIMEOUT, SB_ENONFINITE, SB_EINVAL or SB_ECUDA. */
+sb_status sb_check(void* ws, sb_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIXBIT_H */

@@ -294,15 +294,29 @@ float orc_e4m3_decode(uint8_t c) {
   return (float)(s ? -v : v);
 }
 
-/* Round to nearest, ties to even code, saturate to +-448 (satfinite). */
+/* Round to nearest, ties to even code, saturate to +-448 (satfinite): a search over every
+ * finite non-negative code (their values cached once from orc_e4m3_decode). */
+static double E4M3_POS[127];
+static int E4M3_POS_READY = 0;
+
 uint8_t orc_e4m3_encode(float v) {
+  if (!E4M3_POS_READY) {
+#pragma omp critical(orc_e4m3_table)
+    {
+      if (!E4M3_POS_READY) {
+        for (int c = 0; c < 127; ++c) E4M3_POS[c] = (double)orc_e4m3_decode((uint8_t)c);
+#pragma omp flush
+        E4M3_POS_READY = 1;
+      }
+    }
+  }
   uint8_t sign = signbit(v) ? 0x80 : 0;
   double a = fabs((double)v);
   if (a >= 448.0) return sign | 0x7e;
   int best = 0;
   double bestd = a;
   for (int c = 1; c <= 0x7e; ++c) {
-    double d = fabs(a - (double)orc_e4m3_decode((uint8_t)c));
+    double d = fabs(a - E4M3_POS[c]);
     if (d < bestd || (d == bestd && (c & 1) == 0)) {
       best = c;
       bestd = d;

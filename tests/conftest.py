@@ -23,3 +23,17 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def sbg():
+    """The CUDA library on a B200; fails loudly (no fallback) when either is missing."""
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device (deselect with -m 'not gpu')"
+    major, minor = torch.cuda.get_device_capability()
+    assert major == 10, f"libsixbit targets sm_100a (B200); found sm_{major}{minor}"
+    from video_diffusion_mixed_b200 import build
+    build.build()
+    from video_diffusion_mixed_b200 import sixbit
+    sixbit.lib()
+    return sixbit

@@ -1,0 +1,111 @@
+"""The C-ABI library loads, exports every symbol include/sixbit.h declares, and validates
+arguments on the host (no GPU needed: every case below fails before any CUDA call)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sixbit.h")
+
+
+@pytest.fixture(scope="module")
+def sb():
+    from video_diffusion_mixed_b200 import build
+    build.build()
+    from video_diffusion_mixed_b200 import sixbit
+    sixbit.lib()
+    return sixbit
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sb_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("sb_prepass", "sb_linear", "sb_tdc_step", "sb_tdc_record", "sb_select_precision",
+              "sb_prepare_weight", "sb_check"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(sb):
+    L = sb.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", sb.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (sb_\w+)", out))
+    assert set(declared_functions()) <= exported
+    assert set(sb.EXPORTED) == set(declared_functions())
+
+
+def test_host_only_calls(sb):
+    L = sb.lib()
+    assert L.sb_version().decode().startswith("sixbit")
+    n = ctypes.c_size_t(0)
+    assert L.sb_workspace_size(17776, 3072, ctypes.byref(n)) == sb.SB_OK
+    assert n.value >= 256 + 48 * 556 and n.value % 256 == 0
+    assert L.sb_fp4_sf_bytes(17776, 3072) == 17792 * 192
+    assert L.sb_fp4_sf_bytes(1, 64) == 128 * 4
+    assert L.sb_workspace_size(1, 1, None) == sb.SB_EINVAL
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_argument_validation_without_gpu(sb):
+    L = sb.lib()
+    cfg = sb.config()
+    a4 = sb.Fp4(0x1000, 0x2000, 0x3000, 64, 256)
+    a8 = sb.I8(0x4000, 0x5000, 64, 256)
+    s = None
+    # null X
+    assert L.sb_prepass(None, None, 64, 256, ctypes.byref(cfg), 0, _fake(0x100), ctypes.byref(a4),
+                        ctypes.byref(a8), _fake(0x200), _fake(0x300), s) == sb.SB_EINVAL
+    # misaligned X
+    assert L.sb_prepass(_fake(0x1008), None, 64, 256, ctypes.byref(cfg), 0, _fake(0x100), ctypes.byref(a4),
+                        ctypes.byref(a8), _fake(0x200), _fake(0x300), s) == sb.SB_EALIGN
+    assert "aligned" in L.sb_last_error().decode()
+    # K not a multiple of the block / of 64, bad block
+    bad = sb.config(block=96)
+    assert L.sb_prepass(_fake(0x1000), None, 64, 256, ctypes.byref(bad), 0, _fake(0x100), ctypes.byref(a4),
+                        ctypes.byref(a8), _fake(0x200), _fake(0x300), s) == sb.SB_EUNSUPPORTED
+    assert L.sb_prepass(_fake(0x1000), None, 64, 200, ctypes.byref(cfg), 0, _fake(0x100), ctypes.byref(a4),
+                        ctypes.byref(a8), _fake(0x200), _fake(0x300), s) == sb.SB_EUNSUPPORTED
+    assert L.sb_prepass(_fake(0x1000), None, 0, 256, ctypes.byref(cfg), 0, _fake(0x100), ctypes.byref(a4),
+                        ctypes.byref(a8), _fake(0x200), _fake(0x300), s) == sb.SB_ESHAPE
+    # shape mismatch between X and the a4 descriptor
+    a4b = sb.Fp4(0x1000, 0x2000, 0x3000, 65, 256)
+    assert L.sb_prepass(_fake(0x1000), None, 64, 256, ctypes.byref(cfg), 0, _fake(0x100), ctypes.byref(a4b),
+                        ctypes.byref(a8), _fake(0x200), _fake(0x300), s) == sb.SB_ESHAPE
+    # QUANT mode needs the quantized outputs
+    assert L.sb_prepass(_fake(0x1000), None, 64, 256, ctypes.byref(cfg), 0, _fake(0x100), None, None,
+                        _fake(0x200), _fake(0x300), s) == sb.SB_EINVAL
+    # K above the supported maximum
+    assert L.sb_prepass(_fake(0x1000), None, 64, 16384 + 64, ctypes.byref(cfg), 1, None, None, None,
+                        _fake(0x200), _fake(0x300), s) == sb.SB_EUNSUPPORTED
+    # linear: N not a multiple of 32, K not a multiple of 128
+    w = sb.WeightC()
+    w.N, w.K, w.block = 100, 256, 128
+    assert L.sb_linear(_fake(0x1000), None, None, _fake(0x100), ctypes.byref(w), 0, 0, _fake(0x2000), 64,
+                       _fake(0x300), s) == sb.SB_EUNSUPPORTED
+    w.N, w.K = 128, 192
+    assert L.sb_linear(_fake(0x1000), None, None, _fake(0x100), ctypes.byref(w), 0, 0, _fake(0x2000), 64,
+                       _fake(0x300), s) == sb.SB_EUNSUPPORTED
+    w.N, w.K = 128, 256
+    assert L.sb_linear(None, None, None, _fake(0x100), ctypes.byref(w), 0, 0, _fake(0x2000), 64,
+                       _fake(0x300), s) == sb.SB_EINVAL
+    assert L.sb_linear(_fake(0x1000), None, None, _fake(0x100), ctypes.byref(w), 7, 0, _fake(0x2000), 64,
+                       _fake(0x300), s) == sb.SB_EINVAL
+    # tdc record: C not a multiple of 8
+    assert L.sb_tdc_record(_fake(0x1000), _fake(0x2000), 4, 12, None, 1, _fake(0x300), _fake(0x400),
+                           s) == sb.SB_EUNSUPPORTED
+    # select: bad force value
+    rule = sb.Rule(1.0, 0.0, 0.1)
+    assert L.sb_select_precision(_fake(0x100), ctypes.byref(rule), ctypes.byref(sb.config(force_prec=5)),
+                                 _fake(0x200), s) == sb.SB_EINVAL

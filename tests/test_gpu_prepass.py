@@ -1,0 +1,164 @@
+"""GPU parity of the activation pre-pass against the CPU oracle, through the C ABI.
+
+Bit-exact: rotated values, every FP64 statistic (the reductions follow the same pairwise tree),
+INT8 codes and per-token scales, NVFP4 codes, E4M3 block scales (tiled layout, padding
+included), the tensor scale and the PDR precision decision.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from video_diffusion_mixed_b200 import synth
+from gpu_helpers import npy, u16
+
+pytestmark = pytest.mark.gpu
+
+STATS = ("sum_abs", "sum_d2", "sum_ref2", "max_abs", "amax_rot", "ratio", "d")
+
+
+def run_prepass(sb, X, R=None, *, force=-1, prec0=None, block=128, rho=64.0, mode=0):
+    M, K = X.shape
+    ws = sb.Workspace(M, K)
+    a4 = sb.Fp4Tensor(M, K)
+    a8 = sb.I8Tensor(M, K)
+    a4.codes.fill_(0xAB)
+    a4.sf.fill_(0xCD)
+    a8.codes.fill_(0x55)
+    stats = sb.alloc_stats()
+    prec = torch.tensor([prec0 if prec0 is not None else (force if force >= 0 else sb.INT8)], dtype=torch.int32,
+                        device="cuda")
+    cfg = sb.config(rho=rho, block=block, force_prec=force)
+    sb.prepass(X, R, cfg, mode, prec, a4, a8, stats, ws)
+    sb.check(ws)
+    return {"a4": a4, "a8": a8, "stats": sb.decode_stats(stats), "prec": int(prec.item())}
+
+
+@pytest.mark.parametrize("B,M,K", [(16, 3, 256), (32, 40, 512), (64, 9, 1024), (128, 40, 1024), (256, 5, 1024),
+                                   (128, 5, 1920)])
+def test_rotate_bitexact(sbg, B, M, K):
+    X = synth.activations(M, K, n_outlier=3, scale=20.0, seed=B, device="cuda")
+    Y = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    sbg.rotate(X, Y, B)
+    torch.cuda.synchronize()
+    ref = oracle.rotate_rows(u16(X), B)
+    assert np.array_equal(npy(Y).view(np.uint32), ref.view(np.uint32))
+
+
+CASES = [
+    # (name, M, K, with_ref, workload-like generator args)
+    ("tiny", 256, 256, False, dict(n_outlier=4, scale=20.0)),
+    ("ragged_1920", 33, 1920, True, dict(n_outlier=19, scale=30.0, student=True)),
+    ("k3072_ref", 300, 3072, True, dict(n_outlier=15, scale=50.0)),
+    ("k12288", 70, 12288, False, dict()),
+    ("one_row", 1, 7680, True, dict()),
+]
+
+
+@pytest.mark.parametrize("name,M,K,with_ref,gen", CASES, ids=[c[0] for c in CASES])
+def test_prepass_int8_bitexact(sbg, name, M, K, with_ref, gen):
+    X = synth.activations(M, K, seed=1, tensor_id=1, device="cuda", **gen)
+    R = synth.activations(M, K, seed=1, tensor_id=2, device="cuda") if with_ref else None
+    out = run_prepass(sbg, X, R, force=sbg.INT8)
+    ref = oracle.prepass(u16(X), u16(R) if R is not None else None, 128)
+    for k in STATS:
+        assert out["stats"][k] == ref[k], (k, out["stats"][k], ref[k])
+    assert out["stats"]["has_ref"] == int(with_ref)
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    assert np.array_equal(npy(out["a8"].scale).view(np.uint32), s.view(np.uint32))
+    assert np.array_equal(npy(out["a8"].codes), q)
+    assert out["prec"] == sbg.INT8  # forced precision is kept
+
+
+@pytest.mark.parametrize("name,M,K,with_ref,gen", CASES, ids=[c[0] for c in CASES])
+def test_prepass_nvfp4_bitexact(sbg, name, M, K, with_ref, gen):
+    X = synth.activations(M, K, seed=2, tensor_id=1, device="cuda", **gen)
+    out = run_prepass(sbg, X, None, force=sbg.NVFP4)
+    ref = oracle.prepass(u16(X), None, 128)
+    codes, sfl, sft, sg = oracle.quant_nvfp4(ref["y"], ref["amax_rot"])
+    assert np.float32(npy(out["a4"].gscale)[0]) == sg
+    assert np.array_equal(npy(out["a4"].codes), codes)
+    assert np.array_equal(npy(out["a4"].sf), sft)  # includes the zeroed padding rows
+    assert out["stats"]["amax_rot"] == ref["amax_rot"]
+
+
+@pytest.mark.parametrize("B", [16, 64, 256])
+def test_prepass_block_sizes(sbg, B):
+    X = synth.activations(50, 1024, n_outlier=5, scale=10.0, seed=B, device="cuda")
+    ref = oracle.prepass(u16(X), None, B)
+    out8 = run_prepass(sbg, X, force=sbg.INT8, block=B)
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    assert np.array_equal(npy(out8["a8"].codes), q)
+    out4 = run_prepass(sbg, X, force=sbg.NVFP4, block=B)
+    codes, sfl, sft, sg = oracle.quant_nvfp4(ref["y"], ref["amax_rot"])
+    assert np.array_equal(npy(out4["a4"].codes), codes)
+    assert np.array_equal(npy(out4["a4"].sf), sft)
+
+
+@pytest.mark.parametrize("rho", [8.0, 64.0, 1e9])
+def test_pdr_decision_matches_oracle(sbg, rho):
+    X = synth.activations(256, 256, n_outlier=4, scale=20.0, seed=0, device="cuda")
+    ref = oracle.prepass(u16(X), None, 128)
+    for p0 in (sbg.NVFP4, sbg.INT8):
+        out = run_prepass(sbg, X, prec0=p0, rho=rho)
+        assert out["prec"] == oracle.apply_pdr(p0, ref["ratio"], rho), (p0, rho, ref["ratio"])
+        assert out["stats"]["prec_in"] == p0 and out["stats"]["prec_out"] == out["prec"]
+
+
+def test_pdr_ratio_equal_rho_keeps_quantization(sbg):
+    # all ones with one 64: max = 64, mean = (n - 1 + 64) / n; rho set to the exact ratio
+    X = torch.ones((32, 256), dtype=torch.bfloat16, device="cuda")
+    X[3, 17] = 64.0
+    ref = oracle.prepass(u16(X), None, 128)
+    out = run_prepass(sbg, X, prec0=sbg.NVFP4, rho=ref["ratio"])
+    assert out["stats"]["ratio"] == ref["ratio"] and out["prec"] == sbg.NVFP4
+    out = run_prepass(sbg, X, prec0=sbg.NVFP4, rho=np.nextafter(ref["ratio"], 0))
+    assert out["prec"] == sbg.BF16
+
+
+def test_skip_leaves_everything_untouched(sbg):
+    X = synth.activations(64, 256, seed=3, device="cuda")
+    out = run_prepass(sbg, X, prec0=sbg.SKIP)
+    assert out["prec"] == sbg.SKIP
+    assert (npy(out["a8"].codes) == 0x55).all() and (npy(out["a4"].codes) == 0xAB).all()
+    assert all(v == 0 for v in out["stats"].values())
+
+
+def test_zero_input(sbg):
+    X = torch.zeros((40, 512), dtype=torch.bfloat16, device="cuda")
+    out8 = run_prepass(sbg, X, force=sbg.INT8)
+    assert out8["stats"]["ratio"] == float("inf") and out8["stats"]["sum_abs"] == 0.0
+    assert not npy(out8["a8"].codes).any() and not npy(out8["a8"].scale).any()
+    out4 = run_prepass(sbg, X, force=sbg.NVFP4)
+    assert npy(out4["a4"].gscale)[0] == 1.0
+    assert not npy(out4["a4"].codes).any() and not npy(out4["a4"].sf).any()
+
+
+def test_stats_mode_does_not_touch_precision(sbg):
+    X = synth.activations(64, 512, seed=4, device="cuda")
+    R = synth.activations(64, 512, seed=5, device="cuda")
+    ws = sbg.Workspace(64, 512)
+    stats = sbg.alloc_stats()
+    sbg.prepass(X, R, sbg.config(rho=0.0), sbg.PREPASS_STATS, None, None, None, stats, ws)
+    sbg.check(ws)
+    st = sbg.decode_stats(stats)
+    ref = oracle.prepass(u16(X), u16(R), 128)
+    assert st["d"] == ref["d"] and st["ratio"] == ref["ratio"] and st["prec_out"] == -1
+
+
+@pytest.mark.parametrize("wl", ["attn2b", "ffn5b"])
+def test_prepass_full_size(sbg, wl):
+    """Full CogVideoX-sized activations (17776 tokens): statistics, INT8 and NVFP4 bit-exact."""
+    X, _ = synth.workload_inputs(wl, seed=0, device="cuda")
+    R = synth.noisy_copy(X, 0.1, seed=0)
+    out8 = run_prepass(sbg, R, X, force=sbg.INT8)
+    ref = oracle.prepass(u16(R), u16(X), 128)
+    for k in STATS:
+        assert out8["stats"][k] == ref[k], k
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    assert np.array_equal(npy(out8["a8"].codes), q)
+    assert np.array_equal(npy(out8["a8"].scale), s)
+    out4 = run_prepass(sbg, R, None, force=sbg.NVFP4)
+    codes, sfl, sft, sg = oracle.quant_nvfp4(ref["y"], ref["amax_rot"])
+    assert np.array_equal(npy(out4["a4"].codes), codes)
+    assert np.array_equal(npy(out4["a4"].sf), sft)

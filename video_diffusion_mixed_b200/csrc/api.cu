@@ -1,0 +1,362 @@
+// api.cu -- the C ABI declared in include/sixbit.h: argument validation and kernel dispatch.
+//
+// No entry point allocates device memory; scratch lives in the caller's workspace:
+//   [0, 128)    WsHeader (device error word, last-CTA tickets)
+//   [128, 224)  sb_stats scratch (weight preparation)
+//   [224, 228)  int32 precision scratch (weight preparation)
+//   [256, ...)  one 48-byte GroupSlot per aligned group of 32 rows
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "sb_device.cuh"
+#include "sb_kernels.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+sb_status fail(sb_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+sb_status ok() {
+  g_err.clear();
+  return SB_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_block(int b) { return b == 16 || b == 32 || b == 64 || b == 128 || b == 256; }
+
+constexpr size_t kOffStats = 128;
+constexpr size_t kOffPrec = 224;
+constexpr size_t kOffGroups = 256;
+
+void* ws_groups(void* ws) { return static_cast<char*>(ws) + kOffGroups; }
+sb_stats* ws_stats(void* ws) { return reinterpret_cast<sb_stats*>(static_cast<char*>(ws) + kOffStats); }
+int32_t* ws_prec(void* ws) { return reinterpret_cast<int32_t*>(static_cast<char*>(ws) + kOffPrec); }
+
+sb_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SB_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define SB_REQUIRE(cond, status, ...) \
+  do {                                \
+    if (!(cond)) return fail(status, __VA_ARGS__); \
+  } while (0)
+
+#define SB_ALIGNED(p, name) SB_REQUIRE(aligned16(p), SB_EALIGN, "%s is not 16-byte aligned", name)
+
+sb_status check_rows_cols(int64_t M, int64_t K, int32_t block) {
+  SB_REQUIRE(M >= 1, SB_ESHAPE, "M must be >= 1 (got %lld)", (long long)M);
+  SB_REQUIRE(M <= (int64_t)1 << 30, SB_ESHAPE, "M too large (%lld)", (long long)M);
+  SB_REQUIRE(valid_block(block), SB_EUNSUPPORTED, "block must be 16, 32, 64, 128 or 256 (got %d)", block);
+  SB_REQUIRE(K >= 64 && K % 64 == 0, SB_EUNSUPPORTED, "K must be a positive multiple of 64 (got %lld)",
+             (long long)K);
+  SB_REQUIRE(K % block == 0, SB_EUNSUPPORTED, "K (%lld) must be a multiple of the block (%d)", (long long)K, block);
+  SB_REQUIRE(K <= sb::kMaxK, SB_EUNSUPPORTED, "K must be <= %d (got %lld)", sb::kMaxK, (long long)K);
+  return SB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sb_version(void) { return "sixbit 0.1 (sm_100a)"; }
+
+const char* sb_last_error(void) { return g_err.c_str(); }
+
+sb_status sb_workspace_size(int64_t max_M, int64_t max_K, size_t* bytes) {
+  SB_REQUIRE(bytes != nullptr, SB_EINVAL, "bytes is NULL");
+  SB_REQUIRE(max_M >= 0 && max_K >= 0, SB_ESHAPE, "negative size");
+  const size_t groups = (size_t)sb::ceil_div(max_M > 0 ? max_M : 1, sb::kGroupRows);
+  size_t b = kOffGroups + groups * sizeof(sb::GroupSlot);
+  *bytes = (b + 255) & ~(size_t)255;
+  return ok();
+}
+
+sb_status sb_workspace_init(void* ws, size_t bytes, sb_stream stream) {
+  SB_REQUIRE(ws != nullptr, SB_EINVAL, "ws is NULL");
+  SB_ALIGNED(ws, "ws");
+  SB_REQUIRE(bytes >= kOffGroups, SB_ESHAPE, "workspace smaller than %zu bytes", kOffGroups);
+  cudaError_t e = sb::launch_ws_init(ws, bytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_workspace_init");
+  return ok();
+}
+
+int64_t sb_fp4_sf_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return -1;
+  return ((rows + 127) / 128) * 128 * (cols / 16);
+}
+
+sb_status sb_state_init(sb_module_state* state, sb_stream stream) {
+  SB_REQUIRE(state != nullptr, SB_EINVAL, "state is NULL");
+  SB_ALIGNED(state, "state");
+  cudaError_t e = sb::launch_state_init(state, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_state_init");
+  return ok();
+}
+
+sb_status sb_rotate(const void* X, float* Y, int64_t M, int64_t K, int32_t block, sb_stream stream) {
+  SB_REQUIRE(X && Y, SB_EINVAL, "X and Y are required");
+  SB_ALIGNED(X, "X");
+  SB_ALIGNED(Y, "Y");
+  sb_status st = check_rows_cols(M, K, block);
+  if (st != SB_OK) return st;
+  cudaError_t e = sb::launch_rotate(X, Y, M, K, block, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_rotate");
+  return ok();
+}
+
+static sb_status check_fp4(const sb_fp4* t, int64_t rows, int64_t cols, const char* name) {
+  SB_REQUIRE(t->codes && t->sf && t->gscale, SB_EINVAL, "%s: codes, sf and gscale are required", name);
+  SB_ALIGNED(t->codes, name);
+  SB_ALIGNED(t->sf, name);
+  SB_REQUIRE((reinterpret_cast<uintptr_t>(t->gscale) & 3u) == 0, SB_EALIGN, "%s.gscale misaligned", name);
+  SB_REQUIRE(t->rows == rows && t->cols == cols, SB_ESHAPE, "%s is [%lld x %lld], expected [%lld x %lld]", name,
+             (long long)t->rows, (long long)t->cols, (long long)rows, (long long)cols);
+  return SB_OK;
+}
+
+static sb_status check_i8(const sb_i8* t, int64_t rows, int64_t cols, const char* name) {
+  SB_REQUIRE(t->codes && t->scale, SB_EINVAL, "%s: codes and scale are required", name);
+  SB_ALIGNED(t->codes, name);
+  SB_ALIGNED(t->scale, name);
+  SB_REQUIRE(t->rows == rows && t->cols == cols, SB_ESHAPE, "%s is [%lld x %lld], expected [%lld x %lld]", name,
+             (long long)t->rows, (long long)t->cols, (long long)rows, (long long)cols);
+  return SB_OK;
+}
+
+sb_status sb_prepare_weight(const void* W, const void* bias, int64_t N, int64_t K, int32_t block, sb_weight* w,
+                            void* ws, sb_stream stream) {
+  SB_REQUIRE(W && w && ws, SB_EINVAL, "W, w and ws are required");
+  SB_ALIGNED(W, "W");
+  SB_ALIGNED(ws, "ws");
+  if (bias) SB_ALIGNED(bias, "bias");
+  sb_status st = check_rows_cols(N, K, block);
+  if (st != SB_OK) return st;
+  if ((st = check_fp4(&w->w4, N, K, "w->w4")) != SB_OK) return st;
+  if ((st = check_i8(&w->w8, N, K, "w->w8")) != SB_OK) return st;
+  w->w_bf16 = W;
+  w->bias_bf16 = bias;
+  w->N = N;
+  w->K = K;
+  w->block = block;
+  cudaStream_t s = (cudaStream_t)stream;
+  sb::PrepassLaunch p{};
+  p.X = W;
+  p.R = nullptr;
+  p.M = N;
+  p.K = K;
+  p.B = block;
+  p.mode = SB_PREPASS_QUANT;
+  p.prec = nullptr;
+  p.force_int8 = 1;
+  p.q8 = w->w8.codes;
+  p.s8 = w->w8.scale;
+  p.rho = 0.0;
+  p.force = -1;
+  p.groups = ws_groups(ws);
+  p.hdr = ws;
+  p.stats = ws_stats(ws);
+  cudaError_t e = sb::launch_prepass(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_prepare_weight (rotation, INT8)");
+  sb::Nvfp4Launch q{};
+  q.X = W;
+  q.M = N;
+  q.K = K;
+  q.B = block;
+  q.prec = nullptr;
+  q.stats = ws_stats(ws);
+  q.codes = w->w4.codes;
+  q.sf = w->w4.sf;
+  q.gscale = w->w4.gscale;
+  e = sb::launch_nvfp4(q, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_prepare_weight (NVFP4)");
+  return ok();
+}
+
+sb_status sb_tdc_step(sb_module_state* state, const sb_config* cfg, sb_stream stream) {
+  SB_REQUIRE(state && cfg, SB_EINVAL, "state and cfg are required");
+  SB_ALIGNED(state, "state");
+  cudaError_t e = sb::launch_tdc_step(state, cfg->tdc_thresh, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_tdc_step");
+  return ok();
+}
+
+sb_status sb_select_precision(const sb_module_state* state, const sb_rule* rule, const sb_config* cfg,
+                              int32_t* prec, sb_stream stream) {
+  SB_REQUIRE(state && rule && cfg && prec, SB_EINVAL, "state, rule, cfg and prec are required");
+  SB_ALIGNED(state, "state");
+  SB_REQUIRE((reinterpret_cast<uintptr_t>(prec) & 3u) == 0, SB_EALIGN, "prec misaligned");
+  SB_REQUIRE(cfg->force_prec >= -1 && cfg->force_prec <= 2, SB_EINVAL, "force_prec must be -1, 0, 1 or 2");
+  cudaError_t e = sb::launch_select(state, rule->a, rule->b, rule->tau, cfg->force_prec, prec, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_select_precision");
+  return ok();
+}
+
+sb_status sb_prepass(const void* X, const void* X_ref, int64_t M, int64_t K, const sb_config* cfg, int32_t mode,
+                     int32_t* prec, const sb_fp4* a4, const sb_i8* a8, sb_stats* stats, void* ws,
+                     sb_stream stream) {
+  SB_REQUIRE(X && cfg && stats && ws, SB_EINVAL, "X, cfg, stats and ws are required");
+  SB_ALIGNED(X, "X");
+  if (X_ref) SB_ALIGNED(X_ref, "X_ref");
+  SB_ALIGNED(stats, "stats");
+  SB_ALIGNED(ws, "ws");
+  SB_REQUIRE(mode == SB_PREPASS_QUANT || mode == SB_PREPASS_STATS, SB_EINVAL, "mode must be QUANT or STATS");
+  SB_REQUIRE(cfg->force_prec >= -1 && cfg->force_prec <= 2, SB_EINVAL, "force_prec must be -1, 0, 1 or 2");
+  sb_status st = check_rows_cols(M, K, cfg->block);
+  if (st != SB_OK) return st;
+  if (mode == SB_PREPASS_QUANT) {
+    SB_REQUIRE(prec && a4 && a8, SB_EINVAL, "QUANT mode needs prec, a4 and a8");
+    if ((st = check_fp4(a4, M, K, "a4")) != SB_OK) return st;
+    if ((st = check_i8(a8, M, K, "a8")) != SB_OK) return st;
+  }
+  if (prec) SB_REQUIRE((reinterpret_cast<uintptr_t>(prec) & 3u) == 0, SB_EALIGN, "prec misaligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  sb::PrepassLaunch p{};
+  p.X = X;
+  p.R = X_ref;
+  p.M = M;
+  p.K = K;
+  p.B = cfg->block;
+  p.mode = mode;
+  p.prec = prec;
+  p.force_int8 = 0;
+  p.q8 = (mode == SB_PREPASS_QUANT) ? a8->codes : nullptr;
+  p.s8 = (mode == SB_PREPASS_QUANT) ? a8->scale : nullptr;
+  p.rho = cfg->rho;
+  p.force = cfg->force_prec;
+  p.groups = ws_groups(ws);
+  p.hdr = ws;
+  p.stats = stats;
+  cudaError_t e = sb::launch_prepass(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_prepass (statistics)");
+  if (mode == SB_PREPASS_QUANT) {
+    sb::Nvfp4Launch q{};
+    q.X = X;
+    q.M = M;
+    q.K = K;
+    q.B = cfg->block;
+    q.prec = prec;
+    q.stats = stats;
+    q.codes = a4->codes;
+    q.sf = a4->sf;
+    q.gscale = a4->gscale;
+    e = sb::launch_nvfp4(q, s);
+    if (e != cudaSuccess) return cuda_fail(e, "sb_prepass (NVFP4 encode)");
+  }
+  return ok();
+}
+
+sb_status sb_linear(const void* X, const sb_fp4* a4, const sb_i8* a8, const int32_t* prec, const sb_weight* w,
+                    int32_t epilogue, int32_t out_dtype, void* Y, int64_t M, void* ws, sb_stream stream) {
+  SB_REQUIRE(prec && w && Y && ws, SB_EINVAL, "prec, w, Y and ws are required");
+  SB_ALIGNED(Y, "Y");
+  SB_ALIGNED(ws, "ws");
+  SB_REQUIRE(epilogue == SB_EPI_NONE || epilogue == SB_EPI_GELU_TANH, SB_EINVAL, "bad epilogue");
+  SB_REQUIRE(out_dtype == SB_OUT_BF16 || out_dtype == SB_OUT_F32 || out_dtype == SB_OUT_RAW, SB_EINVAL,
+             "bad out_dtype");
+  const int64_t N = w->N, K = w->K;
+  SB_REQUIRE(M >= 1 && M <= (int64_t)1 << 30, SB_ESHAPE, "M out of range (%lld)", (long long)M);
+  SB_REQUIRE(N >= 32 && N % 32 == 0 && N <= (int64_t)1 << 20, SB_EUNSUPPORTED, "N must be a multiple of 32 (got %lld)",
+             (long long)N);
+  SB_REQUIRE(K >= 128 && K % 128 == 0 && K <= (int64_t)1 << 20, SB_EUNSUPPORTED,
+             "K must be a positive multiple of 128 (got %lld)", (long long)K);
+  SB_REQUIRE(valid_block(w->block), SB_EUNSUPPORTED, "weight block %d unsupported", w->block);
+  if (w->bias_bf16) SB_ALIGNED(w->bias_bf16, "bias");
+  sb::GemmLaunch L{};
+  L.M = M;
+  L.N = N;
+  L.K = K;
+  L.B = w->block;
+  L.prec = prec;
+  if (X && w->w_bf16) {
+    SB_ALIGNED(X, "X");
+    SB_ALIGNED(w->w_bf16, "w->w_bf16");
+    L.X = X;
+    L.W16 = w->w_bf16;
+  }
+  sb_status st;
+  if (a8 && a8->codes) {
+    if ((st = check_i8(a8, M, K, "a8")) != SB_OK) return st;
+    if ((st = check_i8(&w->w8, N, K, "w->w8")) != SB_OK) return st;
+    L.A8 = a8->codes;
+    L.sA8 = a8->scale;
+    L.B8 = w->w8.codes;
+    L.sB8 = w->w8.scale;
+  }
+  if (a4 && a4->codes) {
+    if ((st = check_fp4(a4, M, K, "a4")) != SB_OK) return st;
+    if ((st = check_fp4(&w->w4, N, K, "w->w4")) != SB_OK) return st;
+    L.A4 = a4->codes;
+    L.sfA4 = a4->sf;
+    L.gA4 = a4->gscale;
+    L.B4 = w->w4.codes;
+    L.sfB4 = w->w4.sf;
+    L.gB4 = w->w4.gscale;
+  }
+  SB_REQUIRE(L.X || L.A8 || L.A4, SB_EINVAL, "no operand set given (X+w_bf16, a8 or a4)");
+  L.bias = w->bias_bf16;
+  L.epilogue = epilogue;
+  L.out_dtype = out_dtype;
+  L.Y = Y;
+  L.hdr = ws;
+  const char* why = "kernel launch";
+  cudaError_t e = sb::launch_gemm(L, (cudaStream_t)stream, &why);
+  if (e != cudaSuccess) return cuda_fail(e, why);
+  return ok();
+}
+
+sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C, const sb_stats* d_src,
+                        int32_t update_cache, sb_module_state* state, void* ws, sb_stream stream) {
+  SB_REQUIRE(y_new && y_cache && state && ws, SB_EINVAL, "y_new, y_cache, state and ws are required");
+  SB_ALIGNED(y_new, "y_new");
+  SB_ALIGNED(y_cache, "y_cache");
+  SB_ALIGNED(state, "state");
+  SB_ALIGNED(ws, "ws");
+  if (d_src) SB_ALIGNED(d_src, "d_src");
+  SB_REQUIRE(M >= 1 && M <= (int64_t)1 << 30, SB_ESHAPE, "M out of range (%lld)", (long long)M);
+  SB_REQUIRE(C >= 8 && C % 8 == 0 && C <= sb::kMaxK, SB_EUNSUPPORTED, "C must be a multiple of 8 in [8, %d]",
+             sb::kMaxK);
+  sb::TdcLaunch p{};
+  p.Y = y_new;
+  p.Cache = y_cache;
+  p.M = M;
+  p.C = C;
+  p.update = update_cache ? 1 : 0;
+  p.dsrc = d_src;
+  p.st = state;
+  p.groups = ws_groups(ws);
+  p.hdr = ws;
+  cudaError_t e = sb::launch_tdc_record(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_tdc_record");
+  return ok();
+}
+
+sb_status sb_check(void* ws, sb_stream stream) {
+  SB_REQUIRE(ws != nullptr, SB_EINVAL, "ws is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_check (stream synchronize)");
+  uint32_t err = 0;
+  e = cudaMemcpy(&err, ws, sizeof(err), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_check (read error word)");
+  if (err != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "sb_check (clear error word)");
+    return fail((sb_status)err, "device reported status %u", err);
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,462 @@
+// gemm.cu -- quantized linear layer on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// One persistent, warp-specialised kernel serves the three precisions of a layer; the precision
+// is read from the device flag written by the decision/pre-pass kernels, so no host round trip
+// is needed ("write-up" section 一: NVFP4 or INT8 per layer and step; section 三: full precision
+// under PDR; section 四: 4-bit weights).
+//
+//   NVFP4  tcgen05.mma.kind::mxf4nvf4.block_scale.block16  128 x 192 tiles, K-block 256 elements
+//   INT8   tcgen05.mma.kind::i8 (s32 accumulators)          128 x 256 tiles, K-block 128 elements
+//   BF16   tcgen05.mma.kind::f16 (fp32 accumulators)        128 x 256 tiles, K-block  64 elements
+//
+// Every K-block is one 128-byte-wide row slab of A and B (128B swizzle, loaded by TMA without
+// multicast), consumed by four MMAs of 32 bytes of K each. Warp roles (320 threads):
+//   warp 0      TMA producer (one lane): A/B tiles and, for NVFP4, the E4M3 scale atoms
+//   warp 1      TMEM allocator and MMA issuer (one lane); tcgen05.cp moves scales to TMEM
+//   warps 2-9   epilogue: TMEM -> registers, dequant scale, bias, optional GELU, store
+// Two accumulator buffers in TMEM let the epilogue of tile i overlap the mainloop of tile i+1.
+// NVFP4 tiles are 192 wide so both buffers (2 x 192 columns) and the block scales (48 columns)
+// fit the 512 TMEM columns. Every wait is bounded; a wait that gives up records SB_ETIMEOUT.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "sb_device.cuh"
+#include "sb_kernels.h"
+
+namespace sb {
+
+constexpr int kStages = 4;
+constexpr int kOffB = 16384;      // A: 128 rows x 128 B
+constexpr int kOffSFA = 49152;    // B: up to 256 rows x 128 B
+constexpr int kOffSFB = 51200;    // SFA: 4 atoms x 512 B
+constexpr int kStageBytes = 55296;  // SFB: 2 row tiles x 4 atoms x 512 B
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+constexpr uint64_t kDrainNs = 20000000ull;   // 20 ms to let in-flight copies land after an abort
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+
+enum { KIND_FP4 = 0, KIND_I8 = 1, KIND_BF16 = 2 };
+
+struct TMaps {
+  CUtensorMap a[3];
+  CUtensorMap b[3];
+};
+
+struct GemmParams {
+  int M, N, K;
+  float invB;
+  const int32_t* prec;
+  int bn[3];
+  int have[3];
+  const float* sA8;
+  const float* sB8;
+  const uint8_t* sfA4;
+  const uint8_t* sfB4;
+  const float* gA4;
+  const float* gB4;
+  const __nv_bfloat16* bias;
+  void* Y;
+  int out_dtype;
+  int epilogue;
+  WsHeader* hdr;
+};
+
+__device__ __forceinline__ uint32_t idesc_for(int kind, int BN) {
+  const uint32_t n = (uint32_t)(BN >> 3) << 17;
+  const uint32_t m = (uint32_t)(128 >> 4) << 24;
+  switch (kind) {
+    case KIND_FP4:  // block-scaled: A,B = E2M1 (1), scale type UE4M3 (bit 23 = 0), K = 64
+      return (1u << 7) | (1u << 10) | n | m;
+    case KIND_I8:  // D = S32 (2), A,B signed 8-bit (1)
+      return (2u << 4) | (1u << 7) | (1u << 10) | n | m;
+    default:  // D = F32 (1), A,B = BF16 (1)
+      return (1u << 4) | (1u << 7) | (1u << 10) | n | m;
+  }
+}
+
+// tanh-form GELU; tanh(u) = 1 - 2 / (exp(2u) + 1) with |u| clamped at 15 (tanh(15) rounds to 1).
+__device__ __forceinline__ float gelu_tanh(float v) {
+  const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);
+  const float uc = fminf(fmaxf(u, -15.0f), 15.0f);
+  const float e = __expf(2.0f * uc);
+  const float t = 1.0f - __fdividef(2.0f, e + 1.0f);
+  return 0.5f * v * (1.0f + t);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ TMaps tm, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kind = *p.prec;
+  if (kind < 0 || kind > 2) return;  // skipped module: nothing to compute
+  if (!p.have[kind]) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_error(p.hdr, SB_EINVAL);
+    return;
+  }
+  const int M = p.M, N = p.N, K = p.K;
+  const int BN = p.bn[kind];
+  const int kb_elems = (kind == KIND_FP4) ? 256 : (kind == KIND_I8 ? 128 : 64);
+  const int mma_k = kb_elems >> 2;
+  const int nkb = (K + kb_elems - 1) / kb_elems;
+  const int m_tiles = (M + 127) >> 7;
+  const int n_tiles = (N + BN - 1) / BN;
+  const int tiles = m_tiles * n_tiles;
+  if ((int)blockIdx.x >= tiles) return;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t sfa_col = 2u * BN;        // NVFP4: 4 columns per MMA step (128 rows x 4 scales)
+  const uint32_t sfb_col = 2u * BN + 16u;  // NVFP4: 8 columns per MMA step (two 128-row tiles)
+  const int sf_atoms_k = K >> 6;           // 64-element scale atoms along K
+  const int sf_tiles_n = (N + 127) >> 7;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      prefetch_tmap(&tm.a[kind]);
+      prefetch_tmap(&tm.b[kind]);
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        const int mt = tile % m_tiles, nt = tile / m_tiles;
+        const int m0 = mt * 128, n0 = nt * BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStageBytes;
+          uint32_t bytes = 16384u + (uint32_t)BN * 128u;
+          int atoms = 0, btiles = 0;
+          if (kind == KIND_FP4) {
+            atoms = min(4, sf_atoms_k - 4 * kb);
+            const int t0 = n0 >> 7;
+            btiles = min((n0 % 128 + BN + 127) >> 7, sf_tiles_n - t0);
+            bytes += (uint32_t)atoms * 512u * (uint32_t)(1 + btiles);
+          }
+          mbar_arrive_expect_tx(&full[s], bytes);
+          const int x = (kind == KIND_BF16) ? kb * 64 : kb * 128;
+          tma_load_2d(st, &tm.a[kind], &full[s], x, m0);
+          tma_load_2d(st + kOffB, &tm.b[kind], &full[s], x, n0);
+          if (kind == KIND_FP4) {
+            bulk_load(st + kOffSFA, p.sfA4 + ((int64_t)mt * sf_atoms_k + 4 * kb) * 512, atoms * 512u, &full[s]);
+            const int t0 = n0 >> 7;
+            for (int t = 0; t < btiles; ++t)
+              bulk_load(st + kOffSFB + 2048 * t, p.sfB4 + ((int64_t)(t0 + t) * sf_atoms_k + 4 * kb) * 512,
+                        atoms * 512u, &full[s]);
+          }
+          ++issued;
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        set_error(p.hdr, SB_ETIMEOUT);
+        *abort_flag = 1;
+        // let the copies already issued land before the CTA releases its shared memory
+        const int64_t first = issued > kStages ? issued - kStages : 0;
+        for (int64_t k = first; k < issued; ++k)
+          mbar_wait_bounded(&full[k % kStages], (uint32_t)((k / kStages) & 1), nullptr, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      const uint32_t idesc = idesc_for(kind, BN);
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x, ++it) {
+        const int nt = tile / m_tiles;
+        const int n0 = nt * BN;
+        const int b = it & 1;
+        const uint32_t tph = (uint32_t)((it >> 1) & 1);
+        if (!mbar_wait_bounded(&tempty[b], tph ^ 1u, abort_flag, kWaitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
+        const int btiles = (kind == KIND_FP4) ? min((n0 % 128 + BN + 127) >> 7, sf_tiles_n - (n0 >> 7)) : 0;
+        const uint32_t sfb_shift = (uint32_t)((n0 % 128) >> 5);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&full[s], ph, abort_flag, kWaitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_s = smem_u32(smem + s * kStageBytes);
+          const uint32_t b_s = a_s + kOffB;
+          const int nk = min(4, (K - kb * kb_elems) / mma_k);
+          if (kind == KIND_FP4) {
+            for (int j = 0; j < nk; ++j) {
+              tmem_cp_sf(tmem_base + sfa_col + 4u * j, desc_sf(a_s + kOffSFA + 512u * j));
+              for (int t = 0; t < btiles; ++t)
+                tmem_cp_sf(tmem_base + sfb_col + 8u * j + 4u * t, desc_sf(a_s + kOffSFB + 2048u * t + 512u * j));
+            }
+          }
+          for (int j = 0; j < nk; ++j) {
+            const uint64_t ad = desc_sw128(a_s + 32u * j);
+            const uint64_t bd = desc_sw128(b_s + 32u * j);
+            const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
+            if (kind == KIND_FP4)
+              mma_fp4(d_tmem, ad, bd, idesc, tmem_base + sfa_col + 4u * j, tmem_base + sfb_col + 8u * j + sfb_shift,
+                      acc);
+            else if (kind == KIND_I8)
+              mma_i8(d_tmem, ad, bd, idesc, acc);
+            else
+              mma_bf16(d_tmem, ad, bd, idesc, acc);
+          }
+          mma_commit(&empty[s]);  // the stage is free once these MMAs have read it
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (ok) mma_commit(&tfull[b]);  // accumulator ready for the epilogue
+      }
+      if (!ok) {
+        set_error(p.hdr, SB_ETIMEOUT);
+        *abort_flag = 1;
+      }
+      // wait for every MMA issued by this thread before TMEM is released
+      mma_commit(drain);
+      mbar_wait_bounded(drain, 0u, nullptr, kWaitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;          // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;  // two warps per quadrant split the column chunks
+    const int row = 32 * q + lane;
+    float alpha = 1.0f;
+    if (kind == KIND_FP4) alpha = __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      const int m = mt * 128 + row, n0 = nt * BN;
+      const int b = it & 1;
+      const uint32_t tph = (uint32_t)((it >> 1) & 1);
+      if (!mbar_wait_bounded(&tfull[b], tph, abort_flag, kWaitNs)) {
+        set_error(p.hdr, SB_ETIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const bool row_ok = m < M;
+      const float sx = (kind == KIND_I8 && row_ok) ? p.sA8[m] : 0.0f;
+      for (int c = half; c < BN / 32; c += 2) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN + 32 * c), r);
+        tmem_ld_wait();
+        const int n = n0 + 32 * c;
+        if (!row_ok || n >= N) continue;
+        if (p.out_dtype == SB_OUT_RAW) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(p.Y) + (int64_t)m * N + n);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+          continue;
+        }
+        float y[32];
+        if (kind == KIND_I8) {
+          const float sxb = __fmul_rn(sx, p.invB);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__int2float_rn((int)r[i]), __fmul_rn(sxb, __ldg(p.sB8 + n + i)));
+        } else if (kind == KIND_FP4) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
+        }
+        if (p.bias) {
+          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 u = __ldg(bp + i);
+            float bv[8];
+            unpack8(u, bv);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) y[8 * i + j] = __fadd_rn(y[8 * i + j], bv[j]);
+          }
+        }
+        if (p.epilogue == SB_EPI_GELU_TANH) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = gelu_tanh(y[i]);
+        }
+        if (p.out_dtype == SB_OUT_F32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.Y) + (int64_t)m * N + n);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.Y) + (int64_t)m * N + n);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(pack_bf16(y[8 * i], y[8 * i + 1]), pack_bf16(y[8 * i + 2], y[8 * i + 3]),
+                                pack_bf16(y[8 * i + 4], y[8 * i + 5]), pack_bf16(y[8 * i + 6], y[8 * i + 7]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[b]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------------------------
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2-D row-major map: `inner` elements per row, `outer` rows; box = 128 bytes x box_rows, SW128.
+static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
+                     uint64_t outer, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int device_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) {
+    *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
+    return attr_err;
+  }
+  TMaps tm;
+  memset(&tm, 0, sizeof(tm));
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = (int)L.M;
+  p.N = (int)L.N;
+  p.K = (int)L.K;
+  p.invB = 1.0f / (float)L.B;
+  p.prec = L.prec;
+  p.bn[KIND_FP4] = (L.N % 192 == 0) ? 192 : 128;
+  p.bn[KIND_I8] = (L.N % 256 == 0) ? 256 : 128;
+  p.bn[KIND_BF16] = p.bn[KIND_I8];
+  p.sA8 = L.sA8;
+  p.sB8 = L.sB8;
+  p.sfA4 = L.sfA4;
+  p.sfB4 = L.sfB4;
+  p.gA4 = L.gA4;
+  p.gB4 = L.gB4;
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(L.bias);
+  p.Y = L.Y;
+  p.out_dtype = L.out_dtype;
+  p.epilogue = L.epilogue;
+  p.hdr = reinterpret_cast<WsHeader*>(L.hdr);
+  const uint64_t M = (uint64_t)L.M, N = (uint64_t)L.N, K = (uint64_t)L.K;
+  if (L.A4 && L.B4 && L.sfA4 && L.sfB4 && L.gA4 && L.gB4) {
+    if (!make_map(&tm.a[KIND_FP4], L.A4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128) ||
+        !make_map(&tm.b[KIND_FP4], L.B4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, (uint32_t)p.bn[KIND_FP4])) {
+      *why = "cuTensorMapEncodeTiled failed (NVFP4 operands)";
+      return cudaErrorInvalidValue;
+    }
+    p.have[KIND_FP4] = 1;
+  }
+  if (L.A8 && L.B8 && L.sA8 && L.sB8) {
+    if (!make_map(&tm.a[KIND_I8], L.A8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128) ||
+        !make_map(&tm.b[KIND_I8], L.B8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, (uint32_t)p.bn[KIND_I8])) {
+      *why = "cuTensorMapEncodeTiled failed (INT8 operands)";
+      return cudaErrorInvalidValue;
+    }
+    p.have[KIND_I8] = 1;
+  }
+  if (L.X && L.W16) {
+    if (!make_map(&tm.a[KIND_BF16], L.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 128) ||
+        !make_map(&tm.b[KIND_BF16], L.W16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, (uint32_t)p.bn[KIND_BF16])) {
+      *why = "cuTensorMapEncodeTiled failed (BF16 operands)";
+      return cudaErrorInvalidValue;
+    }
+    p.have[KIND_BF16] = 1;
+  }
+  int64_t max_tiles = 0;
+  for (int k = 0; k < 3; ++k) {
+    const int64_t t = ceil_div(L.M, 128) * ceil_div(L.N, p.bn[k]);
+    if (t > max_tiles) max_tiles = t;
+  }
+  const int sms = device_sms();
+  const unsigned grid = (unsigned)(max_tiles < sms ? max_tiles : sms);
+  k_gemm<<<grid, kThreads, kSmemBytes, s>>>(tm, p);
+  return cudaGetLastError();
+}
+
+}  // namespace sb

@@ -1,0 +1,90 @@
+// sb_kernels.h -- internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sixbit.h"
+
+namespace sb {
+
+struct PrepassLaunch {
+  const void* X;
+  const void* R;
+  int64_t M, K;
+  int B;
+  int mode;
+  int32_t* prec;
+  int force_int8;
+  int8_t* q8;
+  float* s8;
+  double rho;
+  int force;
+  void* groups;
+  void* hdr;
+  sb_stats* stats;
+};
+
+struct Nvfp4Launch {
+  const void* X;
+  int64_t M, K;
+  int B;
+  const int32_t* prec;
+  const sb_stats* stats;
+  uint8_t* codes;
+  uint8_t* sf;
+  float* gscale;
+};
+
+struct TdcLaunch {
+  const void* Y;
+  void* Cache;
+  int64_t M, C;
+  int update;
+  const sb_stats* dsrc;
+  sb_module_state* st;
+  void* groups;
+  void* hdr;
+};
+
+struct GemmLaunch {
+  int64_t M, N, K;
+  int B;
+  const int32_t* prec;
+  // BF16 path
+  const void* X;
+  const void* W16;
+  // INT8 path
+  const int8_t* A8;
+  const float* sA8;
+  const int8_t* B8;
+  const float* sB8;
+  // NVFP4 path
+  const uint8_t* A4;
+  const uint8_t* sfA4;
+  const float* gA4;
+  const uint8_t* B4;
+  const uint8_t* sfB4;
+  const float* gB4;
+  const void* bias;
+  int epilogue;
+  int out_dtype;
+  void* Y;
+  void* hdr;
+};
+
+cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s);
+cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s);
+cudaError_t launch_rotate(const void* X, float* Y, int64_t M, int64_t K, int B, cudaStream_t s);
+cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s);
+cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t s, const char** why);
+
+cudaError_t launch_state_init(sb_module_state* st, cudaStream_t s);
+cudaError_t launch_tdc_step(sb_module_state* st, double thr, cudaStream_t s);
+cudaError_t launch_select(const sb_module_state* st, double a, double b, double tau, int force, int32_t* prec,
+                          cudaStream_t s);
+cudaError_t launch_set_i32(int32_t* p, int32_t v, cudaStream_t s);
+cudaError_t launch_ws_init(void* ws, size_t bytes, cudaStream_t s);
+
+}  // namespace sb

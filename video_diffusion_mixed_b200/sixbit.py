@@ -1,0 +1,255 @@
+"""ctypes binding of libsixbit.so (include/sixbit.h), argument marshalling only.
+
+Every function here forwards torch tensors' device pointers and the current CUDA stream to the
+C ABI; all computation happens in the library's sm_100a kernels. Importing this module fails
+loudly when the library has not been built (there is no fallback path).
+
+Allocation helpers (``alloc_fp4``, ``alloc_i8``, ``Workspace``, ``prepare_weight``...) create the
+caller-owned device buffers with torch; the library itself never allocates.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsixbit.so")
+
+SB_OK, SB_EINVAL, SB_ESHAPE, SB_EALIGN, SB_EUNSUPPORTED, SB_ECUDA, SB_ETIMEOUT, SB_ENONFINITE = range(8)
+STATUS_NAMES = ["SB_OK", "SB_EINVAL", "SB_ESHAPE", "SB_EALIGN", "SB_EUNSUPPORTED", "SB_ECUDA", "SB_ETIMEOUT",
+                "SB_ENONFINITE"]
+NVFP4, INT8, BF16, SKIP = 0, 1, 2, 3
+PREC_NAMES = {NVFP4: "nvfp4", INT8: "int8", BF16: "bf16", SKIP: "skip"}
+OUT_BF16, OUT_F32, OUT_RAW = 0, 1, 2
+EPI_NONE, EPI_GELU = 0, 1
+PREPASS_QUANT, PREPASS_STATS = 0, 1
+
+
+class SixbitError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else status}: {msg}")
+        self.status = status
+
+
+class Fp4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("gscale", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+class I8(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64)]
+
+
+class WeightC(ctypes.Structure):
+    _fields_ = [("w_bf16", ctypes.c_void_p), ("bias_bf16", ctypes.c_void_p), ("w4", Fp4), ("w8", I8),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("block", ctypes.c_int32)]
+
+
+class Rule(ctypes.Structure):
+    _fields_ = [("a", ctypes.c_double), ("b", ctypes.c_double), ("tau", ctypes.c_double)]
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("rho", ctypes.c_double), ("tdc_thresh", ctypes.c_double), ("block", ctypes.c_int32),
+                ("force_prec", ctypes.c_int32)]
+
+
+STATE_BYTES = 64
+STATS_BYTES = 96
+STATE_FIELDS = ("prev_d", "acc", "delta", "have_d", "n_out", "last_skipped", "skip", "steps")
+STATS_FIELDS = ("sum_abs", "sum_d2", "sum_ref2", "max_abs", "amax_rot", "ratio", "d", "numel", "has_ref",
+                "prec_in", "prec_out", "nonfinite")
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m video_diffusion_mixed_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+        P = ctypes.POINTER
+        sig = {
+            "sb_version": (ctypes.c_char_p, []),
+            "sb_last_error": (ctypes.c_char_p, []),
+            "sb_workspace_size": (st, [i64, i64, P(ctypes.c_size_t)]),
+            "sb_workspace_init": (st, [vp, ctypes.c_size_t, vp]),
+            "sb_fp4_sf_bytes": (i64, [i64, i64]),
+            "sb_state_init": (st, [vp, vp]),
+            "sb_rotate": (st, [vp, vp, i64, i64, i32, vp]),
+            "sb_prepare_weight": (st, [vp, vp, i64, i64, i32, P(WeightC), vp, vp]),
+            "sb_tdc_step": (st, [vp, P(Config), vp]),
+            "sb_select_precision": (st, [vp, P(Rule), P(Config), vp, vp]),
+            "sb_prepass": (st, [vp, vp, i64, i64, P(Config), i32, vp, P(Fp4), P(I8), vp, vp, vp]),
+            "sb_linear": (st, [vp, P(Fp4), P(I8), vp, P(WeightC), i32, i32, vp, i64, vp, vp]),
+            "sb_tdc_record": (st, [vp, vp, i64, i64, vp, i32, vp, vp, vp]),
+            "sb_check": (st, [vp, vp]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_init", "sb_fp4_sf_bytes",
+            "sb_state_init", "sb_rotate", "sb_prepare_weight", "sb_tdc_step", "sb_select_precision", "sb_prepass",
+            "sb_linear", "sb_tdc_record", "sb_check")
+
+
+def _ck(status: int):
+    if status != SB_OK:
+        raise SixbitError(status, lib().sb_last_error().decode())
+
+
+def _p(t):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "device tensors must be contiguous CUDA tensors"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def version() -> str:
+    return lib().sb_version().decode()
+
+
+# ------------------------------------------------------------------------------------------------
+# Caller-owned buffers
+# ------------------------------------------------------------------------------------------------
+
+class Workspace:
+    def __init__(self, max_M: int, max_K: int, device="cuda", stream=None):
+        n = ctypes.c_size_t(0)
+        _ck(lib().sb_workspace_size(max_M, max_K, ctypes.byref(n)))
+        self.bytes = n.value
+        self.buf = torch.empty(self.bytes, dtype=torch.uint8, device=device)
+        _ck(lib().sb_workspace_init(_p(self.buf), self.bytes, _stream(stream)))
+
+    @property
+    def ptr(self):
+        return _p(self.buf)
+
+
+class Fp4Tensor:
+    def __init__(self, rows: int, cols: int, device="cuda"):
+        self.rows, self.cols = rows, cols
+        self.codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+        self.sf = torch.empty(int(lib().sb_fp4_sf_bytes(rows, cols)), dtype=torch.uint8, device=device)
+        self.gscale = torch.empty(4, dtype=torch.float32, device=device)  # 16-byte slot, element 0 used
+
+    def c(self) -> Fp4:
+        return Fp4(self.codes.data_ptr(), self.sf.data_ptr(), self.gscale.data_ptr(), self.rows, self.cols)
+
+
+class I8Tensor:
+    def __init__(self, rows: int, cols: int, device="cuda"):
+        self.rows, self.cols = rows, cols
+        self.codes = torch.empty((rows, cols), dtype=torch.int8, device=device)
+        self.scale = torch.empty(rows, dtype=torch.float32, device=device)
+
+    def c(self) -> I8:
+        return I8(self.codes.data_ptr(), self.scale.data_ptr(), self.rows, self.cols)
+
+
+class Weight:
+    """A prepared linear layer: original bf16 weight + bias, rotated NVFP4 and INT8 copies."""
+
+    def __init__(self, W: torch.Tensor, bias: torch.Tensor | None, block: int = 128, ws: Workspace | None = None,
+                 stream=None):
+        N, K = W.shape
+        self.W, self.bias, self.N, self.K, self.block = W.contiguous(), bias, N, K, block
+        self.w4 = Fp4Tensor(N, K, W.device)
+        self.w8 = I8Tensor(N, K, W.device)
+        self._c = WeightC()
+        self._c.w4 = self.w4.c()
+        self._c.w8 = self.w8.c()
+        ws = ws or Workspace(N, K, W.device, stream)
+        _ck(lib().sb_prepare_weight(_p(self.W), _p(bias), N, K, block, ctypes.byref(self._c), ws.ptr,
+                                    _stream(stream)))
+
+    def c(self) -> WeightC:
+        return self._c
+
+
+def alloc_state(device="cuda", stream=None) -> torch.Tensor:
+    st = torch.empty(STATE_BYTES, dtype=torch.uint8, device=device)
+    _ck(lib().sb_state_init(_p(st), _stream(stream)))
+    return st
+
+
+def alloc_stats(device="cuda") -> torch.Tensor:
+    return torch.zeros(STATS_BYTES, dtype=torch.uint8, device=device)
+
+
+def decode_state(buf: torch.Tensor) -> dict:
+    h = buf.detach().cpu()
+    d = h[:24].view(torch.float64).tolist()
+    i = h[24:44].view(torch.int32).tolist()
+    return dict(zip(STATE_FIELDS, d + i))
+
+
+def decode_stats(buf: torch.Tensor) -> dict:
+    h = buf.detach().cpu()
+    d = h[:64].view(torch.float64).tolist()
+    i = h[64:80].view(torch.int32).tolist()
+    return dict(zip(STATS_FIELDS, d + i))
+
+
+def config(rho: float = 64.0, tdc_thresh: float = 0.1, block: int = 128, force_prec: int = -1) -> Config:
+    return Config(rho, tdc_thresh, block, force_prec)
+
+
+# ------------------------------------------------------------------------------------------------
+# Entry points (same names as the C ABI, minus the prefix)
+# ------------------------------------------------------------------------------------------------
+
+def rotate(X: torch.Tensor, Y: torch.Tensor, block: int = 128, stream=None):
+    M, K = X.shape
+    _ck(lib().sb_rotate(_p(X), _p(Y), M, K, block, _stream(stream)))
+
+
+def tdc_step(state: torch.Tensor, cfg: Config, stream=None):
+    _ck(lib().sb_tdc_step(_p(state), ctypes.byref(cfg), _stream(stream)))
+
+
+def select_precision(state: torch.Tensor, rule: Rule, cfg: Config, prec: torch.Tensor, stream=None):
+    _ck(lib().sb_select_precision(_p(state), ctypes.byref(rule), ctypes.byref(cfg), _p(prec), _stream(stream)))
+
+
+def prepass(X, X_ref, cfg: Config, mode: int, prec, a4: Fp4Tensor | None, a8: I8Tensor | None, stats, ws: Workspace,
+            stream=None):
+    M, K = X.shape
+    c4 = ctypes.byref(a4.c()) if a4 is not None else None
+    c8 = ctypes.byref(a8.c()) if a8 is not None else None
+    _ck(lib().sb_prepass(_p(X), _p(X_ref), M, K, ctypes.byref(cfg), mode, _p(prec), c4, c8, _p(stats), ws.ptr,
+                         _stream(stream)))
+
+
+def linear(X, a4: Fp4Tensor | None, a8: I8Tensor | None, prec, w: Weight, Y, epilogue: int = EPI_NONE,
+           out_dtype: int = OUT_BF16, ws: Workspace | None = None, stream=None):
+    M = Y.shape[0]
+    c4 = ctypes.byref(a4.c()) if a4 is not None else None
+    c8 = ctypes.byref(a8.c()) if a8 is not None else None
+    _ck(lib().sb_linear(_p(X), c4, c8, _p(prec), ctypes.byref(w.c()), epilogue, out_dtype, _p(Y), M, ws.ptr,
+                        _stream(stream)))
+
+
+def tdc_record(y_new, y_cache, d_src, state, ws: Workspace, update_cache: bool = True, stream=None):
+    M, C = y_new.shape
+    _ck(lib().sb_tdc_record(_p(y_new), _p(y_cache), M, C, _p(d_src), int(update_cache), _p(state), ws.ptr,
+                            _stream(stream)))
+
+
+def check(ws: Workspace, stream=None):
+    _ck(lib().sb_check(ws.ptr, _stream(stream)))
