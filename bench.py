@@ -1,0 +1,458 @@
+"""Benchmark of the 6Bit-Diffusion hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ffn5b] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one synthetic CogVideoX-5B FFN module input
+(17776 tokens x 3072 channels -> 12288 (GELU) -> 3072), run twice: all layers in NVFP4, then all
+layers in INT8 (the precision forced, as the synthetic activations' outlier channels would
+otherwise send every layer to the BF16 PDR path). Each pass: TDC check, precision selection,
+fused pre-pass + quantization of the layer input, tcgen05 GEMM (+GELU), pre-pass + quantization of
+the hidden tensor, tcgen05 GEMM, difference statistic of the module output against its input,
+TDC record (delta + cache refresh). The metric is the effective tensor throughput of the step
+(4 GEMMs of 2*M*N*K each / step time). Under torchrun every rank runs its own replica on its own
+batch (weak scaling, no collective on the data path); time is the max over ranks.
+
+--impl reference times the CPU oracle (the plain C reference) on the machine's host cores on a row
+sample of the same step and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT shapes"
+
+# ncu DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel, from the capture summarised under profiles/; valid only for the gemm.cu it was taken on.
+TRAFFIC = {}
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc, self.lines = index, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------------------------------------
+# Our arm
+# ------------------------------------------------------------------------------------------------
+
+class FfnStep:
+    """All buffers of one FFN module step, allocated once (the library allocates nothing)."""
+
+    def __init__(self, sb, synth, torch, wl, seed, device, tokens=None):
+        self.sb, self.torch = sb, torch
+        X, layers = synth.workload_inputs(wl, seed=seed, device=device, bias_std=0.0, tokens=tokens)
+        self.X = X
+        self.M, self.C = X.shape
+        (self.N1, self.K1, g1), (self.N2, self.K2, g2) = [(l["N"], l["K"], l["gelu"]) for l in layers]
+        self.ws = sb.Workspace(max(self.M, self.N1, self.N2), max(self.K1, self.K2))
+        self.w1 = sb.Weight(layers[0]["W"], layers[0]["bias"], 128, self.ws)
+        self.w2 = sb.Weight(layers[1]["W"], layers[1]["bias"], 128, self.ws)
+        self.ax4, self.ax8 = sb.Fp4Tensor(self.M, self.K1), sb.I8Tensor(self.M, self.K1)
+        self.ah4, self.ah8 = sb.Fp4Tensor(self.M, self.K2), sb.I8Tensor(self.M, self.K2)
+        self.H = torch.empty((self.M, self.N1), dtype=torch.bfloat16, device=device)
+        self.Y = torch.empty((self.M, self.N2), dtype=torch.bfloat16, device=device)
+        self.cache = torch.zeros_like(self.Y)
+        self.state = sb.alloc_state()
+        self.sx, self.sh, self.sy = sb.alloc_stats(), sb.alloc_stats(), sb.alloc_stats()
+        self.p1 = torch.zeros(1, dtype=torch.int32, device=device)
+        self.p2 = torch.zeros(1, dtype=torch.int32, device=device)
+        self.rule = sb.Rule(1.0, 0.0, 0.1)
+        self.events = None
+        torch.cuda.synchronize()
+
+    def gemm_flops(self):
+        return 2.0 * self.M * (self.N1 * self.K1 + self.N2 * self.K2)
+
+    def one_pass(self, prec, ev=None):
+        sb = self.sb
+        cfg = sb.config(rho=64.0, tdc_thresh=-1.0, block=128, force_prec=prec)  # never skip: full work
+        sb.tdc_step(self.state, cfg)
+        sb.select_precision(self.state, self.rule, cfg, self.p1)
+        self._mark(ev, "pre1_0")
+        sb.prepass(self.X, None, cfg, sb.PREPASS_QUANT, self.p1, self.ax4, self.ax8, self.sx, self.ws)
+        self._mark(ev, "pre1_1")
+        sb.linear(self.X, self.ax4, self.ax8, self.p1, self.w1, self.H, epilogue=sb.EPI_GELU, ws=self.ws)
+        self._mark(ev, "gemm1_1")
+        sb.select_precision(self.state, self.rule, cfg, self.p2)
+        self._mark(ev, "pre2_0")
+        sb.prepass(self.H, None, cfg, sb.PREPASS_QUANT, self.p2, self.ah4, self.ah8, self.sh, self.ws)
+        self._mark(ev, "pre2_1")
+        sb.linear(self.H, self.ah4, self.ah8, self.p2, self.w2, self.Y, ws=self.ws)
+        self._mark(ev, "gemm2_1")
+        sb.prepass(self.Y, self.X, cfg, sb.PREPASS_STATS, self.p2, None, None, self.sy, self.ws)
+        self._mark(ev, "d_1")
+        sb.tdc_record(self.Y, self.cache, self.sy, self.state, self.ws)
+        self._mark(ev, "tdc_1")
+
+    def _mark(self, ev, name):
+        if ev is not None:
+            e = self.torch.cuda.Event(enable_timing=True)
+            e.record()
+            ev.append((name, e))
+
+    def step(self, ev=None):
+        for prec in (self.sb.NVFP4, self.sb.INT8):
+            sub = [] if ev is not None else None
+            self.one_pass(prec, sub)
+            if ev is not None:
+                ev.append((prec, sub))
+
+
+LAUNCHES_PER_PASS = 11  # tdc_step, select, prepass(2), gemm, select, prepass(2), gemm, stats prepass, tdc record
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    from video_diffusion_mixed_b200 import build as b
+    b.build()
+    from video_diffusion_mixed_b200 import sixbit as sb
+    from video_diffusion_mixed_b200 import synth
+
+    S = FfnStep(sb, synth, torch, args.workload, seed=rank, device=device, tokens=args.tokens)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)  # > 126 MB L2
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        S.step()
+    sb.check(S.ws)
+    barrier()
+
+    # ---- timed: K steps; an L2 flush before each step, excluded by per-step events
+    clk = ClockSampler(local)
+    clk.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record()
+        S.step()
+        ends[i].record()
+    barrier()
+    t_wall = time.perf_counter() - t_wall0
+    clocks = clk.stop()
+    sb.check(S.ws)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    flops = 2 * S.gemm_flops()  # both precision passes
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+
+    # ---- per-kernel breakdown (a separate, untimed-for-value pass with events between calls)
+    kern = {}
+    reps = max(3, min(args.steps, 10))
+    for _ in range(reps):
+        flush.zero_()
+        ev = []
+        S.step(ev)
+        torch.cuda.synchronize()
+        for prec, sub in ev:
+            tag = sb.PREC_NAMES[prec]
+            d = dict(sub)
+            for name, a, z in (("prepass_x", "pre1_0", "pre1_1"), ("gemm_w1", "pre1_1", "gemm1_1"),
+                               ("prepass_h", "pre2_0", "pre2_1"), ("gemm_w2", "pre2_1", "gemm2_1"),
+                               ("stats_d", "gemm2_1", "d_1"), ("tdc_record", "d_1", "tdc_1")):
+                kern.setdefault(f"{name}_{tag}", []).append(d[a].elapsed_time(d[z]))
+    kern_ms = {k: statistics.median(v) for k, v in kern.items()}
+
+    # ---- end to end through the public API with host buffers (pinned H2D of X, D2H of Y)
+    Xh = torch.empty(S.X.shape, dtype=S.X.dtype, pin_memory=True)
+    Xh.copy_(S.X.cpu())
+    Yh = torch.empty(S.Y.shape, dtype=S.Y.dtype, pin_memory=True)
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        e_s[i].record()
+        S.X.copy_(Xh, non_blocking=True)
+        for prec in (sb.NVFP4, sb.INT8):
+            S.one_pass(prec)
+            Yh.copy_(S.Y, non_blocking=True)
+        e_e[i].record()
+    barrier()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops / (e2e_ms / args.steps * 1e-3) / 1e12
+    h2d = S.X.numel() * S.X.element_size()
+    d2h = 2 * S.Y.numel() * S.Y.element_size()
+
+    # ---- roofline of the dominant kernel and of the fused pre-pass
+    pk = peaks()
+    ratio = {"nvfp4": 4.0, "int8": 2.0}  # nominal dense ratio to bf16 (9 / 4.5 / 2.25 PFLOP/s)
+    M, K1, N1, K2, N2 = S.M, S.K1, S.N1, S.K2, S.N2
+    gemm_flops = {"gemm_w1": 2.0 * M * N1 * K1, "gemm_w2": 2.0 * M * N2 * K2}
+    rows = []
+    for k, ms in kern_ms.items():
+        base, tag = k.rsplit("_", 1)
+        if base in gemm_flops:
+            ach = gemm_flops[base] / (ms * 1e-3) / 1e12
+            peak = pk["bf16_tflops_sustained"] * ratio[tag]
+            rows.append({"kernel": k, "bound": "tensor", "ms": ms, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                         "frac": ach / peak})
+        else:
+            Kx = {"prepass_x": K1, "prepass_h": K2, "stats_d": N2, "tdc_record": N2}[base]
+            el = M * Kx
+            if base in ("prepass_x", "prepass_h"):
+                # algorithmic bytes: read bf16 X, write the quantized form of the chosen precision
+                byt = el * 2 + (el * 1 + M * 4 if tag == "int8" else el * (0.5 + 1 / 16) + 4)
+            elif base == "stats_d":
+                byt = el * 4  # read y and x
+            else:
+                byt = el * 6  # read y_new and the cache, refresh the cache
+            ach = byt / (ms * 1e-3) / 1e9
+            rows.append({"kernel": k, "bound": "hbm", "ms": ms, "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"]})
+    dom = max(rows, key=lambda r: r["ms"])
+    src_sha = file_sha(os.path.join(ROOT, "video_diffusion_mixed_b200", "csrc", "gemm.cu"))
+    tr = TRAFFIC.get(dom["kernel"])
+    traffic = tr["bytes"] if (tr and tr.get("src_sha") == src_sha) else None
+    roofline = {"bound": dom["bound"], "achieved": round(dom["achieved"], 1), "peak": round(dom["peak"], 1),
+                "unit": dom["unit"], "frac": round(dom["frac"], 4), "traffic": traffic, "kernel": dom["kernel"],
+                "peak_src": f"{pk['src']} bf16 sustained x nominal dtype ratio" if dom["bound"] == "tensor"
+                else f"{pk['src']} HBM copy"}
+    pre = [r for r in rows if r["kernel"].startswith("prepass")]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4+int8 (fp32 accumulate), bf16 activations", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: CogVideoX-5B FFN, X [{M} x {K1}] bf16 (0.5% outlier channels x50) "
+                               f"-> W1 [{N1} x {K1}] (GELU) -> W2 [{N2} x {K2}]; NVFP4 pass + INT8 pass per step",
+                   "tokens": M, "hidden": K1, "ffn": N1, "hadamard_block": 128, "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every step (512 MiB memset, outside the per-step events)"},
+        "roofline": roofline,
+        "roofline_prepass": {r["kernel"]: {"achieved_gbs": round(r["achieved"], 1), "frac": round(r["frac"], 4),
+                                           "ms": round(r["ms"], 4)} for r in pre},
+        "kernels": {r["kernel"]: {"ms": round(r["ms"], 4), "achieved": round(r["achieved"], 1), "unit": r["unit"],
+                                  "frac": round(r["frac"], 4)} for r in rows},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": LAUNCHES_PER_PASS * 2 * args.steps,
+        "clocks": clocks,
+        "wall_s_timed": round(t_wall, 3),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args, S.X, S.w1.W, S.w2.W)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# The oracle on host cores (cpu_baseline leg and the reference arm)
+# ------------------------------------------------------------------------------------------------
+
+_WP = {}
+
+
+def oracle_weights(W1_u16, W2_u16, B=128):
+    """Offline weight preparation by the oracle (rotation, NVFP4 and INT8 copies), cached."""
+    import oracle
+    key = (W1_u16.ctypes.data, W2_u16.ctypes.data, B)
+    if key not in _WP:
+        _WP[key] = (oracle.prepare_weight(W1_u16, B), oracle.prepare_weight(W2_u16, B))
+    return _WP[key]
+
+
+def oracle_sample_step(X_u16, W1_u16, W2_u16, rows, B=128):
+    """The oracle's version of one step restricted to `rows` tokens: pre-pass + quantization of
+    the sampled X rows, W1 GEMM (+GELU) in NVFP4 and in INT8, bf16 rounding of the hidden rows,
+    their pre-pass + quantization, W2 GEMM. Weight preparation is offline (not timed).
+    Returns the GEMM FLOPs it performed and the seconds it took."""
+    import numpy as np
+    import oracle
+    xs = np.ascontiguousarray(X_u16[rows])
+    n = len(rows)
+    flops = 0.0
+    wp1, wp2 = oracle_weights(W1_u16, W2_u16, B)
+    t0 = time.perf_counter()
+    st = oracle.prepass(xs, None, B)
+    q8, s8 = oracle.quant_int8(st["y"], st["row_amax"])
+    c4, sf, _, sg = oracle.quant_nvfp4(st["y"], st["amax_rot"])
+    for prec in ("nvfp4", "int8"):
+        if prec == "nvfp4":
+            h = oracle.gemm_nvfp4(c4, sf, sg, wp1["c4"], wp1["sf4"], wp1["sg4"], None, W1_u16.shape[1], B, gelu=True)
+        else:
+            h = oracle.gemm_int8(q8, s8, wp1["q8"], wp1["s8"], None, B, gelu=True)
+        hb = oracle.f32_to_bf16(h.astype(np.float32))
+        sh = oracle.prepass(hb, None, B)
+        if prec == "nvfp4":
+            c, f, _, g = oracle.quant_nvfp4(sh["y"], sh["amax_rot"])
+            oracle.gemm_nvfp4(c, f, g, wp2["c4"], wp2["sf4"], wp2["sg4"], None, W2_u16.shape[1], B)
+        else:
+            q, s = oracle.quant_int8(sh["y"], sh["row_amax"])
+            oracle.gemm_int8(q, s, wp2["q8"], wp2["s8"], None, B)
+        flops += 2.0 * n * (W1_u16.shape[0] * W1_u16.shape[1] + W2_u16.shape[0] * W2_u16.shape[1])
+    return flops, time.perf_counter() - t0
+
+
+def _u16(t):
+    import numpy as np
+    import torch
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def cpu_baseline(args, X, W1, W2):
+    import numpy as np
+    M = X.shape[0]
+    rows = np.linspace(0, M - 1, args.cpu_rows).round().astype(np.int64)
+    flops, secs = oracle_sample_step(_u16(X), _u16(W1), _u16(W2), rows)
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOPS", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{len(rows)} of {M} tokens (evenly spaced), both precision passes of the step; "
+                      f"{secs:.1f} s; weight preparation untimed"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    from video_diffusion_mixed_b200 import synth
+    import oracle
+    oracle.build()
+    X, layers = synth.workload_inputs(args.workload, seed=0, device="cpu", bias_std=0.0)
+    Xu, W1u, W2u = _u16(X), _u16(layers[0]["W"]), _u16(layers[1]["W"])
+    M = X.shape[0]
+    rows = np.linspace(0, M - 1, args.cpu_rows).round().astype(np.int64)
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        oracle_sample_step(Xu, W1u, W2u, rows[:2])
+    tot_f, tot_s = 0.0, 0.0
+    for _ in range(args.steps):
+        f, s = oracle_sample_step(Xu, W1u, W2u, rows)
+        tot_f += f
+        tot_s += s
+    value = tot_f / tot_s / 1e12
+    full_flops = 2 * 2.0 * M * (layers[0]["N"] * layers[0]["K"] + layers[1]["N"] * layers[1]["K"])
+    line = {
+        "metric": METRIC, "impl": "reference", "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(full_flops / (value * 1e12) * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload}: CogVideoX-5B FFN (same as our arm), row sample",
+                   "tokens": M, "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"{len(rows)} of {M} tokens per step, both precision passes"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="ffn5b", choices=["ffn5b", "ffn2b"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=32, help="tokens in the oracle's timed sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the token count (small profiling case; the bench line is then not the metric)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
