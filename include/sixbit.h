@@ -209,6 +209,24 @@ sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C,
                         const sb_stats* d_src, int32_t update_cache, sb_module_state* state,
                         void* ws, sb_stream stream);
 
+/* sb_prepass without a caller workspace. The paper has no counterpart: this exists for callers
+ * that cannot allocate device memory -- e.g. a plugin inside a host program that owns the whole
+ * device-memory pool and forbids other allocations, or a latency-critical loop that must never
+ * call cudaMalloc/cudaFree because they can synchronise the device. The scratch that sb_prepass
+ * keeps in `ws` lives instead in a 256 KiB array compiled into the library (present on every GPU
+ * that loads it, until the process exits); this call allocates nothing. Arguments and results are
+ * exactly those of sb_prepass; M may be at most SB_STATIC_MAX_ROWS (SB_ESHAPE otherwise, nothing
+ * launched). The first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress (that device must be current), so make that first call before any stream
+ * capture. Every call on a device shares the one array: calls that can overlap on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller. Device-side errors are
+ * reported in stats->nonfinite (there is no workspace for sb_check to read). */
+#define SB_STATIC_MAX_ROWS 65536
+sb_status sb_prepass_static(const void* X, const void* X_ref, int64_t M, int64_t K,
+                            const sb_config* cfg /* host */, int32_t mode, int32_t* prec,
+                            const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */, sb_stats* stats,
+                            sb_stream stream);
+
 /* Synchronise `stream`, read and clear the device error word of `ws`. Returns SB_OK,
  * SB_ETIMEOUT, SB_ENONFINITE, SB_EINVAL or SB_ECUDA. */
 sb_status sb_check(void* ws, sb_stream stream);

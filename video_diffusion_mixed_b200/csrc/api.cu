@@ -68,6 +68,11 @@ sb_status check_rows_cols(int64_t M, int64_t K, int32_t block) {
 
 }  // namespace
 
+namespace sb {
+// Lets other translation units of the library report a failure through sb_last_error().
+sb_status report_error(sb_status st, const char* msg) { return fail(st, "%s", msg); }
+}  // namespace sb
+
 extern "C" {
 
 const char* sb_version(void) { return "sixbit 0.1 (sm_100a)"; }

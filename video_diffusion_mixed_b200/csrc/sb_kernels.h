@@ -87,4 +87,6 @@ cudaError_t launch_select(const sb_module_state* st, double a, double b, double 
 cudaError_t launch_set_i32(int32_t* p, int32_t v, cudaStream_t s);
 cudaError_t launch_ws_init(void* ws, size_t bytes, cudaStream_t s);
 
+sb_status report_error(sb_status st, const char* msg);
+
 }  // namespace sb

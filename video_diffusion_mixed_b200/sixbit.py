@@ -89,6 +89,7 @@ def lib():
             "sb_linear": (st, [vp, P(Fp4), P(I8), vp, P(WeightC), i32, i32, vp, i64, vp, vp]),
             "sb_tdc_record": (st, [vp, vp, i64, i64, vp, i32, vp, vp, vp]),
             "sb_check": (st, [vp, vp]),
+            "sb_prepass_static": (st, [vp, vp, i64, i64, P(Config), i32, vp, P(Fp4), P(I8), vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -100,7 +101,7 @@ def lib():
 
 EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_init", "sb_fp4_sf_bytes",
             "sb_state_init", "sb_rotate", "sb_prepare_weight", "sb_tdc_step", "sb_select_precision", "sb_prepass",
-            "sb_linear", "sb_tdc_record", "sb_check")
+            "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static")
 
 
 def _ck(status: int):
@@ -234,6 +235,16 @@ def prepass(X, X_ref, cfg: Config, mode: int, prec, a4: Fp4Tensor | None, a8: I8
     c8 = ctypes.byref(a8.c()) if a8 is not None else None
     _ck(lib().sb_prepass(_p(X), _p(X_ref), M, K, ctypes.byref(cfg), mode, _p(prec), c4, c8, _p(stats), ws.ptr,
                          _stream(stream)))
+
+
+def prepass_static(X, X_ref, cfg: Config, mode: int, prec, a4: Fp4Tensor | None, a8: I8Tensor | None, stats,
+                   stream=None):
+    """sb_prepass with the library's built-in scratch (no workspace; see include/sixbit.h)."""
+    M, K = X.shape
+    c4 = ctypes.byref(a4.c()) if a4 is not None else None
+    c8 = ctypes.byref(a8.c()) if a8 is not None else None
+    _ck(lib().sb_prepass_static(_p(X), _p(X_ref), M, K, ctypes.byref(cfg), mode, _p(prec), c4, c8, _p(stats),
+                                _stream(stream)))
 
 
 def linear(X, a4: Fp4Tensor | None, a8: I8Tensor | None, prec, w: Weight, Y, epilogue: int = EPI_NONE,
