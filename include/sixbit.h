@@ -177,8 +177,9 @@ sb_status sb_select_precision(const sb_module_state* state, const sb_rule* rule 
  * In SB_PREPASS_QUANT mode PDR is applied: a quantized *prec becomes SB_BF16 when
  * stats->ratio > cfg->rho (unless cfg->force_prec >= 0). *prec == SB_SKIP makes every kernel exit
  * at once. SB_PREPASS_STATS computes the record only and leaves *prec unchanged (prec may be
- * NULL). a4/a8 may be NULL in STATS mode; in QUANT mode both must be given (the precision is only
- * known on the device). Requires M*K > 0, K % block == 0, K % 64 == 0, K <= 16384. */
+ * NULL) and does not rotate (stats->amax_rot is then 0). a4/a8 may be NULL in STATS mode; in QUANT
+ * mode both must be given (the precision is only known on the device). Requires M*K > 0,
+ * K % block == 0, K % 64 == 0, K <= 16384. */
 sb_status sb_prepass(const void* X, const void* X_ref, int64_t M, int64_t K,
                      const sb_config* cfg /* host */, int32_t mode, int32_t* prec,
                      const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */, sb_stats* stats,

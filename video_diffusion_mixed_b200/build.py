@@ -21,7 +21,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsixbit.so")
 SOURCES = ["api.cu", "prepass.cu", "decide.cu", "gemm.cu", "prepass_static.cu"]
-HEADERS = ["sb_device.cuh", "sb_kernels.h"]
+HEADERS = ["sb_device.cuh", "sb_kernels.h", "rows.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2,-Wall",
@@ -40,9 +40,14 @@ def _deps_mtime() -> float:
     return max(os.path.getmtime(f) for f in files)
 
 
+# Per-file flags. The streaming kernels must round every multiply and add separately (their
+# codes and statistics are compared bit for bit), so no multiply-add contraction there.
+FILE_FLAGS = {"prepass.cu": ["-fmad=false"]}
+
+
 def _compile(src: str, verbose: bool, extra=()) -> str:
     obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
-    cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
+    cmd = [nvcc(), *ARCH, *FLAGS, *FILE_FLAGS.get(src, []), *extra, "-c", os.path.join(CSRC, src), "-o", obj]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -1,528 +1,37 @@
 // prepass.cu -- streaming kernels of the activation pre-pass and of the Temporal Delta Cache.
 //
-//  k_prepass      one pass over X (and X_ref): block Hadamard rotation, per-token rotated amax,
-//                 per-row FP32 pairwise partials of |x|, (x - x_ref)^2, x_ref^2, FP64 partials
-//                 per aligned group of 32 rows, and (INT8 precision) the per-token INT8 codes.
-//                 The last CTA to finish reduces the groups, writes the statistics record and
-//                 applies Purified Delta Refresh to the layer's precision flag.
+//  k_rows<.., OP_PREPASS>  one pass over X (and X_ref): block Hadamard rotation, per-token rotated
+//                 amax, deterministic statistics (|x|, (x - x_ref)^2, x_ref^2), per-token INT8
+//                 codes when the layer runs in INT8; the last CTA reduces the groups, writes the
+//                 statistics record and applies Purified Delta Refresh to the precision flag.
 //                 ("write-up" sections 一 (difference statistic, block Hadamard), 三 (outlier
 //                 ratio max / mean), 四 (quantization fused with the Hadamard transform).)
+//  k_rows<.., OP_STATS>    the same statistics without rotation (the d of a module output).
+//  k_rows<.., OP_TDC>      relative L1 change between a module's new output and its cached last
+//                 output, cache refresh in the same pass, module-state update by the last CTA.
+//                 ("write-up" section 二; explainer section 3.)
 //  k_nvfp4        re-reads X once the tensor amax is known, rotates again and writes E2M1 codes,
 //                 E4M3 block scales in the tensor-core layout and the FP32 tensor scale.
-//  k_tdc_record   relative L1 change between a module's new output and its cached last output,
-//                 with the same deterministic reductions; the last CTA updates the module state.
-//                 ("write-up" section 二; explainer section 3.)
 //  k_rotate       rotation only (test hook).
-//
-// Row mapping shared by k_prepass and k_tdc_record: a CTA of W warps owns one aligned group of 32
-// rows and walks them in order. Lane l of warp w holds, for c < CPL, the 8 contiguous elements of
-// chunk ci = (c*W + w)*32 + l, so every warp-wide 16-byte load covers one 256-element segment of
-// the row (coalesced) and a Hadamard block of B elements sits in B/8 neighbouring lanes.
-// Per-row sums follow the canonical pairwise tree: 8 elements in a lane, the lane tree inside a
-// segment, then a tree over the (zero-padded) segments.
-#include <cfloat>
-
-#include "sb_device.cuh"
-#include "sb_kernels.h"
+#include "rows.cuh"
 
 namespace sb {
 
-constexpr int kMaxWarps = 8;
-constexpr int kMaxSeg = 64;  // 64 segments x 256 = 16384 = kMaxK
-
-struct PrepassArgs {
-  const __nv_bfloat16* X;
-  const __nv_bfloat16* R;  // nullable
-  int64_t M;
-  int K, B, W;
-  int mode;
-  int32_t* prec;  // nullable: treated as "quantize INT8" when force_int8
-  int force_int8; // weight preparation: always write INT8 codes and never touch *prec
-  int8_t* q8;
-  float* s8;
-  double rho;
-  int force;
-  GroupSlot* groups;
-  WsHeader* hdr;
-  sb_stats* stats;
-};
-
-// Tree over the segment sums of one row (zero-padded to 64), by warp 0; returns on every lane.
-__device__ __forceinline__ float segment_tree(const float* seg, int nseg, int lane) {
-  const float a = (2 * lane < nseg) ? seg[2 * lane] : 0.0f;
-  const float b = (2 * lane + 1 < nseg) ? seg[2 * lane + 1] : 0.0f;
-  return warp_pairwise_f32(__fadd_rn(a, b));
+static int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
 }
 
-template <int CPL, bool HAS_REF>
-__global__ void __launch_bounds__(256) k_prepass(PrepassArgs a) {
-  __shared__ float seg[2][3][kMaxSeg];
-  __shared__ float wmax[2][kMaxWarps];
-  __shared__ float rowpart[3][kGroupRows];
-  __shared__ float rowamax[kGroupRows];
-  __shared__ float cta_max[kMaxWarps];
-  __shared__ int s_last;
-
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, W = a.W;
-  int prec = a.force_int8 ? SB_INT8 : (a.prec ? *a.prec : -1);
-  if (prec == SB_SKIP) return;  // the module is skipped at this step: uniform exit
-  const bool do_int8 = a.force_int8 || (a.mode == SB_PREPASS_QUANT && prec == SB_INT8);
-  const int K = a.K;
-  const int nch = K >> 3;
-  const int nseg = CPL * W;
-  const int lpb = a.B >> 3;
-  const int64_t row0 = (int64_t)blockIdx.x * kGroupRows;
-
-  float tmax = 0.0f;
-  int nonfinite = 0;
-
-  uint4 xn[CPL], rn[CPL];
-  auto issue = [&](int64_t m, uint4 (&xv)[CPL], uint4 (&rv)[CPL]) {
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      const int ci = (c * W + w) * 32 + lane;
-      if (m < a.M && ci < nch) {
-        xv[c] = ldg_nc_v4(a.X + m * K + (int64_t)ci * 8);
-        if (HAS_REF) rv[c] = ldg_nc_v4(a.R + m * K + (int64_t)ci * 8);
-      } else {
-        xv[c] = make_uint4(0, 0, 0, 0);
-        if (HAS_REF) rv[c] = make_uint4(0, 0, 0, 0);
-      }
-    }
-  };
-  issue(row0, xn, rn);
-
-  for (int r = 0; r < kGroupRows; ++r) {
-    const int64_t m = row0 + r;
-    const int par = r & 1;
-    if (m >= a.M) {
-      if (tid == 0) {
-        rowpart[0][r] = rowpart[1][r] = rowpart[2][r] = 0.0f;
-        rowamax[r] = 0.0f;
-      }
-      continue;
-    }
-    uint4 xc[CPL], rc[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      xc[c] = xn[c];
-      if (HAS_REF) rc[c] = rn[c];
-    }
-    if (r + 1 < kGroupRows) issue(m + 1, xn, rn);  // prefetch the next row of the group
-
-    float v[CPL][8];
-    float am = 0.0f;
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      unpack8(xc[c], v[c]);
-      float t0[8], t1[8], t2[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        t0[j] = fabsf(v[c][j]);
-        tmax = fmaxf(tmax, t0[j]);
-      }
-      const float s0 = warp_pairwise_f32(pairwise8(t0));
-      float s1 = 0.0f, s2 = 0.0f;
-      if (HAS_REF) {
-        float rr[8];
-        unpack8(rc[c], rr);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float d = __fsub_rn(v[c][j], rr[j]);
-          t1[j] = __fmul_rn(d, d);
-          t2[j] = __fmul_rn(rr[j], rr[j]);
-        }
-        s1 = warp_pairwise_f32(pairwise8(t1));
-        s2 = warp_pairwise_f32(pairwise8(t2));
-      }
-      if (lane == 0) {
-        seg[par][0][c * W + w] = s0;
-        seg[par][1][c * W + w] = s1;
-        seg[par][2][c * W + w] = s2;
-      }
-      fwht8_in_lane(v[c]);
-      fwht_across_lanes(v[c], lane, lpb);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(v[c][j]));
-    }
-    am = warp_max_f32(am);
-    if (lane == 0) wmax[par][w] = am;
-    __syncthreads();
-
-    float a_m = 0.0f;
-    for (int i = 0; i < W; ++i) a_m = fmaxf(a_m, wmax[par][i]);
-    if (w == 0) {
-      const float p0 = segment_tree(seg[par][0], nseg, lane);
-      const float p1 = segment_tree(seg[par][1], nseg, lane);
-      const float p2 = segment_tree(seg[par][2], nseg, lane);
-      if (lane == 0) {
-        rowpart[0][r] = p0;
-        rowpart[1][r] = p1;
-        rowpart[2][r] = p2;
-        rowamax[r] = a_m;
-        if (!isfinite(p0)) nonfinite = 1;
-      }
-    }
-    if (do_int8) {
-      const bool zero = (a_m == 0.0f);
-      const float inv = zero ? 0.0f : __fdiv_rn(127.0f, a_m);
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        const int ci = (c * W + w) * 32 + lane;
-        if (ci < nch) {
-          uint32_t wd[2] = {0u, 0u};
-          if (!zero) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              int q = __float2int_rn(__fmul_rn(v[c][j], inv));
-              q = max(-127, min(127, q));
-              wd[j >> 2] |= ((uint32_t)(q & 0xff)) << (8 * (j & 3));
-            }
-          }
-          *reinterpret_cast<uint2*>(a.q8 + m * K + (int64_t)ci * 8) = make_uint2(wd[0], wd[1]);
-        }
-      }
-      if (tid == 0) a.s8[m] = zero ? 0.0f : __fdiv_rn(a_m, 127.0f);
-    }
-  }
-  // ---- group partials (FP64 pairwise over the 32 rows) and maxima
-  tmax = warp_max_f32(tmax);
-  if (lane == 0) cta_max[w] = tmax;
-  __syncthreads();
-  if (w == 0) {
-    const double g0 = warp_pairwise_f64((double)rowpart[0][lane]);
-    const double g1 = warp_pairwise_f64((double)rowpart[1][lane]);
-    const double g2 = warp_pairwise_f64((double)rowpart[2][lane]);
-    const float gam = warp_max_f32(rowamax[lane]);
-    const int nf = __any_sync(0xffffffffu, nonfinite);
-    if (lane == 0) {
-      float mx = 0.0f;
-      for (int i = 0; i < W; ++i) mx = fmaxf(mx, cta_max[i]);
-      GroupSlot* gs = a.groups + blockIdx.x;
-      gs->s[0] = g0;
-      gs->s[1] = g1;
-      gs->s[2] = g2;
-      gs->max_abs = mx;
-      gs->amax_rot = gam;
-      gs->nonfinite = nf;
-      __threadfence();
-      const uint32_t t = atomicAdd(&a.hdr->ticket[TICKET_PREPASS], 1u);
-      s_last = (t == gridDim.x - 1);
-    }
-  }
-  __syncthreads();
-  if (!s_last) return;
-  // ---- last CTA: tree over the groups, statistics record, Purified Delta Refresh
-  __threadfence();
-  if (w != 0) return;
-  const int64_t G = gridDim.x;
-  const double S0 = warp_pairwise_f64_global(&a.groups[0].s[0], sizeof(GroupSlot) / 8, G, lane);
-  const double S1 = warp_pairwise_f64_global(&a.groups[0].s[1], sizeof(GroupSlot) / 8, G, lane);
-  const double S2 = warp_pairwise_f64_global(&a.groups[0].s[2], sizeof(GroupSlot) / 8, G, lane);
-  float mx = 0.0f, ar = 0.0f;
-  int nf = 0;
-  for (int64_t g = lane; g < G; g += 32) {
-    const GroupSlot* gs = a.groups + g;
-    mx = fmaxf(mx, __ldcg(&gs->max_abs));
-    ar = fmaxf(ar, __ldcg(&gs->amax_rot));
-    nf |= __ldcg(&gs->nonfinite);
-  }
-  mx = warp_max_f32(mx);
-  ar = warp_max_f32(ar);
-  nf = __any_sync(0xffffffffu, nf);
-  if (lane == 0) {
-    const double numel = (double)a.M * (double)K;
-    double ratio;
-    if (S0 == 0.0) {
-      ratio = __longlong_as_double(0x7ff0000000000000ll);  // +inf
-    } else {
-      const double mean = __ddiv_rn(S0, numel);
-      ratio = __ddiv_rn((double)mx, mean);
-    }
-    double d = 0.0;
-    if (HAS_REF) {
-      const double num = __dsqrt_rn(S1);
-      const double den = __dsqrt_rn(S2);
-      d = (den == 0.0) ? (num == 0.0 ? 0.0 : __longlong_as_double(0x7ff0000000000000ll)) : __ddiv_rn(num, den);
-    }
-    int pout = prec;
-    if (!a.force_int8 && a.mode == SB_PREPASS_QUANT && a.force < 0 && (prec == SB_NVFP4 || prec == SB_INT8) &&
-        ratio > a.rho)
-      pout = SB_BF16;
-    if (a.stats) {
-      sb_stats* st = a.stats;
-      st->sum_abs = S0;
-      st->sum_d2 = S1;
-      st->sum_ref2 = S2;
-      st->max_abs = (double)mx;
-      st->amax_rot = (double)ar;
-      st->ratio = ratio;
-      st->d = d;
-      st->numel = numel;
-      st->has_ref = HAS_REF ? 1 : 0;
-      st->prec_in = prec;
-      st->prec_out = pout;
-      st->nonfinite = nf;
-    }
-    if (pout != prec && a.prec) *a.prec = pout;
-    if (nf) set_error(a.hdr, SB_ENONFINITE);
-    a.hdr->ticket[TICKET_PREPASS] = 0u;  // ready for the next call on this stream
-    __threadfence();
-  }
-}
-
-// ---------------------------------------------------------------------------------------------
-// NVFP4 encode
-// ---------------------------------------------------------------------------------------------
-
-struct Nvfp4Args {
-  const __nv_bfloat16* X;
-  int64_t M;
-  int K, B;
-  const int32_t* prec;  // nullable: always encode
-  const sb_stats* stats;
-  uint8_t* codes;
-  uint8_t* sf;
-  float* gscale;
-};
-
-__device__ __forceinline__ int64_t sf_offset(int64_t m, int64_t g, int64_t K) {
-  return ((m >> 7) * (K >> 6) + (g >> 2)) * 512 + (m & 31) * 16 + ((m & 127) >> 5) * 4 + (g & 3);
-}
-
-__global__ void __launch_bounds__(256) k_nvfp4(Nvfp4Args a) {
-  if (a.prec && *a.prec != SB_NVFP4) return;
-  const int lane = threadIdx.x & 31;
-  const int K = a.K;
-  const int nch = K >> 3;
-  const int nseg = (nch + 31) >> 5;
-  const int lpb = a.B >> 3;
-  const int64_t Mpad = (a.M + 127) & ~(int64_t)127;
-  const float A = (float)a.stats->amax_rot;  // exact: a float widened to double
-  const float s_g = (A == 0.0f) ? 1.0f : __fdiv_rn(A, 2688.0f);
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.gscale = s_g;
-  const int64_t units = Mpad * nseg;
-  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t u = warp0; u < units; u += nwarps) {
-    const int64_t m = u / nseg;
-    const int sgi = (int)(u - m * nseg);
-    const int ci = sgi * 32 + lane;
-    const bool in_row = ci < nch;
-    float v[8];
-    if (m < a.M && in_row) {
-      unpack8(ldg_nc_v4(a.X + m * K + (int64_t)ci * 8), v);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-    }
-    fwht8_in_lane(v);
-    fwht_across_lanes(v, lane, lpb);
-    float am = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(v[j]));
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));  // 16-element group = 2 lanes
-    const float sfv = __fdiv_rn(__fdiv_rn(am, 6.0f), s_g);
-    const uint32_t sb = cvt_e4m3(sfv);
-    const float den = __fmul_rn(e4m3_to_f32(sb), s_g);
-    const float inv = (den == 0.0f) ? 0.0f : __fdiv_rn(1.0f, den);
-    const bool zero = (den == 0.0f) || !(inv <= FLT_MAX);
-    uint32_t word = 0;
-    if (!zero) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        word |= cvt_e2m1x2(__fmul_rn(v[2 * i], inv), __fmul_rn(v[2 * i + 1], inv)) << (8 * i);
-    }
-    if (m < a.M && in_row) *reinterpret_cast<uint32_t*>(a.codes + m * (K >> 1) + (int64_t)ci * 4) = word;
-    // scales: lanes 8j, 8j+2, 8j+4, 8j+6 hold groups 4j .. 4j+3 (one 32-bit word of the layout)
-    const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 2);
-    const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 4);
-    const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 6);
-    if ((lane & 7) == 0 && in_row) {
-      const int64_t g0 = (int64_t)ci >> 1;
-      *reinterpret_cast<uint32_t*>(a.sf + sf_offset(m, g0, K)) = sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------------------------
-// Rotation only
-// ---------------------------------------------------------------------------------------------
-
-__global__ void __launch_bounds__(256) k_rotate(const __nv_bfloat16* X, float* Y, int64_t M, int K, int B) {
-  const int lane = threadIdx.x & 31;
-  const int nch = K >> 3;
-  const int nseg = (nch + 31) >> 5;
-  const int64_t units = M * nseg;
-  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t u = warp0; u < units; u += nwarps) {
-    const int64_t m = u / nseg;
-    const int ci = (int)(u - m * nseg) * 32 + lane;
-    float v[8];
-    if (ci < nch) {
-      unpack8(ldg_nc_v4(X + m * K + (int64_t)ci * 8), v);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-    }
-    fwht8_in_lane(v);
-    fwht_across_lanes(v, lane, B >> 3);
-    if (ci < nch) {
-      float4* dst = reinterpret_cast<float4*>(Y + m * K + (int64_t)ci * 8);
-      dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-      dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------------------------
-// Temporal Delta Cache record
-// ---------------------------------------------------------------------------------------------
-
-struct TdcArgs {
-  const __nv_bfloat16* Y;  // new output
-  __nv_bfloat16* Cache;    // last computed output (refreshed when update)
-  int64_t M;
-  int C, W;
-  int update;
-  const sb_stats* dsrc;
-  sb_module_state* st;
-  GroupSlot* groups;
-  WsHeader* hdr;
-};
-
-template <int CPL>
-__global__ void __launch_bounds__(256) k_tdc_record(TdcArgs a) {
-  __shared__ float seg[2][2][kMaxSeg];
-  __shared__ float rowpart[2][kGroupRows];
-  __shared__ int s_last;
-  if (a.st->skip) return;
-  const int have_prev = a.st->n_out >= 1;
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, W = a.W;
-  const int C = a.C;
-  const int nch = C >> 3;
-  const int nseg = CPL * W;
-  const int64_t row0 = (int64_t)blockIdx.x * kGroupRows;
-  for (int r = 0; r < kGroupRows; ++r) {
-    const int64_t m = row0 + r;
-    const int par = r & 1;
-    if (m >= a.M) {
-      if (tid == 0) rowpart[0][r] = rowpart[1][r] = 0.0f;
-      continue;
-    }
-    uint4 yv[CPL], cv[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      const int ci = (c * W + w) * 32 + lane;
-      const bool ok = ci < nch;
-      yv[c] = ok ? ldg_nc_v4(a.Y + m * C + (int64_t)ci * 8) : make_uint4(0, 0, 0, 0);
-      cv[c] = (ok && have_prev) ? ldg_v4(a.Cache + m * C + (int64_t)ci * 8) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      const int ci = (c * W + w) * 32 + lane;
-      float yn[8], yl[8], t0[8], t1[8];
-      unpack8(yv[c], yn);
-      unpack8(cv[c], yl);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        t0[j] = fabsf(__fsub_rn(yn[j], yl[j]));
-        t1[j] = fabsf(yl[j]);
-      }
-      const float s0 = warp_pairwise_f32(pairwise8(t0));
-      const float s1 = warp_pairwise_f32(pairwise8(t1));
-      if (lane == 0) {
-        seg[par][0][c * W + w] = s0;
-        seg[par][1][c * W + w] = s1;
-      }
-      if (a.update && ci < nch) *reinterpret_cast<uint4*>(a.Cache + m * C + (int64_t)ci * 8) = yv[c];
-    }
-    __syncthreads();
-    if (w == 0) {
-      const float p0 = segment_tree(seg[par][0], nseg, lane);
-      const float p1 = segment_tree(seg[par][1], nseg, lane);
-      if (lane == 0) {
-        rowpart[0][r] = p0;
-        rowpart[1][r] = p1;
-      }
-    }
-  }
-  __syncthreads();
-  if (w == 0) {
-    const double g0 = warp_pairwise_f64((double)rowpart[0][lane]);
-    const double g1 = warp_pairwise_f64((double)rowpart[1][lane]);
-    if (lane == 0) {
-      GroupSlot* gs = a.groups + blockIdx.x;
-      gs->s[0] = g0;
-      gs->s[1] = g1;
-      __threadfence();
-      const uint32_t t = atomicAdd(&a.hdr->ticket[TICKET_TDC], 1u);
-      s_last = (t == gridDim.x - 1);
-    }
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  if (w != 0) return;
-  const int64_t G = gridDim.x;
-  const double S0 = warp_pairwise_f64_global(&a.groups[0].s[0], sizeof(GroupSlot) / 8, G, lane);
-  const double S1 = warp_pairwise_f64_global(&a.groups[0].s[1], sizeof(GroupSlot) / 8, G, lane);
-  if (lane == 0) {
-    sb_module_state* st = a.st;
-    if (have_prev)
-      st->delta = (S1 == 0.0) ? __longlong_as_double(0x7ff0000000000000ll) : __ddiv_rn(S0, S1);
-    st->n_out += 1;
-    st->acc = 0.0;
-    st->last_skipped = 0;
-    if (a.dsrc && a.dsrc->has_ref) {
-      st->prev_d = a.dsrc->d;
-      st->have_d = 1;
-    } else {
-      st->have_d = 0;
-    }
-    a.hdr->ticket[TICKET_TDC] = 0u;
-    __threadfence();
-  }
-}
-
-// ---------------------------------------------------------------------------------------------
-// Host launchers
-// ---------------------------------------------------------------------------------------------
-
-// Warps per row W and chunks per lane CPL with W*CPL segments covering the row.
-static void row_tiling(int K, int* W, int* CPL) {
-  const int S = (int)ceil_div(K, 256);
-  const int cpl = (int)ceil_div(S, kMaxWarps);
-  *CPL = cpl;
-  *W = (int)ceil_div(S, cpl);
-}
-
-template <bool HAS_REF>
-static cudaError_t launch_prepass_t(const PrepassArgs& a0, int64_t groups, cudaStream_t s) {
-  PrepassArgs a = a0;
-  int W, CPL;
-  row_tiling(a.K, &W, &CPL);
-  a.W = W;
-  const dim3 grid((unsigned)groups), block(32 * W);
-  switch (CPL) {
-    case 1: k_prepass<1, HAS_REF><<<grid, block, 0, s>>>(a); break;
-    case 2: k_prepass<2, HAS_REF><<<grid, block, 0, s>>>(a); break;
-    case 3: k_prepass<3, HAS_REF><<<grid, block, 0, s>>>(a); break;
-    case 4: k_prepass<4, HAS_REF><<<grid, block, 0, s>>>(a); break;
-    case 5: k_prepass<5, HAS_REF><<<grid, block, 0, s>>>(a); break;
-    case 6: k_prepass<6, HAS_REF><<<grid, block, 0, s>>>(a); break;
-    case 7: k_prepass<7, HAS_REF><<<grid, block, 0, s>>>(a); break;
-    case 8: k_prepass<8, HAS_REF><<<grid, block, 0, s>>>(a); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s) {
-  PrepassArgs a{};
+static RowArgs row_args_from(const PrepassLaunch& p) {
+  RowArgs a{};
   a.X = reinterpret_cast<const __nv_bfloat16*>(p.X);
-  a.R = reinterpret_cast<const __nv_bfloat16*>(p.R);
+  a.R = const_cast<__nv_bfloat16*>(reinterpret_cast<const __nv_bfloat16*>(p.R));
   a.M = p.M;
   a.K = (int)p.K;
   a.B = p.B;
@@ -536,19 +45,157 @@ cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s) {
   a.groups = reinterpret_cast<GroupSlot*>(p.groups);
   a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
   a.stats = p.stats;
-  const int64_t groups = ceil_div(p.M, kGroupRows);
-  return p.R ? launch_prepass_t<true>(a, groups, s) : launch_prepass_t<false>(a, groups, s);
+  return a;
 }
 
-static int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s) {
+  const RowArgs a = row_args_from(p);
+  const int sms = sm_count();
+  if (p.mode == SB_PREPASS_STATS && !p.force_int8)
+    return p.R ? launch_rows_t<OP_STATS, true>(a, s, sms) : launch_rows_t<OP_STATS, false>(a, s, sms);
+  return p.R ? launch_rows_t<OP_PREPASS, true>(a, s, sms) : launch_rows_t<OP_PREPASS, false>(a, s, sms);
+}
+
+cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s) {
+  RowArgs a{};
+  a.X = reinterpret_cast<const __nv_bfloat16*>(p.Y);
+  a.R = reinterpret_cast<__nv_bfloat16*>(p.Cache);
+  a.M = p.M;
+  a.K = (int)p.C;
+  a.B = 0;
+  a.update = p.update;
+  a.dsrc = p.dsrc;
+  a.st = p.st;
+  a.groups = reinterpret_cast<GroupSlot*>(p.groups);
+  a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
+  return launch_rows_t<OP_TDC, true>(a, s, sm_count());
+}
+
+// ---------------------------------------------------------------------------------------------
+// NVFP4 encode: one warp per 1024-element segment of a row; a lane's 32 values are two 16-value
+// scale groups, so group maxima need no shuffle.
+// ---------------------------------------------------------------------------------------------
+
+struct Nvfp4Args {
+  const __nv_bfloat16* X;
+  int64_t M;
+  int K, B;
+  const int32_t* prec;  // null: always encode
+  const sb_stats* stats;
+  uint8_t* codes;
+  uint8_t* sf;
+  float* gscale;
+};
+
+__device__ __forceinline__ int64_t sf_offset(int64_t m, int64_t g, int64_t K) {
+  return ((m >> 7) * (K >> 6) + (g >> 2)) * 512 + (m & 31) * 16 + ((m & 127) >> 5) * 4 + (g & 3);
+}
+
+// E4M3 block scale of one 16-value group and the reciprocal used for its codes.
+__device__ __forceinline__ void group_scale(float amax, float s_g, uint32_t* sb, float* inv, bool* zero) {
+  const float sfv = __fdiv_rn(__fdiv_rn(amax, 6.0f), s_g);
+  *sb = cvt_e4m3(sfv);
+  const float den = __fmul_rn(e4m3_to_f32(*sb), s_g);
+  *inv = (den == 0.0f) ? 0.0f : __fdiv_rn(1.0f, den);
+  *zero = (den == 0.0f) || !(*inv <= FLT_MAX);
+}
+
+__global__ void __launch_bounds__(256) k_nvfp4(Nvfp4Args a) {
+  if (a.prec && *a.prec != SB_NVFP4) return;
+  const int lane = threadIdx.x & 31;
+  const int K = a.K;
+  const int nseg = (K + 1023) >> 10;
+  const int64_t Mpad = (a.M + 127) & ~(int64_t)127;
+  const float A = (float)a.stats->amax_rot;  // exact: a float widened to double
+  const float s_g = (A == 0.0f) ? 1.0f : __fdiv_rn(A, 2688.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.gscale = s_g;
+  const int64_t units = Mpad * nseg;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t u = warp0; u < units; u += nwarps) {
+    const int64_t m = u / nseg;
+    const int sgi = (int)(u - m * nseg);
+    const int e0 = sgi * 1024 + lane * 32;
+    const bool in_row = e0 < K;
+    Raw32 raw;
+    load_raw(raw, a.X + m * K, e0, K, in_row && m < a.M);
+    float2 p[16];
+    unpack_pairs(raw, p);
+    fwht_pairs(p, lane, a.B);
+    // group 0 = elements 0..15 = the x halves, group 1 = elements 16..31 = the y halves
+    float am0 = 0.0f, am1 = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 16; k += 2) {
+      am0 = max3(am0, fabsf(p[k].x), fabsf(p[k + 1].x));
+      am1 = max3(am1, fabsf(p[k].y), fabsf(p[k + 1].y));
+    }
+    uint32_t sb0, sb1;
+    float inv0, inv1;
+    bool z0, z1;
+    group_scale(am0, s_g, &sb0, &inv0, &z0);
+    group_scale(am1, s_g, &sb1, &inv1, &z1);
+    const float2 inv2 = make_float2(inv0, inv1);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) p[k] = mul2(p[k], inv2);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // word q = elements 8q..8q+7 (group 0 for q < 2)
+      const bool hi = q >= 2;
+      const bool z = hi ? z1 : z0;
+      uint32_t word = 0;
+      if (!z) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int k = 8 * (q & 1) + 2 * b;
+          word |= cvt_e2m1x2(hi ? p[k].y : p[k].x, hi ? p[k + 1].y : p[k + 1].x) << (8 * b);
+        }
+      }
+      w[q] = word;
+    }
+    if (m < a.M && in_row)
+      *reinterpret_cast<uint4*>(a.codes + m * (K >> 1) + (e0 >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
+    // scale word of groups 4j..4j+3 = lanes 2j (groups 4j, 4j+1) and 2j+1 (4j+2, 4j+3)
+    const uint32_t mine = sb0 | (sb1 << 8);
+    const uint32_t other = __shfl_down_sync(0xffffffffu, mine, 1);
+    if ((lane & 1) == 0 && in_row)
+      *reinterpret_cast<uint32_t*>(a.sf + sf_offset(m, e0 >> 4, K)) = mine | (other << 16);
   }
-  return n;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Rotation only
+// ---------------------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) k_rotate(const __nv_bfloat16* X, float* Y, int64_t M, int K, int B) {
+  const int lane = threadIdx.x & 31;
+  const int nseg = (K + 1023) >> 10;
+  const int64_t units = M * nseg;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t u = warp0; u < units; u += nwarps) {
+    const int64_t m = u / nseg;
+    const int e0 = (int)(u - m * nseg) * 1024 + lane * 32;
+    const bool ok = e0 < K;
+    Raw32 raw;
+    load_raw(raw, X + m * K, e0, K, ok);
+    float2 p[16];
+    unpack_pairs(raw, p);
+    fwht_pairs(p, lane, B);
+    if (ok) {
+      float4* dst = reinterpret_cast<float4*>(Y + m * K + e0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        dst[q] = make_float4(p[4 * q].x, p[4 * q + 1].x, p[4 * q + 2].x, p[4 * q + 3].x);
+        dst[4 + q] = make_float4(p[4 * q].y, p[4 * q + 1].y, p[4 * q + 2].y, p[4 * q + 3].y);
+      }
+    }
+  }
+}
+
+static unsigned stream_grid(int64_t units) {
+  const int64_t want = ceil_div(units, 8);  // 8 warps per CTA, one unit each
+  const int64_t cap = (int64_t)sm_count() * 8;
+  return (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
 cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s) {
@@ -562,49 +209,14 @@ cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s) {
   a.codes = p.codes;
   a.sf = p.sf;
   a.gscale = p.gscale;
-  const int64_t units = ((p.M + 127) & ~(int64_t)127) * ceil_div(p.K / 8, 32);
-  const int64_t want = ceil_div(units, 8);  // 8 warps per CTA, one unit each
-  const int64_t cap = (int64_t)sm_count() * 8;
-  const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
-  k_nvfp4<<<grid, 256, 0, s>>>(a);
+  const int64_t units = ((p.M + 127) & ~(int64_t)127) * ceil_div(p.K, 1024);
+  k_nvfp4<<<stream_grid(units), 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_rotate(const void* X, float* Y, int64_t M, int64_t K, int B, cudaStream_t s) {
-  const int64_t units = M * ceil_div(K / 8, 32);
-  const int64_t want = ceil_div(units, 8);
-  const int64_t cap = (int64_t)sm_count() * 8;
-  const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
-  k_rotate<<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(X), Y, M, (int)K, B);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s) {
-  TdcArgs a{};
-  a.Y = reinterpret_cast<const __nv_bfloat16*>(p.Y);
-  a.Cache = reinterpret_cast<__nv_bfloat16*>(p.Cache);
-  a.M = p.M;
-  a.C = (int)p.C;
-  a.update = p.update;
-  a.dsrc = p.dsrc;
-  a.st = p.st;
-  a.groups = reinterpret_cast<GroupSlot*>(p.groups);
-  a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
-  int W, CPL;
-  row_tiling(a.C, &W, &CPL);
-  a.W = W;
-  const dim3 grid((unsigned)ceil_div(p.M, kGroupRows)), block(32 * W);
-  switch (CPL) {
-    case 1: k_tdc_record<1><<<grid, block, 0, s>>>(a); break;
-    case 2: k_tdc_record<2><<<grid, block, 0, s>>>(a); break;
-    case 3: k_tdc_record<3><<<grid, block, 0, s>>>(a); break;
-    case 4: k_tdc_record<4><<<grid, block, 0, s>>>(a); break;
-    case 5: k_tdc_record<5><<<grid, block, 0, s>>>(a); break;
-    case 6: k_tdc_record<6><<<grid, block, 0, s>>>(a); break;
-    case 7: k_tdc_record<7><<<grid, block, 0, s>>>(a); break;
-    case 8: k_tdc_record<8><<<grid, block, 0, s>>>(a); break;
-    default: return cudaErrorInvalidValue;
-  }
+  const int64_t units = M * ceil_div(K, 1024);
+  k_rotate<<<stream_grid(units), 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(X), Y, M, (int)K, B);
   return cudaGetLastError();
 }
 
