@@ -26,17 +26,24 @@
 
 namespace sb {
 
-constexpr int kStages = 4;
-constexpr int kOffB = 16384;      // A: 128 rows x 128 B
-constexpr int kOffSFA = 49152;    // B: up to 256 rows x 128 B
-constexpr int kOffSFB = 51200;    // SFA: 4 atoms x 512 B
-constexpr int kStageBytes = 55296;  // SFB: 2 row tiles x 4 atoms x 512 B
+// NVFP4 (one CTA per 128 x 192 tile): A 16 KB | B 24 KB | SFA 2 KB | SFB 4 KB, 4 stages.
+// INT8 / BF16 (a CTA pair per 256 x 256 tile): A 16 KB | B half 16 KB per CTA, 6 stages.
+constexpr int kOffB = 16384;
+constexpr int kOffSFA = 49152;
+constexpr int kOffSFB = 51200;
+constexpr int kStageBytesSingle = 55296;
+constexpr int kStagesSingle = 4;
+constexpr int kStageBytesPair = 32768;
+constexpr int kStagesPair = 6;
+constexpr int kMaxStages = 6;
+constexpr int kStageArea = kStagesSingle * kStageBytesSingle;  // >= kStagesPair * kStageBytesPair
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr uint64_t kDrainNs = 20000000ull;   // 20 ms to let in-flight copies land after an abort
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr int kSmemBytes = kStageArea + 1024 + 512;
+static_assert(kStagesPair * kStageBytesPair <= kStageArea, "stage area");
 
 enum { KIND_FP4 = 0, KIND_I8 = 1, KIND_BF16 = 2 };
 
@@ -64,9 +71,9 @@ struct GemmParams {
   WsHeader* hdr;
 };
 
-__device__ __forceinline__ uint32_t idesc_for(int kind, int BN) {
+__device__ __forceinline__ uint32_t idesc_for(int kind, int BM, int BN) {
   const uint32_t n = (uint32_t)(BN >> 3) << 17;
-  const uint32_t m = (uint32_t)(128 >> 4) << 24;
+  const uint32_t m = (uint32_t)(BM >> 4) << 24;
   switch (kind) {
     case KIND_FP4:  // block-scaled: A,B = E2M1 (1), scale type UE4M3 (bit 23 = 0), K = 64
       return (1u << 7) | (1u << 10) | n | m;
@@ -91,12 +98,31 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ TMaps tm, const GemmParams p) {
+// Grouped tile order: kGroupM consecutive M-tiles are swept across all N-tiles before the next
+// group starts, so the A rows of a group stay in L2 while every N-tile reuses them (A of the
+// second FFN layer is larger than L2 and would otherwise be re-read from HBM for each N-tile).
+constexpr int kGroupM = 8;
+
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int* mt, int* nt) {
+  const int group = kGroupM * n_tiles;
+  const int g = t / group, r = t - g * group;
+  const int first = g * kGroupM;
+  const int gm = min(kGroupM, m_tiles - first);
+  *mt = first + r % gm;
+  *nt = r / gm;
+}
+
+// Launched as clusters of two CTAs. INT8 and BF16 run "pair" tiles: the two CTAs of a cluster
+// share one 256 x BN tile; each loads its own 128 rows of A and its half of B, the even CTA (the
+// leader) issues tcgen05.mma.cta_group::2 with M = 256 and both CTAs' accumulators receive their
+// 128 rows. NVFP4 runs one 128 x BN tile per CTA and ignores the cluster.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    k_gemm(const __grid_constant__ TMaps tm, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStageArea);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -104,38 +130,53 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ TM
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kind = *p.prec;
-  if (kind < 0 || kind > 2) return;  // skipped module: nothing to compute
+  if (kind < 0 || kind > 2) return;  // skipped module: nothing to compute (uniform)
   if (!p.have[kind]) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_error(p.hdr, SB_EINVAL);
     return;
   }
+  const bool pair = (kind != KIND_FP4);
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
   const int M = p.M, N = p.N, K = p.K;
   const int BN = p.bn[kind];
+  const int BM = pair ? 256 : 128;
   const int kb_elems = (kind == KIND_FP4) ? 256 : (kind == KIND_I8 ? 128 : 64);
   const int mma_k = kb_elems >> 2;
   const int nkb = (K + kb_elems - 1) / kb_elems;
-  const int m_tiles = (M + 127) >> 7;
+  const int m_tiles = (M + BM - 1) / BM;
   const int n_tiles = (N + BN - 1) / BN;
   const int tiles = m_tiles * n_tiles;
-  if ((int)blockIdx.x >= tiles) return;
+  const int unit = pair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int nunits = pair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  if (unit >= tiles) return;  // pair mode: both CTAs of the cluster leave together
+  const int stages = pair ? kStagesPair : kStagesSingle;
+  const int stage_bytes = pair ? kStageBytesPair : kStageBytesSingle;
+  const int row_off = pair ? 128 * (int)rank : 0;  // this CTA's rows inside the tile
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kEpiWarps);
+      mbar_init(&tempty[b], pair ? 2 * kEpiWarps : kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  if (pair) cluster_sync();  // the peer's barriers exist before any remote arrive or copy
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if (pair) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -151,40 +192,47 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ TM
     if (elect_one()) {
       prefetch_tmap(&tm.a[kind]);
       prefetch_tmap(&tm.b[kind]);
+      const uint32_t full_leader = pair ? cluster_addr(&full[0], 0) : 0u;
       int s = 0;
       uint32_t ph = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
-        const int mt = tile % m_tiles, nt = tile / m_tiles;
-        const int m0 = mt * 128, n0 = nt * BN;
+      for (int tile = unit; ok && tile < tiles; tile += nunits) {
+        int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
+        const int m0 = mt * BM + row_off, n0 = nt * BN;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitNs)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * kStageBytes;
-          uint32_t bytes = 16384u + (uint32_t)BN * 128u;
-          int atoms = 0, btiles = 0;
-          if (kind == KIND_FP4) {
-            atoms = min(4, sf_atoms_k - 4 * kb);
-            const int t0 = n0 >> 7;
-            btiles = min((n0 % 128 + BN + 127) >> 7, sf_tiles_n - t0);
-            bytes += (uint32_t)atoms * 512u * (uint32_t)(1 + btiles);
-          }
-          mbar_arrive_expect_tx(&full[s], bytes);
+          uint8_t* st = smem + s * stage_bytes;
           const int x = (kind == KIND_BF16) ? kb * 64 : kb * 128;
-          tma_load_2d(st, &tm.a[kind], &full[s], x, m0);
-          tma_load_2d(st + kOffB, &tm.b[kind], &full[s], x, n0);
-          if (kind == KIND_FP4) {
-            bulk_load(st + kOffSFA, p.sfA4 + ((int64_t)mt * sf_atoms_k + 4 * kb) * 512, atoms * 512u, &full[s]);
-            const int t0 = n0 >> 7;
-            for (int t = 0; t < btiles; ++t)
-              bulk_load(st + kOffSFB + 2048 * t, p.sfB4 + ((int64_t)(t0 + t) * sf_atoms_k + 4 * kb) * 512,
-                        atoms * 512u, &full[s]);
+          if (pair) {
+            if (leader) mbar_arrive_expect_tx(&full[s], 2u * (16384u + (uint32_t)(BN / 2) * 128u));
+            tma_load_2d_pair(st, &tm.a[kind], full_leader + 8u * s, x, m0);
+            tma_load_2d_pair(st + kOffB, &tm.b[kind], full_leader + 8u * s, x, n0 + (BN / 2) * (int)rank);
+          } else {
+            uint32_t bytes = 16384u + (uint32_t)BN * 128u;
+            int atoms = 0, btiles = 0;
+            if (kind == KIND_FP4) {
+              atoms = min(4, sf_atoms_k - 4 * kb);
+              btiles = min((n0 % 128 + BN + 127) >> 7, sf_tiles_n - (n0 >> 7));
+              bytes += (uint32_t)atoms * 512u * (uint32_t)(1 + btiles);
+            }
+            mbar_arrive_expect_tx(&full[s], bytes);
+            tma_load_2d(st, &tm.a[kind], &full[s], x, m0);
+            tma_load_2d(st + kOffB, &tm.b[kind], &full[s], x, n0);
+            if (kind == KIND_FP4) {
+              bulk_load(st + kOffSFA, p.sfA4 + ((int64_t)mt * sf_atoms_k + 4 * kb) * 512, atoms * 512u, &full[s]);
+              const int t0 = n0 >> 7;
+              for (int t = 0; t < btiles; ++t)
+                bulk_load(st + kOffSFB + 2048 * t, p.sfB4 + ((int64_t)(t0 + t) * sf_atoms_k + 4 * kb) * 512,
+                          atoms * 512u, &full[s]);
+            }
           }
           ++issued;
-          if (++s == kStages) {
+          if (++s == stages) {
             s = 0;
             ph ^= 1u;
           }
@@ -193,23 +241,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ TM
       if (!ok) {
         set_error(p.hdr, SB_ETIMEOUT);
         *abort_flag = 1;
-        // let the copies already issued land before the CTA releases its shared memory
-        const int64_t first = issued > kStages ? issued - kStages : 0;
-        for (int64_t k = first; k < issued; ++k)
-          mbar_wait_bounded(&full[k % kStages], (uint32_t)((k / kStages) & 1), nullptr, kDrainNs);
+        if (!pair) {  // let the copies already issued land before the CTA releases its smem
+          const int64_t first = issued > stages ? issued - stages : 0;
+          for (int64_t k = first; k < issued; ++k)
+            mbar_wait_bounded(&full[k % stages], (uint32_t)((k / stages) & 1), nullptr, kDrainNs);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
-      const uint32_t idesc = idesc_for(kind, BN);
+    if ((!pair || leader) && elect_one()) {
+      const uint32_t idesc = idesc_for(kind, BM, BN);
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x, ++it) {
-        const int nt = tile / m_tiles;
+      for (int tile = unit; ok && tile < tiles; tile += nunits, ++it) {
+        int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
         const int n0 = nt * BN;
         const int b = it & 1;
         const uint32_t tph = (uint32_t)((it >> 1) & 1);
@@ -227,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ TM
             break;
           }
           tc_fence_after();
-          const uint32_t a_s = smem_u32(smem + s * kStageBytes);
+          const uint32_t a_s = smem_u32(smem + s * stage_bytes);
           const uint32_t b_s = a_s + kOffB;
           const int nk = min(4, (K - kb * kb_elems) / mma_k);
           if (kind == KIND_FP4) {
@@ -245,38 +295,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ TM
               mma_fp4(d_tmem, ad, bd, idesc, tmem_base + sfa_col + 4u * j, tmem_base + sfb_col + 8u * j + sfb_shift,
                       acc);
             else if (kind == KIND_I8)
-              mma_i8(d_tmem, ad, bd, idesc, acc);
+              mma_i8_pair(d_tmem, ad, bd, idesc, acc);
             else
-              mma_bf16(d_tmem, ad, bd, idesc, acc);
+              mma_bf16_pair(d_tmem, ad, bd, idesc, acc);
           }
-          mma_commit(&empty[s]);  // the stage is free once these MMAs have read it
-          if (++s == kStages) {
+          if (pair)
+            mma_commit_pair(&empty[s], (uint16_t)3);  // frees the stage in both CTAs
+          else
+            mma_commit(&empty[s]);
+          if (++s == stages) {
             s = 0;
             ph ^= 1u;
           }
         }
-        if (ok) mma_commit(&tfull[b]);  // accumulator ready for the epilogue
+        if (ok) {
+          if (pair)
+            mma_commit_pair(&tfull[b], (uint16_t)3);  // both CTAs' accumulators are ready
+          else
+            mma_commit(&tfull[b]);
+        }
       }
       if (!ok) {
         set_error(p.hdr, SB_ETIMEOUT);
         *abort_flag = 1;
       }
       // wait for every MMA issued by this thread before TMEM is released
-      mma_commit(drain);
+      if (pair)
+        mma_commit_pair(drain, (uint16_t)1);
+      else
+        mma_commit(drain);
       mbar_wait_bounded(drain, 0u, nullptr, kWaitNs);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp & 3;          // TMEM lane quadrant this warp may access
+    const int q = warp & 3;            // TMEM lane quadrant this warp may access
     const int half = (warp - 2) >> 2;  // two warps per quadrant split the column chunks
     const int row = 32 * q + lane;
+    const uint32_t tempty_leader = pair ? cluster_addr(&tempty[0], 0) : 0u;
     float alpha = 1.0f;
     if (kind == KIND_FP4) alpha = __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB);
     int it = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
-      const int mt = tile % m_tiles, nt = tile / m_tiles;
-      const int m = mt * 128 + row, n0 = nt * BN;
+    for (int tile = unit; tile < tiles; tile += nunits, ++it) {
+      int mt, nt;
+      tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
+      const int m = mt * BM + row_off + row, n0 = nt * BN;
       const int b = it & 1;
       const uint32_t tph = (uint32_t)((it >> 1) & 1);
       if (!mbar_wait_bounded(&tfull[b], tph, abort_flag, kWaitNs)) {
@@ -340,14 +403,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ TM
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[b]);
+      if (lane == 0) {
+        if (pair)
+          mbar_arrive_cluster(tempty_leader + 8u * b);  // the leader's MMA waits for both CTAs
+        else
+          mbar_arrive(&tempty[b]);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (pair) cluster_sync();  // the peer is done with this pair's TMEM and barriers
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (pair)
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    else
+      tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -434,7 +506,7 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   }
   if (L.A8 && L.B8 && L.sA8 && L.sB8) {
     if (!make_map(&tm.a[KIND_I8], L.A8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128) ||
-        !make_map(&tm.b[KIND_I8], L.B8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, (uint32_t)p.bn[KIND_I8])) {
+        !make_map(&tm.b[KIND_I8], L.B8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, (uint32_t)p.bn[KIND_I8] / 2)) {
       *why = "cuTensorMapEncodeTiled failed (INT8 operands)";
       return cudaErrorInvalidValue;
     }
@@ -442,19 +514,21 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   }
   if (L.X && L.W16) {
     if (!make_map(&tm.a[KIND_BF16], L.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 128) ||
-        !make_map(&tm.b[KIND_BF16], L.W16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, (uint32_t)p.bn[KIND_BF16])) {
+        !make_map(&tm.b[KIND_BF16], L.W16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N,
+                  (uint32_t)p.bn[KIND_BF16] / 2)) {
       *why = "cuTensorMapEncodeTiled failed (BF16 operands)";
       return cudaErrorInvalidValue;
     }
     p.have[KIND_BF16] = 1;
   }
-  int64_t max_tiles = 0;
-  for (int k = 0; k < 3; ++k) {
-    const int64_t t = ceil_div(L.M, 128) * ceil_div(L.N, p.bn[k]);
-    if (t > max_tiles) max_tiles = t;
-  }
-  const int sms = device_sms();
-  const unsigned grid = (unsigned)(max_tiles < sms ? max_tiles : sms);
+  // CTAs needed: NVFP4 one per 128-row tile, INT8 / BF16 two per 256-row tile
+  int64_t want = ceil_div(L.M, 128) * ceil_div(L.N, p.bn[KIND_FP4]);
+  const int64_t pair_ctas = 2 * ceil_div(L.M, 256) * ceil_div(L.N, p.bn[KIND_I8]);
+  if (pair_ctas > want) want = pair_ctas;
+  const int sms = device_sms() & ~1;
+  int64_t g = want < sms ? want : sms;
+  g = (g + 1) & ~(int64_t)1;  // whole clusters of two
+  const unsigned grid = (unsigned)g;
   k_gemm<<<grid, kThreads, kSmemBytes, s>>>(tm, p);
   return cudaGetLastError();
 }
