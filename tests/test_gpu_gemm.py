@@ -68,8 +68,10 @@ def test_weight_preparation_bitexact(sbg):
 SHAPES = [
     ("tiny", 256, 256, 256),
     ("ragged_m", 300, 256, 512),
-    ("n1920_k1920", 200, 1920, 1920),   # NVFP4: 192-wide tiles with shifted scale atoms, half K-block
+    ("n1920_k1920", 200, 1920, 1920),   # 128-wide tiles (N % 256 != 0), NVFP4 half K-block
     ("n384_k640", 129, 384, 640),
+    ("small_m", 96, 512, 768),          # the second CTA of each pair holds no rows at all
+    ("multi_tile", 700, 1024, 1280),    # 3 x 4 tiles of 256 x 256, ragged last row tile
 ]
 
 

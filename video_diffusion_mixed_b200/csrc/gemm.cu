@@ -5,18 +5,32 @@
 // is needed ("write-up" section 一: NVFP4 or INT8 per layer and step; section 三: full precision
 // under PDR; section 四: 4-bit weights).
 //
-//   NVFP4  tcgen05.mma.kind::mxf4nvf4.block_scale.block16  128 x 192 tiles, K-block 256 elements
-//   INT8   tcgen05.mma.kind::i8 (s32 accumulators)          128 x 256 tiles, K-block 128 elements
-//   BF16   tcgen05.mma.kind::f16 (fp32 accumulators)        128 x 256 tiles, K-block  64 elements
+//   NVFP4  tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16  K-block 256 elements
+//   INT8   tcgen05.mma.cta_group::2.kind::i8 (s32 accumulators)          K-block 128 elements
+//   BF16   tcgen05.mma.cta_group::2.kind::f16 (fp32 accumulators)        K-block  64 elements
 //
-// Every K-block is one 128-byte-wide row slab of A and B (128B swizzle, loaded by TMA without
-// multicast), consumed by four MMAs of 32 bytes of K each. Warp roles (320 threads):
-//   warp 0      TMA producer (one lane): A/B tiles and, for NVFP4, the E4M3 scale atoms
-//   warp 1      TMEM allocator and MMA issuer (one lane); tcgen05.cp moves scales to TMEM
-//   warps 2-9   epilogue: TMEM -> registers, dequant scale, bias, optional GELU, store
-// Two accumulator buffers in TMEM let the epilogue of tile i overlap the mainloop of tile i+1.
-// NVFP4 tiles are 192 wide so both buffers (2 x 192 columns) and the block scales (48 columns)
-// fit the 512 TMEM columns. Every wait is bounded; a wait that gives up records SB_ETIMEOUT.
+// The kernel runs as clusters of two CTAs on the two SMs of a pair. A cluster owns a 256 x BN
+// output tile (BN = 256, or 128 when N is not a multiple of 256): each CTA loads its own 128 rows
+// of A and one half of B -- and, for NVFP4, the E4M3 scales of its rows and of all BN columns --
+// with TMA (no multicast) into its own shared memory; the even CTA (the leader) issues MMAs with
+// M = 256 that read both CTAs' operands, and each CTA's tensor memory receives its 128 rows. Per
+// SM this halves the B traffic through shared memory, whose port is shared by the TMA writes and
+// the MMA reads and otherwise limits the MMA rate.
+//
+// Every K-block is one 128-byte-wide row slab (128B swizzle), consumed by four MMAs of 32 bytes
+// of K. Warp roles (384 threads = 3 warpgroups per CTA):
+//   warp 0      TMA producer (one lane), in both CTAs
+//   warp 1      TMEM allocation (both CTAs); scale copies to TMEM and MMA issue (leader only)
+//   warps 2-3   idle
+//   warps 4-11  epilogue: TMEM -> registers, release the accumulator, then dequant scale, bias,
+//               optional GELU, store
+// The first warpgroup gives registers up (setmaxnreg) so that each epilogue thread can hold 128
+// accumulator values: 40 x 128 + 224 x 256 registers, within the 168 x 384 of the launch.
+// Accumulators: two buffers of BN columns when they fit next to the NVFP4 scale columns (the
+// epilogue of tile i then overlaps the mainloop of tile i + 1), else one; either way the
+// epilogue drains its columns into registers and releases the buffer before computing, so the
+// next tile's MMAs start after the drain. Every wait is bounded; a wait that gives up records
+// SB_ETIMEOUT.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -26,42 +40,49 @@
 
 namespace sb {
 
-// NVFP4 (one CTA per 128 x 192 tile): A 16 KB | B 24 KB | SFA 2 KB | SFB 4 KB, 4 stages.
-// INT8 / BF16 (a CTA pair per 256 x 256 tile): A 16 KB | B half 16 KB per CTA, 6 stages.
+// Per-stage shared memory of one CTA: A 128 rows x 128 B | B half (BN/2 rows) x 128 B | NVFP4
+// only: SFA 4 atoms x 512 B | SFB 2 column tiles x 4 atoms x 512 B. Stage sizes are multiples
+// of 1024 B (the 128B-swizzle atom).
 constexpr int kOffB = 16384;
-constexpr int kOffSFA = 49152;
-constexpr int kOffSFB = 51200;
-constexpr int kStageBytesSingle = 55296;
-constexpr int kStagesSingle = 4;
-constexpr int kStageBytesPair = 32768;
-constexpr int kStagesPair = 6;
+constexpr int kOffSFA = 32768;
+constexpr int kOffSFB = 34816;
+constexpr int kStageBytesQ = 32768;  // INT8 / BF16
+constexpr int kStagesQ = 6;
+constexpr int kStageBytesF = 38912;  // NVFP4
+constexpr int kStagesF = 5;
 constexpr int kMaxStages = 6;
-constexpr int kStageArea = kStagesSingle * kStageBytesSingle;  // >= kStagesPair * kStageBytesPair
-constexpr int kThreads = 320;
+constexpr int kStageArea = kStagesQ * kStageBytesQ;
+constexpr int kThreads = 384;
+constexpr int kEpiWarp0 = 4;  // first epilogue warp
 constexpr int kEpiWarps = 8;
+constexpr uint32_t kRegsCtl = 40;   // producer / MMA warpgroup
+constexpr uint32_t kRegsEpi = 224;  // epilogue warpgroups
+constexpr int kRegsNeeded = (int)(kRegsCtl * 128 + kRegsEpi * 256);
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfCols = 48;             // NVFP4: 16 SFA + 32 SFB columns per K-block
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr uint64_t kDrainNs = 20000000ull;   // 20 ms to let in-flight copies land after an abort
 constexpr int kSmemBytes = kStageArea + 1024 + 512;
-static_assert(kStagesPair * kStageBytesPair <= kStageArea, "stage area");
+static_assert(kStagesF * kStageBytesF <= kStageArea, "NVFP4 stages exceed the stage area");
+static_assert(kOffSFB + 2 * 2048 <= kStageBytesF, "NVFP4 stage layout");
 
 enum { KIND_FP4 = 0, KIND_I8 = 1, KIND_BF16 = 2 };
 
 struct TMaps {
   CUtensorMap a[3];
   CUtensorMap b[3];
+  CUtensorMap sfa;  // NVFP4 scales of A, 3-D: 128 words x K/64 atoms x 128-row tiles
+  CUtensorMap sfb;  // NVFP4 scales of B, same shape over the N rows of the weight
 };
 
 struct GemmParams {
   int M, N, K;
+  int BN;
   float invB;
   const int32_t* prec;
-  int bn[3];
   int have[3];
   const float* sA8;
   const float* sB8;
-  const uint8_t* sfA4;
-  const uint8_t* sfB4;
   const float* gA4;
   const float* gB4;
   const __nv_bfloat16* bias;
@@ -112,10 +133,54 @@ __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int
   *nt = r / gm;
 }
 
-// Launched as clusters of two CTAs. INT8 and BF16 run "pair" tiles: the two CTAs of a cluster
-// share one 256 x BN tile; each loads its own 128 rows of A and its half of B, the even CTA (the
-// leader) issues tcgen05.mma.cta_group::2 with M = 256 and both CTAs' accumulators receive their
-// 128 rows. NVFP4 runs one 128 x BN tile per CTA and ignores the cluster.
+// Epilogue of 32 accumulator columns [n, n + 32) of row m: dequant scale, bias, GELU, store.
+__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int kind, int m, int n, float sxb, float alpha,
+                                               const uint32_t (&r)[32]) {
+  if (p.out_dtype == SB_OUT_RAW) {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(p.Y) + (int64_t)m * p.N + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+    return;
+  }
+  float y[32];
+  if (kind == KIND_I8) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__int2float_rn((int)r[i]), __fmul_rn(sxb, __ldg(p.sB8 + n + i)));
+  } else if (kind == KIND_FP4) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
+  }
+  if (p.bias) {
+    const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 u = __ldg(bp + i);
+      float bv[8];
+      unpack8(u, bv);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[8 * i + j] = __fadd_rn(y[8 * i + j], bv[j]);
+    }
+  }
+  if (p.epilogue == SB_EPI_GELU_TANH) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = gelu_tanh(y[i]);
+  }
+  if (p.out_dtype == SB_OUT_F32) {
+    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.Y) + (int64_t)m * p.N + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.Y) + (int64_t)m * p.N + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      dst[i] = make_uint4(pack_bf16(y[8 * i], y[8 * i + 1]), pack_bf16(y[8 * i + 2], y[8 * i + 3]),
+                          pack_bf16(y[8 * i + 4], y[8 * i + 5]), pack_bf16(y[8 * i + 6], y[8 * i + 7]));
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ TMaps tm, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -135,24 +200,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (blockIdx.x == 0 && threadIdx.x == 0) set_error(p.hdr, SB_EINVAL);
     return;
   }
-  const bool pair = (kind != KIND_FP4);
   const uint32_t rank = cluster_ctarank();
   const bool leader = (rank == 0);
-  const int M = p.M, N = p.N, K = p.K;
-  const int BN = p.bn[kind];
-  const int BM = pair ? 256 : 128;
-  const int kb_elems = (kind == KIND_FP4) ? 256 : (kind == KIND_I8 ? 128 : 64);
+  const bool fp4 = (kind == KIND_FP4);
+  const int M = p.M, N = p.N, K = p.K, BN = p.BN;
+  const int kb_elems = fp4 ? 256 : (kind == KIND_I8 ? 128 : 64);
   const int mma_k = kb_elems >> 2;
   const int nkb = (K + kb_elems - 1) / kb_elems;
-  const int m_tiles = (M + BM - 1) / BM;
+  const int m_tiles = (M + 255) / 256;
   const int n_tiles = (N + BN - 1) / BN;
   const int tiles = m_tiles * n_tiles;
-  const int unit = pair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-  const int nunits = pair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  if (unit >= tiles) return;  // pair mode: both CTAs of the cluster leave together
-  const int stages = pair ? kStagesPair : kStagesSingle;
-  const int stage_bytes = pair ? kStageBytesPair : kStageBytesSingle;
-  const int row_off = pair ? 128 * (int)rank : 0;  // this CTA's rows inside the tile
+  const int unit = (int)(blockIdx.x >> 1);
+  const int nunits = (int)(gridDim.x >> 1);
+  if (unit >= tiles) return;  // both CTAs of the cluster leave together
+  const int stages = fp4 ? kStagesF : kStagesQ;
+  const int stage_bytes = fp4 ? kStageBytesF : kStageBytesQ;
+  const int row_off = 128 * (int)rank;  // this CTA's rows inside the 256-row tile
+  const int sf_tiles = BN / 128;        // NVFP4: 128-column scale tiles of B per output tile
+  const int nacc = (2 * BN + (fp4 ? (int)kSfCols : 0) <= (int)kTmemCols) ? 2 : 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMaxStages; ++s) {
@@ -161,265 +226,195 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], pair ? 2 * kEpiWarps : kEpiWarps);
+      mbar_init(&tempty[b], 2 * kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (pair) cluster_sync();  // the peer's barriers exist before any remote arrive or copy
+  cluster_sync();  // the peer's barriers exist before any remote arrive or copy
   if (warp == 1) {
-    if (pair) {
-      tmem_alloc_pair(tmem_slot, kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t sfa_col = 2u * BN;        // NVFP4: 4 columns per MMA step (128 rows x 4 scales)
-  const uint32_t sfb_col = 2u * BN + 16u;  // NVFP4: 8 columns per MMA step (two 128-row tiles)
-  const int sf_atoms_k = K >> 6;           // 64-element scale atoms along K
-  const int sf_tiles_n = (N + 127) >> 7;
+  const uint32_t sfa_col = (uint32_t)(nacc * BN);  // NVFP4: 4 columns per MMA (128 rows x 4 scales)
+  const uint32_t sfb_col = sfa_col + 16u;          // NVFP4: 8 columns per MMA (up to 2 column tiles)
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (elect_one()) {
-      prefetch_tmap(&tm.a[kind]);
-      prefetch_tmap(&tm.b[kind]);
-      const uint32_t full_leader = pair ? cluster_addr(&full[0], 0) : 0u;
-      int s = 0;
-      uint32_t ph = 0;
-      int64_t issued = 0;
-      bool ok = true;
-      for (int tile = unit; ok && tile < tiles; tile += nunits) {
-        int mt, nt;
-        tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
-        const int m0 = mt * BM + row_off, n0 = nt * BN;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitNs)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = smem + s * stage_bytes;
-          const int x = (kind == KIND_BF16) ? kb * 64 : kb * 128;
-          if (pair) {
-            if (leader) mbar_arrive_expect_tx(&full[s], 2u * (16384u + (uint32_t)(BN / 2) * 128u));
-            tma_load_2d_pair(st, &tm.a[kind], full_leader + 8u * s, x, m0);
-            tma_load_2d_pair(st + kOffB, &tm.b[kind], full_leader + 8u * s, x, n0 + (BN / 2) * (int)rank);
-          } else {
-            uint32_t bytes = 16384u + (uint32_t)BN * 128u;
-            int atoms = 0, btiles = 0;
-            if (kind == KIND_FP4) {
-              atoms = min(4, sf_atoms_k - 4 * kb);
-              btiles = min((n0 % 128 + BN + 127) >> 7, sf_tiles_n - (n0 >> 7));
-              bytes += (uint32_t)atoms * 512u * (uint32_t)(1 + btiles);
+  if (warp < kEpiWarp0) {
+    setmaxnreg_dec<kRegsCtl>();  // one instruction for the whole first warpgroup
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer (both CTAs)
+      if (elect_one()) {
+        prefetch_tmap(&tm.a[kind]);
+        prefetch_tmap(&tm.b[kind]);
+        if (fp4) {
+          prefetch_tmap(&tm.sfa);
+          prefetch_tmap(&tm.sfb);
+        }
+        const uint32_t full_leader = cluster_addr(&full[0], 0);
+        // bytes both CTAs deliver to the leader's barrier per stage
+        const uint32_t stage_tx = 2u * (16384u + (uint32_t)(BN / 2) * 128u + (fp4 ? 2048u * (1u + sf_tiles) : 0u));
+        int s = 0;
+        uint32_t ph = 0;
+        int64_t issued = 0;
+        bool ok = true;
+        for (int tile = unit; ok && tile < tiles; tile += nunits) {
+          int mt, nt;
+          tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
+          const int m0 = mt * 256 + row_off, n0 = nt * BN;
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitNs)) {
+              ok = false;
+              break;
             }
-            mbar_arrive_expect_tx(&full[s], bytes);
-            tma_load_2d(st, &tm.a[kind], &full[s], x, m0);
-            tma_load_2d(st + kOffB, &tm.b[kind], &full[s], x, n0);
-            if (kind == KIND_FP4) {
-              bulk_load(st + kOffSFA, p.sfA4 + ((int64_t)mt * sf_atoms_k + 4 * kb) * 512, atoms * 512u, &full[s]);
-              const int t0 = n0 >> 7;
-              for (int t = 0; t < btiles; ++t)
-                bulk_load(st + kOffSFB + 2048 * t, p.sfB4 + ((int64_t)(t0 + t) * sf_atoms_k + 4 * kb) * 512,
-                          atoms * 512u, &full[s]);
+            uint8_t* st = smem + s * stage_bytes;
+            const uint32_t fb = full_leader + 8u * s;
+            if (leader) mbar_arrive_expect_tx(&full[s], stage_tx);
+            const int x = (kind == KIND_BF16) ? kb * 64 : kb * 128;  // 128-byte column slab
+            tma_load_2d_pair(st, &tm.a[kind], fb, x, m0);
+            tma_load_2d_pair(st + kOffB, &tm.b[kind], fb, x, n0 + (BN / 2) * (int)rank);
+            if (fp4) {
+              // 4 scale atoms (64 K-elements each) of this CTA's 128 rows and of every 128-column
+              // tile of B; atoms past K and rows past M read as zero
+              tma_load_3d_pair(st + kOffSFA, &tm.sfa, fb, 0, 4 * kb, m0 >> 7);
+              for (int t = 0; t < sf_tiles; ++t)
+                tma_load_3d_pair(st + kOffSFB + 2048 * t, &tm.sfb, fb, 0, 4 * kb, (n0 >> 7) + t);
+            }
+            ++issued;
+            if (++s == stages) {
+              s = 0;
+              ph ^= 1u;
             }
           }
-          ++issued;
-          if (++s == stages) {
-            s = 0;
-            ph ^= 1u;
+        }
+        if (!ok) {
+          set_error(p.hdr, SB_ETIMEOUT);
+          *abort_flag = 1;
+          if (leader) {  // both CTAs' copies complete on the leader's barriers: let them land
+            const int64_t first = issued > stages ? issued - stages : 0;
+            for (int64_t k = first; k < issued; ++k)
+              mbar_wait_bounded(&full[k % stages], (uint32_t)((k / stages) & 1), nullptr, kDrainNs);
           }
         }
       }
-      if (!ok) {
-        set_error(p.hdr, SB_ETIMEOUT);
-        *abort_flag = 1;
-        if (!pair) {  // let the copies already issued land before the CTA releases its smem
-          const int64_t first = issued > stages ? issued - stages : 0;
-          for (int64_t k = first; k < issued; ++k)
-            mbar_wait_bounded(&full[k % stages], (uint32_t)((k / stages) & 1), nullptr, kDrainNs);
-        }
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if ((!pair || leader) && elect_one()) {
-      const uint32_t idesc = idesc_for(kind, BM, BN);
-      int s = 0;
-      uint32_t ph = 0;
-      int it = 0;
-      bool ok = true;
-      for (int tile = unit; ok && tile < tiles; tile += nunits, ++it) {
-        int mt, nt;
-        tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
-        const int n0 = nt * BN;
-        const int b = it & 1;
-        const uint32_t tph = (uint32_t)((it >> 1) & 1);
-        if (!mbar_wait_bounded(&tempty[b], tph ^ 1u, abort_flag, kWaitNs)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
-        const int btiles = (kind == KIND_FP4) ? min((n0 % 128 + BN + 127) >> 7, sf_tiles_n - (n0 >> 7)) : 0;
-        const uint32_t sfb_shift = (uint32_t)((n0 % 128) >> 5);
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait_bounded(&full[s], ph, abort_flag, kWaitNs)) {
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issue (leader)
+      if (leader && elect_one()) {
+        const uint32_t idesc = idesc_for(kind, 256, BN);
+        int s = 0;
+        uint32_t ph = 0;
+        int it = 0;
+        bool ok = true;
+        for (int tile = unit; ok && tile < tiles; tile += nunits, ++it) {
+          const int b = it % nacc;
+          const uint32_t tph = (uint32_t)((it / nacc) & 1);
+          if (!mbar_wait_bounded(&tempty[b], tph ^ 1u, abort_flag, kWaitNs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_s = smem_u32(smem + s * stage_bytes);
-          const uint32_t b_s = a_s + kOffB;
-          const int nk = min(4, (K - kb * kb_elems) / mma_k);
-          if (kind == KIND_FP4) {
+          const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait_bounded(&full[s], ph, abort_flag, kWaitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_s = smem_u32(smem + s * stage_bytes);
+            const uint32_t b_s = a_s + kOffB;
+            const int nk = min(4, (K - kb * kb_elems) / mma_k);
+            if (fp4) {
+              // scales of MMA j: SFA atom j -> 4 columns, SFB atom j of tile t -> 4 columns at 4t
+              for (int j = 0; j < nk; ++j) {
+                tmem_cp_sf_pair(tmem_base + sfa_col + 4u * j, desc_sf(a_s + kOffSFA + 512u * j));
+                for (int t = 0; t < sf_tiles; ++t)
+                  tmem_cp_sf_pair(tmem_base + sfb_col + 8u * j + 4u * t, desc_sf(a_s + kOffSFB + 2048u * t + 512u * j));
+              }
+            }
             for (int j = 0; j < nk; ++j) {
-              tmem_cp_sf(tmem_base + sfa_col + 4u * j, desc_sf(a_s + kOffSFA + 512u * j));
-              for (int t = 0; t < btiles; ++t)
-                tmem_cp_sf(tmem_base + sfb_col + 8u * j + 4u * t, desc_sf(a_s + kOffSFB + 2048u * t + 512u * j));
+              const uint64_t ad = desc_sw128(a_s + 32u * j);
+              const uint64_t bd = desc_sw128(b_s + 32u * j);
+              const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
+              if (fp4)
+                mma_fp4_pair(d_tmem, ad, bd, idesc, tmem_base + sfa_col + 4u * j, tmem_base + sfb_col + 8u * j, acc);
+              else if (kind == KIND_I8)
+                mma_i8_pair(d_tmem, ad, bd, idesc, acc);
+              else
+                mma_bf16_pair(d_tmem, ad, bd, idesc, acc);
+            }
+            mma_commit_pair(&empty[s], (uint16_t)3);  // frees the stage in both CTAs
+            if (++s == stages) {
+              s = 0;
+              ph ^= 1u;
             }
           }
-          for (int j = 0; j < nk; ++j) {
-            const uint64_t ad = desc_sw128(a_s + 32u * j);
-            const uint64_t bd = desc_sw128(b_s + 32u * j);
-            const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
-            if (kind == KIND_FP4)
-              mma_fp4(d_tmem, ad, bd, idesc, tmem_base + sfa_col + 4u * j, tmem_base + sfb_col + 8u * j + sfb_shift,
-                      acc);
-            else if (kind == KIND_I8)
-              mma_i8_pair(d_tmem, ad, bd, idesc, acc);
-            else
-              mma_bf16_pair(d_tmem, ad, bd, idesc, acc);
-          }
-          if (pair)
-            mma_commit_pair(&empty[s], (uint16_t)3);  // frees the stage in both CTAs
-          else
-            mma_commit(&empty[s]);
-          if (++s == stages) {
-            s = 0;
-            ph ^= 1u;
-          }
+          if (ok) mma_commit_pair(&tfull[b], (uint16_t)3);  // both CTAs' accumulators are ready
         }
-        if (ok) {
-          if (pair)
-            mma_commit_pair(&tfull[b], (uint16_t)3);  // both CTAs' accumulators are ready
-          else
-            mma_commit(&tfull[b]);
+        if (!ok) {
+          set_error(p.hdr, SB_ETIMEOUT);
+          *abort_flag = 1;
         }
-      }
-      if (!ok) {
-        set_error(p.hdr, SB_ETIMEOUT);
-        *abort_flag = 1;
-      }
-      // wait for every MMA issued by this thread before TMEM is released
-      if (pair)
+        // wait for every MMA issued by this thread before TMEM is released
         mma_commit_pair(drain, (uint16_t)1);
-      else
-        mma_commit(drain);
-      mbar_wait_bounded(drain, 0u, nullptr, kWaitNs);
+        mbar_wait_bounded(drain, 0u, nullptr, kWaitNs);
+      }
+      __syncwarp();
     }
-    __syncwarp();
   } else {
-    // ------------------------------------------------------------------ epilogue
-    const int q = warp & 3;            // TMEM lane quadrant this warp may access
-    const int half = (warp - 2) >> 2;  // two warps per quadrant split the column chunks
+    setmaxnreg_inc<kRegsEpi>();
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;                    // TMEM lane quadrant this warp may access
+    const int half = (warp - kEpiWarp0) >> 2;  // two warps per quadrant split the tile's columns
     const int row = 32 * q + lane;
-    const uint32_t tempty_leader = pair ? cluster_addr(&tempty[0], 0) : 0u;
-    float alpha = 1.0f;
-    if (kind == KIND_FP4) alpha = __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB);
+    const int nch = BN / 64;                   // 32-column chunks per warp: 2 or 4
+    const uint32_t tempty_leader = cluster_addr(&tempty[0], 0);
+    const float alpha = fp4 ? __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB) : 1.0f;
     int it = 0;
     for (int tile = unit; tile < tiles; tile += nunits, ++it) {
       int mt, nt;
       tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
-      const int m = mt * BM + row_off + row, n0 = nt * BN;
-      const int b = it & 1;
-      const uint32_t tph = (uint32_t)((it >> 1) & 1);
+      const int m = mt * 256 + row_off + row;
+      const int n0 = nt * BN + half * (BN / 2);
+      const int b = it % nacc;
+      const uint32_t tph = (uint32_t)((it / nacc) & 1);
       if (!mbar_wait_bounded(&tfull[b], tph, abort_flag, kWaitNs)) {
         set_error(p.hdr, SB_ETIMEOUT);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const bool row_ok = m < M;
-      const float sx = (kind == KIND_I8 && row_ok) ? p.sA8[m] : 0.0f;
-      for (int c = half; c < BN / 32; c += 2) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN + 32 * c), r);
-        tmem_ld_wait();
-        const int n = n0 + 32 * c;
-        if (!row_ok || n >= N) continue;
-        if (p.out_dtype == SB_OUT_RAW) {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(p.Y) + (int64_t)m * N + n);
+      // drain this warp's columns into registers, then hand the buffer back to the MMA
+      uint32_t r[4][32];
+      const uint32_t tcol = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN + half * (BN / 2));
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-          continue;
-        }
-        float y[32];
-        if (kind == KIND_I8) {
-          const float sxb = __fmul_rn(sx, p.invB);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__int2float_rn((int)r[i]), __fmul_rn(sxb, __ldg(p.sB8 + n + i)));
-        } else if (kind == KIND_FP4) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
-        }
-        if (p.bias) {
-          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 u = __ldg(bp + i);
-            float bv[8];
-            unpack8(u, bv);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) y[8 * i + j] = __fadd_rn(y[8 * i + j], bv[j]);
-          }
-        }
-        if (p.epilogue == SB_EPI_GELU_TANH) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = gelu_tanh(y[i]);
-        }
-        if (p.out_dtype == SB_OUT_F32) {
-          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.Y) + (int64_t)m * N + n);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.Y) + (int64_t)m * N + n);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pack_bf16(y[8 * i], y[8 * i + 1]), pack_bf16(y[8 * i + 2], y[8 * i + 3]),
-                                pack_bf16(y[8 * i + 4], y[8 * i + 5]), pack_bf16(y[8 * i + 6], y[8 * i + 7]));
-        }
-      }
+      for (int c = 0; c < 4; ++c)
+        if (c < nch) tmem_ld32(tcol + 32u * c, r[c]);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        if (pair)
-          mbar_arrive_cluster(tempty_leader + 8u * b);  // the leader's MMA waits for both CTAs
-        else
-          mbar_arrive(&tempty[b]);
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * b);  // the leader waits for both CTAs
+      if (m < M) {
+        const float sxb = (kind == KIND_I8) ? __fmul_rn(p.sA8[m], p.invB) : 0.0f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int n = n0 + 32 * c;
+          if (c < nch && n < N) epilogue_chunk(p, kind, m, n, sxb, alpha, r[c]);
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (pair) cluster_sync();  // the peer is done with this pair's TMEM and barriers
+  cluster_sync();  // the peer is done with this pair's TMEM, barriers and shared memory
   if (warp == 1) {
     tc_fence_after();
-    if (pair)
-      tmem_dealloc_pair(tmem_base, kTmemCols);
-    else
-      tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -455,6 +450,21 @@ static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over an NVFP4 block-scale array in the tensor-core layout (512-byte atoms of 128 rows x
+// 4 groups, K/64 atoms per 128-row tile): 128 32-bit words per atom x K/64 atoms x row tiles;
+// box = 4 atoms of one row tile (2 KB), no swizzle.
+static bool make_sf_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, K / 64, (rows + 127) / 128};
+  cuuint64_t strides[2] = {512, (K / 64) * 512};
+  cuuint32_t box[3] = {128, 4, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int device_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -472,6 +482,21 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
     *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
     return attr_err;
   }
+  // The register split of the kernel must fit what a CTA is launched with, or the epilogue's
+  // setmaxnreg.inc would wait for registers that never come free.
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, k_gemm) != cudaSuccess) {
+      *why = "cudaFuncGetAttributes(k_gemm) failed";
+      return cudaErrorInvalidValue;
+    }
+    regs = fa.numRegs;
+  }
+  if (regs * kThreads < kRegsNeeded) {
+    *why = "k_gemm was compiled with fewer registers per thread than its warpgroup split needs";
+    return cudaErrorInvalidConfiguration;
+  }
   TMaps tm;
   memset(&tm, 0, sizeof(tm));
   GemmParams p;
@@ -479,15 +504,11 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   p.M = (int)L.M;
   p.N = (int)L.N;
   p.K = (int)L.K;
+  p.BN = (L.N % 256 == 0) ? 256 : 128;
   p.invB = 1.0f / (float)L.B;
   p.prec = L.prec;
-  p.bn[KIND_FP4] = (L.N % 192 == 0) ? 192 : 128;
-  p.bn[KIND_I8] = (L.N % 256 == 0) ? 256 : 128;
-  p.bn[KIND_BF16] = p.bn[KIND_I8];
   p.sA8 = L.sA8;
   p.sB8 = L.sB8;
-  p.sfA4 = L.sfA4;
-  p.sfB4 = L.sfB4;
   p.gA4 = L.gA4;
   p.gB4 = L.gB4;
   p.bias = reinterpret_cast<const __nv_bfloat16*>(L.bias);
@@ -496,9 +517,11 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   p.epilogue = L.epilogue;
   p.hdr = reinterpret_cast<WsHeader*>(L.hdr);
   const uint64_t M = (uint64_t)L.M, N = (uint64_t)L.N, K = (uint64_t)L.K;
+  const uint32_t half = (uint32_t)p.BN / 2;  // B rows each CTA of the pair loads
   if (L.A4 && L.B4 && L.sfA4 && L.sfB4 && L.gA4 && L.gB4) {
     if (!make_map(&tm.a[KIND_FP4], L.A4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128) ||
-        !make_map(&tm.b[KIND_FP4], L.B4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, (uint32_t)p.bn[KIND_FP4])) {
+        !make_map(&tm.b[KIND_FP4], L.B4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, half) ||
+        !make_sf_map(&tm.sfa, L.sfA4, K, M) || !make_sf_map(&tm.sfb, L.sfB4, K, N)) {
       *why = "cuTensorMapEncodeTiled failed (NVFP4 operands)";
       return cudaErrorInvalidValue;
     }
@@ -506,7 +529,7 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   }
   if (L.A8 && L.B8 && L.sA8 && L.sB8) {
     if (!make_map(&tm.a[KIND_I8], L.A8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128) ||
-        !make_map(&tm.b[KIND_I8], L.B8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, (uint32_t)p.bn[KIND_I8] / 2)) {
+        !make_map(&tm.b[KIND_I8], L.B8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, half)) {
       *why = "cuTensorMapEncodeTiled failed (INT8 operands)";
       return cudaErrorInvalidValue;
     }
@@ -514,21 +537,16 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   }
   if (L.X && L.W16) {
     if (!make_map(&tm.a[KIND_BF16], L.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 128) ||
-        !make_map(&tm.b[KIND_BF16], L.W16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N,
-                  (uint32_t)p.bn[KIND_BF16] / 2)) {
+        !make_map(&tm.b[KIND_BF16], L.W16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, half)) {
       *why = "cuTensorMapEncodeTiled failed (BF16 operands)";
       return cudaErrorInvalidValue;
     }
     p.have[KIND_BF16] = 1;
   }
-  // CTAs needed: NVFP4 one per 128-row tile, INT8 / BF16 two per 256-row tile
-  int64_t want = ceil_div(L.M, 128) * ceil_div(L.N, p.bn[KIND_FP4]);
-  const int64_t pair_ctas = 2 * ceil_div(L.M, 256) * ceil_div(L.N, p.bn[KIND_I8]);
-  if (pair_ctas > want) want = pair_ctas;
+  // one cluster of two CTAs per 256 x BN tile, at most one CTA per SM
+  const int64_t want = 2 * ceil_div(L.M, 256) * ceil_div(L.N, p.BN);
   const int sms = device_sms() & ~1;
-  int64_t g = want < sms ? want : sms;
-  g = (g + 1) & ~(int64_t)1;  // whole clusters of two
-  const unsigned grid = (unsigned)g;
+  const unsigned grid = (unsigned)(want < sms ? want : sms);
   k_gemm<<<grid, kThreads, kSmemBytes, s>>>(tm, p);
   return cudaGetLastError();
 }
