@@ -25,7 +25,7 @@
 //   warps 4-11  epilogue: TMEM -> registers, release the accumulator, then dequant scale, bias,
 //               optional GELU, store
 // The first warpgroup gives registers up (setmaxnreg) so that each epilogue thread can hold 128
-// accumulator values: 40 x 128 + 224 x 256 registers, within the 168 x 384 of the launch.
+// accumulator values: 72 x 128 + 216 x 256 registers, exactly the 168 x 384 of the launch.
 // Accumulators: two buffers of BN columns when they fit next to the NVFP4 scale columns (the
 // epilogue of tile i then overlaps the mainloop of tile i + 1), else one; either way the
 // epilogue drains its columns into registers and releases the buffer before computing, so the
@@ -55,8 +55,8 @@ constexpr int kStageArea = kStagesQ * kStageBytesQ;
 constexpr int kThreads = 384;
 constexpr int kEpiWarp0 = 4;  // first epilogue warp
 constexpr int kEpiWarps = 8;
-constexpr uint32_t kRegsCtl = 40;   // producer / MMA warpgroup
-constexpr uint32_t kRegsEpi = 224;  // epilogue warpgroups
+constexpr uint32_t kRegsCtl = 72;   // producer / MMA warpgroup
+constexpr uint32_t kRegsEpi = 216;  // epilogue warpgroups
 constexpr int kRegsNeeded = (int)(kRegsCtl * 128 + kRegsEpi * 256);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCols = 48;             // NVFP4: 16 SFA + 32 SFB columns per K-block
@@ -179,6 +179,98 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int kind, in
       dst[i] = make_uint4(pack_bf16(y[8 * i], y[8 * i + 1]), pack_bf16(y[8 * i + 2], y[8 * i + 3]),
                           pack_bf16(y[8 * i + 4], y[8 * i + 5]), pack_bf16(y[8 * i + 6], y[8 * i + 7]));
   }
+}
+
+// ---------------------------------------------------------------------------------------------
+// MMA issue (one thread of the leader CTA). The loop is instantiated per precision and number of
+// 128-column scale tiles so that a full K-block is straight-line code: shared-memory descriptors
+// are advanced by adding to their 14-bit start-address field (addresses stay below 256 KB), and
+// TMEM addresses are precomputed.
+// ---------------------------------------------------------------------------------------------
+
+struct Issuer {
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  volatile int* abort;
+  uint32_t smem;      // shared address of stage 0
+  uint32_t stage16;   // stage size in 16-byte units
+  int stages, nkb, tail_nk, tiles, unit, nunits, BN, nacc;
+  uint32_t tmem, sfa, sfb, idesc;  // TMEM base, scale columns (absolute), instruction descriptor
+};
+
+template <int KIND>
+__device__ __forceinline__ void mma_one(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t sfa,
+                                        uint32_t sfb, uint32_t acc) {
+  if constexpr (KIND == KIND_FP4)
+    mma_fp4_pair(d, ad, bd, idesc, sfa, sfb, acc);
+  else if constexpr (KIND == KIND_I8)
+    mma_i8_pair(d, ad, bd, idesc, acc);
+  else
+    mma_bf16_pair(d, ad, bd, idesc, acc);
+}
+
+// One K-block: NVFP4 scale copies (SFA atom j -> 4 columns at 4j; SFB atom j of column tile t ->
+// 4 columns at 8j + 4t), then the nk MMAs of 32 bytes of K each.
+template <int KIND, int SFT>
+__device__ __forceinline__ void issue_kblock(const Issuer& c, uint32_t d, uint64_t ad, uint64_t bd, uint64_t fa,
+                                             uint64_t fb, int nk, bool first) {
+  if (nk == 4) {
+    if constexpr (KIND == KIND_FP4) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        tmem_cp_sf_pair(c.sfa + 4u * j, fa + 32u * j);
+#pragma unroll
+        for (int t = 0; t < SFT; ++t) tmem_cp_sf_pair(c.sfb + 8u * j + 4u * t, fb + 128u * t + 32u * j);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      mma_one<KIND>(d, ad + 2u * j, bd + 2u * j, c.idesc, c.sfa + 4u * j, c.sfb + 8u * j, (first && j == 0) ? 0u : 1u);
+  } else {
+    if constexpr (KIND == KIND_FP4) {
+      for (int j = 0; j < nk; ++j) {
+        tmem_cp_sf_pair(c.sfa + 4u * j, fa + 32u * j);
+#pragma unroll
+        for (int t = 0; t < SFT; ++t) tmem_cp_sf_pair(c.sfb + 8u * j + 4u * t, fb + 128u * t + 32u * j);
+      }
+    }
+    for (int j = 0; j < nk; ++j)
+      mma_one<KIND>(d, ad + 2u * j, bd + 2u * j, c.idesc, c.sfa + 4u * j, c.sfb + 8u * j, (first && j == 0) ? 0u : 1u);
+  }
+}
+
+// Returns false when a wait gave up.
+template <int KIND, int SFT>
+__device__ __noinline__ bool issue_all(const Issuer c) {
+  const uint64_t dsw = desc_sw128(c.smem);
+  const uint64_t dsf = desc_sf(c.smem);
+  int s = 0;
+  uint32_t ph = 0;
+  int it = 0;
+  for (int tile = c.unit; tile < c.tiles; tile += c.nunits, ++it) {
+    const int b = (c.nacc == 1) ? 0 : (it & 1);
+    const uint32_t tph = (uint32_t)(((c.nacc == 1) ? it : (it >> 1)) & 1);
+    if (!mbar_wait_bounded(&c.tempty[b], tph ^ 1u, c.abort, kWaitNs)) return false;
+    tc_fence_after();
+    const uint32_t d = c.tmem + (uint32_t)(b * c.BN);
+    for (int kb = 0; kb < c.nkb; ++kb) {
+      if (!mbar_wait_bounded(&c.full[s], ph, c.abort, kWaitNs)) return false;
+      tc_fence_after();
+      const uint32_t so = (uint32_t)s * c.stage16;
+      const uint64_t ad = dsw + so;
+      issue_kblock<KIND, SFT>(c, d, ad, ad + (kOffB >> 4), dsf + so + (kOffSFA >> 4), dsf + so + (kOffSFB >> 4),
+                              (kb == c.nkb - 1) ? c.tail_nk : 4, kb == 0);
+      mma_commit_pair(&c.empty[s], (uint16_t)3);  // frees the stage in both CTAs
+      if (++s == c.stages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    mma_commit_pair(&c.tfull[b], (uint16_t)3);  // both CTAs' accumulators are ready
+  }
+  return true;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -306,56 +398,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ------------------------------------------------------------------ MMA issue (leader)
       if (leader && elect_one()) {
-        const uint32_t idesc = idesc_for(kind, 256, BN);
-        int s = 0;
-        uint32_t ph = 0;
-        int it = 0;
-        bool ok = true;
-        for (int tile = unit; ok && tile < tiles; tile += nunits, ++it) {
-          const int b = it % nacc;
-          const uint32_t tph = (uint32_t)((it / nacc) & 1);
-          if (!mbar_wait_bounded(&tempty[b], tph ^ 1u, abort_flag, kWaitNs)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
-          for (int kb = 0; kb < nkb; ++kb) {
-            if (!mbar_wait_bounded(&full[s], ph, abort_flag, kWaitNs)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a_s = smem_u32(smem + s * stage_bytes);
-            const uint32_t b_s = a_s + kOffB;
-            const int nk = min(4, (K - kb * kb_elems) / mma_k);
-            if (fp4) {
-              // scales of MMA j: SFA atom j -> 4 columns, SFB atom j of tile t -> 4 columns at 4t
-              for (int j = 0; j < nk; ++j) {
-                tmem_cp_sf_pair(tmem_base + sfa_col + 4u * j, desc_sf(a_s + kOffSFA + 512u * j));
-                for (int t = 0; t < sf_tiles; ++t)
-                  tmem_cp_sf_pair(tmem_base + sfb_col + 8u * j + 4u * t, desc_sf(a_s + kOffSFB + 2048u * t + 512u * j));
-              }
-            }
-            for (int j = 0; j < nk; ++j) {
-              const uint64_t ad = desc_sw128(a_s + 32u * j);
-              const uint64_t bd = desc_sw128(b_s + 32u * j);
-              const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
-              if (fp4)
-                mma_fp4_pair(d_tmem, ad, bd, idesc, tmem_base + sfa_col + 4u * j, tmem_base + sfb_col + 8u * j, acc);
-              else if (kind == KIND_I8)
-                mma_i8_pair(d_tmem, ad, bd, idesc, acc);
-              else
-                mma_bf16_pair(d_tmem, ad, bd, idesc, acc);
-            }
-            mma_commit_pair(&empty[s], (uint16_t)3);  // frees the stage in both CTAs
-            if (++s == stages) {
-              s = 0;
-              ph ^= 1u;
-            }
-          }
-          if (ok) mma_commit_pair(&tfull[b], (uint16_t)3);  // both CTAs' accumulators are ready
-        }
+        Issuer c;
+        c.full = full;
+        c.empty = empty;
+        c.tfull = tfull;
+        c.tempty = tempty;
+        c.abort = abort_flag;
+        c.smem = smem_u32(smem);
+        c.stage16 = (uint32_t)stage_bytes >> 4;
+        c.stages = stages;
+        c.nkb = nkb;
+        c.tail_nk = min(4, (K - (nkb - 1) * kb_elems) / mma_k);
+        c.tiles = tiles;
+        c.unit = unit;
+        c.nunits = nunits;
+        c.BN = BN;
+        c.nacc = nacc;
+        c.tmem = tmem_base;
+        c.sfa = tmem_base + sfa_col;
+        c.sfb = tmem_base + sfb_col;
+        c.idesc = idesc_for(kind, 256, BN);
+        bool ok;
+        if (fp4)
+          ok = (sf_tiles == 2) ? issue_all<KIND_FP4, 2>(c) : issue_all<KIND_FP4, 1>(c);
+        else if (kind == KIND_I8)
+          ok = issue_all<KIND_I8, 0>(c);
+        else
+          ok = issue_all<KIND_BF16, 0>(c);
         if (!ok) {
           set_error(p.hdr, SB_ETIMEOUT);
           *abort_flag = 1;
