@@ -62,7 +62,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCols = 48;             // NVFP4: 16 SFA + 32 SFB columns per K-block
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr uint64_t kDrainNs = 20000000ull;   // 20 ms to let in-flight copies land after an abort
-constexpr int kSmemBytes = kStageArea + 1024 + 512;
+// After the stages: 1 KB of barriers, then the epilogue's output staging (bf16 output): two
+// 32 x 32 bf16 boxes (2 KB each, 64B swizzle) per epilogue warp.
+constexpr int kBarBytes = 1024;
+constexpr int kOutOff = kStageArea + kBarBytes;
+constexpr int kOutBox = 2048;
+constexpr int kOutBytes = 8 * 2 * kOutBox;
+constexpr int kSmemBytes = kOutOff + kOutBytes + 1024;  // + alignment of the dynamic base to 1 KB
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kStagesF * kStageBytesF <= kStageArea, "NVFP4 stages exceed the stage area");
 static_assert(kOffSFB + 2 * 2048 <= kStageBytesF, "NVFP4 stage layout");
 
@@ -73,6 +80,7 @@ struct TMaps {
   CUtensorMap b[3];
   CUtensorMap sfa;  // NVFP4 scales of A, 3-D: 128 words x K/64 atoms x 128-row tiles
   CUtensorMap sfb;  // NVFP4 scales of B, same shape over the N rows of the weight
+  CUtensorMap y;    // bf16 output, box 32 columns x 32 rows, 64B swizzle
 };
 
 struct GemmParams {
@@ -89,6 +97,7 @@ struct GemmParams {
   void* Y;
   int out_dtype;
   int epilogue;
+  int tma_store;  // bf16 output through shared memory and TMA stores
   WsHeader* hdr;
 };
 
@@ -105,13 +114,18 @@ __device__ __forceinline__ uint32_t idesc_for(int kind, int BM, int BN) {
   }
 }
 
-// tanh-form GELU; tanh(u) = 1 - 2 / (exp(2u) + 1) with |u| clamped at 15 (tanh(15) rounds to 1).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// tanh-form GELU, 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), with the SFU's tanh
+// approximation (relative error about 2^-11, below the 2^-9 rounding of the bf16 output).
 __device__ __forceinline__ float gelu_tanh(float v) {
-  const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);
-  const float uc = fminf(fmaxf(u, -15.0f), 15.0f);
-  const float e = __expf(2.0f * uc);
-  const float t = 1.0f - __fdividef(2.0f, e + 1.0f);
-  return 0.5f * v * (1.0f + t);
+  const float u = v * fmaf(0.7978845608028654f * 0.044715f, v * v, 0.7978845608028654f);
+  const float h = 0.5f * v;
+  return fmaf(h, tanh_approx(u), h);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -133,26 +147,10 @@ __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int
   *nt = r / gm;
 }
 
-// Epilogue of 32 accumulator columns [n, n + 32) of row m: dequant scale, bias, GELU, store.
-__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int kind, int m, int n, float sxb, float alpha,
-                                               const uint32_t (&r)[32]) {
-  if (p.out_dtype == SB_OUT_RAW) {
-    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(p.Y) + (int64_t)m * p.N + n);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-    return;
-  }
-  float y[32];
-  if (kind == KIND_I8) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__int2float_rn((int)r[i]), __fmul_rn(sxb, __ldg(p.sB8 + n + i)));
-  } else if (kind == KIND_FP4) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]);
-  }
+// Epilogue arithmetic of 32 accumulator columns [n, n + 32) of one row: dequant scale and bias
+// in one FMA, optional GELU.
+__device__ __forceinline__ void epilogue_math(const GemmParams& p, int kind, int n, float sxb, float alpha,
+                                              const uint32_t (&r)[32], float (&y)[32]) {
   if (p.bias) {
     const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
 #pragma unroll
@@ -161,13 +159,46 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int kind, in
       float bv[8];
       unpack8(u, bv);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) y[8 * i + j] = __fadd_rn(y[8 * i + j], bv[j]);
+      for (int j = 0; j < 8; ++j) y[8 * i + j] = bv[j];
     }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = 0.0f;
+  }
+  if (kind == KIND_I8) {
+    const float4* sp = reinterpret_cast<const float4*>(p.sB8 + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 sc = __ldg(sp + i);
+      y[4 * i + 0] = fmaf(__int2float_rn((int)r[4 * i + 0]), sxb * sc.x, y[4 * i + 0]);
+      y[4 * i + 1] = fmaf(__int2float_rn((int)r[4 * i + 1]), sxb * sc.y, y[4 * i + 1]);
+      y[4 * i + 2] = fmaf(__int2float_rn((int)r[4 * i + 2]), sxb * sc.z, y[4 * i + 2]);
+      y[4 * i + 3] = fmaf(__int2float_rn((int)r[4 * i + 3]), sxb * sc.w, y[4 * i + 3]);
+    }
+  } else if (kind == KIND_FP4) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = fmaf(__uint_as_float(r[i]), alpha, y[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]) + y[i];
   }
   if (p.epilogue == SB_EPI_GELU_TANH) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) y[i] = gelu_tanh(y[i]);
   }
+}
+
+// Direct global stores of one row's 32 columns (FP32 / raw outputs, or bf16 without TMA).
+__device__ __forceinline__ void epilogue_store_direct(const GemmParams& p, int kind, int m, int n, float sxb,
+                                                      float alpha, const uint32_t (&r)[32]) {
+  if (p.out_dtype == SB_OUT_RAW) {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(p.Y) + (int64_t)m * p.N + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+    return;
+  }
+  float y[32];
+  epilogue_math(p, kind, n, sxb, alpha, r, y);
   if (p.out_dtype == SB_OUT_F32) {
     float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.Y) + (int64_t)m * p.N + n);
 #pragma unroll
@@ -179,6 +210,18 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int kind, in
       dst[i] = make_uint4(pack_bf16(y[8 * i], y[8 * i + 1]), pack_bf16(y[8 * i + 2], y[8 * i + 3]),
                           pack_bf16(y[8 * i + 4], y[8 * i + 5]), pack_bf16(y[8 * i + 6], y[8 * i + 7]));
   }
+}
+
+// bf16 row chunk into a 32 x 32 staging box (row = lane, 64 bytes): 16-byte granule g of row r
+// sits at granule g ^ ((r >> 1) & 3), the TMA 64B swizzle, so the 32 lanes' writes hit distinct
+// banks in groups of eight.
+__device__ __forceinline__ void stage_bf16_row(uint32_t box, int lane, const float (&y)[32]) {
+  const uint32_t row = box + 64u * (uint32_t)lane;
+  const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    st_shared_v4(row + 16u * ((uint32_t)g ^ sw), pack_bf16(y[8 * g], y[8 * g + 1]), pack_bf16(y[8 * g + 2], y[8 * g + 3]),
+                 pack_bf16(y[8 * g + 4], y[8 * g + 5]), pack_bf16(y[8 * g + 6], y[8 * g + 7]));
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -444,6 +487,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int nch = BN / 64;                   // 32-column chunks per warp: 2 or 4
     const uint32_t tempty_leader = cluster_addr(&tempty[0], 0);
     const float alpha = fp4 ? __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB) : 1.0f;
+    const uint32_t out_box0 = smem_u32(smem + kOutOff) + (uint32_t)(2 * (warp - kEpiWarp0) * kOutBox);
+    uint32_t oc = 0;  // staged chunks of this warp (selects one of its two boxes)
     int it = 0;
     for (int tile = unit; tile < tiles; tile += nunits, ++it) {
       int mt, nt;
@@ -468,15 +513,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * b);  // the leader waits for both CTAs
-      if (m < M) {
-        const float sxb = (kind == KIND_I8) ? __fmul_rn(p.sA8[m], p.invB) : 0.0f;
+      const float sxb = (kind == KIND_I8 && m < M) ? __fmul_rn(p.sA8[m], p.invB) : 0.0f;
+      if (p.tma_store) {
+        // bf16: each 32-row x 32-column chunk goes through a staging box and one TMA store
+        // (rows past M are clipped by the store)
+        const int m_warp = mt * 256 + row_off + 32 * q;
+        if (m_warp < M) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int n = n0 + 32 * c;
+            if (c < nch && n < N) {
+              float y[32];
+              epilogue_math(p, kind, n, sxb, alpha, r[c], y);
+              const uint32_t box = out_box0 + (oc & 1u) * (uint32_t)kOutBox;
+              if (lane == 0) bulk_wait_read<1>();  // the store issued from this box before has read it
+              __syncwarp();
+              stage_bf16_row(box, lane, y);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tm.y, box, n, m_warp);
+                bulk_commit();
+              }
+              ++oc;
+            }
+          }
+        }
+      } else if (m < M) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int n = n0 + 32 * c;
-          if (c < nch && n < N) epilogue_chunk(p, kind, m, n, sxb, alpha, r[c]);
+          if (c < nch && n < N) epilogue_store_direct(p, kind, m, n, sxb, alpha, r[c]);
         }
       }
     }
+    if (lane == 0) bulk_wait_all();  // staged outputs are read and written before the CTA exits
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -585,6 +657,17 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   p.out_dtype = L.out_dtype;
   p.epilogue = L.epilogue;
   p.hdr = reinterpret_cast<WsHeader*>(L.hdr);
+  // bf16 output through TMA stores when the output satisfies their alignment (else direct stores)
+  if (L.out_dtype == SB_OUT_BF16 && (reinterpret_cast<uintptr_t>(L.Y) & 15) == 0) {
+    auto fn = encode_fn();
+    cuuint64_t dims[2] = {(cuuint64_t)L.N, (cuuint64_t)L.M};
+    cuuint64_t strides[1] = {(cuuint64_t)L.N * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    p.tma_store = fn && fn(&tm.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L.Y, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   const uint64_t M = (uint64_t)L.M, N = (uint64_t)L.N, K = (uint64_t)L.K;
   const uint32_t half = (uint32_t)p.BN / 2;  // B rows each CTA of the pair loads
   if (L.A4 && L.B4 && L.sfA4 && L.sfB4 && L.gA4 && L.gB4) {
