@@ -68,9 +68,13 @@ constexpr int kBarBytes = 1024;
 constexpr int kOutOff = kStageArea + kBarBytes;
 constexpr int kOutBox = 2048;
 constexpr int kOutBytes = 8 * 2 * kOutBox;
+constexpr int kStoreLane = 31;  // epilogue lane that issues a warp's TMA stores
 constexpr int kSmemBytes = kOutOff + kOutBytes + 1024;  // + alignment of the dynamic base to 1 KB
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kStagesF * kStageBytesF <= kStageArea, "NVFP4 stages exceed the stage area");
+// NVFP4 leaves the end of the stage area free: each epilogue warp's 128-column bias slice (bf16).
+constexpr int kBiasOffF = kStagesF * kStageBytesF;
+static_assert(kBiasOffF + 8 * 256 <= kStageArea, "NVFP4 bias slices");
 static_assert(kOffSFB + 2 * 2048 <= kStageBytesF, "NVFP4 stage layout");
 
 enum { KIND_FP4 = 0, KIND_I8 = 1, KIND_BF16 = 2 };
@@ -85,7 +89,7 @@ struct TMaps {
 
 struct GemmParams {
   int M, N, K;
-  int BN;
+  int bn[3];  // tile width per precision: 256, 192 (NVFP4) or 128
   float invB;
   const int32_t* prec;
   int have[3];
@@ -147,81 +151,219 @@ __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int
   *nt = r / gm;
 }
 
-// Epilogue arithmetic of 32 accumulator columns [n, n + 32) of one row: dequant scale and bias
-// in one FMA, optional GELU.
-__device__ __forceinline__ void epilogue_math(const GemmParams& p, int kind, int n, float sxb, float alpha,
-                                              const uint32_t (&r)[32], float (&y)[32]) {
+// Per-column epilogue operands of a 32-column chunk: bias (bf16) and, for INT8, the weight's
+// per-output-channel scale. They are loaded a chunk ahead of their use (the shared-memory stages
+// leave little L1, so they come from L2).
+template <int KIND>
+struct ColOps {
+  uint4 b[4];
+  float4 s[KIND == KIND_I8 ? 8 : 1];
+};
+
+template <int KIND>
+__device__ __forceinline__ void load_colops(const GemmParams& p, int n, ColOps<KIND>& o) {
   if (p.bias) {
     const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 u = __ldg(bp + i);
-      float bv[8];
-      unpack8(u, bv);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) y[8 * i + j] = bv[j];
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = 0.0f;
+    for (int i = 0; i < 4; ++i) o.b[i] = __ldg(bp + i);
   }
-  if (kind == KIND_I8) {
+  if constexpr (KIND == KIND_I8) {
     const float4* sp = reinterpret_cast<const float4*>(p.sB8 + n);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 sc = __ldg(sp + i);
-      y[4 * i + 0] = fmaf(__int2float_rn((int)r[4 * i + 0]), sxb * sc.x, y[4 * i + 0]);
-      y[4 * i + 1] = fmaf(__int2float_rn((int)r[4 * i + 1]), sxb * sc.y, y[4 * i + 1]);
-      y[4 * i + 2] = fmaf(__int2float_rn((int)r[4 * i + 2]), sxb * sc.z, y[4 * i + 2]);
-      y[4 * i + 3] = fmaf(__int2float_rn((int)r[4 * i + 3]), sxb * sc.w, y[4 * i + 3]);
-    }
-  } else if (kind == KIND_FP4) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = fmaf(__uint_as_float(r[i]), alpha, y[i]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(r[i]) + y[i];
+    for (int i = 0; i < 8; ++i) o.s[i] = __ldg(sp + i);
   }
-  if (p.epilogue == SB_EPI_GELU_TANH) {
+}
+
+// Epilogue arithmetic of 32 accumulator columns of one row, in place: the accumulator words become
+// the FP32 outputs. Dequant scale and bias are one FMA, then the optional GELU.
+template <int KIND>
+__device__ __forceinline__ void epilogue_math(const GemmParams& p, const ColOps<KIND>& o, float sxb, float alpha,
+                                              uint32_t (&r)[32]) {
+  const bool has_bias = p.bias != nullptr, gelu = p.epilogue == SB_EPI_GELU_TANH;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = gelu_tanh(y[i]);
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t w = (i & 7) < 2 ? o.b[i >> 3].x : (i & 7) < 4 ? o.b[i >> 3].y : (i & 7) < 6 ? o.b[i >> 3].z : o.b[i >> 3].w;
+    const float bias = has_bias ? __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16)) : 0.0f;
+    float y;
+    if constexpr (KIND == KIND_I8) {
+      const float4 sc = o.s[i >> 2];
+      const float c = (i & 3) == 0 ? sc.x : (i & 3) == 1 ? sc.y : (i & 3) == 2 ? sc.z : sc.w;
+      y = fmaf(__int2float_rn((int)r[i]), sxb * c, bias);
+    } else if constexpr (KIND == KIND_FP4) {
+      y = fmaf(__uint_as_float(r[i]), alpha, bias);
+    } else {
+      y = __uint_as_float(r[i]) + bias;
+    }
+    if (gelu) y = gelu_tanh(y);
+    r[i] = __float_as_uint(y);
   }
 }
 
 // Direct global stores of one row's 32 columns (FP32 / raw outputs, or bf16 without TMA).
-__device__ __forceinline__ void epilogue_store_direct(const GemmParams& p, int kind, int m, int n, float sxb,
-                                                      float alpha, const uint32_t (&r)[32]) {
+template <int KIND>
+__device__ __forceinline__ void store_direct(const GemmParams& p, int m, int n, float sxb, float alpha,
+                                             uint32_t (&r)[32]) {
   if (p.out_dtype == SB_OUT_RAW) {
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(p.Y) + (int64_t)m * p.N + n);
 #pragma unroll
     for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
     return;
   }
-  float y[32];
-  epilogue_math(p, kind, n, sxb, alpha, r, y);
+  ColOps<KIND> o;
+  load_colops<KIND>(p, n, o);
+  epilogue_math<KIND>(p, o, sxb, alpha, r);
   if (p.out_dtype == SB_OUT_F32) {
-    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.Y) + (int64_t)m * p.N + n);
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.Y) + (int64_t)m * p.N + n);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+    for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
   } else {
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.Y) + (int64_t)m * p.N + n);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      dst[i] = make_uint4(pack_bf16(y[8 * i], y[8 * i + 1]), pack_bf16(y[8 * i + 2], y[8 * i + 3]),
-                          pack_bf16(y[8 * i + 4], y[8 * i + 5]), pack_bf16(y[8 * i + 6], y[8 * i + 7]));
+      dst[i] = make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                          pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                          pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                          pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
   }
 }
 
 // bf16 row chunk into a 32 x 32 staging box (row = lane, 64 bytes): 16-byte granule g of row r
 // sits at granule g ^ ((r >> 1) & 3), the TMA 64B swizzle, so the 32 lanes' writes hit distinct
 // banks in groups of eight.
-__device__ __forceinline__ void stage_bf16_row(uint32_t box, int lane, const float (&y)[32]) {
+__device__ __forceinline__ void stage_bf16_row(uint32_t box, int lane, const uint32_t (&y)[32]) {
   const uint32_t row = box + 64u * (uint32_t)lane;
   const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
 #pragma unroll
-  for (int g = 0; g < 4; ++g)
-    st_shared_v4(row + 16u * ((uint32_t)g ^ sw), pack_bf16(y[8 * g], y[8 * g + 1]), pack_bf16(y[8 * g + 2], y[8 * g + 3]),
-                 pack_bf16(y[8 * g + 4], y[8 * g + 5]), pack_bf16(y[8 * g + 6], y[8 * g + 7]));
+  for (int g = 0; g < 4; ++g) {
+    const float* v = reinterpret_cast<const float*>(&y[8 * g]);
+    st_shared_v4(row + 16u * ((uint32_t)g ^ sw), pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                 pack_bf16(v[6], v[7]));
+  }
+}
+
+// What the epilogue warps of one CTA share.
+struct EpiCtx {
+  uint64_t* tfull;
+  uint32_t tempty_leader;  // shared::cluster address of the leader's tempty[0]
+  volatile int* abort;
+  uint32_t tmem;
+  int unit, tiles, nunits, m_tiles, n_tiles, nacc, BN, M, N, row_off, q, half, lane;
+  uint32_t out_box;  // this warp's two staging boxes
+  uint32_t bias_s;   // NVFP4: this warp's bias slice in shared memory
+  float alpha;
+};
+
+// One 32 x 32 bf16 chunk (a row per lane) through a staging box and one TMA store; rows past M
+// are clipped by the store. Lane kStoreLane issues the stores and owns their bulk groups, so lane
+// 0's release-arrive on the accumulator barrier never waits for them.
+__device__ __forceinline__ void store_chunk_tma(const CUtensorMap* ty, const EpiCtx& e, const uint32_t (&r)[32],
+                                                int n, int m_warp, uint32_t& oc) {
+  const uint32_t box = e.out_box + (oc & 1u) * (uint32_t)kOutBox;
+  if (e.lane == kStoreLane) bulk_wait_read<1>();  // the store issued from this box before has read it
+  __syncwarp();
+  stage_bf16_row(box, e.lane, r);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (e.lane == kStoreLane) {
+    tma_store_2d(ty, box, n, m_warp);
+    bulk_commit();
+  }
+  ++oc;
+}
+
+// The epilogue of every tile of this CTA. DRAIN_ALL (one accumulator buffer): the warp's columns
+// are moved to registers and the buffer released before any arithmetic, so the next tile's MMAs
+// can start. Otherwise (two buffers) 32-column chunks are loaded as they are processed and the
+// buffer is released after the last load.
+template <int KIND, bool DRAIN_ALL>
+__device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtensorMap* ty, const EpiCtx& e) {
+  const int nch = e.BN / 64;  // 32-column chunks per warp: 2 or 4
+  const int row = 32 * e.q + e.lane;
+  uint32_t oc = 0;
+  int it = 0;
+  for (int tile = e.unit; tile < e.tiles; tile += e.nunits, ++it) {
+    int mt, nt;
+    tile_coords(tile, e.m_tiles, e.n_tiles, &mt, &nt);
+    const int m = mt * 256 + e.row_off + row;
+    const int m_warp = mt * 256 + e.row_off + 32 * e.q;
+    const int n0 = nt * e.BN + e.half * (e.BN / 2);
+    const int b = it % e.nacc;
+    const uint32_t tph = (uint32_t)((it / e.nacc) & 1);
+    const bool tma = p.tma_store && m_warp < e.M;
+    // operands that do not depend on the accumulator are loaded before waiting for it
+    const float sxb = (KIND == KIND_I8 && m < e.M) ? __fmul_rn(__ldg(p.sA8 + m), p.invB) : 0.0f;
+    ColOps<KIND> ops;
+    if constexpr (DRAIN_ALL) {
+      // the warp's bias slice (128 columns, 256 bytes) goes to shared memory asynchronously
+      if (tma && p.bias && e.lane < 16) cp_async16(e.bias_s + 16u * (uint32_t)e.lane, p.bias + n0 + 8 * e.lane);
+      cp_async_commit();
+    } else {
+      if (tma) load_colops<KIND>(p, n0, ops);
+    }
+    if (!mbar_wait_bounded(&e.tfull[b], tph, e.abort, kWaitNs)) {
+      set_error(p.hdr, SB_ETIMEOUT);
+      *e.abort = 1;
+      break;
+    }
+    tc_fence_after();
+    const uint32_t tcol = e.tmem + ((uint32_t)(32 * e.q) << 16) + (uint32_t)(b * e.BN + e.half * (e.BN / 2));
+    if constexpr (DRAIN_ALL) {
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < nch) tmem_ld32(tcol + 32u * c, r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (e.lane == 0) mbar_arrive_cluster(e.tempty_leader + 8u * b);  // the leader waits for both CTAs
+      cp_async_wait_all();
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int n = n0 + 32 * c;
+        if (c < nch && n < e.N) {
+          if (tma) {
+            if (p.bias) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) ops.b[i] = ld_shared_v4(e.bias_s + 64u * c + 16u * i);
+            }
+            epilogue_math<KIND>(p, ops, sxb, e.alpha, r[c]);
+            store_chunk_tma(ty, e, r[c], n, m_warp, oc);
+          } else if (m < e.M) {
+            store_direct<KIND>(p, m, n, sxb, e.alpha, r[c]);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c < nch) {
+          uint32_t r[32];
+          tmem_ld32(tcol + 32u * c, r);
+          tmem_ld_wait();
+          if (c == nch - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (e.lane == 0) mbar_arrive_cluster(e.tempty_leader + 8u * b);
+          }
+          const int n = n0 + 32 * c;
+          if (n < e.N) {
+            if (tma) {
+              ColOps<KIND> next;
+              if (c + 1 < nch && n + 32 < e.N) load_colops<KIND>(p, n + 32, next);
+              epilogue_math<KIND>(p, ops, sxb, e.alpha, r);
+              store_chunk_tma(ty, e, r, n, m_warp, oc);
+              ops = next;
+            } else if (m < e.M) {
+              store_direct<KIND>(p, m, n, sxb, e.alpha, r);
+            }
+          }
+        }
+      }
+    }
+  }
+  if (e.lane == kStoreLane) bulk_wait_all();  // staged outputs are read and written before the CTA exits
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -239,7 +381,7 @@ struct Issuer {
   volatile int* abort;
   uint32_t smem;      // shared address of stage 0
   uint32_t stage16;   // stage size in 16-byte units
-  int stages, nkb, tail_nk, tiles, unit, nunits, BN, nacc;
+  int stages, nkb, tail_nk, tiles, unit, nunits, BN, nacc, m_tiles, n_tiles;
   uint32_t tmem, sfa, sfb, idesc;  // TMEM base, scale columns (absolute), instruction descriptor
 };
 
@@ -255,10 +397,12 @@ __device__ __forceinline__ void mma_one(uint32_t d, uint64_t ad, uint64_t bd, ui
 }
 
 // One K-block: NVFP4 scale copies (SFA atom j -> 4 columns at 4j; SFB atom j of column tile t ->
-// 4 columns at 8j + 4t), then the nk MMAs of 32 bytes of K each.
+// 4 columns at 8j + 4t), then the nk MMAs of 32 bytes of K each. The MMA reads the scales of
+// output column n from column (n / 32) of its SFB columns, so a tile that starts 64 columns into
+// a 128-column scale tile (192-wide tiles) passes its SFB address advanced by `shift` = 2.
 template <int KIND, int SFT>
 __device__ __forceinline__ void issue_kblock(const Issuer& c, uint32_t d, uint64_t ad, uint64_t bd, uint64_t fa,
-                                             uint64_t fb, int nk, bool first) {
+                                             uint64_t fb, int nk, bool first, uint32_t shift) {
   if (nk == 4) {
     if constexpr (KIND == KIND_FP4) {
 #pragma unroll
@@ -270,7 +414,8 @@ __device__ __forceinline__ void issue_kblock(const Issuer& c, uint32_t d, uint64
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      mma_one<KIND>(d, ad + 2u * j, bd + 2u * j, c.idesc, c.sfa + 4u * j, c.sfb + 8u * j, (first && j == 0) ? 0u : 1u);
+      mma_one<KIND>(d, ad + 2u * j, bd + 2u * j, c.idesc, c.sfa + 4u * j, c.sfb + 8u * j + shift,
+                    (first && j == 0) ? 0u : 1u);
   } else {
     if constexpr (KIND == KIND_FP4) {
       for (int j = 0; j < nk; ++j) {
@@ -280,7 +425,8 @@ __device__ __forceinline__ void issue_kblock(const Issuer& c, uint32_t d, uint64
       }
     }
     for (int j = 0; j < nk; ++j)
-      mma_one<KIND>(d, ad + 2u * j, bd + 2u * j, c.idesc, c.sfa + 4u * j, c.sfb + 8u * j, (first && j == 0) ? 0u : 1u);
+      mma_one<KIND>(d, ad + 2u * j, bd + 2u * j, c.idesc, c.sfa + 4u * j, c.sfb + 8u * j + shift,
+                    (first && j == 0) ? 0u : 1u);
   }
 }
 
@@ -298,13 +444,19 @@ __device__ __noinline__ bool issue_all(const Issuer c) {
     if (!mbar_wait_bounded(&c.tempty[b], tph ^ 1u, c.abort, kWaitNs)) return false;
     tc_fence_after();
     const uint32_t d = c.tmem + (uint32_t)(b * c.BN);
+    uint32_t shift = 0;
+    if (KIND == KIND_FP4) {
+      int mt, nt;
+      tile_coords(tile, c.m_tiles, c.n_tiles, &mt, &nt);
+      shift = (uint32_t)(((nt * c.BN) & 127) >> 5);
+    }
     for (int kb = 0; kb < c.nkb; ++kb) {
       if (!mbar_wait_bounded(&c.full[s], ph, c.abort, kWaitNs)) return false;
       tc_fence_after();
       const uint32_t so = (uint32_t)s * c.stage16;
       const uint64_t ad = dsw + so;
       issue_kblock<KIND, SFT>(c, d, ad, ad + (kOffB >> 4), dsf + so + (kOffSFA >> 4), dsf + so + (kOffSFB >> 4),
-                              (kb == c.nkb - 1) ? c.tail_nk : 4, kb == 0);
+                              (kb == c.nkb - 1) ? c.tail_nk : 4, kb == 0, shift);
       mma_commit_pair(&c.empty[s], (uint16_t)3);  // frees the stage in both CTAs
       if (++s == c.stages) {
         s = 0;
@@ -338,7 +490,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = (rank == 0);
   const bool fp4 = (kind == KIND_FP4);
-  const int M = p.M, N = p.N, K = p.K, BN = p.BN;
+  const int M = p.M, N = p.N, K = p.K, BN = p.bn[kind];
   const int kb_elems = fp4 ? 256 : (kind == KIND_I8 ? 128 : 64);
   const int mma_k = kb_elems >> 2;
   const int nkb = (K + kb_elems - 1) / kb_elems;
@@ -351,7 +503,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int stages = fp4 ? kStagesF : kStagesQ;
   const int stage_bytes = fp4 ? kStageBytesF : kStageBytesQ;
   const int row_off = 128 * (int)rank;  // this CTA's rows inside the 256-row tile
-  const int sf_tiles = BN / 128;        // NVFP4: 128-column scale tiles of B per output tile
+  const int sf_tiles = (BN + 127) / 128;  // NVFP4: 128-column scale tiles of B per output tile
   const int nacc = (2 * BN + (fp4 ? (int)kSfCols : 0) <= (int)kTmemCols) ? 2 : 1;
 
   if (threadIdx.x == 0) {
@@ -456,6 +608,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         c.unit = unit;
         c.nunits = nunits;
         c.BN = BN;
+        c.m_tiles = m_tiles;
+        c.n_tiles = n_tiles;
         c.nacc = nacc;
         c.tmem = tmem_base;
         c.sfa = tmem_base + sfa_col;
@@ -481,74 +635,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     setmaxnreg_inc<kRegsEpi>();
     // ------------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;                    // TMEM lane quadrant this warp may access
-    const int half = (warp - kEpiWarp0) >> 2;  // two warps per quadrant split the tile's columns
-    const int row = 32 * q + lane;
-    const int nch = BN / 64;                   // 32-column chunks per warp: 2 or 4
-    const uint32_t tempty_leader = cluster_addr(&tempty[0], 0);
-    const float alpha = fp4 ? __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB) : 1.0f;
-    const uint32_t out_box0 = smem_u32(smem + kOutOff) + (uint32_t)(2 * (warp - kEpiWarp0) * kOutBox);
-    uint32_t oc = 0;  // staged chunks of this warp (selects one of its two boxes)
-    int it = 0;
-    for (int tile = unit; tile < tiles; tile += nunits, ++it) {
-      int mt, nt;
-      tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
-      const int m = mt * 256 + row_off + row;
-      const int n0 = nt * BN + half * (BN / 2);
-      const int b = it % nacc;
-      const uint32_t tph = (uint32_t)((it / nacc) & 1);
-      if (!mbar_wait_bounded(&tfull[b], tph, abort_flag, kWaitNs)) {
-        set_error(p.hdr, SB_ETIMEOUT);
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      // drain this warp's columns into registers, then hand the buffer back to the MMA
-      uint32_t r[4][32];
-      const uint32_t tcol = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN + half * (BN / 2));
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < nch) tmem_ld32(tcol + 32u * c, r[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * b);  // the leader waits for both CTAs
-      const float sxb = (kind == KIND_I8 && m < M) ? __fmul_rn(p.sA8[m], p.invB) : 0.0f;
-      if (p.tma_store) {
-        // bf16: each 32-row x 32-column chunk goes through a staging box and one TMA store
-        // (rows past M are clipped by the store)
-        const int m_warp = mt * 256 + row_off + 32 * q;
-        if (m_warp < M) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int n = n0 + 32 * c;
-            if (c < nch && n < N) {
-              float y[32];
-              epilogue_math(p, kind, n, sxb, alpha, r[c], y);
-              const uint32_t box = out_box0 + (oc & 1u) * (uint32_t)kOutBox;
-              if (lane == 0) bulk_wait_read<1>();  // the store issued from this box before has read it
-              __syncwarp();
-              stage_bf16_row(box, lane, y);
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&tm.y, box, n, m_warp);
-                bulk_commit();
-              }
-              ++oc;
-            }
-          }
-        }
-      } else if (m < M) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int n = n0 + 32 * c;
-          if (c < nch && n < N) epilogue_store_direct(p, kind, m, n, sxb, alpha, r[c]);
-        }
-      }
-    }
-    if (lane == 0) bulk_wait_all();  // staged outputs are read and written before the CTA exits
-    __syncwarp();
+    EpiCtx e;
+    e.tfull = tfull;
+    e.tempty_leader = cluster_addr(&tempty[0], 0);
+    e.abort = abort_flag;
+    e.tmem = tmem_base;
+    e.unit = unit;
+    e.tiles = tiles;
+    e.nunits = nunits;
+    e.m_tiles = m_tiles;
+    e.n_tiles = n_tiles;
+    e.nacc = nacc;
+    e.BN = BN;
+    e.M = M;
+    e.N = N;
+    e.row_off = row_off;
+    e.q = warp & 3;                    // TMEM lane quadrant this warp may access
+    e.half = (warp - kEpiWarp0) >> 2;  // two warps per quadrant split the tile's columns
+    e.lane = lane;
+    e.out_box = smem_u32(smem + kOutOff) + (uint32_t)(2 * (warp - kEpiWarp0) * kOutBox);
+    e.bias_s = smem_u32(smem + kBiasOffF) + 256u * (uint32_t)(warp - kEpiWarp0);
+    e.alpha = fp4 ? __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB) : 1.0f;
+    if (fp4)
+      epilogue_loop<KIND_FP4, true>(p, &tm.y, e);
+    else if (kind == KIND_I8)
+      epilogue_loop<KIND_I8, false>(p, &tm.y, e);
+    else
+      epilogue_loop<KIND_BF16, false>(p, &tm.y, e);
   }
   tc_fence_before();
   __syncthreads();
@@ -645,7 +758,13 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   p.M = (int)L.M;
   p.N = (int)L.N;
   p.K = (int)L.K;
-  p.BN = (L.N % 256 == 0) ? 256 : 128;
+  // Tile width per precision: 256, or 128 when N is not a multiple of 256; the kernel also takes
+  // 192-wide NVFP4 tiles (two accumulators next to the scale columns), which measured slower than
+  // one 256-wide accumulator on the FFN shapes.
+  const int bn_q = (L.N % 256 == 0) ? 256 : 128;
+  const int bn_f = bn_q;
+  p.bn[KIND_FP4] = bn_f;
+  p.bn[KIND_I8] = p.bn[KIND_BF16] = bn_q;
   p.invB = 1.0f / (float)L.B;
   p.prec = L.prec;
   p.sA8 = L.sA8;
@@ -669,10 +788,10 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   }
   const uint64_t M = (uint64_t)L.M, N = (uint64_t)L.N, K = (uint64_t)L.K;
-  const uint32_t half = (uint32_t)p.BN / 2;  // B rows each CTA of the pair loads
+  const uint32_t half = (uint32_t)bn_q / 2;  // B rows each CTA of the pair loads (INT8 / BF16)
   if (L.A4 && L.B4 && L.sfA4 && L.sfB4 && L.gA4 && L.gB4) {
     if (!make_map(&tm.a[KIND_FP4], L.A4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128) ||
-        !make_map(&tm.b[KIND_FP4], L.B4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, half) ||
+        !make_map(&tm.b[KIND_FP4], L.B4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, (uint32_t)bn_f / 2) ||
         !make_sf_map(&tm.sfa, L.sfA4, K, M) || !make_sf_map(&tm.sfb, L.sfB4, K, N)) {
       *why = "cuTensorMapEncodeTiled failed (NVFP4 operands)";
       return cudaErrorInvalidValue;
@@ -696,7 +815,7 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
     p.have[KIND_BF16] = 1;
   }
   // one cluster of two CTAs per 256 x BN tile, at most one CTA per SM
-  const int64_t want = 2 * ceil_div(L.M, 256) * ceil_div(L.N, p.BN);
+  const int64_t want = 2 * ceil_div(L.M, 256) * ceil_div(L.N, bn_q < bn_f ? bn_q : bn_f);
   const int sms = device_sms() & ~1;
   const unsigned grid = (unsigned)(want < sms ? want : sms);
   k_gemm<<<grid, kThreads, kSmemBytes, s>>>(tm, p);
