@@ -37,6 +37,7 @@
 
 #include "sb_device.cuh"
 #include "sb_kernels.h"
+#include "tmap.h"
 
 namespace sb {
 
@@ -676,19 +677,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // Host side: tensor maps and launch
 // ---------------------------------------------------------------------------------------------
 
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return tmap_encoder(); }
 
 // 2-D row-major map: `inner` elements per row, `outer` rows; box = 128 bytes x box_rows, SW128.
 static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,

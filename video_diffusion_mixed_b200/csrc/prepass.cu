@@ -14,6 +14,7 @@
 //                 E4M3 block scales in the tensor-core layout and the FP32 tensor scale.
 //  k_rotate       rotation only (test hook).
 #include "rows.cuh"
+#include "tmap.h"
 
 namespace sb {
 
@@ -48,12 +49,21 @@ static RowArgs row_args_from(const PrepassLaunch& p) {
   return a;
 }
 
+// TMA maps of a row kernel's tensors; a.tma stays 0 (direct loads) when a row is not a whole
+// number of 128-byte chunks or a map cannot be built.
+static void row_maps(RowArgs& a, RowMaps& mp, const void* X, const void* R) {
+  memset(&mp, 0, sizeof(mp));
+  a.tma = make_row_segment_map(&mp.x, X, a.M, a.K) && (!R || make_row_segment_map(&mp.r, R, a.M, a.K)) ? 1 : 0;
+}
+
 cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s) {
-  const RowArgs a = row_args_from(p);
+  RowArgs a = row_args_from(p);
+  RowMaps mp;
+  row_maps(a, mp, p.X, p.R);
   const int sms = sm_count();
   if (p.mode == SB_PREPASS_STATS && !p.force_int8)
-    return p.R ? launch_rows_t<OP_STATS, true>(a, s, sms) : launch_rows_t<OP_STATS, false>(a, s, sms);
-  return p.R ? launch_rows_t<OP_PREPASS, true>(a, s, sms) : launch_rows_t<OP_PREPASS, false>(a, s, sms);
+    return p.R ? launch_rows_t<OP_STATS, true>(a, mp, s, sms) : launch_rows_t<OP_STATS, false>(a, mp, s, sms);
+  return p.R ? launch_rows_t<OP_PREPASS, true>(a, mp, s, sms) : launch_rows_t<OP_PREPASS, false>(a, mp, s, sms);
 }
 
 cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s) {
@@ -68,7 +78,9 @@ cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s) {
   a.st = p.st;
   a.groups = reinterpret_cast<GroupSlot*>(p.groups);
   a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
-  return launch_rows_t<OP_TDC, true>(a, s, sm_count());
+  RowMaps mp;
+  row_maps(a, mp, p.Y, p.Cache);
+  return launch_rows_t<OP_TDC, true>(a, mp, s, sm_count());
 }
 
 // ---------------------------------------------------------------------------------------------

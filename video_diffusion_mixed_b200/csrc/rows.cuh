@@ -10,7 +10,15 @@
 // Reductions follow the canonical pairwise tree of the oracle: 32 terms inside a lane, lanes
 // 1..16 apart inside a segment, then a tree over the (zero-padded) segments of the row; rows meet
 // in FP64 over aligned groups of kG rows (warp 0 of the CTA), groups in FP64 in the last CTA.
+//
+// Loads: every warp keeps a ring of D row slots in shared memory, filled by TMA a few rows ahead of
+// the row it processes (one 2 KB box per 1024-element segment and tensor, 128B swizzle), so that
+// enough bytes are in flight to cover the memory latency with only 8 warps per SM. Each lane then
+// reads its 64 bytes from the slot without bank conflicts. Rows whose length is not a multiple of
+// 64 elements (possible for the TDC record) use direct global loads instead.
 #pragma once
+
+#include <cudaTypedefs.h>
 
 #include <cfloat>
 
@@ -42,6 +50,29 @@ struct RowArgs {
   GroupSlot* groups;
   WsHeader* hdr;
   sb_stats* stats;
+  int tma;  // rows arrive through the TMA rings (the maps below are valid)
+};
+
+// TMA maps of the row tensors (make_row_segment_map): x = X (TDC: the new output), r = x_ref
+// (TDC: the cache).
+struct RowMaps {
+  CUtensorMap x;
+  CUtensorMap r;
+};
+
+constexpr uint64_t kRowWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+constexpr uint64_t kRowDrainNs = 20000000ull;
+
+// Ring geometry of one k_rows instantiation: NT tensors per row, SPW 2 KB segments per tensor and
+// warp, D slots per warp (2..4, about 200 KB per CTA at most).
+template <int SPW, int OP, bool REF>
+struct RowRing {
+  static constexpr int NT = (OP == OP_TDC || REF) ? 2 : 1;
+  static constexpr int SEG = 2048;
+  static constexpr int SLOT = NT * SPW * SEG;
+  static constexpr int D0 = (200 * 1024) / (kRowWarps * SLOT);
+  static constexpr int D = D0 < 2 ? 2 : (D0 > 4 ? 4 : D0);
+  static constexpr int BYTES = kRowWarps * D * SLOT;
 };
 
 struct Raw32 {
@@ -64,6 +95,16 @@ __device__ __forceinline__ void load_raw(Raw32& r, const __nv_bfloat16* row, int
       r.q[2 * h + 1] = (ok && e + 8 < K) ? ldg_nc_v4(row + e + 8) : make_uint4(0, 0, 0, 0);
     }
   }
+}
+
+// The lane's 64 bytes of a 2 KB segment box written by TMA with 128B swizzle: lane l owns bytes
+// [64 l, 64 l + 64), i.e. granules 4 (l & 1) .. +3 of 128-byte chunk l / 2, stored at granule
+// g ^ (chunk & 7). In each load the 8 lanes of a quarter-warp touch 8 distinct granules.
+__device__ __forceinline__ void read_seg_sw128(Raw32& r, uint32_t seg, int lane) {
+  const uint32_t ch = (uint32_t)lane >> 1, h = (uint32_t)lane & 1u;
+  const uint32_t base = seg + 128u * ch;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) r.q[j] = ld_shared_v4(base + 16u * ((4u * h + (uint32_t)j) ^ (ch & 7u)));
 }
 
 __device__ __forceinline__ void load_raw_coherent(Raw32& r, const __nv_bfloat16* row, int e0, int K, bool ok) {
@@ -254,7 +295,8 @@ __device__ __forceinline__ void team_sync(int team, int T) {
 }
 
 template <int T, int SPW, int OP, bool REF>
-__global__ void __launch_bounds__(256) k_rows(RowArgs a) {
+__global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__ RowMaps mp) {
+  using RG = RowRing<SPW, OP, REF>;
   constexpr int NTEAM = kRowWarps / T;
   constexpr int NSEG = T * SPW;
   constexpr int NSEG2 = pow2_at_least(NSEG);
@@ -267,8 +309,14 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a) {
   __shared__ float s_rowmax[2][kG];
   __shared__ int s_rownf[2][kG];
   __shared__ int s_last;
-  __shared__ double s_fin[kFinChunk];
   __shared__ double s_fwarp[kRowWarps];
+  __shared__ uint64_t s_bar[kRowWarps][4];
+  extern __shared__ uint8_t dsm_raw[];
+  // dynamic shared memory: the rings (1024-byte aligned for the swizzled boxes); the last CTA
+  // reuses it for the final reduction
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~(uintptr_t)1023);
+  double* s_fin = reinterpret_cast<double*>(ring);
+  static_assert(RG::BYTES >= kFinChunk * 8, "final-reduction buffer");
   __shared__ float s_fmax[kRowWarps][2];
   __shared__ int s_fnf[kRowWarps];
 
@@ -289,28 +337,41 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a) {
   const int64_t ngroups = ceil_div(a.M, kG);
 
   // A team walks its rows of the CTA's groups in order: row i = team + NTEAM * j (j < RPT) of
-  // group g = blockIdx.x + n * gridDim.x. The plain pre-pass (no x_ref) prefetches the next row
-  // of the walk while it processes the current one.
+  // group g = blockIdx.x + n * gridDim.x.
   constexpr int RPT = kG / NTEAM;
-  constexpr bool PREFETCH = (OP == OP_PREPASS) && !REF;
-  Raw32 xn[PREFETCH ? SPW : 1];
   auto row_of = [&](int64_t it, int64_t* g, int* i) {
     *g = blockIdx.x + (it / RPT) * (int64_t)gridDim.x;
     *i = team + (int)(it % RPT) * NTEAM;
   };
-  auto load_row = [&](Raw32 (&dst)[PREFETCH ? SPW : 1], int64_t g, int i) {
-    const int64_t m = g * kG + i;
+  // this warp's ring: slot s holds, per tensor t and segment c, the box of segment c*T + wt
+  const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * RG::D * RG::SLOT);
+  const bool use_tma = a.tma != 0;
+  auto issue_row = [&](int64_t it) {  // lane 0
+    int64_t g;
+    int i;
+    row_of(it, &g, &i);
+    if (g >= ngroups) return;
+    const int m = (int)(g * kG + i);  // rows past M read as zero
+    const int slot = (int)(it % RG::D);
+    const uint32_t bar = smem_u32(&s_bar[warp][slot]);
+    mbar_arrive_expect_tx_u32(bar, (uint32_t)RG::SLOT);
 #pragma unroll
-    for (int c = 0; c < (PREFETCH ? SPW : 1); ++c) {
-      const int e0 = (c * T + wt) * 1024 + lane * 32;
-      load_raw(dst[c], a.X + m * K, e0, K, g < ngroups && m < a.M);
+    for (int t = 0; t < RG::NT; ++t) {
+#pragma unroll
+      for (int c = 0; c < SPW; ++c)
+        tma_load_3d(ring_w + (uint32_t)(slot * RG::SLOT + (t * SPW + c) * RG::SEG), t == 0 ? &mp.x : &mp.r, bar, 0,
+                    (c * T + wt) * 16, m);
     }
   };
-  if (PREFETCH) {
-    int64_t g0;
-    int i0;
-    row_of(0, &g0, &i0);
-    load_row(xn, g0, i0);
+  int64_t bad_it = -1;  // last row whose wait gave up (its copy may still be in flight)
+  if (use_tma) {
+    if (lane == 0) {
+#pragma unroll
+      for (int d = 0; d < RG::D; ++d) mbar_init(&s_bar[warp][d], 1);
+      fence_barrier_init();
+      for (int d = 0; d < RG::D; ++d) issue_row(d);
+    }
+    __syncwarp();
   }
 
   for (int64_t it = 0;; ++it) {
@@ -323,19 +384,32 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a) {
     const bool group_end = (it % RPT) == RPT - 1;
     const int64_t m = g * kG + i;
     Raw32 xr[SPW], rr[SPW];
-    if (PREFETCH) {
+    if (use_tma) {
+      // this row's slot: wait for its boxes, copy the lane's part to registers, refill the slot
+      // with the row D steps ahead
+      const int slot = (int)(it % RG::D);
+      if (!mbar_wait_bounded(&s_bar[warp][slot], (uint32_t)((it / RG::D) & 1), nullptr, kRowWaitNs)) {
+        if (lane == 0) set_error(a.hdr, SB_ETIMEOUT);
+        bad_it = it;
+      }
+      const uint32_t sl = ring_w + (uint32_t)(slot * RG::SLOT);
 #pragma unroll
-      for (int c = 0; c < SPW; ++c) xr[c] = xn[(PREFETCH ? c : 0)];
-      int64_t g1;
-      int i1;
-      row_of(it + 1, &g1, &i1);
-      load_row(xn, g1, i1);
+      for (int c = 0; c < SPW; ++c) read_seg_sw128(xr[c], sl + (uint32_t)(c * RG::SEG), lane);
+      if (RG::NT == 2) {
+#pragma unroll
+        for (int c = 0; c < SPW; ++c) read_seg_sw128(rr[c], sl + (uint32_t)((SPW + c) * RG::SEG), lane);
+      }
+      __syncwarp();
+      if (lane == 0) issue_row(it + RG::D);
+      if (OP == OP_TDC && !have_prev) {  // no cached output yet: it reads as zero
+#pragma unroll
+        for (int c = 0; c < SPW; ++c) rr[c].q[0] = rr[c].q[1] = rr[c].q[2] = rr[c].q[3] = make_uint4(0, 0, 0, 0);
+      }
     }
     if (m < a.M) {
       const __nv_bfloat16* xrow = a.X + m * K;
       __nv_bfloat16* rrow = (OP == OP_TDC || REF) ? a.R + m * K : nullptr;
-      // ---- issue every load of this warp's part of the row (already in flight when prefetching)
-      if (!PREFETCH) {
+      if (!use_tma) {
 #pragma unroll
         for (int c = 0; c < SPW; ++c) {
           const int e0 = (c * T + wt) * 1024 + lane * 32;
@@ -512,6 +586,10 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a) {
       }
     }
   }
+  // a copy whose wait gave up may still be in flight: give it a bounded chance to land before the
+  // ring is reused or the CTA exits
+  if (use_tma && bad_it >= 0 && lane == 0)
+    mbar_wait_bounded(&s_bar[warp][bad_it % RG::D], (uint32_t)((bad_it / RG::D) & 1), nullptr, kRowDrainNs);
   // ---- last CTA: tree over the groups (whole CTA, shared memory)
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -608,21 +686,23 @@ inline void pick_row_tiling(int K, int* T, int* SPW) {
 }
 
 template <int OP, bool REF>
-cudaError_t launch_rows_t(const RowArgs& a, cudaStream_t s, int sms) {
+cudaError_t launch_rows_t(const RowArgs& a, const RowMaps& mp, cudaStream_t s, int sms) {
   int T, SPW;
   pick_row_tiling(a.K, &T, &SPW);
   const int64_t ngroups = ceil_div(a.M, kG);
-#define SB_ROWS_CASE(TT, SS)                                                                          \
-  if (T == TT && SPW == SS) {                                                                         \
-    static int occ = 0;                                                                               \
-    if (occ == 0) {                                                                                   \
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_rows<TT, SS, OP, REF>, kRowWarps * 32, 0); \
-      if (occ <= 0) occ = 1;                                                                          \
-    }                                                                                                 \
-    const int64_t cap = (int64_t)sms * occ; /* persistent: one wave of resident CTAs */               \
-    const unsigned grid = (unsigned)(ngroups < cap ? ngroups : cap);                                  \
-    k_rows<TT, SS, OP, REF><<<grid, kRowWarps * 32, 0, s>>>(a);                                       \
-    return cudaGetLastError();                                                                        \
+#define SB_ROWS_CASE(TT, SS)                                                                              \
+  if (T == TT && SPW == SS) {                                                                             \
+    constexpr int dsm = RowRing<SS, OP, REF>::BYTES + 1024;                                               \
+    static int occ = 0;                                                                                   \
+    if (occ == 0) {                                                                                       \
+      cudaFuncSetAttribute(k_rows<TT, SS, OP, REF>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);    \
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_rows<TT, SS, OP, REF>, kRowWarps * 32, dsm); \
+      if (occ <= 0) occ = 1;                                                                              \
+    }                                                                                                     \
+    const int64_t cap = (int64_t)sms * occ; /* persistent: one wave of resident CTAs */                   \
+    const unsigned grid = (unsigned)(ngroups < cap ? ngroups : cap);                                      \
+    k_rows<TT, SS, OP, REF><<<grid, kRowWarps * 32, dsm, s>>>(a, mp);                                     \
+    return cudaGetLastError();                                                                            \
   }
   SB_ROWS_CASE(1, 1)
   SB_ROWS_CASE(1, 2)
