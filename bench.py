@@ -33,14 +33,29 @@ if ROOT not in sys.path:
 
 METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT shapes"
 
-# ncu DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernel, from the capture summarised under profiles/; valid only for the gemm.cu it was taken on.
-TRAFFIC = {}
+# ncu DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the kernels that
+# can be the dominant one, from the 8192-token captures summarised under profiles/ scaled to 17776
+# tokens (every term grows with the token count), for the ffn5b workload at full size only. An
+# entry is valid only for the sources it was measured on (sha over the listed files of csrc/).
+_GEMM_SRC = ("gemm.cu", "sb_device.cuh")
+_ROWS_SRC = ("prepass.cu", "rows.cuh", "sb_device.cuh")
+TRAFFIC = {
+    "gemm_w1_int8": {"bytes": 750.6e6, "files": _GEMM_SRC, "sha": "c7275c8b5a60ac65"},
+    "gemm_w2_int8": {"bytes": 795.5e6, "files": _GEMM_SRC, "sha": "c7275c8b5a60ac65"},
+    "gemm_w1_nvfp4": {"bytes": 496.0e6, "files": _GEMM_SRC, "sha": "c7275c8b5a60ac65"},
+    "gemm_w2_nvfp4": {"bytes": 279.0e6, "files": _GEMM_SRC, "sha": "c7275c8b5a60ac65"},
+    "prepass_h_nvfp4": {"bytes": 974.7e6, "files": _ROWS_SRC, "sha": "25c4aecd182a1187"},  # k_rows + k_nvfp4
+    "prepass_h_int8": {"bytes": 575.2e6, "files": _ROWS_SRC, "sha": "25c4aecd182a1187"},
+}
+TRAFFIC_TOKENS = 17776
 
 
-def file_sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def src_sha(files):
+    h = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(ROOT, "video_diffusion_mixed_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def peaks():
@@ -302,9 +317,9 @@ def run_ours(args):
             rows.append({"kernel": k, "bound": "hbm", "ms": ms, "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / pk["hbm_gbs"]})
     dom = max(rows, key=lambda r: r["ms"])
-    src_sha = file_sha(os.path.join(ROOT, "video_diffusion_mixed_b200", "csrc", "gemm.cu"))
     tr = TRAFFIC.get(dom["kernel"])
-    traffic = tr["bytes"] if (tr and tr.get("src_sha") == src_sha) else None
+    valid = tr is not None and args.workload == "ffn5b" and M == TRAFFIC_TOKENS and src_sha(tr["files"]) == tr["sha"]
+    traffic = int(tr["bytes"]) if valid else None  # bytes per launch
     roofline = {"bound": dom["bound"], "achieved": round(dom["achieved"], 1), "peak": round(dom["peak"], 1),
                 "unit": dom["unit"], "frac": round(dom["frac"], 4), "traffic": traffic, "kernel": dom["kernel"],
                 "peak_src": f"{pk['src']} bf16 {'burst' if burst else 'sustained'} x nominal dtype ratio"
