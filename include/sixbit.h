@@ -228,6 +228,17 @@ sb_status sb_prepass_static(const void* X, const void* X_ref, int64_t M, int64_t
                             const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */, sb_stats* stats,
                             sb_stream stream);
 
+/* Bounded device-side wait, the library's failure-detection primitive (the pages have no
+ * counterpart). Enqueues on `stream` a one-thread kernel that polls the device int32 at `flag`
+ * (acquire loads, ~1 us apart) until it equals `value`. If `limit_ns` nanoseconds of device time
+ * (%globaltimer) pass first, the kernel records SB_ETIMEOUT in `ws` and returns, so the stream and
+ * the context stay usable; sb_check() reports the timeout. The flag must be written by something
+ * that does not need this kernel to finish or to be co-scheduled with it: the host (mapped or
+ * managed memory), a copy or kernel that completes before this launch, or another device -- never
+ * a kernel launched later on the same GPU. flag: 4-byte aligned device pointer (SB_EALIGN);
+ * limit_ns in [1, 1e10] (SB_EINVAL otherwise). */
+sb_status sb_wait_flag(const int32_t* flag, int32_t value, uint64_t limit_ns, void* ws, sb_stream stream);
+
 /* Synchronise `stream`, read and clear the device error word of `ws`. Returns SB_OK,
  * SB_ETIMEOUT, SB_ENONFINITE, SB_EINVAL or SB_ECUDA. */
 sb_status sb_check(void* ws, sb_stream stream);

@@ -58,6 +58,15 @@ def _fake(addr):
     return ctypes.c_void_p(addr)
 
 
+def test_wait_flag_validation_without_gpu(sb):
+    L = sb.lib()
+    assert L.sb_wait_flag(None, 1, 1000, _fake(0x100), None) == sb.SB_EINVAL
+    assert L.sb_wait_flag(_fake(0x1002), 1, 1000, _fake(0x100), None) == sb.SB_EALIGN
+    assert L.sb_wait_flag(_fake(0x1000), 1, 0, _fake(0x100), None) == sb.SB_EINVAL
+    assert L.sb_wait_flag(_fake(0x1000), 1, 10_000_000_001, _fake(0x100), None) == sb.SB_EINVAL
+    assert "limit_ns" in L.sb_last_error().decode()
+
+
 def test_argument_validation_without_gpu(sb):
     L = sb.lib()
     cfg = sb.config()

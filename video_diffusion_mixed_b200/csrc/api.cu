@@ -347,6 +347,16 @@ sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C, 
   return ok();
 }
 
+sb_status sb_wait_flag(const int32_t* flag, int32_t value, uint64_t limit_ns, void* ws, sb_stream stream) {
+  SB_REQUIRE(flag && ws, SB_EINVAL, "flag and ws are required");
+  SB_REQUIRE((reinterpret_cast<uintptr_t>(flag) & 3u) == 0, SB_EALIGN, "flag misaligned");
+  SB_REQUIRE(limit_ns >= 1 && limit_ns <= 10000000000ull, SB_EINVAL, "limit_ns must be in [1, 1e10] (got %llu)",
+             (unsigned long long)limit_ns);
+  cudaError_t e = sb::launch_wait_flag(flag, value, limit_ns, ws, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "k_wait_flag launch");
+  return ok();
+}
+
 sb_status sb_check(void* ws, sb_stream stream) {
   SB_REQUIRE(ws != nullptr, SB_EINVAL, "ws is NULL");
   cudaStream_t s = (cudaStream_t)stream;

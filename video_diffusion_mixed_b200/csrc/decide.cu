@@ -83,6 +83,27 @@ cudaError_t launch_select(const sb_module_state* st, double a, double b, double 
   return cudaGetLastError();
 }
 
+// Bounded wait for *flag == value: acquire loads, a short sleep between polls, %globaltimer for
+// the deadline. On timeout the workspace error word records SB_ETIMEOUT and the kernel returns.
+__global__ void k_wait_flag(const int32_t* flag, int32_t value, uint64_t limit_ns, WsHeader* hdr) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    int32_t v;
+    asm volatile("ld.acquire.sys.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == value) return;
+    if (globaltimer() - t0 > limit_ns) {
+      set_error(hdr, SB_ETIMEOUT);
+      return;
+    }
+    __nanosleep(1000);
+  }
+}
+
+cudaError_t launch_wait_flag(const int32_t* flag, int32_t value, uint64_t limit_ns, void* hdr, cudaStream_t s) {
+  k_wait_flag<<<1, 1, 0, s>>>(flag, value, limit_ns, reinterpret_cast<WsHeader*>(hdr));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_set_i32(int32_t* p, int32_t v, cudaStream_t s) {
   k_set_i32<<<1, 32, 0, s>>>(p, v);
   return cudaGetLastError();

@@ -90,6 +90,7 @@ def lib():
             "sb_tdc_record": (st, [vp, vp, i64, i64, vp, i32, vp, vp, vp]),
             "sb_check": (st, [vp, vp]),
             "sb_prepass_static": (st, [vp, vp, i64, i64, P(Config), i32, vp, P(Fp4), P(I8), vp, vp]),
+            "sb_wait_flag": (st, [vp, i32, ctypes.c_uint64, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -101,7 +102,7 @@ def lib():
 
 EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_init", "sb_fp4_sf_bytes",
             "sb_state_init", "sb_rotate", "sb_prepare_weight", "sb_tdc_step", "sb_select_precision", "sb_prepass",
-            "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static")
+            "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static", "sb_wait_flag")
 
 
 def _ck(status: int):
@@ -264,3 +265,9 @@ def tdc_record(y_new, y_cache, d_src, state, ws: Workspace, update_cache: bool =
 
 def check(ws: Workspace, stream=None):
     _ck(lib().sb_check(ws.ptr, _stream(stream)))
+
+
+def wait_flag(flag, value: int, limit_ns: int, ws: Workspace, stream=None):
+    """Enqueue a bounded device-side wait until flag[0] == value (see sb_wait_flag)."""
+    assert flag.dtype == torch.int32
+    _ck(lib().sb_wait_flag(_p(flag), int(value), int(limit_ns), ws.ptr, _stream(stream)))
