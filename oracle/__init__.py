@@ -68,6 +68,8 @@ def lib():
             "orc_gemm_int8": (None, [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, i64, vp, vp]),
             "orc_gemm_bf16": (None, [vp, vp, vp, i64, i64, i64, i32, vp, i64, vp]),
             "orc_tdc_delta": (f64, [vp, vp, i64, i64, vp]),
+            "orc_tdc_refresh": (None, [vp, vp, i64, vp]),
+            "orc_tdc_reuse": (None, [vp, vp, i64, vp]),
             "orc_state_init": (None, [vp]),
             "orc_tdc_step": (None, [vp, f64]),
             "orc_select_precision": (i32, [vp, f64, f64, f64, i32]),
@@ -328,6 +330,26 @@ def tdc_delta(ynew_bf16, ylast_bf16):
     out = np.zeros(2, dtype=np.float64)
     d = lib().orc_tdc_delta(_P(a), _P(b), M, C, _P(out))
     return d, float(out[0]), float(out[1])
+
+
+def tdc_refresh(x_bf16, y_bf16):
+    """R-REUSE: the residual kept at a computed step, D = bf16(y - x) (bf16 bit patterns)."""
+    x = _u16(x_bf16)
+    y = _u16(y_bf16)
+    assert x.shape == y.shape
+    d = np.empty_like(x)
+    lib().orc_tdc_refresh(_P(x), _P(y), x.size, _P(d))
+    return d
+
+
+def tdc_reuse(x_bf16, d_bf16):
+    """R-REUSE: the output of a skipped step, y = bf16(x + D) (bf16 bit patterns)."""
+    x = _u16(x_bf16)
+    d = _u16(d_bf16)
+    assert x.shape == d.shape
+    y = np.empty_like(x)
+    lib().orc_tdc_reuse(_P(x), _P(d), x.size, _P(y))
+    return y
 
 
 class State(ctypes.Structure):

@@ -25,6 +25,9 @@
  *   R-RULE  INT8 iff a * d_prev + b > tau (FP64, no fused multiply-add); restart -> INT8.
  *   R-TDC   delta = sum|y_new - y_last| / sum|y_last|; acc += delta each later step;
  *           skip iff acc <= threshold; a computed step resets acc to 0.
+ *   R-REUSE the cache keeps the module's residual D = y - x of its last computed step (bf16: the
+ *           FP32 difference of the bf16 values, rounded to nearest even); a skipped step
+ *           returns y = x + D (FP32 sum of the bf16 values, rounded to nearest even).
  * Parity of R-RULE constants, R-TDC accumulator semantics and R-PDR granularity is pinned only
  * to these definitions ("parity unpinned" against the pages, which print no constants).
  *
@@ -521,6 +524,18 @@ double orc_tdc_delta(const uint16_t* ynew, const uint16_t* ylast, int64_t M, int
     out[1] = S[1];
   }
   return (S[1] == 0.0) ? INFINITY : S[0] / S[1];
+}
+
+/* R-REUSE ([VU] 二: a skipped module reuses the cached result; [GS] 3: the old outcome is used
+ * and adjusted very slightly; [VU] 七: the cache holds historical results). At a computed step
+ * the module's residual is kept, D = bf16(y - x); at a skipped step y = bf16(x + D). n elements,
+ * all bf16 bit patterns. */
+void orc_tdc_refresh(const uint16_t* x, const uint16_t* y, int64_t n, uint16_t* d) {
+  for (int64_t i = 0; i < n; ++i) d[i] = orc_f32_to_bf16(bf16_to_f32(y[i]) - bf16_to_f32(x[i]));
+}
+
+void orc_tdc_reuse(const uint16_t* x, const uint16_t* d, int64_t n, uint16_t* y) {
+  for (int64_t i = 0; i < n; ++i) y[i] = orc_f32_to_bf16(bf16_to_f32(x[i]) + bf16_to_f32(d[i]));
 }
 
 /* Per-module state of the Temporal Delta Cache and of the precision rule. */

@@ -351,6 +351,34 @@ def test_tdc_delta_closed_form(orc):
     assert d0 == math.inf
 
 
+def test_tdc_reuse_matches_ml_dtypes_rounding(orc):
+    """R-REUSE through an independent bf16 implementation: ml_dtypes' float32 -> bfloat16 cast
+    (round to nearest even) of the FP32 difference / sum of the bf16 values."""
+    ml = pytest.importorskip("ml_dtypes")
+    rng = np.random.default_rng(11)
+    # values of very different magnitude, so the FP32 difference and the bf16 rounding both bite
+    x = (rng.standard_normal(6000) * np.exp2(rng.integers(-20, 20, 6000))).astype(np.float32).astype(ml.bfloat16)
+    y = (rng.standard_normal(6000) * np.exp2(rng.integers(-20, 20, 6000))).astype(np.float32).astype(ml.bfloat16)
+    xb, yb = x.view(np.uint16), y.view(np.uint16)
+    ref_d = (y.astype(np.float32) - x.astype(np.float32)).astype(ml.bfloat16)
+    d = orc.tdc_refresh(xb, yb)
+    assert np.array_equal(d, ref_d.view(np.uint16))
+    ref_y = (x.astype(np.float32) + ref_d.astype(np.float32)).astype(ml.bfloat16)
+    assert np.array_equal(orc.tdc_reuse(xb, d), ref_y.view(np.uint16))
+
+
+def test_tdc_reuse_closed_form(orc):
+    """Small integers: every step is exact, so a reuse with the same input returns the output;
+    a zero residual returns the input; equal input and output keep a +0 residual."""
+    x = _bf16(np.arange(-64, 64, dtype=np.float64).reshape(8, 16))
+    y = _bf16((np.arange(-64, 64, dtype=np.float64) * 3 + 5).reshape(8, 16))
+    xb, yb = x.view(torch.int16).numpy().view(np.uint16), y.view(torch.int16).numpy().view(np.uint16)
+    d = orc.tdc_refresh(xb, yb)
+    assert np.array_equal(orc.tdc_reuse(xb, d), yb)
+    assert np.array_equal(orc.tdc_reuse(xb, np.zeros_like(xb)), xb)
+    assert np.array_equal(orc.tdc_refresh(xb, xb), np.zeros_like(xb))  # +0, not -0
+
+
 def test_tdc_schedule_dyadic(orc):
     """delta = 1/32, threshold 1/8: after the two warm-up outputs, four skips then a compute."""
     s = orc.State()
