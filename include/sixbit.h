@@ -228,6 +228,20 @@ sb_status sb_prepass_static(const void* X, const void* X_ref, int64_t M, int64_t
                             const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */, sb_stats* stats,
                             sb_stream stream);
 
+/* Temporal Delta Cache, reuse path ("write-up" section 二: a skipped module reuses the cached
+ * result; explainer section 3: the old outcome is used and adjusted very slightly). The cache
+ * keeps the module's residual D = y - x of its last computed step:
+ *   sb_tdc_refresh: if the module computed this step (state->skip == 0), delta = bf16(y - x);
+ *   sb_tdc_reuse:   if the module is skipped this step (state->skip == 1), y = bf16(x + delta);
+ * each element as the FP32 difference / sum of the bf16 values, rounded to nearest even. The other
+ * case writes nothing, so both calls can be enqueued every step after sb_tdc_step. x, y, delta:
+ * bf16 [M][C] row-major, caller-owned, 16-byte aligned (SB_EALIGN); C a multiple of 8
+ * (SB_EUNSUPPORTED); state: device sb_module_state. */
+sb_status sb_tdc_refresh(const void* x, const void* y, void* delta, int64_t M, int64_t C, const sb_module_state* state,
+                         sb_stream stream);
+sb_status sb_tdc_reuse(const void* x, const void* delta, void* y, int64_t M, int64_t C, const sb_module_state* state,
+                       sb_stream stream);
+
 /* Bounded device-side wait, the library's failure-detection primitive (the pages have no
  * counterpart). Enqueues on `stream` a one-thread kernel that polls the device int32 at `flag`
  * (acquire loads, ~1 us apart) until it equals `value`. If `limit_ns` nanoseconds of device time

@@ -58,6 +58,15 @@ def _fake(addr):
     return ctypes.c_void_p(addr)
 
 
+def test_tdc_reuse_validation_without_gpu(sb):
+    L = sb.lib()
+    ok = (_fake(0x1000), _fake(0x2000), _fake(0x3000))
+    assert L.sb_tdc_refresh(*ok, 4, 64, None, None) == sb.SB_EINVAL
+    assert L.sb_tdc_reuse(_fake(0x1008), _fake(0x2000), _fake(0x3000), 4, 64, _fake(0x4000), None) == sb.SB_EALIGN
+    assert L.sb_tdc_reuse(*ok, 4, 60, _fake(0x4000), None) == sb.SB_EUNSUPPORTED
+    assert L.sb_tdc_refresh(*ok, 0, 64, _fake(0x4000), None) == sb.SB_ESHAPE
+
+
 def test_wait_flag_validation_without_gpu(sb):
     L = sb.lib()
     assert L.sb_wait_flag(None, 1, 1000, _fake(0x100), None) == sb.SB_EINVAL

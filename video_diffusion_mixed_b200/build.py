@@ -20,7 +20,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsixbit.so")
-SOURCES = ["api.cu", "prepass.cu", "decide.cu", "gemm.cu", "prepass_static.cu"]
+SOURCES = ["api.cu", "prepass.cu", "decide.cu", "gemm.cu", "prepass_static.cu", "reuse.cu"]
 HEADERS = ["sb_device.cuh", "sb_kernels.h", "rows.cuh", "tmap.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

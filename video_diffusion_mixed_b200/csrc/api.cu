@@ -347,6 +347,36 @@ sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C, 
   return ok();
 }
 
+static sb_status tdc_combine_args(const void* a, const void* b, const void* out, int64_t M, int64_t C,
+                                  const sb_module_state* state) {
+  SB_REQUIRE(a && b && out && state, SB_EINVAL, "x, the residual, the output and state are required");
+  SB_ALIGNED(a, "x");
+  SB_ALIGNED(b, "second input");
+  SB_ALIGNED(out, "output");
+  SB_REQUIRE(M >= 1 && M <= (int64_t)1 << 30, SB_ESHAPE, "M out of range (%lld)", (long long)M);
+  SB_REQUIRE(C >= 8 && C % 8 == 0 && C <= (int64_t)1 << 20, SB_EUNSUPPORTED, "C must be a multiple of 8 (got %lld)",
+             (long long)C);
+  return SB_OK;
+}
+
+sb_status sb_tdc_refresh(const void* x, const void* y, void* delta, int64_t M, int64_t C, const sb_module_state* state,
+                         sb_stream stream) {
+  const sb_status st = tdc_combine_args(x, y, delta, M, C, state);
+  if (st != SB_OK) return st;
+  cudaError_t e = sb::launch_tdc_refresh(x, y, delta, M * C, state, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "k_tdc_combine (refresh) launch");
+  return ok();
+}
+
+sb_status sb_tdc_reuse(const void* x, const void* delta, void* y, int64_t M, int64_t C, const sb_module_state* state,
+                       sb_stream stream) {
+  const sb_status st = tdc_combine_args(x, delta, y, M, C, state);
+  if (st != SB_OK) return st;
+  cudaError_t e = sb::launch_tdc_reuse(x, delta, y, M * C, state, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "k_tdc_combine (reuse) launch");
+  return ok();
+}
+
 sb_status sb_wait_flag(const int32_t* flag, int32_t value, uint64_t limit_ns, void* ws, sb_stream stream) {
   SB_REQUIRE(flag && ws, SB_EINVAL, "flag and ws are required");
   SB_REQUIRE((reinterpret_cast<uintptr_t>(flag) & 3u) == 0, SB_EALIGN, "flag misaligned");

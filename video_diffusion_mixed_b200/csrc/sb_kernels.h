@@ -86,6 +86,10 @@ cudaError_t launch_select(const sb_module_state* st, double a, double b, double 
                           cudaStream_t s);
 cudaError_t launch_set_i32(int32_t* p, int32_t v, cudaStream_t s);
 cudaError_t launch_wait_flag(const int32_t* flag, int32_t value, uint64_t limit_ns, void* hdr, cudaStream_t s);
+cudaError_t launch_tdc_refresh(const void* x, const void* y, void* d, int64_t n, const sb_module_state* st,
+                               cudaStream_t s);
+cudaError_t launch_tdc_reuse(const void* x, const void* d, void* y, int64_t n, const sb_module_state* st,
+                             cudaStream_t s);
 cudaError_t launch_ws_init(void* ws, size_t bytes, cudaStream_t s);
 
 sb_status report_error(sb_status st, const char* msg);

@@ -91,6 +91,8 @@ def lib():
             "sb_check": (st, [vp, vp]),
             "sb_prepass_static": (st, [vp, vp, i64, i64, P(Config), i32, vp, P(Fp4), P(I8), vp, vp]),
             "sb_wait_flag": (st, [vp, i32, ctypes.c_uint64, vp, vp]),
+            "sb_tdc_refresh": (st, [vp, vp, vp, i64, i64, vp, vp]),
+            "sb_tdc_reuse": (st, [vp, vp, vp, i64, i64, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -102,7 +104,8 @@ def lib():
 
 EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_init", "sb_fp4_sf_bytes",
             "sb_state_init", "sb_rotate", "sb_prepare_weight", "sb_tdc_step", "sb_select_precision", "sb_prepass",
-            "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static", "sb_wait_flag")
+            "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static", "sb_wait_flag", "sb_tdc_refresh",
+            "sb_tdc_reuse")
 
 
 def _ck(status: int):
@@ -265,6 +268,18 @@ def tdc_record(y_new, y_cache, d_src, state, ws: Workspace, update_cache: bool =
 
 def check(ws: Workspace, stream=None):
     _ck(lib().sb_check(ws.ptr, _stream(stream)))
+
+
+def tdc_refresh(x, y, delta, state, stream=None):
+    """At a computed step keep the module's residual: delta = bf16(y - x) (sb_tdc_refresh)."""
+    M, C = x.shape
+    _ck(lib().sb_tdc_refresh(_p(x), _p(y), _p(delta), M, C, _p(state), _stream(stream)))
+
+
+def tdc_reuse(x, delta, y, state, stream=None):
+    """At a skipped step produce the output from the kept residual: y = bf16(x + delta)."""
+    M, C = x.shape
+    _ck(lib().sb_tdc_reuse(_p(x), _p(delta), _p(y), M, C, _p(state), _stream(stream)))
 
 
 def wait_flag(flag, value: int, limit_ns: int, ws: Workspace, stream=None):
