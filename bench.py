@@ -150,25 +150,27 @@ class FfnStep:
     def gemm_flops(self):
         return 2.0 * self.M * (self.N1 * self.K1 + self.N2 * self.K2)
 
-    def one_pass(self, prec, ev=None):
+    def one_pass(self, prec, ev=None, X=None, Y=None):
         sb = self.sb
+        X = self.X if X is None else X
+        Y = self.Y if Y is None else Y
         cfg = sb.config(rho=64.0, tdc_thresh=-1.0, block=128, force_prec=prec)  # never skip: full work
         sb.tdc_step(self.state, cfg)
         sb.select_precision(self.state, self.rule, cfg, self.p1)
         self._mark(ev, "pre1_0")
-        sb.prepass(self.X, None, cfg, sb.PREPASS_QUANT, self.p1, self.ax4, self.ax8, self.sx, self.ws)
+        sb.prepass(X, None, cfg, sb.PREPASS_QUANT, self.p1, self.ax4, self.ax8, self.sx, self.ws)
         self._mark(ev, "pre1_1")
-        sb.linear(self.X, self.ax4, self.ax8, self.p1, self.w1, self.H, epilogue=sb.EPI_GELU, ws=self.ws)
+        sb.linear(X, self.ax4, self.ax8, self.p1, self.w1, self.H, epilogue=sb.EPI_GELU, ws=self.ws)
         self._mark(ev, "gemm1_1")
         sb.select_precision(self.state, self.rule, cfg, self.p2)
         self._mark(ev, "pre2_0")
         sb.prepass(self.H, None, cfg, sb.PREPASS_QUANT, self.p2, self.ah4, self.ah8, self.sh, self.ws)
         self._mark(ev, "pre2_1")
-        sb.linear(self.H, self.ah4, self.ah8, self.p2, self.w2, self.Y, ws=self.ws)
+        sb.linear(self.H, self.ah4, self.ah8, self.p2, self.w2, Y, ws=self.ws)
         self._mark(ev, "gemm2_1")
-        sb.prepass(self.Y, self.X, cfg, sb.PREPASS_STATS, self.p2, None, None, self.sy, self.ws)
+        sb.prepass(Y, X, cfg, sb.PREPASS_STATS, self.p2, None, None, self.sy, self.ws)
         self._mark(ev, "d_1")
-        sb.tdc_record(self.Y, self.cache, self.sy, self.state, self.ws)
+        sb.tdc_record(Y, self.cache, self.sy, self.state, self.ws)
         self._mark(ev, "tdc_1")
 
     def _mark(self, ev, name):
@@ -261,23 +263,56 @@ def run_ours(args):
                 kern.setdefault(f"{name}_{tag}", []).append(d[a].elapsed_time(d[z]))
     kern_ms = {k: statistics.median(v) for k, v in kern.items()}
 
-    # ---- end to end through the public API with host buffers (pinned H2D of X, D2H of Y)
+    # ---- end to end through the public API with host buffers: every step uploads its X from
+    # pinned host memory and downloads both passes' outputs. A deployment pipelines the transfers:
+    # the upload of step i + 1 (copy stream U) and the download of each pass's output (copy
+    # stream D) overlap the compute of the neighbouring passes on the compute stream, through
+    # double-buffered device inputs and outputs ordered by events. The timed span runs from the
+    # first upload to the last download; the L2 flush stays inside it on the compute stream.
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     Xh = torch.empty(S.X.shape, dtype=S.X.dtype, pin_memory=True)
     Xh.copy_(S.X.cpu())
-    Yh = torch.empty(S.Y.shape, dtype=S.Y.dtype, pin_memory=True)
-    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    Yh = [torch.empty(S.Y.shape, dtype=S.Y.dtype, pin_memory=True) for _ in range(2)]
+    Xd = [S.X, torch.empty_like(S.X)]
+    Yd = [S.Y, torch.empty_like(S.Y)]
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    x_free = [None, None]      # compute finished with Xd[b]
+    y_free = [None, None]      # download finished with Yd[p]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
     barrier()
     for i in range(args.steps):
+        b = i % 2
+        with torch.cuda.stream(up):
+            if i == 0:
+                t0.record()
+            if x_free[b] is not None:
+                up.wait_event(x_free[b])
+            Xd[b].copy_(Xh, non_blocking=True)
+            x_ready = ev()
+            x_ready.record()
+        comp.wait_event(x_ready)
         flush.zero_()
-        e_s[i].record()
-        S.X.copy_(Xh, non_blocking=True)
-        for prec in (sb.NVFP4, sb.INT8):
-            S.one_pass(prec)
-            Yh.copy_(S.Y, non_blocking=True)
-        e_e[i].record()
+        for p, prec in enumerate((sb.NVFP4, sb.INT8)):
+            if y_free[p] is not None:
+                comp.wait_event(y_free[p])
+            S.one_pass(prec, X=Xd[b], Y=Yd[p])
+            y_ready = ev()
+            y_ready.record()
+            with torch.cuda.stream(down):
+                down.wait_event(y_ready)
+                Yh[p].copy_(Yd[p], non_blocking=True)
+                y_free[p] = ev()
+                y_free[p].record()
+        x_free[b] = ev()
+        x_free[b].record()
+    with torch.cuda.stream(down):
+        down.wait_event(x_free[(args.steps - 1) % 2])
+        t1.record()
+    torch.cuda.synchronize()
     barrier()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
+    e2e_ms = t0.elapsed_time(t1)
     if world > 1:
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
