@@ -163,20 +163,28 @@ def test_missing_operands_reported(sbg):
     assert e.value.status == sbg.SB_EINVAL
 
 
-@pytest.mark.parametrize("layer", ["w1", "w2"])
+FULL = [  # (id, N, K, GELU): CogVideoX-5B FFN, CogVideoX-2B attention projection and FFN
+    ("5b_w1", 12288, 3072, True), ("5b_w2", 3072, 12288, False),
+    ("2b_attn", 1920, 1920, False), ("2b_w1", 7680, 1920, True), ("2b_w2", 1920, 7680, False),
+]
+
+
+@pytest.mark.parametrize("name,N,K,gelu", FULL, ids=[f[0] for f in FULL])
 @pytest.mark.parametrize("prec", [0, 1], ids=["nvfp4", "int8"])
-def test_full_size_5b_ffn_sampled(sbg, layer, prec):
-    """CogVideoX-5B FFN at full shape (17776 tokens), every 64th row plus the last one checked."""
+def test_full_size_sampled(sbg, name, N, K, gelu, prec):
+    """DiT layers at full shape (17776 tokens): every 64th row plus the last one against the
+    oracle (FP32 output), and the bf16 output -- the TMA-store epilogue, last tile clipped at
+    M -- equal to the RNE rounding of the kernel's FP32 result over every element."""
     M = synth.TOKENS
-    N, K = (12288, 3072) if layer == "w1" else (3072, 12288)
-    L = Layer(sbg, M, N, K, seed=10, gen=dict(n_outlier=15, scale=50.0) if layer == "w1" else {})
-    Y = L.run(prec, sbg.OUT_F32, gelu=(layer == "w1"))
+    L = Layer(sbg, M, N, K, seed=10, gen=dict(n_outlier=15, scale=50.0) if gelu else {})
+    Y = L.run(prec, sbg.OUT_F32, gelu=gelu)
+    Yb = L.run(prec, sbg.OUT_BF16, gelu=gelu)
+    assert torch.equal(Yb, Y.to(torch.bfloat16))
     rows = sample_rows(M)
     wp, xp = L.oracle_ops()
     if prec == 0:
         ref = oracle.gemm_nvfp4(xp["c4"], xp["sf4"], xp["sg4"], wp["c4"], wp["sf4"], wp["sg4"], u16(L.bias), K, 128,
-                                gelu=(layer == "w1"), rows=rows)
+                                gelu=gelu, rows=rows)
     else:
-        ref = oracle.gemm_int8(xp["q8"], xp["s8"], wp["q8"], wp["s8"], u16(L.bias), 128, gelu=(layer == "w1"),
-                               rows=rows)
+        ref = oracle.gemm_int8(xp["q8"], xp["s8"], wp["q8"], wp["s8"], u16(L.bias), 128, gelu=gelu, rows=rows)
     assert rel_fro(npy(Y)[rows], ref) <= TOL

@@ -109,20 +109,22 @@ def test_decision_kernels_follow_the_oracle_state_machine(sbg):
         k_out += 1
 
 
-def test_trajectory_decisions_bitexact(sbg):
-    """30 DiT blocks x 50 steps (hidden 3072, tokens reduced to 256 so the oracle finishes in
-    seconds): difference-driven NVFP4/INT8, PDR BF16 fallback (rho 64), TDC threshold 0.1.
-    The decision log and every delta and d must equal the oracle's."""
-    blocks, steps, M, C = 30, 50, 256, 3072
+@pytest.mark.parametrize("M,ks", [(256, tuple(range(30))), (17776, (0, 7, 14, 22, 29))],
+                         ids=["256tok_30blocks", "17776tok_5blocks"])
+def test_trajectory_decisions_bitexact(sbg, M, ks):
+    """DiT blocks x 50 steps (hidden 3072): difference-driven NVFP4/INT8, PDR BF16 fallback
+    (rho 64), TDC threshold 0.1; all 30 blocks at 256 tokens, and a spread of 5 blocks at the full
+    17776 tokens. The decision log and every delta and d must equal the oracle's."""
+    blocks, steps, C = 30, 50, 3072
     cfg = sbg.config(rho=64.0, tdc_thresh=0.1)
     rule = sbg.Rule(1.0, 0.0, 0.1)
     ws = sbg.Workspace(M, C)
     a4, a8 = sbg.Fp4Tensor(M, C), sbg.I8Tensor(M, C)
     sx, sy = sbg.alloc_stats(), sbg.alloc_stats()
     prec = torch.zeros(1, dtype=torch.int32, device="cuda")
-    log_gpu = np.zeros((blocks, steps), np.int32)
-    log_ref = np.zeros((blocks, steps), np.int32)
-    for k in range(blocks):
+    log_gpu = np.zeros((len(ks), steps), np.int32)
+    log_ref = np.zeros((len(ks), steps), np.int32)
+    for kk, k in enumerate(ks):
         traj = synth.Trajectory(M, C, k, blocks=blocks, steps=steps, seed=0, device="cuda")
         st = sbg.alloc_state()
         os_ = oracle.State()
@@ -136,7 +138,7 @@ def test_trajectory_decisions_bitexact(sbg):
             sbg.prepass(y, x, cfg, sbg.PREPASS_STATS, prec, None, None, sy, ws)
             sbg.tdc_record(y, cache, sy, st, ws)
             sbg.check(ws)
-            log_gpu[k, t] = int(prec.item())
+            log_gpu[kk, t] = int(prec.item())
             # oracle
             oracle.tdc_step(os_, 0.1)
             p = oracle.select_precision(os_, 1.0, 0.0, 0.1)
@@ -148,7 +150,7 @@ def test_trajectory_decisions_bitexact(sbg):
                 delta = oracle.tdc_delta(yb, last_y)[0] if last_y is not None else None
                 oracle.tdc_record(os_, delta, ry["d"])
                 last_y = yb
-            log_ref[k, t] = p
+            log_ref[kk, t] = p
             g = gstate_dict(sbg, st)
             assert g == ostate_dict(os_), (k, t, g, ostate_dict(os_))
             if t + 1 < steps:
