@@ -602,15 +602,66 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   __threadfence();
   const int64_t G = ngroups;
   double S[NST];
-#pragma unroll
-  for (int s = 0; s < NST; ++s) S[s] = cta_pairwise_f64(&a.groups[0].s[s], sizeof(GroupSlot) / 8, G, s_fin, s_fwarp);
   float mx = 0.0f, ar = 0.0f;
   int nf = 0;
-  for (int64_t gg = threadIdx.x; gg < G; gg += blockDim.x) {
-    const GroupSlot* gs = a.groups + gg;
-    mx = fmaxf(mx, __ldcg(&gs->max_abs));
-    ar = fmaxf(ar, __ldcg(&gs->amax_rot));
-    nf |= __ldcg(&gs->nonfinite);
+  int64_t P = 256;
+  while (P < G) P <<= 1;
+  if (P <= 256 * 16) {
+    // One pass over the group slots for every statistic and maximum: thread t owns the aligned
+    // run [t R, (t + 1) R) of the zero-padded slots (R = P / 256 <= 16, padded to 16 with zeros),
+    // then the warp trees and the tree of the 8 warp sums -- the same halving tree as
+    // cta_pairwise_f64 with a single chunk.
+    const int R = (int)(P / 256);
+    double t3[NST][16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int64_t gi = (int64_t)threadIdx.x * R + k;
+      const bool in = k < R && gi < G;
+      const GroupSlot* gs = a.groups + (in ? gi : 0);
+#pragma unroll
+      for (int st = 0; st < NST; ++st) t3[st][k] = in ? __ldcg(&gs->s[st]) : 0.0;
+      if (in) {
+        mx = fmaxf(mx, __ldcg(&gs->max_abs));
+        ar = fmaxf(ar, __ldcg(&gs->amax_rot));
+        nf |= __ldcg(&gs->nonfinite);
+      }
+    }
+    double* s_w3 = s_fin;  // [warp][statistic]
+#pragma unroll
+    for (int st = 0; st < NST; ++st) {
+#pragma unroll
+      for (int len = 16; len > 1; len >>= 1) {
+#pragma unroll
+        for (int i = 0; i < len / 2; ++i) t3[st][i] = __dadd_rn(t3[st][2 * i], t3[st][2 * i + 1]);
+      }
+      const double wsum = warp_pairwise_f64(t3[st][0]);
+      if (lane == 0) s_w3[warp * NST + st] = wsum;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+#pragma unroll
+      for (int st = 0; st < NST; ++st) {
+        double u[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) u[w] = s_w3[w * NST + st];
+#pragma unroll
+        for (int len = 8; len > 1; len >>= 1) {
+#pragma unroll
+          for (int i = 0; i < len / 2; ++i) u[i] = __dadd_rn(u[2 * i], u[2 * i + 1]);
+        }
+        S[st] = u[0];
+      }
+    }
+  } else {
+#pragma unroll
+    for (int st = 0; st < NST; ++st)
+      S[st] = cta_pairwise_f64(&a.groups[0].s[st], sizeof(GroupSlot) / 8, G, s_fin, s_fwarp);
+    for (int64_t gg = threadIdx.x; gg < G; gg += blockDim.x) {
+      const GroupSlot* gs = a.groups + gg;
+      mx = fmaxf(mx, __ldcg(&gs->max_abs));
+      ar = fmaxf(ar, __ldcg(&gs->amax_rot));
+      nf |= __ldcg(&gs->nonfinite);
+    }
   }
   mx = warp_max_f32(mx);
   ar = warp_max_f32(ar);
