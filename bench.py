@@ -119,6 +119,25 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------
+# Multi-rank bookkeeping (replicas: every rank runs its own full step on its own batch)
+# ------------------------------------------------------------------------------------------------
+
+def max_over_ranks(ms, world, dist, device):
+    """Device time of the whole job: the slowest rank's. Every rank calls it in the same order."""
+    if world > 1:
+        import torch
+        t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def whole_job_tflops(world, flops_per_rank_step, ms_per_step):
+    """Throughput of all ranks together: each rank processed its own batch in ms_per_step."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
+# ------------------------------------------------------------------------------------------------
 # Our arm
 # ------------------------------------------------------------------------------------------------
 
@@ -237,14 +256,10 @@ def run_ours(args):
     clocks = clk.stop()
     sb.check(S.ws)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dist, device)
     ms_per_step = total_ms / args.steps
     flops = 2 * S.gemm_flops()  # both precision passes
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops, ms_per_step)
 
     # ---- per-kernel breakdown (a separate, untimed-for-value pass with events between calls)
     kern = {}
@@ -312,12 +327,8 @@ def run_ours(args):
         t1.record()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops / (e2e_ms / args.steps * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, dist, device)
+    e2e_value = whole_job_tflops(world, flops, e2e_ms / args.steps)
     h2d = S.X.numel() * S.X.element_size()
     d2h = 2 * S.Y.numel() * S.Y.element_size()
 
