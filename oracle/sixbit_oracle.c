@@ -233,7 +233,8 @@ void orc_prepass(const uint16_t* X, const uint16_t* Xref, int64_t M, int64_t K, 
 /* ------------------------------------------------------------------------------------------ */
 
 /* Symmetric per-row INT8 of the rotated rows: s_m = a_m / 127, q = clamp(rne(y * (127/a_m))).
- * a_m = 0 gives s_m = 0 and all codes 0. */
+ * a_m = 0 gives s_m = 0 and all codes 0; when 127/a_m overflows, nonzero y clamp to +-127 and
+ * y = 0 gives 0. */
 void orc_quant_int8(const float* y, int64_t M, int64_t K, const float* row_amax, int8_t* q,
                     float* s) {
 #pragma omp parallel for schedule(static)
@@ -251,6 +252,9 @@ void orc_quant_int8(const float* y, int64_t M, int64_t K, const float* row_amax,
       float r = nearbyintf(v); /* default rounding mode: nearest, ties to even */
       if (r > 127.0f) r = 127.0f;
       if (r < -127.0f) r = -127.0f;
+      /* 127/a overflows to +inf for a below 127/FLT_MAX: y = 0 then gives 0 * inf = NaN, whose
+       * exact value y * (127/a) is 0 */
+      if (r != r) r = 0.0f;
       q[m * K + k] = (int8_t)r;
     }
   }

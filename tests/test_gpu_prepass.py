@@ -82,7 +82,7 @@ def test_prepass_nvfp4_bitexact(sbg, name, M, K, with_ref, gen):
     assert out["stats"]["amax_rot"] == ref["amax_rot"]
 
 
-@pytest.mark.parametrize("B", [16, 64, 256])
+@pytest.mark.parametrize("B", [16, 32, 64, 256])
 def test_prepass_block_sizes(sbg, B):
     X = synth.activations(50, 1024, n_outlier=5, scale=10.0, seed=B, device="cuda")
     ref = oracle.prepass(u16(X), None, B)
@@ -158,7 +158,71 @@ def test_prepass_full_size(sbg, wl):
     q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
     assert np.array_equal(npy(out8["a8"].codes), q)
     assert np.array_equal(npy(out8["a8"].scale), s)
+    out8n = run_prepass(sbg, R, None, force=sbg.INT8)  # no x_ref: the block-per-lane kernel
+    for k in ("sum_abs", "max_abs", "amax_rot", "ratio"):
+        assert out8n["stats"][k] == ref[k], k
+    assert np.array_equal(npy(out8n["a8"].codes), q)
+    assert np.array_equal(npy(out8n["a8"].scale), s)
+    del out8n
     out4 = run_prepass(sbg, R, None, force=sbg.NVFP4)
+    codes, sfl, sft, sg = oracle.quant_nvfp4(ref["y"], ref["amax_rot"])
+    assert np.array_equal(npy(out4["a4"].codes), codes)
+    assert np.array_equal(npy(out4["a4"].sf), sft)
+
+
+# Row shapes for every team shape of the block-per-lane pre-pass: several rows per warp (K = 128,
+# 384, 1920, 2048), rows straddling warps (640, 3072, 12288, 16384), idle lanes (128, 384, 640,
+# 1920, 7680) and a ragged last group of rows.
+GEOMS = [(1, 128), (17, 384), (33, 640), (129, 3072), (300, 1920), (7, 12288), (40, 16384), (1000, 2048),
+         (20, 7680)]
+
+
+@pytest.mark.parametrize("M,K", GEOMS, ids=[f"{m}x{k}" for m, k in GEOMS])
+def test_prepass_team_shapes(sbg, M, K):
+    X = synth.activations(M, K, n_outlier=max(1, K // 200), scale=25.0, seed=M, tensor_id=K, device="cuda")
+    ref = oracle.prepass(u16(X), None, 128)
+    out8 = run_prepass(sbg, X, force=sbg.INT8)
+    for k in ("sum_abs", "max_abs", "amax_rot", "ratio"):
+        assert out8["stats"][k] == ref[k], (k, out8["stats"][k], ref[k])
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    assert np.array_equal(npy(out8["a8"].codes), q)
+    assert np.array_equal(npy(out8["a8"].scale).view(np.uint32), s.view(np.uint32))
+    out4 = run_prepass(sbg, X, force=sbg.NVFP4)
+    codes, sfl, sft, sg = oracle.quant_nvfp4(ref["y"], ref["amax_rot"])
+    assert np.array_equal(npy(out4["a4"].codes), codes)
+    assert np.array_equal(npy(out4["a4"].sf), sft)
+
+
+@pytest.mark.parametrize("B,with_ref", [(128, False), (256, False), (128, True)])
+def test_int8_rows_below_overflow_threshold(sbg, B, with_ref):
+    """Rows of subnormal magnitude: 127 / a_m overflows in FP32, so every nonzero code clamps to
+    +-127 and zeros stay 0 (both pre-pass kernels, with and without x_ref)."""
+    X = (synth.activations(24, 512, seed=11, device="cuda").float() * 1e-39).to(torch.bfloat16)
+    X[3] = 0.0                 # an all-zero row: a_m = 0
+    X[5, ::3] = 0.0            # zeros inside a tiny row
+    X[7] = (X[7].double() * 1e40).to(torch.bfloat16)  # one ordinary row (1e40 overflows FP32)
+    R = synth.activations(24, 512, seed=12, device="cuda") if with_ref else None
+    ref = oracle.prepass(u16(X), u16(R) if R is not None else None, B)
+    assert (ref["row_amax"][[0, 1, 2, 4, 5]] < np.float32(127.0) / np.finfo(np.float32).max).all()
+    out8 = run_prepass(sbg, X, R, force=sbg.INT8, block=B)
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    assert np.array_equal(npy(out8["a8"].codes), q)
+    assert np.array_equal(npy(out8["a8"].scale).view(np.uint32), s.view(np.uint32))
+
+
+def test_prepass_hidden_full_size(sbg):
+    """The FFN hidden tensor of CogVideoX-5B (17776 x 12288): statistics, INT8 and NVFP4 of the
+    block-per-lane pre-pass, bit-exact over every element."""
+    X = synth.activations(17776, 12288, n_outlier=61, scale=20.0, seed=0, tensor_id=7, device="cuda")
+    ref = oracle.prepass(u16(X), None, 128)
+    out8 = run_prepass(sbg, X, force=sbg.INT8)
+    for k in ("sum_abs", "max_abs", "amax_rot", "ratio"):
+        assert out8["stats"][k] == ref[k], k
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    assert np.array_equal(npy(out8["a8"].codes), q)
+    assert np.array_equal(npy(out8["a8"].scale), s)
+    del out8, q
+    out4 = run_prepass(sbg, X, force=sbg.NVFP4)
     codes, sfl, sft, sg = oracle.quant_nvfp4(ref["y"], ref["amax_rot"])
     assert np.array_equal(npy(out4["a4"].codes), codes)
     assert np.array_equal(npy(out4["a4"].sf), sft)

@@ -180,6 +180,19 @@ def test_int8_quant_properties(orc):
         assert np.array_equal(q[m].astype(np.int64), best)
 
 
+def test_int8_quant_overflowing_reciprocal(orc):
+    """FP32 reading of R-INT8 when 127 / a overflows (a below 127 / FLT_MAX): the reciprocal is +inf,
+    every nonzero y lands on +-127 (numpy's FP32 arithmetic gives the same +-inf products) and y = 0,
+    whose exact product is 0, stays 0; s = a / 127 is still the correctly rounded quotient."""
+    a = np.float32(1e-38)
+    assert np.isinf(np.float32(127) / a)
+    y = np.array([[a, a / 2, 0.0, -a / 4, -a, np.float32(1e-45)]], dtype=np.float32)
+    y = np.pad(y, ((0, 0), (0, 128 - y.shape[1])))
+    q, s = orc.quant_int8(y, np.array([a], dtype=np.float32))
+    assert q[0, :6].tolist() == [127, 127, 0, -127, -127, 127] and not q[0, 6:].any()
+    assert s[0] == np.float32(a / np.float32(127))
+
+
 def test_nvfp4_quant_properties(orc):
     rng = np.random.default_rng(6)
     y = (rng.standard_normal((9, 128)) * rng.uniform(0.01, 30, (9, 1))).astype(np.float32)

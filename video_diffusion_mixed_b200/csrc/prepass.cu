@@ -13,6 +13,7 @@
 //  k_nvfp4        re-reads X once the tensor amax is known, rotates again and writes E2M1 codes,
 //                 E4M3 block scales in the tensor-core layout and the FP32 tensor scale.
 //  k_rotate       rotation only (test hook).
+#include "prepass_blk.cuh"
 #include "rows.cuh"
 #include "tmap.h"
 
@@ -56,11 +57,41 @@ static void row_maps(RowArgs& a, RowMaps& mp, const void* X, const void* R) {
   a.tma = make_row_segment_map(&mp.x, X, a.M, a.K) && (!R || make_row_segment_map(&mp.r, R, a.M, a.K)) ? 1 : 0;
 }
 
+// The block-per-lane pre-pass (k_prepass_blk): no x_ref, B <= 128, whole 128-channel blocks and a
+// team shape and tensor map that fit. Returns false (nothing launched) otherwise.
+static bool launch_prepass_blk(const RowArgs& a, cudaStream_t s, int sms, cudaError_t* err) {
+  if (a.R || a.B > 128 || a.K % 128 != 0) return false;
+  PbGeom gm;
+  if (!pick_pb_geom(a.K / 128, &gm)) return false;
+  CUtensorMap mx;
+  if (!make_halfblock_map(&mx, a.X, a.M, a.K)) return false;
+  constexpr int dsm = kPbRing + 1024;
+  const int64_t groups = ceil_div(a.M, kG);  // a team's unit of work
+  const unsigned grid = (unsigned)(groups < sms ? groups : sms);
+  auto go = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
+    kern<<<grid, kPbThreads, dsm, s>>>(a, gm, mx);
+    *err = cudaGetLastError();
+    return true;
+  };
+  switch (a.B) {
+    case 16: return go(k_prepass_blk<16>);
+    case 32: return go(k_prepass_blk<32>);
+    case 64: return go(k_prepass_blk<64>);
+    case 128: return go(k_prepass_blk<128>);
+    default: return false;
+  }
+}
+
 cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s) {
   RowArgs a = row_args_from(p);
+  const int sms = sm_count();
+  if (!(p.mode == SB_PREPASS_STATS && !p.force_int8) && !p.R) {
+    cudaError_t e;
+    if (launch_prepass_blk(a, s, sms, &e)) return e;
+  }
   RowMaps mp;
   row_maps(a, mp, p.X, p.R);
-  const int sms = sm_count();
   if (p.mode == SB_PREPASS_STATS && !p.force_int8)
     return p.R ? launch_rows_t<OP_STATS, true>(a, mp, s, sms) : launch_rows_t<OP_STATS, false>(a, mp, s, sms);
   return p.R ? launch_rows_t<OP_PREPASS, true>(a, mp, s, sms) : launch_rows_t<OP_PREPASS, false>(a, mp, s, sms);

@@ -171,6 +171,7 @@ __device__ __forceinline__ float2 sq2(float2 a) { return make_float2(__fmul_rn(a
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {  // a - b = fma(b, -1, a): one rounding
   return fma2(b, make_float2(-1.0f, -1.0f), a);
 }
+__device__ __forceinline__ float sign127(float v) { return v > 0.0f ? 127.0f : (v < 0.0f ? -127.0f : 0.0f); }
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -238,8 +239,8 @@ __device__ __forceinline__ void fwht_pairs(float2 (&p)[16], int lane, int B) {
 
 constexpr int kFinChunk = 4096;  // group sums reduced per pass of the last CTA
 
-// Pairwise FP64 tree over n strided values zero-padded to a power of two P >= 256, by a whole CTA
-// of 256 threads. Chunks of up to 4096 values are staged in shared memory; thread t reduces the
+// Pairwise FP64 tree over n strided values zero-padded to a power of two P >= 256, by the first
+// 256 threads of the CTA (every thread calls it: it holds CTA barriers). Chunks of up to 4096 values are staged in shared memory; thread t reduces the
 // aligned run [t*R, (t+1)*R) of its chunk (R = chunk/256 <= 16, zero-padded to 16, which leaves a
 // power-of-two run's sum unchanged), the warps combine 32 runs, thread 0 combines the 8 warps and
 // then, in order, the chunk sums with a stack of partial sums. Every addition is one of the
@@ -252,25 +253,26 @@ __device__ inline double cta_pairwise_f64(const double* p, int64_t stride, int64
   const int R = L / 256;
   const int64_t nchunks = P / L;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool act = tid < 256;
   double stack[40];
   int sp = 0;
   for (int64_t b = 0; b < nchunks; ++b) {
     const int64_t lo = b * L;
-    for (int i = tid; i < L; i += 256) {
+    for (int i = tid; act && i < L; i += 256) {
       const int64_t idx = lo + i;
       sbuf[i] = (idx < n) ? __ldcg(p + idx * stride) : 0.0;
     }
     __syncthreads();
     double t[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) t[k] = (k < R) ? sbuf[tid * R + k] : 0.0;
+    for (int k = 0; k < 16; ++k) t[k] = (act && k < R) ? sbuf[tid * R + k] : 0.0;
 #pragma unroll
     for (int len = 16; len > 1; len >>= 1) {
 #pragma unroll
       for (int i = 0; i < len / 2; ++i) t[i] = __dadd_rn(t[2 * i], t[2 * i + 1]);
     }
     const double wsum = warp_pairwise_f64(t[0]);
-    if (lane == 0) swarp[warp] = wsum;
+    if (act && lane == 0) swarp[warp] = wsum;
     __syncthreads();
     if (tid == 0) {
       double u[8];
@@ -288,6 +290,158 @@ __device__ inline double cta_pairwise_f64(const double* p, int64_t stride, int64
     __syncthreads();
   }
   return stack[0];
+}
+
+// The last CTA to finish reduces the group slots (FP64, the canonical halving tree over the groups
+// zero-padded to a power of two), writes the statistics record or the module state and applies
+// Purified Delta Refresh to the precision flag. Every thread of the CTA calls it (it holds CTA
+// barriers); the first 256 threads do the work. s_fin: at least kFinChunk doubles of shared memory
+// that nothing else uses any more.
+template <int OP, bool REF>
+__device__ void rows_finish(const RowArgs& a, int64_t ngroups, int prec, bool have_prev, double* s_fin) {
+  constexpr int NST = (OP == OP_TDC) ? 2 : 3;
+  constexpr int NW = 8;  // working warps
+  __shared__ int s_last;
+  __shared__ double s_fwarp[NW];
+  __shared__ float s_fmax[NW][2];
+  __shared__ int s_fnf[NW];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool act = threadIdx.x < NW * 32;
+  const int K = a.K;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t tk = atomicAdd(&a.hdr->ticket[OP == OP_TDC ? TICKET_TDC : TICKET_PREPASS], 1u);
+    s_last = (tk == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int64_t G = ngroups;
+  double S[NST];
+  float mx = 0.0f, ar = 0.0f;
+  int nf = 0;
+  int64_t P = 256;
+  while (P < G) P <<= 1;
+  if (P <= 256 * 16) {
+    // One pass over the group slots for every statistic and maximum: thread t owns the aligned
+    // run [t R, (t + 1) R) of the zero-padded slots (R = P / 256 <= 16, padded to 16 with zeros),
+    // then the warp trees and the tree of the 8 warp sums -- the same halving tree as
+    // cta_pairwise_f64 with a single chunk.
+    const int R = (int)(P / 256);
+    double t3[NST][16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int64_t gi = (int64_t)threadIdx.x * R + k;
+      const bool in = act && k < R && gi < G;
+      const GroupSlot* gs = a.groups + (in ? gi : 0);
+#pragma unroll
+      for (int st = 0; st < NST; ++st) t3[st][k] = in ? __ldcg(&gs->s[st]) : 0.0;
+      if (in) {
+        mx = fmaxf(mx, __ldcg(&gs->max_abs));
+        ar = fmaxf(ar, __ldcg(&gs->amax_rot));
+        nf |= __ldcg(&gs->nonfinite);
+      }
+    }
+    double* s_w3 = s_fin;  // [warp][statistic]
+#pragma unroll
+    for (int st = 0; st < NST; ++st) {
+#pragma unroll
+      for (int len = 16; len > 1; len >>= 1) {
+#pragma unroll
+        for (int i = 0; i < len / 2; ++i) t3[st][i] = __dadd_rn(t3[st][2 * i], t3[st][2 * i + 1]);
+      }
+      const double wsum = warp_pairwise_f64(t3[st][0]);
+      if (act && lane == 0) s_w3[warp * NST + st] = wsum;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+#pragma unroll
+      for (int st = 0; st < NST; ++st) {
+        double u[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) u[w] = s_w3[w * NST + st];
+#pragma unroll
+        for (int len = 8; len > 1; len >>= 1) {
+#pragma unroll
+          for (int i = 0; i < len / 2; ++i) u[i] = __dadd_rn(u[2 * i], u[2 * i + 1]);
+        }
+        S[st] = u[0];
+      }
+    }
+  } else {
+#pragma unroll
+    for (int st = 0; st < NST; ++st)
+      S[st] = cta_pairwise_f64(&a.groups[0].s[st], sizeof(GroupSlot) / 8, G, s_fin, s_fwarp);
+    for (int64_t gg = threadIdx.x; act && gg < G; gg += NW * 32) {
+      const GroupSlot* gs = a.groups + gg;
+      mx = fmaxf(mx, __ldcg(&gs->max_abs));
+      ar = fmaxf(ar, __ldcg(&gs->amax_rot));
+      nf |= __ldcg(&gs->nonfinite);
+    }
+  }
+  mx = warp_max_f32(mx);
+  ar = warp_max_f32(ar);
+  nf = __any_sync(0xffffffffu, nf);
+  if (act && lane == 0) {
+    s_fmax[warp][0] = mx;
+    s_fmax[warp][1] = ar;
+    s_fnf[warp] = nf;
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  for (int w = 1; w < NW; ++w) {
+    mx = fmaxf(mx, s_fmax[w][0]);
+    ar = fmaxf(ar, s_fmax[w][1]);
+    nf |= s_fnf[w];
+  }
+  const double inf = __longlong_as_double(0x7ff0000000000000ll);
+  if (OP == OP_TDC) {
+    sb_module_state* st = a.st;
+    if (have_prev) st->delta = (S[1] == 0.0) ? inf : __ddiv_rn(S[0], S[1]);
+    st->n_out += 1;
+    st->acc = 0.0;
+    st->last_skipped = 0;
+    if (a.dsrc && a.dsrc->has_ref) {
+      st->prev_d = a.dsrc->d;
+      st->have_d = 1;
+    } else {
+      st->have_d = 0;
+    }
+    a.hdr->ticket[TICKET_TDC] = 0u;
+  } else {
+    const double numel = (double)a.M * (double)K;
+    const double ratio = (S[0] == 0.0) ? inf : __ddiv_rn((double)mx, __ddiv_rn(S[0], numel));
+    double d = 0.0;
+    if (REF) {
+      const double num = __dsqrt_rn(S[1]);
+      const double den = __dsqrt_rn(S[2]);
+      d = (den == 0.0) ? (num == 0.0 ? 0.0 : inf) : __ddiv_rn(num, den);
+    }
+    int pout = prec;
+    if (OP == OP_PREPASS && !a.force_int8 && a.mode == SB_PREPASS_QUANT && a.force < 0 &&
+        (prec == SB_NVFP4 || prec == SB_INT8) && ratio > a.rho)
+      pout = SB_BF16;
+    if (a.stats) {
+      sb_stats* so = a.stats;
+      so->sum_abs = S[0];
+      so->sum_d2 = S[1];
+      so->sum_ref2 = S[2];
+      so->max_abs = (double)mx;
+      so->amax_rot = (double)ar;
+      so->ratio = ratio;
+      so->d = d;
+      so->numel = numel;
+      so->has_ref = REF ? 1 : 0;
+      so->prec_in = prec;
+      so->prec_out = pout;
+      so->nonfinite = nf;
+    }
+    if (pout != prec && a.prec) *a.prec = pout;
+    if (nf) set_error(a.hdr, SB_ENONFINITE);
+    a.hdr->ticket[TICKET_PREPASS] = 0u;
+  }
+  __threadfence();
 }
 
 __device__ __forceinline__ void team_sync(int team, int T) {
@@ -308,8 +462,6 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   __shared__ float s_rowamax[2][kG];
   __shared__ float s_rowmax[2][kG];
   __shared__ int s_rownf[2][kG];
-  __shared__ int s_last;
-  __shared__ double s_fwarp[kRowWarps];
   __shared__ uint64_t s_bar[kRowWarps][4];
   extern __shared__ uint8_t dsm_raw[];
   // dynamic shared memory: the rings (1024-byte aligned for the swizzled boxes); the last CTA
@@ -317,8 +469,6 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~(uintptr_t)1023);
   double* s_fin = reinterpret_cast<double*>(ring);
   static_assert(RG::BYTES >= kFinChunk * 8, "final-reduction buffer");
-  __shared__ float s_fmax[kRowWarps][2];
-  __shared__ int s_fnf[kRowWarps];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int team = warp / T, wt = warp % T;
@@ -536,6 +686,10 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
             float2 f[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) f[k] = mul2(vr[c][k], inv2);
+            if (!(inv <= FLT_MAX)) {  // 127 / a_m overflowed: +-inf * y clamps to +-127, y = 0 gives 0
+#pragma unroll
+              for (int k = 0; k < 16; ++k) f[k] = make_float2(sign127(vr[c][k].x), sign127(vr[c][k].y));
+            }
             uint32_t w[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {  // word i = elements 4i..4i+3 (x halves for i < 4)
@@ -590,141 +744,7 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   // ring is reused or the CTA exits
   if (use_tma && bad_it >= 0 && lane == 0)
     mbar_wait_bounded(&s_bar[warp][bad_it % RG::D], (uint32_t)((bad_it / RG::D) & 1), nullptr, kRowDrainNs);
-  // ---- last CTA: tree over the groups (whole CTA, shared memory)
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const uint32_t tk = atomicAdd(&a.hdr->ticket[OP == OP_TDC ? TICKET_TDC : TICKET_PREPASS], 1u);
-    s_last = (tk == gridDim.x - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const int64_t G = ngroups;
-  double S[NST];
-  float mx = 0.0f, ar = 0.0f;
-  int nf = 0;
-  int64_t P = 256;
-  while (P < G) P <<= 1;
-  if (P <= 256 * 16) {
-    // One pass over the group slots for every statistic and maximum: thread t owns the aligned
-    // run [t R, (t + 1) R) of the zero-padded slots (R = P / 256 <= 16, padded to 16 with zeros),
-    // then the warp trees and the tree of the 8 warp sums -- the same halving tree as
-    // cta_pairwise_f64 with a single chunk.
-    const int R = (int)(P / 256);
-    double t3[NST][16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int64_t gi = (int64_t)threadIdx.x * R + k;
-      const bool in = k < R && gi < G;
-      const GroupSlot* gs = a.groups + (in ? gi : 0);
-#pragma unroll
-      for (int st = 0; st < NST; ++st) t3[st][k] = in ? __ldcg(&gs->s[st]) : 0.0;
-      if (in) {
-        mx = fmaxf(mx, __ldcg(&gs->max_abs));
-        ar = fmaxf(ar, __ldcg(&gs->amax_rot));
-        nf |= __ldcg(&gs->nonfinite);
-      }
-    }
-    double* s_w3 = s_fin;  // [warp][statistic]
-#pragma unroll
-    for (int st = 0; st < NST; ++st) {
-#pragma unroll
-      for (int len = 16; len > 1; len >>= 1) {
-#pragma unroll
-        for (int i = 0; i < len / 2; ++i) t3[st][i] = __dadd_rn(t3[st][2 * i], t3[st][2 * i + 1]);
-      }
-      const double wsum = warp_pairwise_f64(t3[st][0]);
-      if (lane == 0) s_w3[warp * NST + st] = wsum;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-#pragma unroll
-      for (int st = 0; st < NST; ++st) {
-        double u[8];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) u[w] = s_w3[w * NST + st];
-#pragma unroll
-        for (int len = 8; len > 1; len >>= 1) {
-#pragma unroll
-          for (int i = 0; i < len / 2; ++i) u[i] = __dadd_rn(u[2 * i], u[2 * i + 1]);
-        }
-        S[st] = u[0];
-      }
-    }
-  } else {
-#pragma unroll
-    for (int st = 0; st < NST; ++st)
-      S[st] = cta_pairwise_f64(&a.groups[0].s[st], sizeof(GroupSlot) / 8, G, s_fin, s_fwarp);
-    for (int64_t gg = threadIdx.x; gg < G; gg += blockDim.x) {
-      const GroupSlot* gs = a.groups + gg;
-      mx = fmaxf(mx, __ldcg(&gs->max_abs));
-      ar = fmaxf(ar, __ldcg(&gs->amax_rot));
-      nf |= __ldcg(&gs->nonfinite);
-    }
-  }
-  mx = warp_max_f32(mx);
-  ar = warp_max_f32(ar);
-  nf = __any_sync(0xffffffffu, nf);
-  if (lane == 0) {
-    s_fmax[warp][0] = mx;
-    s_fmax[warp][1] = ar;
-    s_fnf[warp] = nf;
-  }
-  __syncthreads();
-  if (threadIdx.x != 0) return;
-  for (int w = 1; w < kRowWarps; ++w) {
-    mx = fmaxf(mx, s_fmax[w][0]);
-    ar = fmaxf(ar, s_fmax[w][1]);
-    nf |= s_fnf[w];
-  }
-  const double inf = __longlong_as_double(0x7ff0000000000000ll);
-  if (OP == OP_TDC) {
-    sb_module_state* st = a.st;
-    if (have_prev) st->delta = (S[1] == 0.0) ? inf : __ddiv_rn(S[0], S[1]);
-    st->n_out += 1;
-    st->acc = 0.0;
-    st->last_skipped = 0;
-    if (a.dsrc && a.dsrc->has_ref) {
-      st->prev_d = a.dsrc->d;
-      st->have_d = 1;
-    } else {
-      st->have_d = 0;
-    }
-    a.hdr->ticket[TICKET_TDC] = 0u;
-  } else {
-    const double numel = (double)a.M * (double)K;
-    const double ratio = (S[0] == 0.0) ? inf : __ddiv_rn((double)mx, __ddiv_rn(S[0], numel));
-    double d = 0.0;
-    if (REF) {
-      const double num = __dsqrt_rn(S[1]);
-      const double den = __dsqrt_rn(S[2]);
-      d = (den == 0.0) ? (num == 0.0 ? 0.0 : inf) : __ddiv_rn(num, den);
-    }
-    int pout = prec;
-    if (OP == OP_PREPASS && !a.force_int8 && a.mode == SB_PREPASS_QUANT && a.force < 0 &&
-        (prec == SB_NVFP4 || prec == SB_INT8) && ratio > a.rho)
-      pout = SB_BF16;
-    if (a.stats) {
-      sb_stats* so = a.stats;
-      so->sum_abs = S[0];
-      so->sum_d2 = S[1];
-      so->sum_ref2 = S[2];
-      so->max_abs = (double)mx;
-      so->amax_rot = (double)ar;
-      so->ratio = ratio;
-      so->d = d;
-      so->numel = numel;
-      so->has_ref = REF ? 1 : 0;
-      so->prec_in = prec;
-      so->prec_out = pout;
-      so->nonfinite = nf;
-    }
-    if (pout != prec && a.prec) *a.prec = pout;
-    if (nf) set_error(a.hdr, SB_ENONFINITE);
-    a.hdr->ticket[TICKET_PREPASS] = 0u;
-  }
-  __threadfence();
+  rows_finish<OP, REF>(a, ngroups, prec, have_prev, s_fin);
 }
 
 // Team size T and segments per warp SPW for a row of K elements: T*SPW >= ceil(K/1024), SPW <= 3.

@@ -39,4 +39,22 @@ inline bool make_row_segment_map(CUtensorMap* m, const void* base, int64_t rows,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A [rows][K] bf16 row-major tensor (K a multiple of 64) seen as one column of 128-byte half
+// blocks: dims {64, rows * K / 64}; one box = 64 consecutive half blocks = 32 Hadamard blocks of
+// 128 channels (8 KB), 128B swizzle. Half blocks past the end read as zero. The half-block count
+// must fit a signed 32-bit coordinate.
+inline bool make_halfblock_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
+  auto fn = tmap_encoder();
+  if (!fn || K % 64 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
+  const int64_t n = rows * (K / 64);
+  if (n <= 0 || n >= (int64_t(1) << 31)) return false;
+  cuuint64_t dims[2] = {64, (cuuint64_t)n};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace sb
