@@ -184,6 +184,7 @@ sb_status sb_prepare_weight(const void* W, const void* bias, int64_t N, int64_t 
   q.codes = w->w4.codes;
   q.sf = w->w4.sf;
   q.gscale = w->w4.gscale;
+  q.hdr = ws;
   e = sb::launch_nvfp4(q, s);
   if (e != cudaSuccess) return cuda_fail(e, "sb_prepare_weight (NVFP4)");
   return ok();
@@ -256,6 +257,7 @@ sb_status sb_prepass(const void* X, const void* X_ref, int64_t M, int64_t K, con
     q.codes = a4->codes;
     q.sf = a4->sf;
     q.gscale = a4->gscale;
+    q.hdr = ws;
     e = sb::launch_nvfp4(q, s);
     if (e != cudaSuccess) return cuda_fail(e, "sb_prepass (NVFP4 encode)");
   }

@@ -128,6 +128,7 @@ struct Nvfp4Args {
   uint8_t* codes;
   uint8_t* sf;
   float* gscale;
+  WsHeader* hdr;
 };
 
 __device__ __forceinline__ int64_t sf_offset(int64_t m, int64_t g, int64_t K) {
@@ -206,6 +207,125 @@ __global__ void __launch_bounds__(256) k_nvfp4(Nvfp4Args a) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// NVFP4 encode with one 128-channel block per lane (B <= 128, K a multiple of 128): a lane's 8
+// scale groups are its own, so warps never meet. A warp encodes 32 consecutive blocks of the
+// row-padded tensor per task (TMA ring as in k_prepass_blk; rows past M read as zero, which writes
+// the zero scale factors of the padding rows).
+// ---------------------------------------------------------------------------------------------
+
+// Eight values -> one word of E2M1 codes: byte t holds values 2t (low nibble) and 2t + 1.
+__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                                           float v7) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
+      "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+      : "=r"(w)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+  return w;
+}
+
+template <int B>
+__global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB, const __grid_constant__ CUtensorMap mx) {
+  extern __shared__ uint8_t pb_dsm[];
+  __shared__ uint64_t s_bar[kPbWarps][kPbD];
+  if (a.prec && *a.prec != SB_NVFP4) return;
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pb_dsm) + 1023) & ~(uintptr_t)1023);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int K = a.K;
+  const float A = (float)a.stats->amax_rot;  // exact: a float widened to double
+  const float s_g = (A == 0.0f) ? 1.0f : __fdiv_rn(A, 2688.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.gscale = s_g;
+  const int64_t Mpad = (a.M + 127) & ~(int64_t)127;
+  const int64_t nblk = Mpad * NB;
+  const int ntask = (int)ceil_div(nblk, 32);
+  const int nw = (int)gridDim.x * kPbWarps;
+  const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * kPbD * kPbSlot);
+  auto issue = [&](int t, int slot) {  // lane 0
+    if (t >= ntask) return;
+    const uint32_t bar = smem_u32(&s_bar[warp][slot]);
+    mbar_arrive_expect_tx_u32(bar, (uint32_t)kPbSlot);
+    tma_load_2d_u32(ring_w + (uint32_t)(slot * kPbSlot), &mx, bar, 0, 64 * t);
+  };
+  const int t0 = (int)blockIdx.x * kPbWarps + warp;
+  if (lane == 0) {
+    mbar_init(&s_bar[warp][0], 1);
+    mbar_init(&s_bar[warp][1], 1);
+    fence_barrier_init();
+    issue(t0, 0);
+    issue(t0 + nw, 1);
+  }
+  __syncwarp();
+  int bad_it = -1;
+  for (int it = 0, t = t0; t < ntask; ++it, t += nw) {
+    const int slot = it & 1;
+    if (lane == 0 && it > 0) issue(t + nw, slot ^ 1);  // the previous task's slot, read there
+    if (!mbar_wait_bounded(&s_bar[warp][slot], (uint32_t)((it >> 1) & 1), nullptr, kRowWaitNs)) {
+      if (lane == 0) set_error(a.hdr, SB_ETIMEOUT);
+      bad_it = it;
+    }
+    float2 P[64];
+    pb_load_block(ring_w + (uint32_t)(slot * kPbSlot), lane, P);
+#pragma unroll
+    for (int k = 0; k < 64; k += 2) {
+      const float2 x = P[k], y = P[k + 1];
+      P[k] = add2(x, y);
+      P[k + 1] = sub2(x, y);
+    }
+    (void)pb_stages_rest<B>(P);
+    const int64_t f = (int64_t)t * 32 + lane;
+    if (f >= nblk) continue;
+    const int64_t m = f / NB;
+    const int blk = (int)(f - m * NB);
+    // groups i (elements 16i.., the x halves of P[16i..16i+15]) and i + 4 (the y halves)
+    uint32_t w[16];
+    uint32_t sbx = 0, sby = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float ax = 0.0f, ay = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 16; u += 2) {
+        ax = max3(ax, fabsf(P[16 * i + u].x), fabsf(P[16 * i + u + 1].x));
+        ay = max3(ay, fabsf(P[16 * i + u].y), fabsf(P[16 * i + u + 1].y));
+      }
+      uint32_t bx, by;
+      float ix, iy;
+      bool zx, zy;
+      group_scale(ax, s_g, &bx, &ix, &zx);
+      group_scale(ay, s_g, &by, &iy, &zy);
+      sbx |= bx << (8 * i);
+      sby |= by << (8 * i);
+      const float2 inv2 = make_float2(ix, iy);
+      float2 q[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) q[u] = mul2(P[16 * i + u], inv2);
+      w[2 * i] = zx ? 0u : e2m1x8(q[0].x, q[1].x, q[2].x, q[3].x, q[4].x, q[5].x, q[6].x, q[7].x);
+      w[2 * i + 1] = zx ? 0u : e2m1x8(q[8].x, q[9].x, q[10].x, q[11].x, q[12].x, q[13].x, q[14].x, q[15].x);
+      w[8 + 2 * i] = zy ? 0u : e2m1x8(q[0].y, q[1].y, q[2].y, q[3].y, q[4].y, q[5].y, q[6].y, q[7].y);
+      w[9 + 2 * i] = zy ? 0u : e2m1x8(q[8].y, q[9].y, q[10].y, q[11].y, q[12].y, q[13].y, q[14].y, q[15].y);
+    }
+    if (m < a.M) {
+      uint8_t* dst = a.codes + m * (K >> 1) + (int64_t)blk * 64;
+      if (aligned32(dst)) {
+        stg_v8(dst, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+        stg_v8(dst + 32, make_uint4(w[8], w[9], w[10], w[11]), make_uint4(w[12], w[13], w[14], w[15]));
+      } else {
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
+    }
+    *reinterpret_cast<uint32_t*>(a.sf + sf_offset(m, 8 * (int64_t)blk, K)) = sbx;
+    *reinterpret_cast<uint32_t*>(a.sf + sf_offset(m, 8 * (int64_t)blk + 4, K)) = sby;
+  }
+  if (bad_it >= 0 && lane == 0)
+    mbar_wait_bounded(&s_bar[warp][bad_it & 1], (uint32_t)((bad_it >> 1) & 1), nullptr, kRowDrainNs);
+}
+
+// ---------------------------------------------------------------------------------------------
 // Rotation only
 // ---------------------------------------------------------------------------------------------
 
@@ -252,7 +372,30 @@ cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s) {
   a.codes = p.codes;
   a.sf = p.sf;
   a.gscale = p.gscale;
-  const int64_t units = ((p.M + 127) & ~(int64_t)127) * ceil_div(p.K, 1024);
+  a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
+  const int64_t Mpad = (p.M + 127) & ~(int64_t)127;
+  CUtensorMap mx;
+  if (p.B <= 128 && p.K % 128 == 0 && p.B >= 16 && Mpad * (p.K / 64) < (int64_t(1) << 31) &&
+      make_halfblock_map(&mx, p.X, p.M, p.K)) {
+    constexpr int dsm = kPbRing + 1024;
+    const int NB = (int)(p.K / 128);
+    const int64_t tasks = ceil_div(Mpad * NB, 32);
+    const int64_t want = ceil_div(tasks, kPbWarps);
+    const unsigned grid = (unsigned)(want < sm_count() ? want : sm_count());
+    auto go = [&](auto kern) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
+      kern<<<grid, kPbThreads, dsm, s>>>(a, NB, mx);
+      return cudaGetLastError();
+    };
+    switch (p.B) {
+      case 16: return go(k_nvfp4_blk<16>);
+      case 32: return go(k_nvfp4_blk<32>);
+      case 64: return go(k_nvfp4_blk<64>);
+      case 128: return go(k_nvfp4_blk<128>);
+      default: break;
+    }
+  }
+  const int64_t units = Mpad * ceil_div(p.K, 1024);
   k_nvfp4<<<stream_grid(units), 256, 0, s>>>(a);
   return cudaGetLastError();
 }

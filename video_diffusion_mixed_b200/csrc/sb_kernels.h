@@ -35,6 +35,7 @@ struct Nvfp4Launch {
   uint8_t* codes;
   uint8_t* sf;
   float* gscale;
+  void* hdr;  // workspace header: error word
 };
 
 struct TdcLaunch {
