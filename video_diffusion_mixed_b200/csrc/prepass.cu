@@ -57,6 +57,18 @@ static void row_maps(RowArgs& a, RowMaps& mp, const void* X, const void* R) {
   a.tma = make_row_segment_map(&mp.x, X, a.M, a.K) && (!R || make_row_segment_map(&mp.r, R, a.M, a.K)) ? 1 : 0;
 }
 
+template <int B>
+static cudaError_t launch_pb(const RowArgs& a, const PbGeom& gm, const CUtensorMap& mx, unsigned grid, cudaStream_t s) {
+  constexpr int dsm = kPbRing + 1024;
+  static bool attr = false;  // once per instantiation
+  if (!attr) {
+    cudaFuncSetAttribute(k_prepass_blk<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
+    attr = true;
+  }
+  k_prepass_blk<B><<<grid, kPbThreads, dsm, s>>>(a, gm, mx);
+  return cudaGetLastError();
+}
+
 // The block-per-lane pre-pass (k_prepass_blk): no x_ref, B <= 128, whole 128-channel blocks and a
 // team shape and tensor map that fit. Returns false (nothing launched) otherwise.
 static bool launch_prepass_blk(const RowArgs& a, cudaStream_t s, int sms, cudaError_t* err) {
@@ -65,20 +77,13 @@ static bool launch_prepass_blk(const RowArgs& a, cudaStream_t s, int sms, cudaEr
   if (!pick_pb_geom(a.K / 128, &gm)) return false;
   CUtensorMap mx;
   if (!make_halfblock_map(&mx, a.X, a.M, a.K)) return false;
-  constexpr int dsm = kPbRing + 1024;
   const int64_t groups = ceil_div(a.M, kG);  // a team's unit of work
   const unsigned grid = (unsigned)(groups < sms ? groups : sms);
-  auto go = [&](auto kern) {
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
-    kern<<<grid, kPbThreads, dsm, s>>>(a, gm, mx);
-    *err = cudaGetLastError();
-    return true;
-  };
   switch (a.B) {
-    case 16: return go(k_prepass_blk<16>);
-    case 32: return go(k_prepass_blk<32>);
-    case 64: return go(k_prepass_blk<64>);
-    case 128: return go(k_prepass_blk<128>);
+    case 16: *err = launch_pb<16>(a, gm, mx, grid, s); return true;
+    case 32: *err = launch_pb<32>(a, gm, mx, grid, s); return true;
+    case 64: *err = launch_pb<64>(a, gm, mx, grid, s); return true;
+    case 128: *err = launch_pb<128>(a, gm, mx, grid, s); return true;
     default: return false;
   }
 }
@@ -361,6 +366,18 @@ static unsigned stream_grid(int64_t units) {
   return (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
+template <int B>
+static cudaError_t launch_nvfp4_blk(const Nvfp4Args& a, int NB, const CUtensorMap& mx, unsigned grid, cudaStream_t s) {
+  constexpr int dsm = kPbRing + 1024;
+  static bool attr = false;  // once per instantiation
+  if (!attr) {
+    cudaFuncSetAttribute(k_nvfp4_blk<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
+    attr = true;
+  }
+  k_nvfp4_blk<B><<<grid, kPbThreads, dsm, s>>>(a, NB, mx);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s) {
   Nvfp4Args a{};
   a.X = reinterpret_cast<const __nv_bfloat16*>(p.X);
@@ -377,21 +394,15 @@ cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s) {
   CUtensorMap mx;
   if (p.B <= 128 && p.K % 128 == 0 && p.B >= 16 && Mpad * (p.K / 64) < (int64_t(1) << 31) &&
       make_halfblock_map(&mx, p.X, p.M, p.K)) {
-    constexpr int dsm = kPbRing + 1024;
     const int NB = (int)(p.K / 128);
     const int64_t tasks = ceil_div(Mpad * NB, 32);
     const int64_t want = ceil_div(tasks, kPbWarps);
     const unsigned grid = (unsigned)(want < sm_count() ? want : sm_count());
-    auto go = [&](auto kern) {
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
-      kern<<<grid, kPbThreads, dsm, s>>>(a, NB, mx);
-      return cudaGetLastError();
-    };
     switch (p.B) {
-      case 16: return go(k_nvfp4_blk<16>);
-      case 32: return go(k_nvfp4_blk<32>);
-      case 64: return go(k_nvfp4_blk<64>);
-      case 128: return go(k_nvfp4_blk<128>);
+      case 16: return launch_nvfp4_blk<16>(a, NB, mx, grid, s);
+      case 32: return launch_nvfp4_blk<32>(a, NB, mx, grid, s);
+      case 64: return launch_nvfp4_blk<64>(a, NB, mx, grid, s);
+      case 128: return launch_nvfp4_blk<128>(a, NB, mx, grid, s);
       default: break;
     }
   }
