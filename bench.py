@@ -38,14 +38,17 @@ METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT sh
 # tokens (every term grows with the token count), for the ffn5b workload at full size only. An
 # entry is valid only for the sources it was measured on (sha over the listed files of csrc/).
 _GEMM_SRC = ("gemm.cu", "sb_device.cuh")
-_ROWS_SRC = ("prepass.cu", "rows.cuh", "sb_device.cuh")
+_ROWS_SRC = ("prepass.cu", "rows.cuh", "prepass_blk.cuh", "sb_device.cuh", "tmap.h")
 TRAFFIC = {
-    "gemm_w1_int8": {"bytes": 750.6e6, "files": _GEMM_SRC, "sha": "c7275c8b5a60ac65"},
-    "gemm_w2_int8": {"bytes": 795.5e6, "files": _GEMM_SRC, "sha": "c7275c8b5a60ac65"},
-    "gemm_w1_nvfp4": {"bytes": 496.0e6, "files": _GEMM_SRC, "sha": "c7275c8b5a60ac65"},
-    "gemm_w2_nvfp4": {"bytes": 279.0e6, "files": _GEMM_SRC, "sha": "c7275c8b5a60ac65"},
-    "prepass_h_nvfp4": {"bytes": 974.7e6, "files": _ROWS_SRC, "sha": "25c4aecd182a1187"},  # k_rows + k_nvfp4
-    "prepass_h_int8": {"bytes": 575.2e6, "files": _ROWS_SRC, "sha": "25c4aecd182a1187"},
+    "gemm_w1_int8": {"bytes": 739.4e6, "files": _GEMM_SRC, "sha": "2f9a3737d827dbc7"},
+    "gemm_w2_int8": {"bytes": 795.8e6, "files": _GEMM_SRC, "sha": "2f9a3737d827dbc7"},
+    "gemm_w1_nvfp4": {"bytes": 486.1e6, "files": _GEMM_SRC, "sha": "2f9a3737d827dbc7"},
+    "gemm_w2_nvfp4": {"bytes": 264.5e6, "files": _GEMM_SRC, "sha": "2f9a3737d827dbc7"},
+    # k_prepass_blk + k_nvfp4_blk (the encode exits at once in the INT8 pass)
+    "prepass_h_nvfp4": {"bytes": 940.7e6, "files": _ROWS_SRC, "sha": "01321ae6d175034e"},
+    "prepass_h_int8": {"bytes": 578.1e6, "files": _ROWS_SRC, "sha": "01321ae6d175034e"},
+    "prepass_x_nvfp4": {"bytes": 218.9e6, "files": _ROWS_SRC, "sha": "01321ae6d175034e"},
+    "prepass_x_int8": {"bytes": 111.6e6, "files": _ROWS_SRC, "sha": "01321ae6d175034e"},
 }
 TRAFFIC_TOKENS = 17776
 

@@ -280,12 +280,13 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB
       P[k] = add2(x, y);
       P[k + 1] = sub2(x, y);
     }
-    (void)pb_stages_rest<B>(P);
+    (void)pb_stages_rest<B>(P, lane);
     const int64_t f = (int64_t)t * 32 + lane;
     if (f >= nblk) continue;
     const int64_t m = f / NB;
     const int blk = (int)(f - m * NB);
-    // groups i (elements 16i.., the x halves of P[16i..16i+15]) and i + 4 (the y halves)
+    // groups i (elements 16i.., the x halves of P[16i..16i+15]) and i + 4 (the y halves); a
+    // swapped lane's halves are the other way round, which only moves where they are stored
     uint32_t w[16];
     uint32_t sbx = 0, sby = 0;
 #pragma unroll
@@ -312,19 +313,24 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB
       w[8 + 2 * i] = zy ? 0u : e2m1x8(q[0].y, q[1].y, q[2].y, q[3].y, q[4].y, q[5].y, q[6].y, q[7].y);
       w[9 + 2 * i] = zy ? 0u : e2m1x8(q[8].y, q[9].y, q[10].y, q[11].y, q[12].y, q[13].y, q[14].y, q[15].y);
     }
+    const int hx = (int)pb_swap(lane), hy = 1 - hx;  // which half of the block x and y are
     if (m < a.M) {
       uint8_t* dst = a.codes + m * (K >> 1) + (int64_t)blk * 64;
       if (aligned32(dst)) {
-        stg_v8(dst, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
-        stg_v8(dst + 32, make_uint4(w[8], w[9], w[10], w[11]), make_uint4(w[12], w[13], w[14], w[15]));
+        stg_v8(dst + 32 * hx, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+        stg_v8(dst + 32 * hy, make_uint4(w[8], w[9], w[10], w[11]), make_uint4(w[12], w[13], w[14], w[15]));
       } else {
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-          *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        for (int v = 0; v < 2; ++v) {
+          *reinterpret_cast<uint4*>(dst + 32 * hx + 16 * v) =
+              make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          *reinterpret_cast<uint4*>(dst + 32 * hy + 16 * v) =
+              make_uint4(w[8 + 4 * v], w[9 + 4 * v], w[10 + 4 * v], w[11 + 4 * v]);
+        }
       }
     }
-    *reinterpret_cast<uint32_t*>(a.sf + sf_offset(m, 8 * (int64_t)blk, K)) = sbx;
-    *reinterpret_cast<uint32_t*>(a.sf + sf_offset(m, 8 * (int64_t)blk + 4, K)) = sby;
+    *reinterpret_cast<uint32_t*>(a.sf + sf_offset(m, 8 * (int64_t)blk + 4 * hx, K)) = sbx;
+    *reinterpret_cast<uint32_t*>(a.sf + sf_offset(m, 8 * (int64_t)blk + 4 * hy, K)) = sby;
   }
   if (bad_it >= 0 && lane == 0)
     mbar_wait_bounded(&s_bar[warp][bad_it & 1], (uint32_t)((bad_it >> 1) & 1), nullptr, kRowDrainNs);

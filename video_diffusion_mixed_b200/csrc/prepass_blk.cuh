@@ -9,7 +9,9 @@
 // Layout: a lane owns one whole 128-element block, so all butterfly stages run inside its
 // registers and no value crosses lanes. Its 128 values live as 64 packed pairs
 // P[k] = (v[k], v[k + 64]): FP32x2 arithmetic covers the stages h = 1..32, the stage h = 64 pairs
-// the two halves of each P[k]. A "team" of T warps (T | 12) owns R rows at a time (R | kG), their
+// the two halves of each P[k]. Lanes 4..7 of every eight hold the halves the other way round,
+// P[k] = (v[k + 64], v[k]) (see pb_load_block); every step but the stage h = 64 and the final
+// stores treats the two halves alike. A "team" of T warps (T | 12) owns R rows at a time (R | kG), their
 // R NB blocks laid out flat over its 32 T lanes (a row may straddle warps; idle lanes compute on
 // whatever the box holds and write nothing). Per task the team meets once at a named barrier:
 // row maxima go through shared-memory atomics, block sums through a shared buffer that one warp
@@ -72,13 +74,20 @@ inline bool pick_pb_geom(int NB, PbGeom* g) {
 
 // The lane's 128 values from its two swizzled half blocks in the slot: half block r = 2 lane + h
 // holds elements 64 h .. 64 h + 63; its 16-byte chunk c sits at chunk position c ^ (r & 7).
+// Lanes with swp = 1 (lanes 4..7 of every eight) read their upper half first, so the eight lanes
+// of each 128-bit load phase touch half blocks with eight different (r & 7): no bank conflicts.
+// Their pairs come out as (v[k + 64], v[k]).
+__device__ __forceinline__ uint32_t pb_swap(int lane) { return ((uint32_t)lane >> 2) & 1u; }
+
 __device__ __forceinline__ void pb_load_block(uint32_t slot, int lane, float2 (&P)[64]) {
-  const uint32_t base = slot + (uint32_t)lane * 256u;
-  const uint32_t sw0 = (2u * (uint32_t)lane) & 7u, sw1 = (2u * (uint32_t)lane + 1u) & 7u;
+  const uint32_t swp = pb_swap(lane);
+  const uint32_t r0 = 2u * (uint32_t)lane + swp, r1 = 2u * (uint32_t)lane + 1u - swp;
+  const uint32_t b0 = slot + 128u * r0, b1 = slot + 128u * r1;
+  const uint32_t sw0 = r0 & 7u, sw1 = r1 & 7u;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
-    const uint4 u0 = ld_shared_v4(base + 16u * ((uint32_t)c ^ sw0));
-    const uint4 u1 = ld_shared_v4(base + 128u + 16u * ((uint32_t)c ^ sw1));
+    const uint4 u0 = ld_shared_v4(b0 + 16u * ((uint32_t)c ^ sw0));
+    const uint4 u1 = ld_shared_v4(b1 + 16u * ((uint32_t)c ^ sw1));
     const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w};
     const uint32_t w1[4] = {u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
@@ -124,9 +133,11 @@ __device__ __forceinline__ float pb_stage1_raw(float2 (&P)[64], float* rmax) {
 
 // Stages h = 2 .. 64 (each while h < B) and the block's rotated amax. B is a template argument:
 // stages chosen at run time would force the compiler to reconcile the pairs' registers at every
-// join and spill.
+// join and spill. The stage h = 64 adds and subtracts the halves of each pair as one fused
+// multiply-add by +-1 each (exact product, one rounding): (x + y, x - y) for a pair (lower, upper)
+// and (y - x, y + x) for a swapped pair (upper, lower) -- the same two results in swapped places.
 template <int B>
-__device__ __forceinline__ float pb_stages_rest(float2 (&P)[64]) {
+__device__ __forceinline__ float pb_stages_rest(float2 (&P)[64], int lane) {
 #pragma unroll
   for (int h = 2; h <= 32; h <<= 1) {
     if (h < B) {
@@ -142,9 +153,10 @@ __device__ __forceinline__ float pb_stages_rest(float2 (&P)[64]) {
   }
   float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent chains
   if (64 < B) {
+    const float cx = pb_swap(lane) ? -1.0f : 1.0f, cy = -cx;
 #pragma unroll
     for (int k = 0; k < 64; ++k) {
-      const float s = __fadd_rn(P[k].x, P[k].y), d = __fsub_rn(P[k].x, P[k].y);
+      const float s = __fmaf_rn(cx, P[k].x, P[k].y), d = __fmaf_rn(cy, P[k].y, P[k].x);
       P[k] = make_float2(s, d);
       am[k & 3] = max3(am[k & 3], fabsf(s), fabsf(d));
     }
@@ -167,8 +179,9 @@ __device__ __forceinline__ uint32_t pb_pack4(float a, float b, float c, float d)
 
 __device__ __forceinline__ uint32_t pb_sign_code(float v) { return v > 0.0f ? 127u : (v < 0.0f ? 0x81u : 0u); }
 
-__device__ __forceinline__ void pb_store_int8(float2 (&P)[64], float a_m, int8_t* dst) {
+__device__ __forceinline__ void pb_store_int8(float2 (&P)[64], float a_m, int8_t* dst, int lane) {
   const float inv = (a_m == 0.0f) ? 0.0f : __fdiv_rn(127.0f, a_m);
+  const int64_t ox = pb_swap(lane) ? 64 : 0, oy = 64 - ox;  // where the x and y halves go
   const bool finite = inv <= FLT_MAX;
   const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
@@ -194,8 +207,8 @@ __device__ __forceinline__ void pb_store_int8(float2 (&P)[64], float a_m, int8_t
         wy[v] = y;
       }
     }
-    *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(wx[0], wx[1], wx[2], wx[3]);
-    *reinterpret_cast<uint4*>(dst + 64 + 4 * i) = make_uint4(wy[0], wy[1], wy[2], wy[3]);
+    *reinterpret_cast<uint4*>(dst + ox + 4 * i) = make_uint4(wx[0], wx[1], wx[2], wx[3]);
+    *reinterpret_cast<uint4*>(dst + oy + 4 * i) = make_uint4(wy[0], wy[1], wy[2], wy[3]);
   }
 }
 
@@ -297,7 +310,7 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
 
     float rmax;
     const float bsum = pb_stage1_raw(P, &rmax);
-    const float am = pb_stages_rest<B>(P);
+    const float am = pb_stages_rest<B>(P, lane);
 
     // ---- row maxima and sums of aligned runs of SUB blocks, then the team meets
     const uint32_t amb = __reduce_max_sync(rowmask, __float_as_uint(am));
@@ -313,7 +326,7 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
 
     const int m = m0 + rl;
     if (do_int8 && qv && m < a.M)
-      pb_store_int8(P, __uint_as_float(s_ram[tb][team][rl]), a.q8 + ((int64_t)m * NB + blk) * 128);
+      pb_store_int8(P, __uint_as_float(s_ram[tb][team][rl]), a.q8 + ((int64_t)m * NB + blk) * 128, lane);
 
     // ---- one warp of the team: row sums, the task's rows into the group, the group's slot
     if (wt == dw) {
