@@ -20,7 +20,8 @@
  *           across rows: the same pairwise tree in FP64 over the row partials.
  *   R-D     d = sqrt(sum (y - x)^2) / sqrt(sum x^2), FP64.
  *   R-PDR   ratio = max|x| / (sum|x| / numel) on the raw (unrotated) layer input, FP64.
- *   R-INT8  symmetric per-token: s = a / 127, q = clamp(rne(y * (127 / a)), -127, 127), FP32.
+ *   R-INT8  symmetric per-token: s = a / 127, q = clamp(rne(y * (127 / a)), -127, 127), FP32;
+ *           when 127 / a overflows, y = 0 gives 0 (its exact product) instead of 0 * inf.
  *   R-FP4   NVFP4: E2M1 codes, one E4M3 scale per 16 elements, FP32 tensor scale A / (6 * 448).
  *   R-RULE  INT8 iff a * d_prev + b > tau (FP64, no fused multiply-add); restart -> INT8.
  *   R-TDC   delta = sum|y_new - y_last| / sum|y_last|; acc += delta each later step;
