@@ -226,3 +226,19 @@ def test_prepass_hidden_full_size(sbg):
     codes, sfl, sft, sg = oracle.quant_nvfp4(ref["y"], ref["amax_rot"])
     assert np.array_equal(npy(out4["a4"].codes), codes)
     assert np.array_equal(npy(out4["a4"].sf), sft)
+
+
+@pytest.mark.parametrize("K,B,with_ref", [(128, 128, False), (256, 256, False), (128, 128, True)])
+def test_prepass_many_groups(sbg, K, B, with_ref):
+    """More than 4096 groups of 16 rows (70001 tokens): the last CTA folds the FP64 group sums in
+    several chunks of its shared buffer (both pre-pass kernels, with and without x_ref)."""
+    M = 70001
+    X = synth.activations(M, K, n_outlier=1, scale=30.0, seed=9, device="cuda")
+    R = synth.activations(M, K, seed=10, device="cuda") if with_ref else None
+    ref = oracle.prepass(u16(X), u16(R) if R is not None else None, B)
+    out = run_prepass(sbg, X, R, force=sbg.INT8, block=B)
+    for k in STATS:
+        assert out["stats"][k] == ref[k], (k, out["stats"][k], ref[k])
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    assert np.array_equal(npy(out["a8"].codes), q)
+    assert np.array_equal(npy(out["a8"].scale).view(np.uint32), s.view(np.uint32))

@@ -24,7 +24,8 @@ def gstate_dict(sb, st):
     return {k: d[k] for k in ("prev_d", "acc", "delta", "have_d", "n_out", "last_skipped", "skip")}
 
 
-@pytest.mark.parametrize("M,C", [(1, 8), (33, 1920), (256, 3072), (100, 12288)])
+# (70001, 64): more than 4096 groups of 16 rows, so the last CTA folds the group sums in chunks
+@pytest.mark.parametrize("M,C", [(1, 8), (33, 1920), (256, 3072), (100, 12288), (70001, 64)])
 def test_tdc_record_delta_bitexact(sbg, M, C):
     ws = sbg.Workspace(M, C)
     st = sbg.alloc_state()

@@ -125,12 +125,38 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
+// FP32x2 arithmetic for the epilogue (one instruction, two lanes of FP32 work; the epilogue's
+// outputs are compared with a tolerance, so contraction is allowed here).
+__device__ __forceinline__ uint64_t ep_bits(float2 a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+  return r;
+}
+__device__ __forceinline__ float2 ep_f2(uint64_t r) {
+  float2 a;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
+  return a;
+}
+__device__ __forceinline__ float2 ep_mul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ep_bits(a)), "l"(ep_bits(b)));
+  return ep_f2(r);
+}
+__device__ __forceinline__ float2 ep_fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(ep_bits(a)), "l"(ep_bits(b)), "l"(ep_bits(c)));
+  return ep_f2(r);
+}
+
 // tanh-form GELU, 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), with the SFU's tanh
-// approximation (relative error about 2^-11, below the 2^-9 rounding of the bf16 output).
-__device__ __forceinline__ float gelu_tanh(float v) {
-  const float u = v * fmaf(0.7978845608028654f * 0.044715f, v * v, 0.7978845608028654f);
-  const float h = 0.5f * v;
-  return fmaf(h, tanh_approx(u), h);
+// approximation (relative error about 2^-11, below the 2^-9 rounding of the bf16 output), on two
+// values at a time.
+__device__ __forceinline__ float2 gelu_tanh2(float2 v) {
+  const float2 c1 = make_float2(0.7978845608028654f * 0.044715f, 0.7978845608028654f * 0.044715f);
+  const float2 c0 = make_float2(0.7978845608028654f, 0.7978845608028654f);
+  const float2 u = ep_mul2(v, ep_fma2(c1, ep_mul2(v, v), c0));
+  const float2 h = ep_mul2(make_float2(0.5f, 0.5f), v);
+  return ep_fma2(h, make_float2(tanh_approx(u.x), tanh_approx(u.y)), h);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -176,27 +202,33 @@ __device__ __forceinline__ void load_colops(const GemmParams& p, int n, ColOps<K
 }
 
 // Epilogue arithmetic of 32 accumulator columns of one row, in place: the accumulator words become
-// the FP32 outputs. Dequant scale and bias are one FMA, then the optional GELU.
+// the FP32 outputs. Dequant scale and bias are one FMA, then the optional GELU; columns go in
+// pairs through FP32x2 arithmetic.
 template <int KIND>
 __device__ __forceinline__ void epilogue_math(const GemmParams& p, const ColOps<KIND>& o, float sxb, float alpha,
                                               uint32_t (&r)[32]) {
   const bool has_bias = p.bias != nullptr, gelu = p.epilogue == SB_EPI_GELU_TANH;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint32_t w = (i & 7) < 2 ? o.b[i >> 3].x : (i & 7) < 4 ? o.b[i >> 3].y : (i & 7) < 6 ? o.b[i >> 3].z : o.b[i >> 3].w;
-    const float bias = has_bias ? __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16)) : 0.0f;
-    float y;
+  for (int j = 0; j < 16; ++j) {  // columns 2j, 2j + 1
+    const uint4 bq = o.b[j >> 2];
+    const uint32_t w = (j & 3) == 0 ? bq.x : (j & 3) == 1 ? bq.y : (j & 3) == 2 ? bq.z : bq.w;
+    const float2 bias = has_bias ? make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u))
+                                 : make_float2(0.0f, 0.0f);
+    float2 y;
     if constexpr (KIND == KIND_I8) {
-      const float4 sc = o.s[i >> 2];
-      const float c = (i & 3) == 0 ? sc.x : (i & 3) == 1 ? sc.y : (i & 3) == 2 ? sc.z : sc.w;
-      y = fmaf(__int2float_rn((int)r[i]), sxb * c, bias);
+      const float4 sc = o.s[j >> 1];
+      const float2 c = (j & 1) ? make_float2(sc.z, sc.w) : make_float2(sc.x, sc.y);
+      const float2 acc = make_float2(__int2float_rn((int)r[2 * j]), __int2float_rn((int)r[2 * j + 1]));
+      y = ep_fma2(acc, ep_mul2(make_float2(sxb, sxb), c), bias);
     } else if constexpr (KIND == KIND_FP4) {
-      y = fmaf(__uint_as_float(r[i]), alpha, bias);
+      y = ep_fma2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), make_float2(alpha, alpha),
+                  bias);
     } else {
-      y = __uint_as_float(r[i]) + bias;
+      y = make_float2(__uint_as_float(r[2 * j]) + bias.x, __uint_as_float(r[2 * j + 1]) + bias.y);
     }
-    if (gelu) y = gelu_tanh(y);
-    r[i] = __float_as_uint(y);
+    if (gelu) y = gelu_tanh2(y);
+    r[2 * j] = __float_as_uint(y.x);
+    r[2 * j + 1] = __float_as_uint(y.y);
   }
 }
 
