@@ -55,6 +55,7 @@ def lib():
             "orc_pairwise_f64": (f64, [vp, i64]),
             "orc_prepass": (None, [vp, vp, i64, i64, i32, vp, vp, vp, vp]),
             "orc_quant_int8": (None, [vp, i64, i64, vp, vp, vp]),
+            "orc_chunk_stats": (None, [vp, i64, i64, i32, vp]),
             "orc_e2m1_decode": (f32, [ctypes.c_uint8]),
             "orc_e2m1_encode": (ctypes.c_uint8, [f32]),
             "orc_e4m3_decode": (f32, [ctypes.c_uint8]),
@@ -204,6 +205,17 @@ def prepass(x_bf16, xref_bf16=None, B: int = 128, want_rot: bool = True):
     out = np.zeros(8, dtype=np.float64)
     lib().orc_prepass(_P(x), _P(r), M, K, B, _P(y), _P(amax), _P(part), _P(out))
     return {"y": y, "row_amax": amax, "row_part": part, **{n: float(out[i]) for i, n in enumerate(STAT_NAMES)}}
+
+
+def chunk_stats(x_bf16, B: int = 128) -> np.ndarray:
+    """Per aligned 128-channel chunk of every row: [M, K/128, 3] float32 of (max |H_B x|, canonical
+    pairwise sum |x|, max |x|) -- the records the first FFN layer's epilogue hands to the second
+    layer's pre-pass."""
+    x = _u16(x_bf16)
+    M, K = x.shape
+    out = np.empty((M, K // 128, 3), dtype=np.float32)
+    lib().orc_chunk_stats(_P(x), M, K, B, _P(out))
+    return out
 
 
 def quant_int8(y: np.ndarray, row_amax: np.ndarray):

@@ -229,6 +229,40 @@ void orc_prepass(const uint16_t* X, const uint16_t* Xref, int64_t M, int64_t K, 
   if (!row_part) free(rp);
 }
 
+/* Statistics of every aligned 128-channel chunk of every row (K a multiple of 128, B | 128):
+ * out[(m * (K / 128) + c) * 3 + i] for chunk c of row m is
+ *   i = 0: max over the chunk of |H_B x| (its B-blocks rotated as in R-H),
+ *   i = 1: sum of |x| over the chunk's 128 values in the canonical pairwise order (R-RED),
+ *   i = 2: max |x|.
+ * A chunk is an aligned subtree of its row's sum tree, so these records carry everything the
+ * pre-pass needs from the row; they are what the first FFN layer's epilogue produces for the
+ * second layer's pre-pass ("write-up" section 四: quantization work fused into the layers). */
+void orc_chunk_stats(const uint16_t* x, int64_t M, int64_t K, int B, float* out) {
+  const int64_t NC = K / 128;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t c = 0; c < NC; ++c) {
+      float v[128], a[128];
+      float mx = 0.0f;
+      for (int i = 0; i < 128; ++i) {
+        v[i] = bf16_to_f32(x[m * K + c * 128 + i]);
+        a[i] = fabsf(v[i]);
+        if (a[i] > mx) mx = a[i];
+      }
+      for (int len = 128; len > 1; len >>= 1)
+        for (int i = 0; i < len / 2; ++i) a[i] = a[2 * i] + a[2 * i + 1];
+      for (int j = 0; j < 128; j += B) orc_fwht_f32(v + j, B);
+      float am = 0.0f;
+      for (int i = 0; i < 128; ++i)
+        if (fabsf(v[i]) > am) am = fabsf(v[i]);
+      float* o = out + (m * NC + c) * 3;
+      o[0] = am;
+      o[1] = a[0];
+      o[2] = mx;
+    }
+  }
+}
+
 /* ------------------------------------------------------------------------------------------ */
 /* R-INT8                                                                                      */
 /* ------------------------------------------------------------------------------------------ */

@@ -193,6 +193,44 @@ def test_int8_quant_overflowing_reciprocal(orc):
     assert s[0] == np.float32(a / np.float32(127))
 
 
+def test_chunk_stats_closed_forms(orc):
+    """Chunk records against exact arithmetic: small integers make every FP32 sum exact, so the
+    rotated amax is max |x H_B^T| from the explicit +-1 matrix and the sum is the integer sum."""
+    rng = np.random.default_rng(21)
+    M, K = 5, 512
+    xi = rng.integers(-8, 9, size=(M, K))
+    xi[2] = 0
+    xi[3, :] = 1  # a constant row: the rotation puts 128 (B = 128) or B in the first slot of a block
+    x = orc.f32_to_bf16(xi.astype(np.float32))
+    for B in (16, 128):
+        H = np.array([[orc.hadamard_entry(i, j) for j in range(B)] for i in range(B)], dtype=np.int64)
+        cs = orc.chunk_stats(x, B)
+        assert cs.shape == (M, K // 128, 3)
+        for m in range(M):
+            for c in range(K // 128):
+                v = xi[m, 128 * c:128 * (c + 1)]
+                rot = (v.reshape(-1, B) @ H.T).ravel()
+                assert cs[m, c, 0] == np.abs(rot).max()
+                assert cs[m, c, 1] == np.abs(v).sum()
+                assert cs[m, c, 2] == np.abs(v).max()
+        assert (cs[3, :, 0] == B).all() and (cs[3, :, 1] == 128).all() and not cs[2].any()
+
+
+def test_chunk_stats_fold_to_the_row_statistics(orc):
+    """The chunks are aligned subtrees of each row's pairwise tree: folding a row's chunk sums
+    (zero-padded to a power of two) gives the pre-pass row sum bit for bit, and the chunk maxima
+    give the per-token rotated amax and the raw max."""
+    rng = np.random.default_rng(22)
+    M, K = 7, 12288
+    x = orc.f32_to_bf16((rng.standard_normal((M, K)) * rng.uniform(0.01, 40.0, (M, 1))).astype(np.float32))
+    cs = orc.chunk_stats(x, 128)
+    ref = orc.prepass(x, None, 128)
+    for m in range(M):
+        assert np.float32(orc.pairwise_f32(cs[m, :, 1])) == ref["row_part"][m, 0]
+        assert cs[m, :, 0].max() == ref["row_amax"][m]
+    assert float(cs[:, :, 2].max()) == ref["max_abs"]
+
+
 def test_nvfp4_quant_properties(orc):
     rng = np.random.default_rng(6)
     y = (rng.standard_normal((9, 128)) * rng.uniform(0.01, 30, (9, 1))).astype(np.float32)
