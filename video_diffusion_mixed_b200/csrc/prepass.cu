@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB
       P[k] = add2(x, y);
       P[k + 1] = sub2(x, y);
     }
-    (void)pb_stages_rest<B>(P, lane);
+    (void)pb_stages_rest<B>(P, pb_swap(lane) ? -1.0f : 1.0f);
     const int64_t f = (int64_t)t * 32 + lane;
     if (f >= nblk) continue;
     const int64_t m = f / NB;

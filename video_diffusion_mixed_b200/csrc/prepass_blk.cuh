@@ -137,7 +137,7 @@ __device__ __forceinline__ float pb_stage1_raw(float2 (&P)[64], float* rmax) {
 // multiply-add by +-1 each (exact product, one rounding): (x + y, x - y) for a pair (lower, upper)
 // and (y - x, y + x) for a swapped pair (upper, lower) -- the same two results in swapped places.
 template <int B>
-__device__ __forceinline__ float pb_stages_rest(float2 (&P)[64], int lane) {
+__device__ __forceinline__ float pb_stages_rest(float2 (&P)[64], float cx) {  // cx = -1: swapped pairs
 #pragma unroll
   for (int h = 2; h <= 32; h <<= 1) {
     if (h < B) {
@@ -153,7 +153,7 @@ __device__ __forceinline__ float pb_stages_rest(float2 (&P)[64], int lane) {
   }
   float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent chains
   if (64 < B) {
-    const float cx = pb_swap(lane) ? -1.0f : 1.0f, cy = -cx;
+    const float cy = -cx;
 #pragma unroll
     for (int k = 0; k < 64; ++k) {
       const float s = __fmaf_rn(cx, P[k].x, P[k].y), d = __fmaf_rn(cy, P[k].y, P[k].x);
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
 
     float rmax;
     const float bsum = pb_stage1_raw(P, &rmax);
-    const float am = pb_stages_rest<B>(P, lane);
+    const float am = pb_stages_rest<B>(P, pb_swap(lane) ? -1.0f : 1.0f);
 
     // ---- row maxima and sums of aligned runs of SUB blocks, then the team meets
     const uint32_t amb = __reduce_max_sync(rowmask, __float_as_uint(am));
