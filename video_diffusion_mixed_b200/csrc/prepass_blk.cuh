@@ -23,6 +23,8 @@
 // load is always in flight while a task computes.
 #pragma once
 
+#include <type_traits>
+
 #include "rows.cuh"
 
 namespace sb {
@@ -238,6 +240,8 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
   __shared__ float s_gsum[kPbWarps][kG];                   // per row of the current group
   __shared__ float s_gam[kPbWarps][kG];
   __shared__ float s_grm[kPbWarps][kG];
+  __shared__ uint64_t s_full[kPbWarps][2];   // statistics-only pass: the team's task buffers
+  __shared__ uint64_t s_empty[kPbWarps][2];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pb_dsm) + 1023) & ~(uintptr_t)1023);
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -281,6 +285,12 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
   if (lane == 0) {
 #pragma unroll
     for (int d = 0; d < kPbD; ++d) mbar_init(&s_bar[warp][d], 1);
+    if (wt == 0) {
+      mbar_init(&s_full[team][0], (uint32_t)T);
+      mbar_init(&s_full[team][1], (uint32_t)T);
+      mbar_init(&s_empty[team][0], 1);
+      mbar_init(&s_empty[team][1], 1);
+    }
     fence_barrier_init();
   }
   __syncthreads();  // zeroed buffers and initialised barriers
@@ -293,92 +303,122 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
 
   const int SUB = gm.SUB, NBS = NB2 / SUB;  // per row: NBS aligned run sums (zero-padded)
   int bad_it = -1;
-  int g = gteam, j = 0, tb = 0, dw = 0;  // group, task in group, atomics buffer, designated warp
-  for (int it = 0; g < G; ++it) {
-    const int m0 = g * kG + j * R;
-    const int slot = it & 1, pb = it & 1;
-    const int jn = (j + 1 == TPG) ? 0 : j + 1, gn = (j + 1 == TPG) ? g + nteams : g;  // next task
-    // the slot of the previous task was read into registers (and used) there: refill it with the
-    // task after this one
-    if (lane == 0 && it > 0) issue(gn, jn, slot ^ 1);
-    if (!mbar_wait_bounded(&s_bar[warp][slot], (uint32_t)((it >> 1) & 1), nullptr, kRowWaitNs)) {
+  auto bounded = [&](uint64_t* bar, uint32_t parity, int it) {
+    if (!mbar_wait_bounded(bar, parity, nullptr, kRowWaitNs)) {
       if (lane == 0) set_error(a.hdr, SB_ETIMEOUT);
       bad_it = it;
     }
-    float2 P[64];
-    pb_load_block(ring_w + (uint32_t)(slot * kPbSlot), lane, P);
+  };
+  // Q: the INT8 pass. Every lane needs its row's amax before it quantizes, so the team meets at a
+  // named barrier each task, and the maxima are triple-buffered. Otherwise (statistics only) just
+  // the warp that folds the task's rows waits for the others: every warp arrives on
+  // s_full[team][t & 1] and goes on; the folding warp waits there, folds, clears the task's
+  // buffers and arrives on s_empty[team][t & 1]; a warp waits on s_empty only before it writes the
+  // buffers again two tasks later.
+  auto run = [&](auto qtag) {
+    constexpr bool Q = decltype(qtag)::value;
+    int g = gteam, j = 0, tb = 0, dw = 0;  // group, task in group, maxima buffer (Q), folding warp
+    for (int it = 0; g < G; ++it) {
+      const int m0 = g * kG + j * R;
+      const int slot = it & 1, pb = it & 1;
+      const int ab = Q ? tb : pb;  // maxima buffer of this task
+      const int jn = (j + 1 == TPG) ? 0 : j + 1, gn = (j + 1 == TPG) ? g + nteams : g;  // next task
+      // the slot of the previous task was read into registers (and used) there: refill it with the
+      // task after this one
+      if (lane == 0 && it > 0) issue(gn, jn, slot ^ 1);
+      bounded(&s_bar[warp][slot], (uint32_t)((it >> 1) & 1), it);
+      float2 P[64];
+      pb_load_block(ring_w + (uint32_t)(slot * kPbSlot), lane, P);
 
-    float rmax;
-    const float bsum = pb_stage1_raw(P, &rmax);
-    const float am = pb_stages_rest<B>(P, pb_swap(lane) ? -1.0f : 1.0f);
+      float rmax;
+      const float bsum = pb_stage1_raw(P, &rmax);
+      const float am = pb_stages_rest<B>(P, pb_swap(lane) ? -1.0f : 1.0f);
 
-    // ---- row maxima and sums of aligned runs of SUB blocks, then the team meets
-    const uint32_t amb = __reduce_max_sync(rowmask, __float_as_uint(am));
-    const uint32_t rmb = __reduce_max_sync(rowmask, __float_as_uint(rmax));
-    if (qv && leader) {
-      atomicMax(&s_ram[tb][team][rl], amb);
-      atomicMax(&s_rmx[tb][team][rl], rmb);
-    }
-    float run = bsum;
-    for (int sh = 1; sh < SUB; sh <<= 1) run = __fadd_rn(run, __shfl_xor_sync(0xffffffffu, run, sh));
-    if (qv && (blk & (SUB - 1)) == 0) s_bsum[pb][sbase + rl * NBS + blk / SUB] = run;
-    pb_team_sync(team, T);
-
-    const int m = m0 + rl;
-    if (do_int8 && qv && m < a.M)
-      pb_store_int8(P, __uint_as_float(s_ram[tb][team][rl]), a.q8 + ((int64_t)m * NB + blk) * 128, lane);
-
-    // ---- one warp of the team: row sums, the task's rows into the group, the group's slot
-    if (wt == dw) {
-      const int n = R * NBS;
-      const int c = n >= 32 ? n / 32 : 1;
-      const float* bs = &s_bsum[pb][sbase + lane * c];
-      float v;
-      if (c == 1) v = (lane < n) ? bs[0] : 0.0f;
-      else if (c == 2) v = pb_run_sum<2>(bs);
-      else if (c == 4) v = pb_run_sum<4>(bs);
-      else if (c == 8) v = pb_run_sum<8>(bs);
-      else v = pb_run_sum<16>(bs);
-      const int span = NBS / c;  // lanes per row
-      for (int s = 1; s < span; s <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
-      const int r = lane / span;
-      if ((lane & (span - 1)) == 0 && r < R) {
-        const int gi = j * R + r;
-        const float a_m = __uint_as_float(s_ram[tb][team][r]);
-        s_gsum[team][gi] = v;
-        s_gam[team][gi] = a_m;
-        s_grm[team][gi] = __uint_as_float(s_rmx[tb][team][r]);
-        if (do_int8 && m0 + r < a.M) a.s8[m0 + r] = (a_m == 0.0f) ? 0.0f : __fdiv_rn(a_m, 127.0f);
+      // ---- row maxima and sums of aligned runs of SUB blocks, then the team meets
+      if (!Q && it >= 2) bounded(&s_empty[team][pb], (uint32_t)(((it >> 1) & 1) ^ 1), it);
+      const uint32_t amb = __reduce_max_sync(rowmask, __float_as_uint(am));
+      const uint32_t rmb = __reduce_max_sync(rowmask, __float_as_uint(rmax));
+      if (qv && leader) {
+        atomicMax(&s_ram[ab][team][rl], amb);
+        atomicMax(&s_rmx[ab][team][rl], rmb);
       }
-      if (lane < R) {  // the buffers of the task two steps ahead start from zero
-        const int tz = tb == 0 ? 2 : tb - 1;
-        s_ram[tz][team][lane] = 0u;
-        s_rmx[tz][team][lane] = 0u;
-      }
-      if (j == TPG - 1) {
+      float run = bsum;
+      for (int sh = 1; sh < SUB; sh <<= 1) run = __fadd_rn(run, __shfl_xor_sync(0xffffffffu, run, sh));
+      if (qv && (blk & (SUB - 1)) == 0) s_bsum[pb][sbase + rl * NBS + blk / SUB] = run;
+      if (Q) {
+        pb_team_sync(team, T);
+        const int m = m0 + rl;
+        if (qv && m < a.M)
+          pb_store_int8(P, __uint_as_float(s_ram[ab][team][rl]), a.q8 + ((int64_t)m * NB + blk) * 128, lane);
+      } else {
         __syncwarp();
-        const bool in = lane < kG;
-        const float rs = in ? s_gsum[team][lane] : 0.0f;
-        const double gs = warp_pairwise_f64((double)rs);
-        const float gam = warp_max_f32(in ? s_gam[team][lane] : 0.0f);
-        const float gmx = warp_max_f32(in ? s_grm[team][lane] : 0.0f);
-        const int gnf = __any_sync(0xffffffffu, in && !isfinite(rs));
-        if (lane == 0) {
-          GroupSlot* gsl = a.groups + g;
-          gsl->s[0] = gs;
-          gsl->s[1] = 0.0;
-          gsl->s[2] = 0.0;
-          gsl->max_abs = gmx;
-          gsl->amax_rot = gam;
-          gsl->nonfinite = gnf;
+        if (lane == 0) mbar_arrive(&s_full[team][pb]);
+      }
+
+      // ---- one warp of the team: row sums, the task's rows into the group, the group's slot
+      if (wt == dw) {
+        if (!Q) bounded(&s_full[team][pb], (uint32_t)((it >> 1) & 1), it);
+        const int n = R * NBS;
+        const int c = n >= 32 ? n / 32 : 1;
+        const float* bs = &s_bsum[pb][sbase + lane * c];
+        float v;
+        if (c == 1) v = (lane < n) ? bs[0] : 0.0f;
+        else if (c == 2) v = pb_run_sum<2>(bs);
+        else if (c == 4) v = pb_run_sum<4>(bs);
+        else if (c == 8) v = pb_run_sum<8>(bs);
+        else v = pb_run_sum<16>(bs);
+        const int span = NBS / c;  // lanes per row
+        for (int s = 1; s < span; s <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
+        const int r = lane / span;
+        if ((lane & (span - 1)) == 0 && r < R) {
+          const int gi = j * R + r;
+          const float a_m = __uint_as_float(s_ram[ab][team][r]);
+          s_gsum[team][gi] = v;
+          s_gam[team][gi] = a_m;
+          s_grm[team][gi] = __uint_as_float(s_rmx[ab][team][r]);
+          if (Q && m0 + r < a.M) a.s8[m0 + r] = (a_m == 0.0f) ? 0.0f : __fdiv_rn(a_m, 127.0f);
+        }
+        // the maxima buffer used next starts from zero: Q, the one two tasks ahead (the others
+        // have read this task's already); otherwise this task's own, read above
+        if (!Q) __syncwarp();
+        if (lane < R) {
+          const int tz = Q ? (tb == 0 ? 2 : tb - 1) : ab;
+          s_ram[tz][team][lane] = 0u;
+          s_rmx[tz][team][lane] = 0u;
+        }
+        if (j == TPG - 1) {
+          __syncwarp();
+          const bool in = lane < kG;
+          const float rs = in ? s_gsum[team][lane] : 0.0f;
+          const double gs = warp_pairwise_f64((double)rs);
+          const float gam = warp_max_f32(in ? s_gam[team][lane] : 0.0f);
+          const float gmx = warp_max_f32(in ? s_grm[team][lane] : 0.0f);
+          const int gnf = __any_sync(0xffffffffu, in && !isfinite(rs));
+          if (lane == 0) {
+            GroupSlot* gsl = a.groups + g;
+            gsl->s[0] = gs;
+            gsl->s[1] = 0.0;
+            gsl->s[2] = 0.0;
+            gsl->max_abs = gmx;
+            gsl->amax_rot = gam;
+            gsl->nonfinite = gnf;
+          }
+        }
+        if (!Q) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_empty[team][pb]);
         }
       }
+      g = gn;
+      j = jn;
+      tb = tb == 2 ? 0 : tb + 1;
+      dw = dw + 1 == T ? 0 : dw + 1;
     }
-    g = gn;
-    j = jn;
-    tb = tb == 2 ? 0 : tb + 1;
-    dw = dw + 1 == T ? 0 : dw + 1;
-  }
+  };
+  if (do_int8)
+    run(std::true_type{});
+  else
+    run(std::false_type{});
   if (bad_it >= 0 && lane == 0)
     mbar_wait_bounded(&s_bar[warp][bad_it & 1], (uint32_t)((bad_it >> 1) & 1), nullptr, kRowDrainNs);
   rows_finish<OP_PREPASS, false>(a, G, prec, true, reinterpret_cast<double*>(ring));
