@@ -40,15 +40,15 @@ METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT sh
 _GEMM_SRC = ("gemm.cu", "sb_device.cuh")
 _ROWS_SRC = ("prepass.cu", "rows.cuh", "prepass_blk.cuh", "sb_device.cuh", "tmap.h")
 TRAFFIC = {
-    "gemm_w1_int8": {"bytes": 739.4e6, "files": _GEMM_SRC, "sha": "2f9a3737d827dbc7"},
-    "gemm_w2_int8": {"bytes": 795.8e6, "files": _GEMM_SRC, "sha": "2f9a3737d827dbc7"},
-    "gemm_w1_nvfp4": {"bytes": 486.1e6, "files": _GEMM_SRC, "sha": "2f9a3737d827dbc7"},
-    "gemm_w2_nvfp4": {"bytes": 264.5e6, "files": _GEMM_SRC, "sha": "2f9a3737d827dbc7"},
+    "gemm_w1_int8": {"bytes": 743.7e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
+    "gemm_w2_int8": {"bytes": 801.8e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
+    "gemm_w1_nvfp4": {"bytes": 487.6e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
+    "gemm_w2_nvfp4": {"bytes": 269.0e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
     # k_prepass_blk + k_nvfp4_blk (the encode exits at once in the INT8 pass)
-    "prepass_h_nvfp4": {"bytes": 940.7e6, "files": _ROWS_SRC, "sha": "01321ae6d175034e"},
-    "prepass_h_int8": {"bytes": 578.1e6, "files": _ROWS_SRC, "sha": "01321ae6d175034e"},
-    "prepass_x_nvfp4": {"bytes": 218.9e6, "files": _ROWS_SRC, "sha": "01321ae6d175034e"},
-    "prepass_x_int8": {"bytes": 111.6e6, "files": _ROWS_SRC, "sha": "01321ae6d175034e"},
+    "prepass_h_nvfp4": {"bytes": 942.1e6, "files": _ROWS_SRC, "sha": "9e1db27da5e5db9f"},
+    "prepass_h_int8": {"bytes": 577.0e6, "files": _ROWS_SRC, "sha": "9e1db27da5e5db9f"},
+    "prepass_x_nvfp4": {"bytes": 218.7e6, "files": _ROWS_SRC, "sha": "9e1db27da5e5db9f"},
+    "prepass_x_int8": {"bytes": 112.8e6, "files": _ROWS_SRC, "sha": "9e1db27da5e5db9f"},
 }
 TRAFFIC_TOKENS = 17776
 
