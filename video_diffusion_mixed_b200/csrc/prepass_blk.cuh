@@ -11,12 +11,16 @@
 // P[k] = (v[k], v[k + 64]): FP32x2 arithmetic covers the stages h = 1..32, the stage h = 64 pairs
 // the two halves of each P[k]. Lanes 4..7 of every eight hold the halves the other way round,
 // P[k] = (v[k + 64], v[k]) (see pb_load_block); every step but the stage h = 64 and the final
-// stores treats the two halves alike. A "team" of T warps (T | 12) owns R rows at a time (R | kG), their
-// R NB blocks laid out flat over its 32 T lanes (a row may straddle warps; idle lanes compute on
-// whatever the box holds and write nothing). Per task the team meets once at a named barrier:
-// row maxima go through shared-memory atomics, block sums through a shared buffer that one warp
-// of the team (rotating) folds into row sums. A team walks whole groups of kG rows and writes
-// each group's FP64 slot itself; the last CTA finishes as k_rows does.
+// stores treats the two halves alike.
+//
+// Teams: T warps (T | 12) own R rows at a time (R | kG), their R NB blocks laid out flat over the
+// team's 32 T lanes (a row may straddle warps; idle lanes compute on whatever the box holds and
+// write nothing). Row maxima go through shared-memory atomics, sums of aligned runs of blocks
+// through a shared buffer that one warp of the team (rotating) folds into row sums. In the INT8
+// pass the team meets once per task at a named barrier, since every lane needs its row's amax;
+// in a statistics-only pass only the folding warp waits for the others (mbarriers). A team walks
+// whole groups of kG rows and writes each group's FP64 slot itself; the last CTA finishes as
+// k_rows does.
 //
 // Loads: every warp keeps a ring of kPbD slots, each one TMA box of 32 consecutive blocks (8 KB,
 // 128B swizzle); a slot is refilled at the start of the task after the one that read it, so one
