@@ -242,6 +242,59 @@ sb_status sb_tdc_refresh(const void* x, const void* y, void* delta, int64_t M, i
 sb_status sb_tdc_reuse(const void* x, const void* delta, void* y, int64_t M, int64_t C, const sb_module_state* state,
                        sb_stream stream);
 
+/* ---- Token sharding: several GPUs each own a contiguous range of a tensor's rows ----
+ * Every step of the path works row by row except the reductions of the pre-pass and of the TDC
+ * record, which span all rows. A shard runs the row work of its rows and writes its FP64 group
+ * partials (one 48-byte slot per aligned 16-row group) into a slot array covering the whole tensor.
+ * Shards write disjoint ranges of that array, so gathering them is exact: e.g. an int64 all-reduce
+ * SUM of zero-filled copies. Every GPU then runs the same final reduction over the gathered array
+ * and obtains the statistics record, PDR verdict or module-state update of the whole tensor, bit
+ * for bit those of the unsharded call, because the group slots are aligned subtrees of the same
+ * FP64 tree. The weights are replicated, so the GEMMs need no exchange. ("write-up" sections 一,
+ * 二, 三: the difference, the TDC change and the outlier ratio are statistics of whole tensors.)
+ * Shard rules: row0 % 16 == 0, and M % 16 == 0 unless the shard ends the tensor. */
+
+/* Bytes of the slot array of an M_total-row tensor (48 per 16-row group), or -1 if M_total < 1. */
+int64_t sb_group_slots_bytes(int64_t M_total);
+
+/* The row work of sb_prepass on rows [row0, row0 + M) of an M_total-row tensor: X, X_ref and a8
+ * hold only these M rows ([M][K] bf16; a8 codes [M][K], scales [M]). Writes the shard's group
+ * slots at slots + (row0 / 16) * 48 and, in SB_PREPASS_QUANT mode when *prec says INT8, the INT8
+ * codes and per-token scales. Writes no statistics record and leaves *prec unchanged; the NVFP4
+ * codes need the whole tensor's amax (sb_nvfp4_encode after sb_prepass_finish). slots: device,
+ * 16-byte aligned, sb_group_slots_bytes(M_total) bytes. Validation as sb_prepass (SB_ESHAPE for
+ * the shard rules). */
+sb_status sb_prepass_partial(const void* X, const void* X_ref, int64_t M, int64_t K, int64_t row0,
+                             int64_t M_total, const sb_config* cfg /* host */, int32_t mode,
+                             int32_t* prec, const sb_i8* a8 /* host */, void* slots, void* ws,
+                             sb_stream stream);
+
+/* The final reduction of a sharded pre-pass of an M_total x K tensor over the gathered slots:
+ * writes *stats and, in SB_PREPASS_QUANT mode, applies PDR to *prec, as sb_prepass does. has_ref:
+ * whether the shards were given X_ref. */
+sb_status sb_prepass_finish(const void* slots, int64_t M_total, int64_t K, int32_t has_ref,
+                            const sb_config* cfg /* host */, int32_t mode, int32_t* prec,
+                            sb_stats* stats, void* ws, sb_stream stream);
+
+/* NVFP4 codes of the rows X [M][K] (a shard, or a whole tensor) from finished statistics: tensor
+ * scale from stats->amax_rot (the whole tensor's), E4M3 block scales in the tiled layout of these
+ * M rows. Writes a4 only when *prec is SB_NVFP4 (prec NULL: always). */
+sb_status sb_nvfp4_encode(const void* X, int64_t M, int64_t K, const sb_config* cfg /* host */,
+                          const int32_t* prec, const sb_stats* stats, const sb_fp4* a4 /* host */,
+                          void* ws, sb_stream stream);
+
+/* The row work of sb_tdc_record on rows [row0, row0 + M) of an M_total-row module output: the
+ * shard's sums of |y_new - y_cache| and |y_cache| into the slot array, and the cache refresh with
+ * update_cache. The module state is read (skip, whether an output was recorded), not written. */
+sb_status sb_tdc_record_partial(const void* y_new, void* y_cache, int64_t M, int64_t C, int64_t row0,
+                                int64_t M_total, int32_t update_cache,
+                                const sb_module_state* state, void* slots, void* ws, sb_stream stream);
+
+/* The final TDC reduction over the gathered slots: delta and the state update of sb_tdc_record
+ * (d from d_src when given). Does nothing if state->skip. */
+sb_status sb_tdc_finish(const void* slots, int64_t M_total, int64_t C, const sb_stats* d_src,
+                        sb_module_state* state, void* ws, sb_stream stream);
+
 /* Bounded device-side wait, the library's failure-detection primitive (the pages have no
  * counterpart). Enqueues on `stream` a one-thread kernel that polls the device int32 at `flag`
  * (acquire loads, ~1 us apart) until it equals `value`. If `limit_ns` nanoseconds of device time

@@ -127,3 +127,36 @@ def test_argument_validation_without_gpu(sb):
     rule = sb.Rule(1.0, 0.0, 0.1)
     assert L.sb_select_precision(_fake(0x100), ctypes.byref(rule), ctypes.byref(sb.config(force_prec=5)),
                                  _fake(0x200), s) == sb.SB_EINVAL
+
+
+def test_shard_validation_without_gpu(sb):
+    """The token-sharding entry points check the shard rules before any launch."""
+    L = sb.lib()
+    cfg = sb.config()
+    a8 = sb.I8(0x4000, 0x5000, 32, 256)
+    assert L.sb_group_slots_bytes(17776) == 1111 * 48
+    assert L.sb_group_slots_bytes(17) == 2 * 48
+    assert L.sb_group_slots_bytes(0) == -1
+    X, slots, ws, prec = _fake(0x1000), _fake(0x8000), _fake(0x9000), _fake(0x100)
+    # row0 not on a 16-row group boundary
+    assert L.sb_prepass_partial(X, None, 32, 256, 8, 64, ctypes.byref(cfg), 1, None, None, slots, ws,
+                                None) == sb.SB_ESHAPE
+    assert "multiple of 16" in L.sb_last_error().decode()
+    # a shard that does not end the tensor must hold whole groups
+    assert L.sb_prepass_partial(X, None, 20, 256, 0, 64, ctypes.byref(cfg), 1, None, None, slots, ws,
+                                None) == sb.SB_ESHAPE
+    # rows past the tensor
+    assert L.sb_prepass_partial(X, None, 32, 256, 48, 64, ctypes.byref(cfg), 1, None, None, slots, ws,
+                                None) == sb.SB_ESHAPE
+    # QUANT needs prec and a8; misaligned slots
+    assert L.sb_prepass_partial(X, None, 32, 256, 32, 64, ctypes.byref(cfg), 0, None, None, slots, ws,
+                                None) == sb.SB_EINVAL
+    assert L.sb_prepass_partial(X, None, 32, 256, 32, 64, ctypes.byref(cfg), 0, prec, ctypes.byref(a8),
+                                _fake(0x8008), ws, None) == sb.SB_EALIGN
+    # finish and TDC partial / finish
+    assert L.sb_prepass_finish(None, 64, 256, 0, ctypes.byref(cfg), 1, None, _fake(0x200), ws, None) == sb.SB_EINVAL
+    assert L.sb_prepass_finish(slots, 64, 256, 0, ctypes.byref(cfg), 0, None, _fake(0x200), ws, None) == sb.SB_EINVAL
+    assert L.sb_tdc_record_partial(X, _fake(0x2000), 32, 64, 16, 40, 1, _fake(0x300), slots, ws,
+                                   None) == sb.SB_ESHAPE
+    assert L.sb_tdc_finish(slots, 0, 64, None, _fake(0x300), ws, None) == sb.SB_ESHAPE
+    assert L.sb_nvfp4_encode(X, 64, 256, ctypes.byref(cfg), prec, _fake(0x200), None, ws, None) == sb.SB_EINVAL

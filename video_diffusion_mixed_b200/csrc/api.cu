@@ -157,6 +157,7 @@ sb_status sb_prepare_weight(const void* W, const void* bias, int64_t N, int64_t 
   w->block = block;
   cudaStream_t s = (cudaStream_t)stream;
   sb::PrepassLaunch p{};
+  p.finish = 1;
   p.X = W;
   p.R = nullptr;
   p.M = N;
@@ -229,6 +230,7 @@ sb_status sb_prepass(const void* X, const void* X_ref, int64_t M, int64_t K, con
   if (prec) SB_REQUIRE((reinterpret_cast<uintptr_t>(prec) & 3u) == 0, SB_EALIGN, "prec misaligned");
   cudaStream_t s = (cudaStream_t)stream;
   sb::PrepassLaunch p{};
+  p.finish = 1;
   p.X = X;
   p.R = X_ref;
   p.M = M;
@@ -335,6 +337,7 @@ sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C, 
   SB_REQUIRE(C >= 8 && C % 8 == 0 && C <= sb::kMaxK, SB_EUNSUPPORTED, "C must be a multiple of 8 in [8, %d]",
              sb::kMaxK);
   sb::TdcLaunch p{};
+  p.finish = 1;
   p.Y = y_new;
   p.Cache = y_cache;
   p.M = M;
@@ -346,6 +349,176 @@ sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C, 
   p.hdr = ws;
   cudaError_t e = sb::launch_tdc_record(p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "sb_tdc_record");
+  return ok();
+}
+
+// ---------------------------------------------------------------------------------------------
+// Token sharding: partial row work into a slot array, gathered elsewhere, then the final reduction
+// ---------------------------------------------------------------------------------------------
+
+int64_t sb_group_slots_bytes(int64_t M_total) {
+  if (M_total < 1) return -1;
+  return sb::ceil_div(M_total, sb::kGroupRows) * (int64_t)sizeof(sb::GroupSlot);
+}
+
+static sb_status check_shard(int64_t M, int64_t row0, int64_t M_total, const void* slots) {
+  SB_REQUIRE(slots != nullptr, SB_EINVAL, "slots is NULL");
+  SB_ALIGNED(slots, "slots");
+  SB_REQUIRE(M >= 1 && row0 >= 0 && M_total <= (int64_t)1 << 30 && row0 + M <= M_total, SB_ESHAPE,
+             "shard rows [%lld, %lld) outside the tensor's %lld rows", (long long)row0, (long long)(row0 + M),
+             (long long)M_total);
+  SB_REQUIRE(row0 % sb::kGroupRows == 0, SB_ESHAPE, "row0 (%lld) must be a multiple of %d", (long long)row0,
+             sb::kGroupRows);
+  SB_REQUIRE(row0 + M == M_total || M % sb::kGroupRows == 0, SB_ESHAPE,
+             "a shard that does not end the tensor must hold a multiple of %d rows (got %lld)", sb::kGroupRows,
+             (long long)M);
+  return SB_OK;
+}
+
+static char* shard_slots(void* slots, int64_t row0) {
+  return static_cast<char*>(slots) + (row0 / sb::kGroupRows) * (int64_t)sizeof(sb::GroupSlot);
+}
+
+sb_status sb_prepass_partial(const void* X, const void* X_ref, int64_t M, int64_t K, int64_t row0, int64_t M_total,
+                             const sb_config* cfg, int32_t mode, int32_t* prec, const sb_i8* a8, void* slots, void* ws,
+                             sb_stream stream) {
+  SB_REQUIRE(X && cfg && ws, SB_EINVAL, "X, cfg and ws are required");
+  SB_ALIGNED(X, "X");
+  if (X_ref) SB_ALIGNED(X_ref, "X_ref");
+  SB_ALIGNED(ws, "ws");
+  SB_REQUIRE(mode == SB_PREPASS_QUANT || mode == SB_PREPASS_STATS, SB_EINVAL, "mode must be QUANT or STATS");
+  SB_REQUIRE(cfg->force_prec >= -1 && cfg->force_prec <= 2, SB_EINVAL, "force_prec must be -1, 0, 1 or 2");
+  sb_status st = check_rows_cols(M, K, cfg->block);
+  if (st != SB_OK) return st;
+  if ((st = check_shard(M, row0, M_total, slots)) != SB_OK) return st;
+  if (mode == SB_PREPASS_QUANT) {
+    SB_REQUIRE(prec && a8, SB_EINVAL, "QUANT mode needs prec and a8");
+    if ((st = check_i8(a8, M, K, "a8")) != SB_OK) return st;
+  }
+  if (prec) SB_REQUIRE((reinterpret_cast<uintptr_t>(prec) & 3u) == 0, SB_EALIGN, "prec misaligned");
+  sb::PrepassLaunch p{};
+  p.finish = 0;
+  p.X = X;
+  p.R = X_ref;
+  p.M = M;
+  p.K = K;
+  p.B = cfg->block;
+  p.mode = mode;
+  p.prec = prec;
+  p.q8 = (mode == SB_PREPASS_QUANT) ? a8->codes : nullptr;
+  p.s8 = (mode == SB_PREPASS_QUANT) ? a8->scale : nullptr;
+  p.rho = cfg->rho;
+  p.force = cfg->force_prec;
+  p.groups = shard_slots(slots, row0);
+  p.hdr = ws;
+  cudaError_t e = sb::launch_prepass(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_prepass_partial");
+  return ok();
+}
+
+sb_status sb_prepass_finish(const void* slots, int64_t M_total, int64_t K, int32_t has_ref, const sb_config* cfg,
+                            int32_t mode, int32_t* prec, sb_stats* stats, void* ws, sb_stream stream) {
+  SB_REQUIRE(slots && cfg && stats && ws, SB_EINVAL, "slots, cfg, stats and ws are required");
+  SB_ALIGNED(slots, "slots");
+  SB_ALIGNED(stats, "stats");
+  SB_ALIGNED(ws, "ws");
+  SB_REQUIRE(mode == SB_PREPASS_QUANT || mode == SB_PREPASS_STATS, SB_EINVAL, "mode must be QUANT or STATS");
+  SB_REQUIRE(mode == SB_PREPASS_STATS || prec, SB_EINVAL, "QUANT mode needs prec");
+  sb_status st = check_rows_cols(M_total, K, cfg->block);
+  if (st != SB_OK) return st;
+  if (prec) SB_REQUIRE((reinterpret_cast<uintptr_t>(prec) & 3u) == 0, SB_EALIGN, "prec misaligned");
+  sb::FinishLaunch f{};
+  f.op = 0;
+  f.has_ref = has_ref ? 1 : 0;
+  f.M = M_total;
+  f.K = K;
+  f.mode = mode;
+  f.prec = prec;
+  f.rho = cfg->rho;
+  f.force = cfg->force_prec;
+  f.groups = slots;
+  f.hdr = ws;
+  f.stats = stats;
+  cudaError_t e = sb::launch_finish(f, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_prepass_finish");
+  return ok();
+}
+
+sb_status sb_nvfp4_encode(const void* X, int64_t M, int64_t K, const sb_config* cfg, const int32_t* prec,
+                          const sb_stats* stats, const sb_fp4* a4, void* ws, sb_stream stream) {
+  SB_REQUIRE(X && cfg && stats && a4 && ws, SB_EINVAL, "X, cfg, stats, a4 and ws are required");
+  SB_ALIGNED(X, "X");
+  SB_ALIGNED(stats, "stats");
+  SB_ALIGNED(ws, "ws");
+  sb_status st = check_rows_cols(M, K, cfg->block);
+  if (st != SB_OK) return st;
+  if ((st = check_fp4(a4, M, K, "a4")) != SB_OK) return st;
+  if (prec) SB_REQUIRE((reinterpret_cast<uintptr_t>(prec) & 3u) == 0, SB_EALIGN, "prec misaligned");
+  sb::Nvfp4Launch q{};
+  q.X = X;
+  q.M = M;
+  q.K = K;
+  q.B = cfg->block;
+  q.prec = prec;
+  q.stats = stats;
+  q.codes = a4->codes;
+  q.sf = a4->sf;
+  q.gscale = a4->gscale;
+  q.hdr = ws;
+  cudaError_t e = sb::launch_nvfp4(q, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_nvfp4_encode");
+  return ok();
+}
+
+sb_status sb_tdc_record_partial(const void* y_new, void* y_cache, int64_t M, int64_t C, int64_t row0, int64_t M_total,
+                                int32_t update_cache, const sb_module_state* state, void* slots, void* ws,
+                                sb_stream stream) {
+  SB_REQUIRE(y_new && y_cache && state && ws, SB_EINVAL, "y_new, y_cache, state and ws are required");
+  SB_ALIGNED(y_new, "y_new");
+  SB_ALIGNED(y_cache, "y_cache");
+  SB_ALIGNED(state, "state");
+  SB_ALIGNED(ws, "ws");
+  SB_REQUIRE(C >= 8 && C % 8 == 0 && C <= sb::kMaxK, SB_EUNSUPPORTED, "C must be a multiple of 8 in [8, %d]",
+             sb::kMaxK);
+  sb_status st = check_shard(M, row0, M_total, slots);
+  if (st != SB_OK) return st;
+  sb::TdcLaunch p{};
+  p.finish = 0;
+  p.Y = y_new;
+  p.Cache = y_cache;
+  p.M = M;
+  p.C = C;
+  p.update = update_cache ? 1 : 0;
+  p.st = const_cast<sb_module_state*>(state);
+  p.groups = shard_slots(slots, row0);
+  p.hdr = ws;
+  cudaError_t e = sb::launch_tdc_record(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_tdc_record_partial");
+  return ok();
+}
+
+sb_status sb_tdc_finish(const void* slots, int64_t M_total, int64_t C, const sb_stats* d_src, sb_module_state* state,
+                        void* ws, sb_stream stream) {
+  SB_REQUIRE(slots && state && ws, SB_EINVAL, "slots, state and ws are required");
+  SB_ALIGNED(slots, "slots");
+  SB_ALIGNED(state, "state");
+  SB_ALIGNED(ws, "ws");
+  if (d_src) SB_ALIGNED(d_src, "d_src");
+  SB_REQUIRE(M_total >= 1 && M_total <= (int64_t)1 << 30, SB_ESHAPE, "M_total out of range (%lld)",
+             (long long)M_total);
+  SB_REQUIRE(C >= 8 && C % 8 == 0 && C <= sb::kMaxK, SB_EUNSUPPORTED, "C must be a multiple of 8 in [8, %d]",
+             sb::kMaxK);
+  sb::FinishLaunch f{};
+  f.op = 2;
+  f.has_ref = 1;
+  f.M = M_total;
+  f.K = C;
+  f.dsrc = d_src;
+  f.st = state;
+  f.groups = slots;
+  f.hdr = ws;
+  cudaError_t e = sb::launch_finish(f, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_tdc_finish");
   return ok();
 }
 

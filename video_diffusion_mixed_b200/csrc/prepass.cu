@@ -47,6 +47,7 @@ static RowArgs row_args_from(const PrepassLaunch& p) {
   a.groups = reinterpret_cast<GroupSlot*>(p.groups);
   a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
   a.stats = p.stats;
+  a.finish = p.finish;
   return a;
 }
 
@@ -114,9 +115,37 @@ cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s) {
   a.st = p.st;
   a.groups = reinterpret_cast<GroupSlot*>(p.groups);
   a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
+  a.finish = p.finish;
   RowMaps mp;
   row_maps(a, mp, p.Y, p.Cache);
   return launch_rows_t<OP_TDC, true>(a, mp, s, sm_count());
+}
+
+cudaError_t launch_finish(const FinishLaunch& p, cudaStream_t s) {
+  RowArgs a{};
+  a.M = p.M;
+  a.K = (int)p.K;
+  a.mode = p.mode;
+  a.prec = p.prec;
+  a.rho = p.rho;
+  a.force = p.force;
+  a.dsrc = p.dsrc;
+  a.st = p.st;
+  a.groups = const_cast<GroupSlot*>(reinterpret_cast<const GroupSlot*>(p.groups));
+  a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
+  a.stats = p.stats;
+  a.finish = 1;
+  const int64_t G = ceil_div(p.M, kG);
+  if (p.op == 2) {
+    k_finish<OP_TDC, true><<<1, 256, 0, s>>>(a, G);
+  } else if (p.mode == SB_PREPASS_STATS) {
+    if (p.has_ref) k_finish<OP_STATS, true><<<1, 256, 0, s>>>(a, G);
+    else k_finish<OP_STATS, false><<<1, 256, 0, s>>>(a, G);
+  } else {
+    if (p.has_ref) k_finish<OP_PREPASS, true><<<1, 256, 0, s>>>(a, G);
+    else k_finish<OP_PREPASS, false><<<1, 256, 0, s>>>(a, G);
+  }
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
     run(std::false_type{});
   if (bad_it >= 0 && lane == 0)
     mbar_wait_bounded(&s_bar[warp][bad_it & 1], (uint32_t)((bad_it >> 1) & 1), nullptr, kRowDrainNs);
-  rows_finish<OP_PREPASS, false>(a, G, prec, true, reinterpret_cast<double*>(ring));
+  if (a.finish) rows_finish<OP_PREPASS, false>(a, G, prec, true, reinterpret_cast<double*>(ring));
 }
 
 }  // namespace sb

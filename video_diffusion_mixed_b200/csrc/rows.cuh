@@ -51,6 +51,8 @@ struct RowArgs {
   WsHeader* hdr;
   sb_stats* stats;
   int tma;  // rows arrive through the TMA rings (the maps below are valid)
+  int finish;  // 1: the last CTA reduces the group slots; 0: only this launch's slots are written
+               // (one shard of a token-sharded tensor; the slots are folded later)
 };
 
 // TMA maps of the row tensors (make_row_segment_map): x = X (TDC: the new output), r = x_ref
@@ -744,6 +746,23 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   // ring is reused or the CTA exits
   if (use_tma && bad_it >= 0 && lane == 0)
     mbar_wait_bounded(&s_bar[warp][bad_it % RG::D], (uint32_t)((bad_it / RG::D) & 1), nullptr, kRowDrainNs);
+  if (a.finish) rows_finish<OP, REF>(a, ngroups, prec, have_prev, s_fin);
+}
+
+// The final reduction alone, over group slots written by earlier launches (the shards of a
+// token-sharded tensor, gathered): one CTA runs rows_finish over a.groups[0 .. ngroups).
+template <int OP, bool REF>
+__global__ void __launch_bounds__(256) k_finish(RowArgs a, int64_t ngroups) {
+  __shared__ double s_fin[kFinChunk];
+  int prec = -1;
+  bool have_prev = true;
+  if (OP == OP_TDC) {
+    if (a.st->skip) return;
+    have_prev = a.st->n_out >= 1;
+  } else {
+    prec = a.force_int8 ? SB_INT8 : (a.prec ? *a.prec : -1);
+    if (prec == SB_SKIP) return;
+  }
   rows_finish<OP, REF>(a, ngroups, prec, have_prev, s_fin);
 }
 

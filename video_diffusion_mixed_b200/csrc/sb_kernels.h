@@ -24,6 +24,7 @@ struct PrepassLaunch {
   void* groups;
   void* hdr;
   sb_stats* stats;
+  int finish;  // 1: reduce the slots in the last CTA; 0: write this launch's group slots only
 };
 
 struct Nvfp4Launch {
@@ -47,6 +48,24 @@ struct TdcLaunch {
   sb_module_state* st;
   void* groups;
   void* hdr;
+  int finish;
+};
+
+// The final reduction over gathered group slots: op 0 pre-pass (mode, has_ref as in
+// PrepassLaunch), op 2 TDC record. The row kernels' arguments carry M = the whole tensor's rows.
+struct FinishLaunch {
+  int op;
+  int has_ref;
+  int64_t M, K;
+  int mode;
+  int32_t* prec;
+  double rho;
+  int force;
+  const sb_stats* dsrc;
+  sb_module_state* st;
+  const void* groups;
+  void* hdr;
+  sb_stats* stats;
 };
 
 struct GemmLaunch {
@@ -79,6 +98,7 @@ cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s);
 cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s);
 cudaError_t launch_rotate(const void* X, float* Y, int64_t M, int64_t K, int B, cudaStream_t s);
 cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s);
+cudaError_t launch_finish(const FinishLaunch& p, cudaStream_t s);
 cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t s, const char** why);
 
 cudaError_t launch_state_init(sb_module_state* st, cudaStream_t s);

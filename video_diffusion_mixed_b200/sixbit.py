@@ -93,6 +93,12 @@ def lib():
             "sb_wait_flag": (st, [vp, i32, ctypes.c_uint64, vp, vp]),
             "sb_tdc_refresh": (st, [vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_reuse": (st, [vp, vp, vp, i64, i64, vp, vp]),
+            "sb_group_slots_bytes": (i64, [i64]),
+            "sb_prepass_partial": (st, [vp, vp, i64, i64, i64, i64, P(Config), i32, vp, P(I8), vp, vp, vp]),
+            "sb_prepass_finish": (st, [vp, i64, i64, i32, P(Config), i32, vp, vp, vp, vp]),
+            "sb_nvfp4_encode": (st, [vp, i64, i64, P(Config), vp, vp, P(Fp4), vp, vp]),
+            "sb_tdc_record_partial": (st, [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp]),
+            "sb_tdc_finish": (st, [vp, i64, i64, vp, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -105,7 +111,8 @@ def lib():
 EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_init", "sb_fp4_sf_bytes",
             "sb_state_init", "sb_rotate", "sb_prepare_weight", "sb_tdc_step", "sb_select_precision", "sb_prepass",
             "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static", "sb_wait_flag", "sb_tdc_refresh",
-            "sb_tdc_reuse")
+            "sb_tdc_reuse", "sb_group_slots_bytes", "sb_prepass_partial", "sb_prepass_finish", "sb_nvfp4_encode",
+            "sb_tdc_record_partial", "sb_tdc_finish")
 
 
 def _ck(status: int):
@@ -268,6 +275,59 @@ def tdc_record(y_new, y_cache, d_src, state, ws: Workspace, update_cache: bool =
 
 def check(ws: Workspace, stream=None):
     _ck(lib().sb_check(ws.ptr, _stream(stream)))
+
+
+# ---- token sharding (include/sixbit.h): partial row work, slot gathering, final reduction ----
+
+GROUP_ROWS = 16
+SLOT_BYTES = 48
+
+
+def alloc_slots(M_total: int, device="cuda") -> torch.Tensor:
+    """Zero-filled group-slot array of an M_total-row tensor (int64 words, 16-byte aligned)."""
+    n = lib().sb_group_slots_bytes(M_total)
+    if n < 0:
+        raise SixbitError(SB_ESHAPE, f"M_total must be >= 1 (got {M_total})")
+    return torch.zeros(n // 8, dtype=torch.int64, device=device)
+
+
+def gather_slots(slots: torch.Tensor, group=None) -> torch.Tensor:
+    """Combine the shards' slot arrays in place: every rank wrote a disjoint range of its
+    zero-filled copy, so an int64 all-reduce SUM reproduces every written word bit for bit."""
+    import torch.distributed as dist
+    dist.all_reduce(slots, op=dist.ReduceOp.SUM, group=group)
+    return slots
+
+
+def prepass_partial(X, X_ref, row0: int, M_total: int, cfg: Config, mode: int, prec, a8: I8Tensor | None, slots,
+                    ws: Workspace, stream=None):
+    M, K = X.shape
+    c8 = ctypes.byref(a8.c()) if a8 is not None else None
+    _ck(lib().sb_prepass_partial(_p(X), _p(X_ref), M, K, row0, M_total, ctypes.byref(cfg), mode, _p(prec), c8,
+                                 _p(slots), ws.ptr, _stream(stream)))
+
+
+def prepass_finish(slots, M_total: int, K: int, has_ref: bool, cfg: Config, mode: int, prec, stats, ws: Workspace,
+                   stream=None):
+    _ck(lib().sb_prepass_finish(_p(slots), M_total, K, int(has_ref), ctypes.byref(cfg), mode, _p(prec), _p(stats),
+                                ws.ptr, _stream(stream)))
+
+
+def nvfp4_encode(X, cfg: Config, prec, stats, a4: Fp4Tensor, ws: Workspace, stream=None):
+    M, K = X.shape
+    _ck(lib().sb_nvfp4_encode(_p(X), M, K, ctypes.byref(cfg), _p(prec), _p(stats), ctypes.byref(a4.c()), ws.ptr,
+                              _stream(stream)))
+
+
+def tdc_record_partial(y_new, y_cache, row0: int, M_total: int, state, slots, ws: Workspace,
+                       update_cache: bool = True, stream=None):
+    M, C = y_new.shape
+    _ck(lib().sb_tdc_record_partial(_p(y_new), _p(y_cache), M, C, row0, M_total, int(update_cache), _p(state),
+                                    _p(slots), ws.ptr, _stream(stream)))
+
+
+def tdc_finish(slots, M_total: int, C: int, d_src, state, ws: Workspace, stream=None):
+    _ck(lib().sb_tdc_finish(_p(slots), M_total, C, _p(d_src), _p(state), ws.ptr, _stream(stream)))
 
 
 def tdc_refresh(x, y, delta, state, stream=None):
