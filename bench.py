@@ -177,14 +177,12 @@ class FfnStep:
         X = self.X if X is None else X
         Y = self.Y if Y is None else Y
         cfg = sb.config(rho=64.0, tdc_thresh=-1.0, block=128, force_prec=prec)  # never skip: full work
-        sb.tdc_step(self.state, cfg)
-        sb.select_precision(self.state, self.rule, cfg, self.p1)
+        sb.module_decide(self.state, cfg, [self.rule, self.rule], [self.p1, self.p2])  # TDC check, both layers
         self._mark(ev, "pre1_0")
         sb.prepass(X, None, cfg, sb.PREPASS_QUANT, self.p1, self.ax4, self.ax8, self.sx, self.ws)
         self._mark(ev, "pre1_1")
         sb.linear(X, self.ax4, self.ax8, self.p1, self.w1, self.H, epilogue=sb.EPI_GELU, ws=self.ws)
         self._mark(ev, "gemm1_1")
-        sb.select_precision(self.state, self.rule, cfg, self.p2)
         self._mark(ev, "pre2_0")
         sb.prepass(self.H, None, cfg, sb.PREPASS_QUANT, self.p2, self.ah4, self.ah8, self.sh, self.ws)
         self._mark(ev, "pre2_1")
@@ -209,7 +207,7 @@ class FfnStep:
                 ev.append((prec, sub))
 
 
-LAUNCHES_PER_PASS = 11  # tdc_step, select, prepass(2), gemm, select, prepass(2), gemm, stats prepass, tdc record
+LAUNCHES_PER_PASS = 9  # decide, prepass(2), gemm, prepass(2), gemm, stats prepass, tdc record
 
 
 def capture(torch, fn):
@@ -406,7 +404,7 @@ def run_ours(args):
                                f"-> W1 [{N1} x {K1}] (GELU) -> W2 [{N2} x {K2}]; NVFP4 pass + INT8 pass per step",
                    "tokens": M, "hidden": K1, "ffn": N1, "hadamard_block": 128, "parallelism": f"replicas x{world}",
                    "l2": "flushed before every step (512 MiB memset, outside the per-step events)",
-                   "launch": "each step replays one CUDA graph of its 22 kernels"},
+                   "launch": "each step replays one CUDA graph of its 18 kernels"},
         "roofline": roofline,
         "roofline_prepass": {r["kernel"]: {"achieved_gbs": round(r["achieved"], 1), "frac": round(r["frac"], 4),
                                            "ms": round(r["ms"], 4)} for r in pre},

@@ -169,6 +169,13 @@ sb_status sb_tdc_step(sb_module_state* state, const sb_config* cfg /* host */, s
 sb_status sb_select_precision(const sb_module_state* state, const sb_rule* rule /* host */,
                               const sb_config* cfg /* host */, int32_t* prec, sb_stream stream);
 
+/* sb_tdc_step followed by sb_select_precision for each of a module's n layers (1 <= n <= 8), in
+ * one launch: rules[i] (host array) decides *precs[i] (host array of device int32 pointers, 4-byte
+ * aligned) from the state the TDC check leaves. Same results as the separate calls. */
+sb_status sb_module_decide(sb_module_state* state, const sb_config* cfg /* host */, int32_t n,
+                           const sb_rule* rules /* host */, int32_t* const* precs /* host */,
+                           sb_stream stream);
+
 /* Activation pre-pass of one layer input X [M][K] bf16 ("write-up" sections 一, 三, 四).
  * One pass computes the statistics record *stats (PDR ratio on the raw X; d against X_ref when
  * given) and, in SB_PREPASS_QUANT mode, the block-Hadamard-rotated quantized activations for the

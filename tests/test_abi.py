@@ -160,3 +160,19 @@ def test_shard_validation_without_gpu(sb):
                                    None) == sb.SB_ESHAPE
     assert L.sb_tdc_finish(slots, 0, 64, None, _fake(0x300), ws, None) == sb.SB_ESHAPE
     assert L.sb_nvfp4_encode(X, 64, 256, ctypes.byref(cfg), prec, _fake(0x200), None, ws, None) == sb.SB_EINVAL
+
+
+def test_module_decide_validation_without_gpu(sb):
+    L = sb.lib()
+    cfg = sb.config()
+    rules = (sb.Rule * 2)(sb.Rule(1.0, 0.0, 0.1), sb.Rule(1.0, 0.0, 0.2))
+    precs = (ctypes.c_void_p * 2)(0x100, 0x200)
+    r, p = ctypes.cast(rules, ctypes.c_void_p), ctypes.cast(precs, ctypes.c_void_p)
+    st = _fake(0x1000)
+    assert L.sb_module_decide(st, ctypes.byref(cfg), 0, r, p, None) == sb.SB_EINVAL
+    assert L.sb_module_decide(st, ctypes.byref(cfg), 9, r, p, None) == sb.SB_EINVAL
+    assert L.sb_module_decide(None, ctypes.byref(cfg), 2, r, p, None) == sb.SB_EINVAL
+    bad = (ctypes.c_void_p * 2)(0x100, 0x202)
+    assert L.sb_module_decide(st, ctypes.byref(cfg), 2, r, ctypes.cast(bad, ctypes.c_void_p), None) == sb.SB_EALIGN
+    null = (ctypes.c_void_p * 2)(0x100, None)
+    assert L.sb_module_decide(st, ctypes.byref(cfg), 2, r, ctypes.cast(null, ctypes.c_void_p), None) == sb.SB_EINVAL

@@ -72,8 +72,10 @@ def test_tdc_zero_cache_gives_inf(sbg):
     assert sbg.decode_state(st)["delta"] == float("inf")
 
 
-def test_decision_kernels_follow_the_oracle_state_machine(sbg):
-    """Drive the device state with dyadic deltas and ds; compare every field after every call."""
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "module_decide"])
+def test_decision_kernels_follow_the_oracle_state_machine(sbg, fused):
+    """Drive the device state with dyadic deltas and ds; compare every field after every call
+    (the TDC check and the layers' precision choices as separate launches, or as one)."""
     ws = sbg.Workspace(32, 128)
     st = sbg.alloc_state()
     os_ = oracle.State()
@@ -85,13 +87,21 @@ def test_decision_kernels_follow_the_oracle_state_machine(sbg):
     cache = torch.zeros_like(base)
     # outputs y_k = 1 + k/32 so that delta between consecutive computed outputs is dyadic
     k_out = 0
+    rule2 = sbg.Rule(0.5, 0.0625, 0.0625)
+    prec2 = torch.zeros(1, dtype=torch.int32, device="cuda")
     for t in range(24):
-        sbg.tdc_step(st, cfg)
+        if fused:
+            sbg.module_decide(st, cfg, [rule, rule2], [prec, prec2])
+        else:
+            sbg.tdc_step(st, cfg)
+            sbg.select_precision(st, rule, cfg, prec)
+            sbg.select_precision(st, rule2, cfg, prec2)
         oracle.tdc_step(os_, 0.125)
-        sbg.select_precision(st, rule, cfg, prec)
         p_ref = oracle.select_precision(os_, 1.0, 0.0, 0.1)
+        p2_ref = oracle.select_precision(os_, 0.5, 0.0625, 0.0625)
         torch.cuda.synchronize()
         assert int(prec.item()) == p_ref, t
+        assert int(prec2.item()) == p2_ref, t
         assert gstate_dict(sbg, st) == ostate_dict(os_), t
         if p_ref == oracle.SKIP:
             continue

@@ -210,6 +210,27 @@ sb_status sb_select_precision(const sb_module_state* state, const sb_rule* rule,
   return ok();
 }
 
+sb_status sb_module_decide(sb_module_state* state, const sb_config* cfg, int32_t n, const sb_rule* rules,
+                           int32_t* const* precs, sb_stream stream) {
+  SB_REQUIRE(state && cfg && rules && precs, SB_EINVAL, "state, cfg, rules and precs are required");
+  SB_ALIGNED(state, "state");
+  SB_REQUIRE(n >= 1 && n <= sb::kDecideMax, SB_EINVAL, "n must be in [1, %d] (got %d)", sb::kDecideMax, (int)n);
+  SB_REQUIRE(cfg->force_prec >= -1 && cfg->force_prec <= 2, SB_EINVAL, "force_prec must be -1, 0, 1 or 2");
+  sb::DecideLayers L{};
+  L.n = n;
+  for (int i = 0; i < n; ++i) {
+    SB_REQUIRE(precs[i] != nullptr, SB_EINVAL, "precs[%d] is NULL", i);
+    SB_REQUIRE((reinterpret_cast<uintptr_t>(precs[i]) & 3u) == 0, SB_EALIGN, "precs[%d] misaligned", i);
+    L.a[i] = rules[i].a;
+    L.b[i] = rules[i].b;
+    L.tau[i] = rules[i].tau;
+    L.prec[i] = precs[i];
+  }
+  cudaError_t e = sb::launch_decide(state, cfg->tdc_thresh, cfg->force_prec, L, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_module_decide");
+  return ok();
+}
+
 sb_status sb_prepass(const void* X, const void* X_ref, int64_t M, int64_t K, const sb_config* cfg, int32_t mode,
                      int32_t* prec, const sb_fp4* a4, const sb_i8* a8, sb_stats* stats, void* ws,
                      sb_stream stream) {

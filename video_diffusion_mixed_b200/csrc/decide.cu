@@ -24,8 +24,7 @@ __global__ void k_state_init(sb_module_state* st) {
 // "write-up" section 二: two outputs are needed before the change can be predicted; after that
 // the per-step change delta accumulates and the module is skipped while the sum stays within the
 // threshold. A skipped step leaves no input/output difference for the next step (section 三).
-__global__ void k_tdc_step(sb_module_state* st, double thr) {
-  if (threadIdx.x != 0) return;
+__device__ __forceinline__ void tdc_step(sb_module_state* st, double thr) {
   int skip = 0;
   if (st->n_out >= 2) {
     const double acc = __dadd_rn(st->acc, st->delta);
@@ -42,20 +41,28 @@ __global__ void k_tdc_step(sb_module_state* st, double thr) {
 
 // "write-up" sections 一 and 三: INT8 for a changing module (linear rule on the previous step's
 // difference), NVFP4 for a stable one, INT8 after a restart or at the first step.
+__device__ __forceinline__ int32_t select_precision(const sb_module_state* st, double a, double b, double tau,
+                                                    int force) {
+  if (st->skip) return SB_SKIP;
+  if (force >= 0) return force;
+  if (!st->have_d) return SB_INT8;
+  const double v = __dadd_rn(__dmul_rn(a, st->prev_d), b);
+  return (v > tau) ? SB_INT8 : SB_NVFP4;
+}
+
+__global__ void k_tdc_step(sb_module_state* st, double thr) {
+  if (threadIdx.x == 0) tdc_step(st, thr);
+}
+
 __global__ void k_select(const sb_module_state* st, double a, double b, double tau, int force, int32_t* prec) {
+  if (threadIdx.x == 0) *prec = select_precision(st, a, b, tau, force);
+}
+
+// Both in one launch: the module's TDC check, then the precision of each of its layers.
+__global__ void k_decide(sb_module_state* st, double thr, int force, DecideLayers L) {
   if (threadIdx.x != 0) return;
-  int p;
-  if (st->skip) {
-    p = SB_SKIP;
-  } else if (force >= 0) {
-    p = force;
-  } else if (!st->have_d) {
-    p = SB_INT8;
-  } else {
-    const double v = __dadd_rn(__dmul_rn(a, st->prev_d), b);
-    p = (v > tau) ? SB_INT8 : SB_NVFP4;
-  }
-  *prec = p;
+  tdc_step(st, thr);
+  for (int i = 0; i < L.n; ++i) *L.prec[i] = select_precision(st, L.a[i], L.b[i], L.tau[i], force);
 }
 
 __global__ void k_set_i32(int32_t* p, int32_t v) {
@@ -80,6 +87,11 @@ cudaError_t launch_tdc_step(sb_module_state* st, double thr, cudaStream_t s) {
 cudaError_t launch_select(const sb_module_state* st, double a, double b, double tau, int force, int32_t* prec,
                           cudaStream_t s) {
   k_select<<<1, 32, 0, s>>>(st, a, b, tau, force, prec);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decide(sb_module_state* st, double thr, int force, const DecideLayers& L, cudaStream_t s) {
+  k_decide<<<1, 32, 0, s>>>(st, thr, force, L);
   return cudaGetLastError();
 }
 

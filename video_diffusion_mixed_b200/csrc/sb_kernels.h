@@ -99,6 +99,15 @@ cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s);
 cudaError_t launch_rotate(const void* X, float* Y, int64_t M, int64_t K, int B, cudaStream_t s);
 cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s);
 cudaError_t launch_finish(const FinishLaunch& p, cudaStream_t s);
+
+// The decision of one module step: its layers' rules and precision flags (at most kDecideMax).
+constexpr int kDecideMax = 8;
+struct DecideLayers {
+  int n;
+  double a[kDecideMax], b[kDecideMax], tau[kDecideMax];
+  int32_t* prec[kDecideMax];
+};
+cudaError_t launch_decide(sb_module_state* st, double thr, int force, const DecideLayers& L, cudaStream_t s);
 cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t s, const char** why);
 
 cudaError_t launch_state_init(sb_module_state* st, cudaStream_t s);

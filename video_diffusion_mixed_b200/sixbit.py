@@ -99,6 +99,7 @@ def lib():
             "sb_nvfp4_encode": (st, [vp, i64, i64, P(Config), vp, vp, P(Fp4), vp, vp]),
             "sb_tdc_record_partial": (st, [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp]),
             "sb_tdc_finish": (st, [vp, i64, i64, vp, vp, vp, vp]),
+            "sb_module_decide": (st, [vp, P(Config), i32, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -112,7 +113,7 @@ EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_in
             "sb_state_init", "sb_rotate", "sb_prepare_weight", "sb_tdc_step", "sb_select_precision", "sb_prepass",
             "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static", "sb_wait_flag", "sb_tdc_refresh",
             "sb_tdc_reuse", "sb_group_slots_bytes", "sb_prepass_partial", "sb_prepass_finish", "sb_nvfp4_encode",
-            "sb_tdc_record_partial", "sb_tdc_finish")
+            "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide")
 
 
 def _ck(status: int):
@@ -275,6 +276,15 @@ def tdc_record(y_new, y_cache, d_src, state, ws: Workspace, update_cache: bool =
 
 def check(ws: Workspace, stream=None):
     _ck(lib().sb_check(ws.ptr, _stream(stream)))
+
+
+def module_decide(state, cfg: Config, rules, precs, stream=None):
+    """sb_module_decide: the TDC check, then precs[i] from rules[i], in one launch."""
+    n = len(rules)
+    R = (Rule * n)(*rules)
+    Pp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in precs])
+    _ck(lib().sb_module_decide(_p(state), ctypes.byref(cfg), n, ctypes.cast(R, ctypes.c_void_p),
+                               ctypes.cast(Pp, ctypes.c_void_p), _stream(stream)))
 
 
 # ---- token sharding (include/sixbit.h): partial row work, slot gathering, final reduction ----
