@@ -45,10 +45,10 @@ TRAFFIC = {
     "gemm_w1_nvfp4": {"bytes": 487.6e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
     "gemm_w2_nvfp4": {"bytes": 269.0e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
     # k_prepass_blk + k_nvfp4_blk (the encode exits at once in the INT8 pass)
-    "prepass_h_nvfp4": {"bytes": 942.1e6, "files": _ROWS_SRC, "sha": "5974f16fb8c4f6b3"},
-    "prepass_h_int8": {"bytes": 577.0e6, "files": _ROWS_SRC, "sha": "5974f16fb8c4f6b3"},
-    "prepass_x_nvfp4": {"bytes": 218.7e6, "files": _ROWS_SRC, "sha": "5974f16fb8c4f6b3"},
-    "prepass_x_int8": {"bytes": 112.8e6, "files": _ROWS_SRC, "sha": "5974f16fb8c4f6b3"},
+    "prepass_h_nvfp4": {"bytes": 941.1e6, "files": _ROWS_SRC, "sha": "3f4b80ad2d9b6473"},
+    "prepass_h_int8": {"bytes": 577.2e6, "files": _ROWS_SRC, "sha": "3f4b80ad2d9b6473"},
+    "prepass_x_nvfp4": {"bytes": 218.8e6, "files": _ROWS_SRC, "sha": "3f4b80ad2d9b6473"},
+    "prepass_x_int8": {"bytes": 111.7e6, "files": _ROWS_SRC, "sha": "3f4b80ad2d9b6473"},
 }
 TRAFFIC_TOKENS = 17776
 
