@@ -119,3 +119,50 @@ def test_sharded_tdc_record_matches_oracle(sbg, M, C, cuts):
     assert s["delta"] == oracle.tdc_delta(u16(y1), u16(y0))[0]
     assert s["n_out"] == 2 and s["acc"] == 0.0 and s["have_d"] == 0
     assert torch.equal(cache, y1)
+
+
+@pytest.mark.parametrize("block", [256, 64])
+def test_sharded_prepass_other_block_sizes(sbg, block):
+    """B = 256 runs the 32-element row engine, B = 64 the block-per-lane kernel with its B = 64
+    instance: both stop at the group slots when asked to."""
+    M, K = 100, 1024
+    X = synth.activations(M, K, n_outlier=3, scale=25.0, seed=8, device="cuda")
+    ref = oracle.prepass(u16(X), None, block)
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    cfg = sbg.config(rho=64.0, block=block, force_prec=sbg.INT8)
+    ws = sbg.Workspace(M, K)
+    slots = sbg.alloc_slots(M)
+    prec = torch.tensor([sbg.INT8], dtype=torch.int32, device="cuda")
+    parts = []
+    for r0, r1 in ((0, 48), (48, 100)):
+        a8 = sbg.I8Tensor(r1 - r0, K)
+        sbg.prepass_partial(X[r0:r1], None, r0, M, cfg, sbg.PREPASS_QUANT, prec, a8, slots, ws)
+        parts.append(a8)
+    stats = sbg.alloc_stats()
+    sbg.prepass_finish(slots, M, K, False, cfg, sbg.PREPASS_QUANT, prec, stats, ws)
+    sbg.check(ws)
+    st = sbg.decode_stats(stats)
+    for k in STATS:
+        assert st[k] == ref[k], k
+    assert np.array_equal(np.concatenate([npy(a.codes) for a in parts]), q)
+
+
+def test_sharded_difference_statistic(sbg):
+    """The d of a module output against its input (STATS mode with x_ref, the row engine without
+    rotation), sharded: the finished record equals the oracle's and leaves *prec alone."""
+    M, K = 17776, 3072
+    X, _ = synth.workload_inputs("ffn5b", seed=0, device="cuda")
+    Y = synth.noisy_copy(X, 0.1, seed=1)
+    ref = oracle.prepass(u16(Y), u16(X), 128, want_rot=False)
+    cfg = sbg.config(rho=0.0, block=128)
+    ws = sbg.Workspace(M, K)
+    slots = sbg.alloc_slots(M)
+    for r0, r1 in ((0, 6000), (6000, 12000), (12000, M)):
+        sbg.prepass_partial(Y[r0:r1], X[r0:r1], r0, M, cfg, sbg.PREPASS_STATS, None, None, slots, ws)
+    stats = sbg.alloc_stats()
+    sbg.prepass_finish(slots, M, K, True, cfg, sbg.PREPASS_STATS, None, stats, ws)
+    sbg.check(ws)
+    st = sbg.decode_stats(stats)
+    for k in ("sum_abs", "sum_d2", "sum_ref2", "max_abs", "ratio", "d"):
+        assert st[k] == ref[k], (k, st[k], ref[k])
+    assert st["prec_out"] == -1
