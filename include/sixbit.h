@@ -192,6 +192,20 @@ sb_status sb_prepass(const void* X, const void* X_ref, int64_t M, int64_t K,
                      const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */, sb_stats* stats,
                      void* ws, sb_stream stream);
 
+/* sb_prepass for a tensor whose per-chunk statistics its producer already computed (FFN-pair
+ * fusion: the layer that writes X hands these over, so the pre-pass does not read X for them).
+ * chunks: device float4 records [M][K/128], one per aligned 128-channel chunk of a row:
+ * x = max |H_B x| over the chunk (B = cfg->block <= 128), y = the canonical pairwise sum of |x|
+ * over its 128 values, z = max |x|; w is scratch: the call leaves the row's rotated amax in the
+ * w of its first record. The records fold into the same statistics record, PDR verdict and INT8
+ * scales as sb_prepass computes from X; in QUANT mode X is then read once for the codes (INT8
+ * when *prec said INT8 at the start, NVFP4 when it says NVFP4 after PDR). X_ref is not
+ * supported. Requires K % 128 == 0 and block <= 128 (SB_EUNSUPPORTED), else as sb_prepass. */
+sb_status sb_prepass_chunks(const void* X, float* chunks, int64_t M, int64_t K,
+                            const sb_config* cfg /* host */, int32_t mode, int32_t* prec,
+                            const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */, sb_stats* stats,
+                            void* ws, sb_stream stream);
+
 /* Quantized linear layer Y = X W^T + bias ("write-up" section 四; tcgen05 tensor cores):
  *   NVFP4: Y = acc * s_gx * s_gw / B + bias, acc = sum of block-scaled E2M1 products
  *          (tcgen05.mma kind::mxf4nvf4, UE4M3 scales per 16);

@@ -210,6 +210,63 @@ sb_status sb_select_precision(const sb_module_state* state, const sb_rule* rule,
   return ok();
 }
 
+sb_status sb_prepass_chunks(const void* X, float* chunks, int64_t M, int64_t K, const sb_config* cfg, int32_t mode,
+                            int32_t* prec, const sb_fp4* a4, const sb_i8* a8, sb_stats* stats, void* ws,
+                            sb_stream stream) {
+  SB_REQUIRE(X && chunks && cfg && stats && ws, SB_EINVAL, "X, chunks, cfg, stats and ws are required");
+  SB_ALIGNED(X, "X");
+  SB_ALIGNED(chunks, "chunks");
+  SB_ALIGNED(stats, "stats");
+  SB_ALIGNED(ws, "ws");
+  SB_REQUIRE(mode == SB_PREPASS_QUANT || mode == SB_PREPASS_STATS, SB_EINVAL, "mode must be QUANT or STATS");
+  SB_REQUIRE(cfg->force_prec >= -1 && cfg->force_prec <= 2, SB_EINVAL, "force_prec must be -1, 0, 1 or 2");
+  sb_status st = check_rows_cols(M, K, cfg->block);
+  if (st != SB_OK) return st;
+  SB_REQUIRE(cfg->block <= 128 && K % 128 == 0, SB_EUNSUPPORTED,
+             "chunk records need block <= 128 and K a multiple of 128 (got block %d, K %lld)", (int)cfg->block,
+             (long long)K);
+  if (mode == SB_PREPASS_QUANT) {
+    SB_REQUIRE(prec && a4 && a8, SB_EINVAL, "QUANT mode needs prec, a4 and a8");
+    if ((st = check_fp4(a4, M, K, "a4")) != SB_OK) return st;
+    if ((st = check_i8(a8, M, K, "a8")) != SB_OK) return st;
+  }
+  if (prec) SB_REQUIRE((reinterpret_cast<uintptr_t>(prec) & 3u) == 0, SB_EALIGN, "prec misaligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  sb::PrepassLaunch p{};
+  p.finish = 1;
+  p.X = X;
+  p.M = M;
+  p.K = K;
+  p.B = cfg->block;
+  p.mode = mode;
+  p.prec = prec;
+  p.q8 = (mode == SB_PREPASS_QUANT) ? a8->codes : nullptr;
+  p.s8 = (mode == SB_PREPASS_QUANT) ? a8->scale : nullptr;
+  p.rho = cfg->rho;
+  p.force = cfg->force_prec;
+  p.groups = ws_groups(ws);
+  p.hdr = ws;
+  p.stats = stats;
+  cudaError_t e = sb::launch_prepass_chunks(p, chunks, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_prepass_chunks");
+  if (mode == SB_PREPASS_QUANT) {
+    sb::Nvfp4Launch q{};
+    q.X = X;
+    q.M = M;
+    q.K = K;
+    q.B = cfg->block;
+    q.prec = prec;
+    q.stats = stats;
+    q.codes = a4->codes;
+    q.sf = a4->sf;
+    q.gscale = a4->gscale;
+    q.hdr = ws;
+    e = sb::launch_nvfp4(q, s);
+    if (e != cudaSuccess) return cuda_fail(e, "sb_prepass_chunks (NVFP4 encode)");
+  }
+  return ok();
+}
+
 sb_status sb_module_decide(sb_module_state* state, const sb_config* cfg, int32_t n, const sb_rule* rules,
                            int32_t* const* precs, sb_stream stream) {
   SB_REQUIRE(state && cfg && rules && precs, SB_EINVAL, "state, cfg, rules and precs are required");

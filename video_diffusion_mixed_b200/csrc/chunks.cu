@@ -1,0 +1,213 @@
+// chunks.cu -- the pre-pass of a tensor whose per-chunk statistics are already known.
+//
+// The second linear layer of an FFN reads the tensor the first one wrote. If that layer's
+// producer also hands over, for every aligned 128-channel chunk of every row, the chunk's rotated
+// amax, its canonical pairwise sum of |x| and its max |x|, the pre-pass no longer needs a
+// statistics pass over the tensor: the records fold into the row statistics (a chunk is an
+// aligned subtree of its row's sum tree), the group slots and, in the last CTA, the statistics
+// record and the Purified Delta Refresh verdict ("write-up" sections 一, 三, 四). Only the
+// quantization pass reads the tensor: the NVFP4 encode as in sb_prepass, or a streaming INT8
+// pass that knows every row's amax in advance and so needs no team of warps per row.
+//
+//  k_fold_chunks   one warp per 16-row group: per row, the tree over the chunk sums and the
+//                  chunk maxima; INT8 scales; the group's FP64 slot; rows_finish in the last CTA.
+//                  The row's rotated amax is left in the fourth float of its first record.
+//  k_int8_blk      INT8 codes, one 128-channel block per lane (as the NVFP4 encode).
+#include "prepass_blk.cuh"
+#include "tmap.h"
+
+namespace sb {
+
+constexpr int kFoldWarps = 8;
+
+// Canonical pairwise tree over 16 values whose tail is zero (the run of a lane).
+__device__ __forceinline__ float tree16(float (&t)[16]) {
+#pragma unroll
+  for (int len = 16; len > 1; len >>= 1) {
+#pragma unroll
+    for (int i = 0; i < len / 2; ++i) t[i] = __fadd_rn(t[2 * i], t[2 * i + 1]);
+  }
+  return t[0];
+}
+
+__global__ void __launch_bounds__(kFoldWarps * 32) k_fold_chunks(RowArgs a, float4* chunks, int NB) {
+  __shared__ double s_fin[kFinChunk];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int prec = a.prec ? *a.prec : -1;
+  if (prec == SB_SKIP) return;
+  const bool do_int8 = a.mode == SB_PREPASS_QUANT && prec == SB_INT8;
+  const int64_t G = ceil_div(a.M, kG);
+  int NB2 = 1;
+  while (NB2 < NB) NB2 <<= 1;
+  const int c = NB2 >= 32 ? NB2 / 32 : 1;  // chunk sums per lane (a power of two <= 16)
+  const int span = NB2 / c;                // lanes covering one row
+  for (int64_t g = (int64_t)blockIdx.x * kFoldWarps + warp; g < G; g += (int64_t)gridDim.x * kFoldWarps) {
+    float rs = 0.0f, ram = 0.0f, rmx = 0.0f;  // lane i < kG: row i of the group
+    for (int i = 0; i < kG; ++i) {
+      const int64_t m = g * kG + i;
+      float t[16];
+      float am = 0.0f, mx = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int idx = lane * c + u;
+        t[u] = 0.0f;
+        if (m < a.M && u < c && idx < NB) {
+          const float4 r = chunks[m * NB + idx];
+          t[u] = r.y;
+          am = fmaxf(am, r.x);
+          mx = fmaxf(mx, r.z);
+        }
+      }
+      float v = tree16(t);
+      for (int s = 1; s < span; s <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
+      v = __shfl_sync(0xffffffffu, v, 0);  // lanes 0 .. span-1 hold the row; past them only zeros
+      am = warp_max_f32(am);
+      mx = warp_max_f32(mx);
+      if (lane == i) {
+        rs = v;
+        ram = am;
+        rmx = mx;
+      }
+      if (lane == 0 && m < a.M) {
+        chunks[m * NB].w = am;
+        if (do_int8) a.s8[m] = (am == 0.0f) ? 0.0f : __fdiv_rn(am, 127.0f);
+      }
+    }
+    const bool in = lane < kG;
+    const double gs = warp_pairwise_f64(in ? (double)rs : 0.0);
+    const float gam = warp_max_f32(in ? ram : 0.0f);
+    const float gmx = warp_max_f32(in ? rmx : 0.0f);
+    const int gnf = __any_sync(0xffffffffu, in && !isfinite(rs));
+    if (lane == 0) {
+      GroupSlot* gsl = a.groups + g;
+      gsl->s[0] = gs;
+      gsl->s[1] = 0.0;
+      gsl->s[2] = 0.0;
+      gsl->max_abs = gmx;
+      gsl->amax_rot = gam;
+      gsl->nonfinite = gnf;
+    }
+  }
+  rows_finish<OP_PREPASS, false>(a, G, prec, true, s_fin);
+}
+
+// INT8 codes of the rows, with every row's amax known: a warp streams 32 consecutive blocks per
+// task through a two-slot TMA ring, a lane rotates its block and writes its 128 codes. Written
+// when the flag said INT8 when the pre-pass began (stats->prec_in), as sb_prepass writes them.
+template <int B>
+__global__ void __launch_bounds__(kPbThreads, 1) k_int8_blk(RowArgs a, const float4* chunks, int NB,
+                                                           const __grid_constant__ CUtensorMap mx) {
+  extern __shared__ uint8_t pb_dsm[];
+  __shared__ uint64_t s_bar[kPbWarps][kPbD];
+  const int p = a.prec ? *a.prec : -1;
+  if (p == SB_SKIP || a.mode != SB_PREPASS_QUANT || a.stats->prec_in != SB_INT8) return;
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pb_dsm) + 1023) & ~(uintptr_t)1023);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t nblk = a.M * NB;
+  const int ntask = (int)ceil_div(nblk, 32);
+  const int nw = (int)gridDim.x * kPbWarps;
+  const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * kPbD * kPbSlot);
+  auto issue = [&](int t, int slot) {  // lane 0
+    if (t >= ntask) return;
+    const uint32_t bar = smem_u32(&s_bar[warp][slot]);
+    mbar_arrive_expect_tx_u32(bar, (uint32_t)kPbSlot);
+    tma_load_2d_u32(ring_w + (uint32_t)(slot * kPbSlot), &mx, bar, 0, 64 * t);
+  };
+  const int t0 = (int)blockIdx.x * kPbWarps + warp;
+  if (lane == 0) {
+    mbar_init(&s_bar[warp][0], 1);
+    mbar_init(&s_bar[warp][1], 1);
+    fence_barrier_init();
+    issue(t0, 0);
+    issue(t0 + nw, 1);
+  }
+  __syncwarp();
+  int bad_it = -1;
+  for (int it = 0, t = t0; t < ntask; ++it, t += nw) {
+    const int slot = it & 1;
+    if (lane == 0 && it > 0) issue(t + nw, slot ^ 1);  // the previous task's slot, read there
+    if (!mbar_wait_bounded(&s_bar[warp][slot], (uint32_t)((it >> 1) & 1), nullptr, kRowWaitNs)) {
+      if (lane == 0) set_error(a.hdr, SB_ETIMEOUT);
+      bad_it = it;
+    }
+    float2 P[64];
+    pb_load_block(ring_w + (uint32_t)(slot * kPbSlot), lane, P);
+#pragma unroll
+    for (int k = 0; k < 64; k += 2) {
+      const float2 x = P[k], y = P[k + 1];
+      P[k] = add2(x, y);
+      P[k + 1] = sub2(x, y);
+    }
+    (void)pb_stages_rest<B>(P, pb_swap(lane) ? -1.0f : 1.0f);
+    const int64_t f = (int64_t)t * 32 + lane;
+    if (f >= nblk) continue;
+    const int64_t m = f / NB;
+    pb_store_int8(P, chunks[m * NB].w, a.q8 + f * 128, lane);
+  }
+  if (bad_it >= 0 && lane == 0)
+    mbar_wait_bounded(&s_bar[warp][bad_it & 1], (uint32_t)((bad_it >> 1) & 1), nullptr, kRowDrainNs);
+}
+
+static int chunks_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int B>
+static cudaError_t launch_int8_blk(const RowArgs& a, const float4* chunks, int NB, const CUtensorMap& mx,
+                                   cudaStream_t s) {
+  constexpr int dsm = kPbRing + 1024;
+  static bool attr = false;  // once per instantiation
+  if (!attr) {
+    cudaFuncSetAttribute(k_int8_blk<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
+    attr = true;
+  }
+  const int64_t want = ceil_div(ceil_div(a.M * NB, 32), kPbWarps);
+  const int sms = chunks_sms();
+  const unsigned grid = (unsigned)(want < sms ? want : sms);
+  k_int8_blk<B><<<grid, kPbThreads, dsm, s>>>(a, chunks, NB, mx);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prepass_chunks(const PrepassLaunch& p, float* chunks, cudaStream_t s) {
+  RowArgs a{};
+  a.X = reinterpret_cast<const __nv_bfloat16*>(p.X);
+  a.M = p.M;
+  a.K = (int)p.K;
+  a.B = p.B;
+  a.mode = p.mode;
+  a.prec = p.prec;
+  a.q8 = p.q8;
+  a.s8 = p.s8;
+  a.rho = p.rho;
+  a.force = p.force;
+  a.groups = reinterpret_cast<GroupSlot*>(p.groups);
+  a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
+  a.stats = p.stats;
+  a.finish = 1;
+  const int NB = (int)(p.K / 128);
+  float4* c4 = reinterpret_cast<float4*>(chunks);
+  const int64_t G = ceil_div(p.M, kG);
+  const int64_t want = ceil_div(G, kFoldWarps);
+  const int sms = chunks_sms();
+  k_fold_chunks<<<(unsigned)(want < sms ? want : sms), kFoldWarps * 32, 0, s>>>(a, c4, NB);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.mode != SB_PREPASS_QUANT) return e;
+  CUtensorMap mx;
+  if (!make_halfblock_map(&mx, p.X, p.M, p.K)) return cudaErrorInvalidValue;
+  switch (p.B) {
+    case 16: return launch_int8_blk<16>(a, c4, NB, mx, s);
+    case 32: return launch_int8_blk<32>(a, c4, NB, mx, s);
+    case 64: return launch_int8_blk<64>(a, c4, NB, mx, s);
+    case 128: return launch_int8_blk<128>(a, c4, NB, mx, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace sb

@@ -99,6 +99,7 @@ cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s);
 cudaError_t launch_rotate(const void* X, float* Y, int64_t M, int64_t K, int B, cudaStream_t s);
 cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s);
 cudaError_t launch_finish(const FinishLaunch& p, cudaStream_t s);
+cudaError_t launch_prepass_chunks(const PrepassLaunch& p, float* chunks, cudaStream_t s);
 
 // The decision of one module step: its layers' rules and precision flags (at most kDecideMax).
 constexpr int kDecideMax = 8;

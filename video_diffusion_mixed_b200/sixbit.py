@@ -100,6 +100,7 @@ def lib():
             "sb_tdc_record_partial": (st, [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp]),
             "sb_tdc_finish": (st, [vp, i64, i64, vp, vp, vp, vp]),
             "sb_module_decide": (st, [vp, P(Config), i32, vp, vp, vp]),
+            "sb_prepass_chunks": (st, [vp, vp, i64, i64, P(Config), i32, vp, P(Fp4), P(I8), vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -113,7 +114,7 @@ EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_in
             "sb_state_init", "sb_rotate", "sb_prepare_weight", "sb_tdc_step", "sb_select_precision", "sb_prepass",
             "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static", "sb_wait_flag", "sb_tdc_refresh",
             "sb_tdc_reuse", "sb_group_slots_bytes", "sb_prepass_partial", "sb_prepass_finish", "sb_nvfp4_encode",
-            "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide")
+            "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide", "sb_prepass_chunks")
 
 
 def _ck(status: int):
@@ -247,6 +248,16 @@ def prepass(X, X_ref, cfg: Config, mode: int, prec, a4: Fp4Tensor | None, a8: I8
     c8 = ctypes.byref(a8.c()) if a8 is not None else None
     _ck(lib().sb_prepass(_p(X), _p(X_ref), M, K, ctypes.byref(cfg), mode, _p(prec), c4, c8, _p(stats), ws.ptr,
                          _stream(stream)))
+
+
+def prepass_chunks(X, chunks, cfg: Config, mode: int, prec, a4: Fp4Tensor | None, a8: I8Tensor | None, stats,
+                   ws: Workspace, stream=None):
+    """sb_prepass_chunks: the pre-pass from the producer's chunk records (float32 [M, K/128, 4])."""
+    M, K = X.shape
+    c4 = ctypes.byref(a4.c()) if a4 is not None else None
+    c8 = ctypes.byref(a8.c()) if a8 is not None else None
+    _ck(lib().sb_prepass_chunks(_p(X), _p(chunks), M, K, ctypes.byref(cfg), mode, _p(prec), c4, c8, _p(stats),
+                                ws.ptr, _stream(stream)))
 
 
 def prepass_static(X, X_ref, cfg: Config, mode: int, prec, a4: Fp4Tensor | None, a8: I8Tensor | None, stats,
