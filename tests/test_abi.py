@@ -176,3 +176,21 @@ def test_module_decide_validation_without_gpu(sb):
     assert L.sb_module_decide(st, ctypes.byref(cfg), 2, r, ctypes.cast(bad, ctypes.c_void_p), None) == sb.SB_EALIGN
     null = (ctypes.c_void_p * 2)(0x100, None)
     assert L.sb_module_decide(st, ctypes.byref(cfg), 2, r, ctypes.cast(null, ctypes.c_void_p), None) == sb.SB_EINVAL
+
+
+def test_prepass_chunks_validation_without_gpu(sb):
+    L = sb.lib()
+    cfg = sb.config()
+    a4 = sb.Fp4(0x1000, 0x2000, 0x3000, 64, 1024)
+    a8 = sb.I8(0x4000, 0x5000, 64, 1024)
+    X, chunks, stats, ws, prec = _fake(0x10000), _fake(0x20000), _fake(0x200), _fake(0x300), _fake(0x100)
+    ok = (ctypes.byref(a4), ctypes.byref(a8), stats, ws, None)
+    assert L.sb_prepass_chunks(X, None, 64, 1024, ctypes.byref(cfg), 0, prec, *ok) == sb.SB_EINVAL
+    assert L.sb_prepass_chunks(X, _fake(0x20008), 64, 1024, ctypes.byref(cfg), 0, prec, *ok) == sb.SB_EALIGN
+    # chunk records need whole 128-channel chunks and a Hadamard block that fits one
+    big = sb.config(block=256)
+    assert L.sb_prepass_chunks(X, chunks, 64, 1024, ctypes.byref(big), 0, prec, *ok) == sb.SB_EUNSUPPORTED
+    assert L.sb_prepass_chunks(X, chunks, 64, 960, ctypes.byref(cfg), 0, prec, *ok) == sb.SB_EUNSUPPORTED
+    assert "128" in L.sb_last_error().decode()
+    assert L.sb_prepass_chunks(X, chunks, 64, 1024, ctypes.byref(cfg), 0, prec, None, None, stats, ws,
+                               None) == sb.SB_EINVAL
