@@ -13,8 +13,10 @@
  *  - Pointers are DEVICE pointers unless the parameter is marked "host". Structs passed by
  *    pointer (sb_config, sb_rule, sb_weight, sb_fp4, sb_i8) are HOST structs whose pointer
  *    fields are device pointers; sb_module_state and sb_stats live in DEVICE memory.
- *  - The caller owns all memory. The library allocates no device memory and keeps no device
- *    state between calls; scratch lives in the caller's workspace `ws` (sb_workspace_size).
+ *  - The caller owns all memory. The library allocates no device memory; scratch lives in the
+ *    caller's workspace `ws` (sb_workspace_size). The one exception is sb_prepass_static, whose
+ *    scratch is a fixed array compiled into the library (see there); no other call keeps device
+ *    state between calls.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; 0 = legacy default stream).
  *    Calls that share a workspace must be ordered on one stream.
  *  - Arguments are validated synchronously; on failure nothing is launched, the status is
@@ -109,8 +111,9 @@ typedef struct {
   int32_t reserved[3];
 } sb_module_state;
 
-/* Pre-pass statistics (device memory, 96 bytes). Sums are the deterministic pairwise reductions
- * (FP32 per row, FP64 across rows) so that every decision is reproducible bit for bit. */
+/* Pre-pass statistics (device memory, 88 bytes; the Python binding allocates 96). Sums are the
+ * deterministic pairwise reductions (FP32 per row, FP64 across rows) so that every decision is
+ * reproducible bit for bit. */
 typedef struct {
   double sum_abs;   /* sum |x| */
   double sum_d2;    /* sum (x - x_ref)^2 (0 without x_ref) */
@@ -123,7 +126,9 @@ typedef struct {
   int32_t has_ref;  /* d is valid */
   int32_t prec_in;  /* precision on entry */
   int32_t prec_out; /* precision after PDR */
-  int32_t nonfinite;
+  int32_t nonfinite; /* the input X held Inf or NaN (a row's max |x| is Inf or its sum |x| NaN) */
+  int32_t error;     /* written by sb_prepass_static only: the device error word of its call */
+  int32_t reserved;
 } sb_stats;
 
 const char* sb_version(void);
@@ -241,8 +246,11 @@ sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C,
  * launched). The first call on a device looks up the array's device address with
  * cudaGetSymbolAddress (that device must be current), so make that first call before any stream
  * capture. Every call on a device shares the one array: calls that can overlap on the GPU (other
- * streams, other host threads) race and must be serialised by the caller. Device-side errors are
- * reported in stats->nonfinite (there is no workspace for sb_check to read). */
+ * streams, other host threads) race and must be serialised by the caller. There is no workspace
+ * for sb_check to read, so the call ends by copying the array's device error word into
+ * stats->error: SB_OK, SB_ETIMEOUT (a bounded wait gave up; codes and statistics are then
+ * undefined), SB_ENONFINITE (X held Inf/NaN; also in stats->nonfinite) or SB_EINVAL. The next
+ * call clears the word, so read stats->error after each call. */
 #define SB_STATIC_MAX_ROWS 65536
 sb_status sb_prepass_static(const void* X, const void* X_ref, int64_t M, int64_t K,
                             const sb_config* cfg /* host */, int32_t mode, int32_t* prec,

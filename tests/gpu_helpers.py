@@ -39,3 +39,22 @@ def sample_rows(M: int, step: int = 64) -> np.ndarray:
     if r[-1] != M - 1:
         r.append(M - 1)
     return np.array(r, dtype=np.int64)
+
+
+def assert_close(got, ref, tol: float = 1e-3):
+    """The output tolerance of the quantized and BF16 linear layers, checked two ways:
+    relative Frobenius error <= tol over the whole compared block, and elementwise
+    |got - ref| <= tol * max|ref| + tol * |ref|, which a localized error (one wrong column group,
+    one wrong tile) would break even when it is too small to move the Frobenius norm. The
+    elementwise bound holds for every correct kernel here: FP32 accumulation and the FP32
+    dequant/bias epilogue err by a few FP32 ulps of the row's magnitude, the SFU tanh of the GELU
+    by about 2^-11 of 0.5 |v|, both far below 1e-3 of the block's largest output."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    fro = rel_fro(got, ref)
+    assert fro <= tol, f"relative Frobenius error {fro:.3e} > {tol:g}"
+    bound = tol * float(np.max(np.abs(ref))) + tol * np.abs(ref)
+    err = np.abs(got - ref)
+    bad = np.argwhere(err > bound)
+    assert bad.size == 0, (f"{len(bad)} elements outside the elementwise bound; first at {tuple(bad[0])}: "
+                           f"got {got[tuple(bad[0])]!r}, ref {ref[tuple(bad[0])]!r}")

@@ -77,3 +77,44 @@ def test_chunk_records_pdr_verdict_and_int8_codes(sbg):
     assert st["ratio"] == ref["ratio"] > 64.0
     assert p == oracle.apply_pdr(sbg.INT8, ref["ratio"], 64.0) == sbg.BF16
     assert np.array_equal(npy(a8.codes), q)
+
+
+def test_chunk_records_stats_mode(sbg):
+    """STATS mode: the records fold into the statistics record only; no quantization kernel
+    runs, the precision flag may be absent, the quantized tensors are not touched."""
+    M, K = 300, 3072
+    X = synth.activations(M, K, n_outlier=15, scale=50.0, seed=41, device="cuda")
+    ref = oracle.prepass(u16(X), None, 128)
+    ws = sbg.Workspace(M, K)
+    stats = sbg.alloc_stats()
+    sbg.prepass_chunks(X, _records(X, 128), sbg.config(block=128), sbg.PREPASS_STATS, None, None, None, stats, ws)
+    sbg.check(ws)
+    st = sbg.decode_stats(stats)
+    for k in STATS:
+        assert st[k] == ref[k], (k, st[k], ref[k])
+    assert st["numel"] == M * K and st["nonfinite"] == 0
+
+
+def test_chunk_records_skip_writes_nothing(sbg):
+    """*prec == SB_SKIP: every kernel exits at once -- no statistics, codes or scales are written
+    -- and the workspace's last-CTA ticket stays clean for the next call, which must be exact."""
+    M, K = 200, 1024
+    X = synth.activations(M, K, seed=42, device="cuda")
+    ws = sbg.Workspace(M, K)
+    a4, a8 = sbg.Fp4Tensor(M, K), sbg.I8Tensor(M, K)
+    a4.codes.fill_(0xAB)
+    a8.codes.fill_(0x55)
+    a8.scale.fill_(-1.0)
+    stats = sbg.alloc_stats()
+    stats.fill_(0xEE)
+    prec = torch.tensor([sbg.SKIP], dtype=torch.int32, device="cuda")
+    sbg.prepass_chunks(X, _records(X, 128), sbg.config(block=128), sbg.PREPASS_QUANT, prec, a4, a8, stats, ws)
+    sbg.check(ws)
+    assert int(prec.item()) == sbg.SKIP
+    assert (npy(a4.codes) == 0xAB).all() and (npy(a8.codes) == 0x55).all() and (npy(a8.scale) == -1.0).all()
+    assert (npy(stats) == 0xEE).all()
+    ref = oracle.prepass(u16(X), None, 128)
+    q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
+    a4, a8, st, p = _run(sbg, X, _records(X, 128), sbg.INT8, force=sbg.INT8)
+    assert st["sum_abs"] == ref["sum_abs"] and p == sbg.INT8
+    assert np.array_equal(npy(a8.codes), q)

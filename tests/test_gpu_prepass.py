@@ -242,3 +242,73 @@ def test_prepass_many_groups(sbg, K, B, with_ref):
     q, s = oracle.quant_int8(ref["y"], ref["row_amax"])
     assert np.array_equal(npy(out["a8"].codes), q)
     assert np.array_equal(npy(out["a8"].scale).view(np.uint32), s.view(np.uint32))
+
+
+def _block_scale_code(amax: np.float32, s_g: np.float32) -> int:
+    """E4M3(RN(RN(amax / 6) / s_g)) with numpy's IEEE FP32 divisions and the oracle's E4M3 cast;
+    used only to place inputs on the scale boundaries (expected values come from the oracle)."""
+    with np.errstate(over="ignore"):
+        q = np.float32(np.float32(amax) / np.float32(6.0))
+        return oracle.e4m3_encode(float(np.float32(q / np.float32(s_g))))
+
+
+def _scale_boundaries(s_g: np.float32) -> list:
+    """For every block-scale code c >= 1 reachable from finite amax: the smallest FP32 amax whose
+    scale code is >= c (bisection over the ordered bit patterns of non-negative floats)."""
+    out = []
+    top = _block_scale_code(np.float32(np.finfo(np.float32).max), s_g)
+    for c in range(1, top + 1):
+        lo, hi = 0, 0x7F7FFFFF
+        while lo + 1 < hi:
+            mid = (lo + hi) // 2
+            if _block_scale_code(np.uint32(mid).view(np.float32), s_g) >= c:
+                hi = mid
+            else:
+                lo = mid
+        out.append(np.uint32(hi).view(np.float32))
+    return out
+
+
+def _bf16_parts(v: np.float32):
+    """v = p0 + p1 + p2 exactly, each part a bf16 value (8 significant bits apiece)."""
+    b = int(np.float32(v).view(np.uint32))
+    e, m = (b >> 23) & 0xFF, (b & 0x7FFFFF) | (0x800000 if (b >> 23) & 0xFF else 0)
+    scale = 2.0 ** ((e if e else 1) - 150)
+    parts = [((m >> 16) << 16) * scale, (((m >> 8) & 0xFF) << 8) * scale, (m & 0xFF) * scale]
+    assert sum(parts) == float(v)
+    return parts
+
+
+@pytest.mark.parametrize("A", [1000.0, 0.75, 24576.0])  # bf16-exact tensor maxima
+def test_nvfp4_block_scales_on_every_boundary(sbg, A):
+    """Group maxima placed exactly on, one ulp below and one ulp above every block-scale rounding
+    boundary, for three tensor scales: with B = 16 a block with x0 + x1 + x2 in its first three
+    channels (each part a bf16 value) rotates to a group whose amax is exactly the FP32 value
+    x0 + x1 + x2. The encode's table-driven scale choice must match the oracle's plain arithmetic
+    (two IEEE divisions, then the E4M3 cast) on every such group, codes and scales alike."""
+    s_g = np.float32(np.float32(A) / np.float32(2688.0))
+    targets = []
+    for T in _scale_boundaries(s_g):
+        for v in (np.nextafter(T, np.float32(0)), T, np.nextafter(T, np.float32(np.inf))):
+            if 0 < v < A:
+                targets.append(v)
+    K = 2048  # 128 groups of 16 per row
+    rows = (len(targets) + 127) // 128 + 1
+    X = torch.zeros((rows, K), dtype=torch.float32)
+    X[0, 0] = A  # the tensor amax: sets s_g
+    for i, v in enumerate(targets):
+        r, g = 1 + i // 128, i % 128
+        for j, p in enumerate(_bf16_parts(v)):
+            X[r, 16 * g + j] = p
+    Xb = X.to(torch.bfloat16)
+    assert torch.equal(Xb.float(), X)  # every part is bf16-exact
+    Xb = Xb.cuda()
+    ref = oracle.prepass(u16(Xb), None, 16)
+    assert ref["amax_rot"] == A
+    out = run_prepass(sbg, Xb, force=sbg.NVFP4, block=16)
+    codes, sfl, sft, sg = oracle.quant_nvfp4(ref["y"], ref["amax_rot"])
+    assert np.float32(npy(out["a4"].gscale)[0]) == sg == s_g
+    # the groups really sit on distinct scale codes on both sides of each boundary
+    assert len(np.unique(sfl[1:])) >= 100
+    assert np.array_equal(npy(out["a4"].sf), sft)
+    assert np.array_equal(npy(out["a4"].codes), codes)

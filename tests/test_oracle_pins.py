@@ -88,6 +88,43 @@ def test_pairwise_order_hand_worked(orc):
     assert orc.pairwise_f32(np.zeros(0, np.float32)) == 0.0
 
 
+def test_pairwise_f64_order_hand_worked(orc):
+    """The FP64 tree across row groups: the same hand-worked cases one precision up, which a
+    left-to-right (or right-to-left) FP64 fold gets wrong."""
+    big = 2.0 ** 53
+    # [2^53,1,1,1]: (2^53+1 -> 2^53, tie to even) + (1+1) = 2^53+2; a left-to-right sum gives 2^53
+    assert orc.pairwise_f64(np.array([big, 1, 1, 1])) == big + 2
+    # n=3 pads with one zero: 2^53 + (1+0) -> 2^53 (tie, even)
+    assert orc.pairwise_f64(np.array([big, 1, 1])) == big
+    # n=5 pads to 8: (2^53 + 2) + 1 = 2^53+3 -> tie between +2 and +4 -> 2^53+4
+    assert orc.pairwise_f64(np.array([big, 1, 1, 1, 1])) == big + 4
+    # right-to-left would give (1+1+1) + 2^53 = 2^53+4 for the first case; the tree gives +2
+    assert orc.pairwise_f64(np.array([1, 1, 1, big])) == big + 2
+    # [1, 2^53, 1, 1]: (1+2^53 -> 2^53) + (1+1) = 2^53+2
+    assert orc.pairwise_f64(np.array([1, big, 1, 1])) == big + 2
+    assert orc.pairwise_f64(np.zeros(0)) == 0.0
+
+
+def test_f32_to_bf16_matches_ml_dtypes(orc):
+    """The comparison helper that rounds FP64/FP32 references to bf16 agrees with ml_dtypes' own
+    round-to-nearest-even cast on random values of every magnitude, on every tie (the 16 low bits
+    exactly 0x8000, with an even and an odd kept bit), on subnormals, at the overflow edge and on
+    infinities; a NaN stays a NaN."""
+    ml = pytest.importorskip("ml_dtypes")
+    rng = np.random.default_rng(17)
+    bits = rng.integers(0, 2 ** 32, 200000, dtype=np.uint64).astype(np.uint32)
+    ties = (rng.integers(0, 2 ** 16, 5000, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000
+    edge = np.array([0x7F7F7FFF, 0x7F7F8000, 0x7F7FFFFF, 0xFF7F8000, 0x00008000, 0x00018000, 0x0000FFFF,
+                     0x80008000, 0x7F800000, 0xFF800000, 0x00000000, 0x80000000, 0x3F808000, 0x3F818000],
+                    dtype=np.uint32)
+    x = np.concatenate([bits, ties, edge]).view(np.float32)
+    x = x[~np.isnan(x)]
+    ref = x.astype(ml.bfloat16).view(np.uint16)
+    assert np.array_equal(orc.f32_to_bf16(x), ref)
+    nan = np.array([np.nan, -np.nan], dtype=np.float32)
+    assert np.isnan(orc.bf16_to_f32(orc.f32_to_bf16(nan))).all()
+
+
 def test_pairwise_accuracy(orc):
     rng = np.random.default_rng(3)
     t = rng.random(10007).astype(np.float32)

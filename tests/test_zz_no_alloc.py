@@ -54,6 +54,24 @@ def test_static_scratch_matches_workspace_version_twice_in_a_row(sbg):
             assert torch.equal(got["g4"], ref["g4"])
         st = sbg.decode_stats(got["stats"])
         assert st["nonfinite"] == 0 and st["numel"] == M * K
+        assert st["error"] == sbg.SB_OK  # the static scratch's device error word, copied out
+
+
+def test_static_scratch_reports_device_errors_in_stats(sbg):
+    """There is no workspace for sb_check to read, so a device-side error of the call reaches the
+    caller through stats->error: a NaN in X gives SB_ENONFINITE there. The next call starts from a
+    cleared error word and reports SB_OK."""
+    M, K = 256, 1024
+    X = synth.activations(M, K, seed=24, device="cuda")
+    X.view(torch.int16)[17, 99] = 0x7FC0  # a bf16 NaN
+    got = _run(sbg, "static", X, None, sbg.INT8)
+    st = sbg.decode_stats(got["stats"])
+    assert st["error"] == sbg.SB_ENONFINITE and st["nonfinite"] == 1
+    Xf = synth.activations(M, K, seed=25, device="cuda")
+    got = _run(sbg, "static", Xf, None, sbg.INT8)
+    ref = _run(sbg, "ws", Xf, None, sbg.INT8, sbg.Workspace(M, K))
+    assert sbg.decode_stats(got["stats"])["error"] == sbg.SB_OK
+    assert torch.equal(got["stats"], ref["stats"]) and torch.equal(got["q8"], ref["q8"])
 
 
 def test_static_scratch_rejects_too_many_rows(sbg):

@@ -21,7 +21,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsixbit.so")
 SOURCES = ["api.cu", "prepass.cu", "decide.cu", "gemm.cu", "prepass_static.cu", "reuse.cu", "chunks.cu"]
-HEADERS = ["sb_device.cuh", "sb_kernels.h", "rows.cuh", "prepass_blk.cuh", "tmap.h"]
+HEADERS = ["sb_device.cuh", "sb_kernels.h", "rows.cuh", "prepass_blk.cuh", "tmap.h", "launch_util.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2,-Wall",

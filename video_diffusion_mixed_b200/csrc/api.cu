@@ -4,7 +4,7 @@
 //   [0, 128)    WsHeader (device error word, last-CTA tickets)
 //   [128, 224)  sb_stats scratch (weight preparation)
 //   [224, 228)  int32 precision scratch (weight preparation)
-//   [256, ...)  one 48-byte GroupSlot per aligned group of 32 rows
+//   [256, ...)  one 48-byte GroupSlot per aligned group of 16 rows (kGroupRows)
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>

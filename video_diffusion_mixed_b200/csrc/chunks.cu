@@ -13,6 +13,7 @@
 //                  chunk maxima; INT8 scales; the group's FP64 slot; rows_finish in the last CTA.
 //                  The row's rotated amax is left in the fourth float of its first record.
 //  k_int8_blk      INT8 codes, one 128-channel block per lane (as the NVFP4 encode).
+#include "launch_util.h"
 #include "prepass_blk.cuh"
 #include "tmap.h"
 
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(kFoldWarps * 32) k_fold_chunks(RowArgs a, floa
     const double gs = warp_pairwise_f64(in ? (double)rs : 0.0);
     const float gam = warp_max_f32(in ? ram : 0.0f);
     const float gmx = warp_max_f32(in ? rmx : 0.0f);
-    const int gnf = __any_sync(0xffffffffu, in && !isfinite(rs));
+    const int gnf = __any_sync(0xffffffffu, in && (isnan(rs) || isinf(rmx)));  // Inf or NaN in a row
     if (lane == 0) {
       GroupSlot* gsl = a.groups + g;
       gsl->s[0] = gs;
@@ -125,6 +126,7 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_int8_blk(RowArgs a, const flo
   int bad_it = -1;
   for (int it = 0, t = t0; t < ntask; ++it, t += nw) {
     const int slot = it & 1;
+    __syncwarp();  // every lane has read the previous task's slot (lanes may drift apart)
     if (lane == 0 && it > 0) issue(t + nw, slot ^ 1);  // the previous task's slot, read there
     if (!mbar_wait_bounded(&s_bar[warp][slot], (uint32_t)((it >> 1) & 1), nullptr, kRowWaitNs)) {
       if (lane == 0) set_error(a.hdr, SB_ETIMEOUT);
@@ -148,26 +150,15 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_int8_blk(RowArgs a, const flo
     mbar_wait_bounded(&s_bar[warp][bad_it & 1], (uint32_t)((bad_it >> 1) & 1), nullptr, kRowDrainNs);
 }
 
-static int chunks_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
+static int chunks_sms() { return device_sm_count(); }
 
 template <int B>
 static cudaError_t launch_int8_blk(const RowArgs& a, const float4* chunks, int NB, const CUtensorMap& mx,
                                    cudaStream_t s) {
   constexpr int dsm = kPbRing + 1024;
-  static bool attr = false;  // once per instantiation
-  if (!attr) {
-    cudaFuncSetAttribute(k_int8_blk<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};  // per instantiation, one bit per device
+  const cudaError_t e = smem_attr_once(k_int8_blk<B>, dsm, attr);
+  if (e != cudaSuccess) return e;
   const int64_t want = ceil_div(ceil_div(a.M * NB, 32), kPbWarps);
   const int sms = chunks_sms();
   const unsigned grid = (unsigned)(want < sms ? want : sms);

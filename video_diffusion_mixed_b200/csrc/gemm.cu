@@ -35,6 +35,7 @@
 
 #include <mutex>
 
+#include "launch_util.h"
 #include "sb_device.cuh"
 #include "sb_kernels.h"
 #include "tmap.h"
@@ -103,6 +104,7 @@ struct GemmParams {
   int out_dtype;
   int epilogue;
   int tma_store;  // bf16 output through shared memory and TMA stores
+  int group_m;    // M-tiles per raster group (tile_coords)
   WsHeader* hdr;
 };
 
@@ -164,16 +166,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Grouped tile order: kGroupM consecutive M-tiles are swept across all N-tiles before the next
-// group starts, so the A rows of a group stay in L2 while every N-tile reuses them (A of the
-// second FFN layer is larger than L2 and would otherwise be re-read from HBM for each N-tile).
-constexpr int kGroupM = 8;
-
-__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int* mt, int* nt) {
-  const int group = kGroupM * n_tiles;
+// Grouped tile order: group_m consecutive M-tiles are swept across all N-tiles before the next
+// group starts (M-tile fastest inside a group), so the A rows of a group stay in L2 while every
+// N-tile reuses them (A of the second FFN layer is larger than L2 and would otherwise be re-read
+// from HBM for each N-tile). The host picks group_m (pick_group_m).
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int group_m, int* mt, int* nt) {
+  const int group = group_m * n_tiles;
   const int g = t / group, r = t - g * group;
-  const int first = g * kGroupM;
-  const int gm = min(kGroupM, m_tiles - first);
+  const int first = g * group_m;
+  const int gm = min(group_m, m_tiles - first);
   *mt = first + r % gm;
   *nt = r / gm;
 }
@@ -280,7 +281,7 @@ struct EpiCtx {
   uint32_t tempty_leader;  // shared::cluster address of the leader's tempty[0]
   volatile int* abort;
   uint32_t tmem;
-  int unit, tiles, nunits, m_tiles, n_tiles, nacc, BN, M, N, row_off, q, half, lane;
+  int unit, tiles, nunits, m_tiles, n_tiles, group_m, nacc, BN, M, N, row_off, q, half, lane;
   uint32_t out_box;  // this warp's two staging boxes
   uint32_t bias_s;   // NVFP4: this warp's bias slice in shared memory
   float alpha;
@@ -316,7 +317,7 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
   int it = 0;
   for (int tile = e.unit; tile < e.tiles; tile += e.nunits, ++it) {
     int mt, nt;
-    tile_coords(tile, e.m_tiles, e.n_tiles, &mt, &nt);
+    tile_coords(tile, e.m_tiles, e.n_tiles, e.group_m, &mt, &nt);
     const int m = mt * 256 + e.row_off + row;
     const int m_warp = mt * 256 + e.row_off + 32 * e.q;
     const int n0 = nt * e.BN + e.half * (e.BN / 2);
@@ -414,7 +415,7 @@ struct Issuer {
   volatile int* abort;
   uint32_t smem;      // shared address of stage 0
   uint32_t stage16;   // stage size in 16-byte units
-  int stages, nkb, tail_nk, tiles, unit, nunits, BN, nacc, m_tiles, n_tiles;
+  int stages, nkb, tail_nk, tiles, unit, nunits, BN, nacc, m_tiles, n_tiles, group_m;
   uint32_t tmem, sfa, sfb, idesc;  // TMEM base, scale columns (absolute), instruction descriptor
 };
 
@@ -480,7 +481,7 @@ __device__ __noinline__ bool issue_all(const Issuer c) {
     uint32_t shift = 0;
     if (KIND == KIND_FP4) {
       int mt, nt;
-      tile_coords(tile, c.m_tiles, c.n_tiles, &mt, &nt);
+      tile_coords(tile, c.m_tiles, c.n_tiles, c.group_m, &mt, &nt);
       shift = (uint32_t)(((nt * c.BN) & 127) >> 5);
     }
     for (int kb = 0; kb < c.nkb; ++kb) {
@@ -585,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int tile = unit; ok && tile < tiles; tile += nunits) {
           int mt, nt;
-          tile_coords(tile, m_tiles, n_tiles, &mt, &nt);
+          tile_coords(tile, m_tiles, n_tiles, p.group_m, &mt, &nt);
           const int m0 = mt * 256 + row_off, n0 = nt * BN;
           for (int kb = 0; kb < nkb; ++kb) {
             if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitNs)) {
@@ -643,6 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         c.BN = BN;
         c.m_tiles = m_tiles;
         c.n_tiles = n_tiles;
+        c.group_m = p.group_m;
         c.nacc = nacc;
         c.tmem = tmem_base;
         c.sfa = tmem_base + sfa_col;
@@ -678,6 +680,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     e.nunits = nunits;
     e.m_tiles = m_tiles;
     e.n_tiles = n_tiles;
+    e.group_m = p.group_m;
     e.nacc = nacc;
     e.BN = BN;
     e.M = M;
@@ -740,19 +743,24 @@ static bool make_sf_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t r
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static int device_sms() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+static int device_sms() { return device_sm_count(); }
+
+// M-tiles per raster group. Wide outputs (many N-tiles: the first FFN layer) keep groups of 8
+// M-tiles: A stays in L2 across the N sweep while the weight streams. Narrow outputs (at most 16
+// N-tiles: the second FFN layer, the attention projection) take as many M-tiles as one wave of
+// the persistent grid covers with every N-tile, so a wave reads each A row slab once, shared by
+// all N-tiles at the same K position, and the whole weight, which stays in L2 from wave to wave.
+static int pick_group_m(int64_t m_tiles, int64_t n_tiles, int64_t units) {
+  if (n_tiles > 16) return 8;
+  int64_t g = units / n_tiles;
+  if (g < 1) g = 1;
+  if (g > m_tiles) g = m_tiles;
+  return (int)g;
 }
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  });
+  static std::atomic<uint64_t> attr{0};  // one bit per device
+  const cudaError_t attr_err = smem_attr_once(k_gemm, kSmemBytes, attr);
   if (attr_err != cudaSuccess) {
     *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
     return attr_err;
@@ -839,6 +847,7 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   const int64_t want = 2 * ceil_div(L.M, 256) * ceil_div(L.N, bn_q < bn_f ? bn_q : bn_f);
   const int sms = device_sms() & ~1;
   const unsigned grid = (unsigned)(want < sms ? want : sms);
+  p.group_m = pick_group_m(ceil_div(L.M, 256), ceil_div(L.N, bn_q), grid / 2);
   k_gemm<<<grid, kThreads, kSmemBytes, s>>>(tm, p);
   return cudaGetLastError();
 }

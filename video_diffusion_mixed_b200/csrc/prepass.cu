@@ -13,22 +13,14 @@
 //  k_nvfp4        re-reads X once the tensor amax is known, rotates again and writes E2M1 codes,
 //                 E4M3 block scales in the tensor-core layout and the FP32 tensor scale.
 //  k_rotate       rotation only (test hook).
+#include "launch_util.h"
 #include "prepass_blk.cuh"
 #include "rows.cuh"
 #include "tmap.h"
 
 namespace sb {
 
-static int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
+static int sm_count() { return device_sm_count(); }
 
 static RowArgs row_args_from(const PrepassLaunch& p) {
   RowArgs a{};
@@ -61,11 +53,9 @@ static void row_maps(RowArgs& a, RowMaps& mp, const void* X, const void* R) {
 template <int B>
 static cudaError_t launch_pb(const RowArgs& a, const PbGeom& gm, const CUtensorMap& mx, unsigned grid, cudaStream_t s) {
   constexpr int dsm = kPbRing + 1024;
-  static bool attr = false;  // once per instantiation
-  if (!attr) {
-    cudaFuncSetAttribute(k_prepass_blk<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};  // per instantiation, one bit per device
+  const cudaError_t e = smem_attr_once(k_prepass_blk<B>, dsm, attr);
+  if (e != cudaSuccess) return e;
   k_prepass_blk<B><<<grid, kPbThreads, dsm, s>>>(a, gm, mx);
   return cudaGetLastError();
 }
@@ -262,10 +252,69 @@ __device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v
   return w;
 }
 
+// Per-tensor tables of the block-scale arithmetic, built by every CTA from the tensor scale s_g
+// (a few hundred IEEE divisions per CTA, overlapped with its first loads). The block scale of a
+// 16-value group is sb(amax) = E4M3(RN(RN(amax / 6) / s_g)), a monotone step function of amax,
+// and its codes use inv(sb) = RN(1 / RN(dec(sb) s_g)):
+//   thr[c]  the smallest amax with sb(amax) >= c (NaN when no amax reaches c, so that every
+//           comparison with it is false); thr[0] = 0
+//   inv[c]  inv(c), or 0 when the group's codes are all zero (dec(c) s_g = 0, or 1 / den
+//           overflows)
+// In the encode, c0 = E4M3(RN(amax K)) with K = RN(1 / RN(6 s_g)) is within one code of sb(amax):
+// the two arguments differ by a few FP32 ulps, and E4M3 rounding boundaries are more than 2^-5
+// apart relatively (2^-9 absolutely among its subnormals), so at most one boundary lies between
+// them. Two comparisons with thr then give sb(amax) exactly: three instructions and two
+// shared-memory loads instead of three IEEE divisions per group.
+constexpr int kScaleCodes = 128;
+
+__device__ __forceinline__ uint32_t block_scale_code(float amax, float s_g) {
+  return cvt_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_g));
+}
+
+__device__ __forceinline__ void build_scale_tables(float s_g, float* inv, float* thr) {
+  const int t = (int)threadIdx.x;
+  if (t < kScaleCodes) {
+    const float den = __fmul_rn(e4m3_to_f32((uint32_t)t), s_g);
+    float r = (den == 0.0f) ? 0.0f : __fdiv_rn(1.0f, den);
+    if (!(r <= FLT_MAX)) r = 0.0f;  // 1 / den overflowed (or the NaN code): zero codes
+    inv[t] = r;
+  } else if (t < 2 * kScaleCodes + 1) {
+    const uint32_t c = (uint32_t)(t - kScaleCodes);  // 0 .. 128
+    float v;
+    if (c == 0) {
+      v = 0.0f;
+    } else if (block_scale_code(__uint_as_float(0x7f800000u), s_g) < c) {
+      v = __uint_as_float(0x7fc00000u);  // unreachable code: NaN, never <= amax
+    } else {
+      // smallest non-negative float bit pattern b with sb(b) >= c (non-negative floats order
+      // like their bit patterns, and sb is monotone): invariant sb(lo) < c <= sb(hi)
+      uint32_t lo = 0u, hi = 0x7f800000u;
+      if (block_scale_code(0.0f, s_g) >= c) hi = 0u;
+      while (lo + 1u < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (block_scale_code(__uint_as_float(mid), s_g) >= c) hi = mid;
+        else lo = mid;
+      }
+      v = __uint_as_float(hi);
+    }
+    thr[c] = v;
+  }
+}
+
+// Block scale code of one group from its candidate c0 and the thresholds (see above).
+__device__ __forceinline__ uint32_t scale_from_tables(float amax, const float* thr, uint32_t c0) {
+  uint32_t c = c0;
+  if (amax >= thr[c0 + 1]) c = c0 + 1;
+  else if (amax < thr[c0]) c = c0 - 1;
+  return c;
+}
+
 template <int B>
 __global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB, const __grid_constant__ CUtensorMap mx) {
   extern __shared__ uint8_t pb_dsm[];
   __shared__ uint64_t s_bar[kPbWarps][kPbD];
+  __shared__ float s_inv[kScaleCodes];
+  __shared__ float s_thr[kScaleCodes + 1];
   if (a.prec && *a.prec != SB_NVFP4) return;
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pb_dsm) + 1023) & ~(uintptr_t)1023);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -278,11 +327,13 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB
   const int ntask = (int)ceil_div(nblk, 32);
   const int nw = (int)gridDim.x * kPbWarps;
   const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * kPbD * kPbSlot);
+  // Tasks run from the end of the tensor backwards: the statistics pass that ran just before
+  // read the end last, so that part is still in L2 (all of a tensor that fits).
   auto issue = [&](int t, int slot) {  // lane 0
     if (t >= ntask) return;
     const uint32_t bar = smem_u32(&s_bar[warp][slot]);
     mbar_arrive_expect_tx_u32(bar, (uint32_t)kPbSlot);
-    tma_load_2d_u32(ring_w + (uint32_t)(slot * kPbSlot), &mx, bar, 0, 64 * t);
+    tma_load_2d_u32(ring_w + (uint32_t)(slot * kPbSlot), &mx, bar, 0, 64 * (ntask - 1 - t));
   };
   const int t0 = (int)blockIdx.x * kPbWarps + warp;
   if (lane == 0) {
@@ -292,10 +343,13 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB
     issue(t0, 0);
     issue(t0 + nw, 1);
   }
-  __syncwarp();
+  build_scale_tables(s_g, s_inv, s_thr);
+  __syncthreads();
+  const float kmul = __fdiv_rn(1.0f, __fmul_rn(6.0f, s_g));
   int bad_it = -1;
   for (int it = 0, t = t0; t < ntask; ++it, t += nw) {
     const int slot = it & 1;
+    __syncwarp();  // every lane has read the previous task's slot (lanes may drift apart)
     if (lane == 0 && it > 0) issue(t + nw, slot ^ 1);  // the previous task's slot, read there
     if (!mbar_wait_bounded(&s_bar[warp][slot], (uint32_t)((it >> 1) & 1), nullptr, kRowWaitNs)) {
       if (lane == 0) set_error(a.hdr, SB_ETIMEOUT);
@@ -310,7 +364,7 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB
       P[k + 1] = sub2(x, y);
     }
     (void)pb_stages_rest<B>(P, pb_swap(lane) ? -1.0f : 1.0f);
-    const int64_t f = (int64_t)t * 32 + lane;
+    const int64_t f = (int64_t)(ntask - 1 - t) * 32 + lane;
     if (f >= nblk) continue;
     const int64_t m = f / NB;
     const int blk = (int)(f - m * NB);
@@ -320,27 +374,30 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_nvfp4_blk(Nvfp4Args a, int NB
     uint32_t sbx = 0, sby = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float ax = 0.0f, ay = 0.0f;
+      float ax0 = 0.0f, ay0 = 0.0f, ax1 = 0.0f, ay1 = 0.0f;  // two chains per half
 #pragma unroll
-      for (int u = 0; u < 16; u += 2) {
-        ax = max3(ax, fabsf(P[16 * i + u].x), fabsf(P[16 * i + u + 1].x));
-        ay = max3(ay, fabsf(P[16 * i + u].y), fabsf(P[16 * i + u + 1].y));
+      for (int u = 0; u < 8; u += 2) {
+        ax0 = max3(ax0, fabsf(P[16 * i + u].x), fabsf(P[16 * i + u + 1].x));
+        ay0 = max3(ay0, fabsf(P[16 * i + u].y), fabsf(P[16 * i + u + 1].y));
+        ax1 = max3(ax1, fabsf(P[16 * i + 8 + u].x), fabsf(P[16 * i + 8 + u + 1].x));
+        ay1 = max3(ay1, fabsf(P[16 * i + 8 + u].y), fabsf(P[16 * i + 8 + u + 1].y));
       }
-      uint32_t bx, by;
-      float ix, iy;
-      bool zx, zy;
-      group_scale(ax, s_g, &bx, &ix, &zx);
-      group_scale(ay, s_g, &by, &iy, &zy);
+      const float ax = fmaxf(ax0, ax1), ay = fmaxf(ay0, ay1);
+      uint16_t c2;  // candidate codes of both groups in one conversion: x in the low byte
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c2) : "f"(__fmul_rn(ay, kmul)), "f"(__fmul_rn(ax, kmul)));
+      const uint32_t bx = scale_from_tables(ax, s_thr, (uint32_t)c2 & 0xffu);
+      const uint32_t by = scale_from_tables(ay, s_thr, (uint32_t)c2 >> 8);
+      const float ix = s_inv[bx], iy = s_inv[by];
       sbx |= bx << (8 * i);
       sby |= by << (8 * i);
       const float2 inv2 = make_float2(ix, iy);
       float2 q[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) q[u] = mul2(P[16 * i + u], inv2);
-      w[2 * i] = zx ? 0u : e2m1x8(q[0].x, q[1].x, q[2].x, q[3].x, q[4].x, q[5].x, q[6].x, q[7].x);
-      w[2 * i + 1] = zx ? 0u : e2m1x8(q[8].x, q[9].x, q[10].x, q[11].x, q[12].x, q[13].x, q[14].x, q[15].x);
-      w[8 + 2 * i] = zy ? 0u : e2m1x8(q[0].y, q[1].y, q[2].y, q[3].y, q[4].y, q[5].y, q[6].y, q[7].y);
-      w[9 + 2 * i] = zy ? 0u : e2m1x8(q[8].y, q[9].y, q[10].y, q[11].y, q[12].y, q[13].y, q[14].y, q[15].y);
+      w[2 * i] = (ix == 0.0f) ? 0u : e2m1x8(q[0].x, q[1].x, q[2].x, q[3].x, q[4].x, q[5].x, q[6].x, q[7].x);
+      w[2 * i + 1] = (ix == 0.0f) ? 0u : e2m1x8(q[8].x, q[9].x, q[10].x, q[11].x, q[12].x, q[13].x, q[14].x, q[15].x);
+      w[8 + 2 * i] = (iy == 0.0f) ? 0u : e2m1x8(q[0].y, q[1].y, q[2].y, q[3].y, q[4].y, q[5].y, q[6].y, q[7].y);
+      w[9 + 2 * i] = (iy == 0.0f) ? 0u : e2m1x8(q[8].y, q[9].y, q[10].y, q[11].y, q[12].y, q[13].y, q[14].y, q[15].y);
     }
     const int hx = (int)pb_swap(lane), hy = 1 - hx;  // which half of the block x and y are
     if (m < a.M) {
@@ -404,11 +461,9 @@ static unsigned stream_grid(int64_t units) {
 template <int B>
 static cudaError_t launch_nvfp4_blk(const Nvfp4Args& a, int NB, const CUtensorMap& mx, unsigned grid, cudaStream_t s) {
   constexpr int dsm = kPbRing + 1024;
-  static bool attr = false;  // once per instantiation
-  if (!attr) {
-    cudaFuncSetAttribute(k_nvfp4_blk<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};  // per instantiation, one bit per device
+  const cudaError_t e = smem_attr_once(k_nvfp4_blk<B>, dsm, attr);
+  if (e != cudaSuccess) return e;
   k_nvfp4_blk<B><<<grid, kPbThreads, dsm, s>>>(a, NB, mx);
   return cudaGetLastError();
 }

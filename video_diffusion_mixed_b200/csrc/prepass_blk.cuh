@@ -396,8 +396,11 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
           const float rs = in ? s_gsum[team][lane] : 0.0f;
           const double gs = warp_pairwise_f64((double)rs);
           const float gam = warp_max_f32(in ? s_gam[team][lane] : 0.0f);
-          const float gmx = warp_max_f32(in ? s_grm[team][lane] : 0.0f);
-          const int gnf = __any_sync(0xffffffffu, in && !isfinite(rs));
+          const float rm = in ? s_grm[team][lane] : 0.0f;
+          const float gmx = warp_max_f32(rm);
+          // non-finite input: an infinite |x| makes the row max infinite, a NaN makes the row sum
+          // NaN (a finite row whose sum overflows to +inf is not flagged)
+          const int gnf = __any_sync(0xffffffffu, isnan(rs) || isinf(rm));
           if (lane == 0) {
             GroupSlot* gsl = a.groups + g;
             gsl->s[0] = gs;

@@ -10,6 +10,10 @@
 // In host code the array's name is only a stand-in, never a device address: the address is
 // looked up with cudaGetSymbolAddress, once per device, with that device current, on the first
 // call made on that device; later calls reuse it.
+//
+// Device-side errors (a bounded wait that gave up, non-finite input) land in the array's error
+// word, which no caller can read; the call therefore ends with a one-thread kernel that copies
+// that word into stats->error.
 #include <mutex>
 
 #include "sb_device.cuh"
@@ -24,6 +28,10 @@ __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+
+// The scratch's device error word (the first word of its header) into the caller's statistics
+// record, after the pre-pass kernels on the same stream.
+__global__ void k_copy_error(const uint32_t* err, sb_stats* stats) { stats->error = (int32_t)*err; }
 
 }  // namespace
 
@@ -55,5 +63,10 @@ extern "C" sb_status sb_prepass_static(const void* X, const void* X_ref, int64_t
   // zero, so they are cleared on the stream before the kernels run.
   if (cudaMemsetAsync(scratch, 0, 256, (cudaStream_t)stream) != cudaSuccess)
     return sb::report_error(SB_ECUDA, "sb_prepass_static: clearing the scratch header failed");
-  return sb_prepass(X, X_ref, M, K, cfg, mode, prec, a4, a8, stats, scratch, stream);
+  const sb_status ps = sb_prepass(X, X_ref, M, K, cfg, mode, prec, a4, a8, stats, scratch, stream);
+  if (ps != SB_OK) return ps;
+  k_copy_error<<<1, 1, 0, (cudaStream_t)stream>>>(static_cast<const uint32_t*>(scratch), stats);
+  if (cudaGetLastError() != cudaSuccess)
+    return sb::report_error(SB_ECUDA, "sb_prepass_static: launching the error-word copy failed");
+  return SB_OK;
 }

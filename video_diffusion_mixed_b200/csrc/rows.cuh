@@ -22,6 +22,7 @@
 
 #include <cfloat>
 
+#include "launch_util.h"
 #include "sb_device.cuh"
 #include "sb_kernels.h"
 
@@ -674,7 +675,7 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
         for (int s = 0; s < NST; ++s) s_rowpart[gpar][s][i] = part[s];
         s_rowamax[gpar][i] = a_m;
         s_rowmax[gpar][i] = rmax;
-        s_rownf[gpar][i] = isfinite(part[0]) ? 0 : 1;
+        s_rownf[gpar][i] = (isnan(part[0]) || isinf(rmax)) ? 1 : 0;  // Inf or NaN in the row
       }
       // ---- per-token INT8 of the rotated row held in registers
       if (OP == OP_PREPASS && do_int8) {
@@ -783,12 +784,12 @@ cudaError_t launch_rows_t(const RowArgs& a, const RowMaps& mp, cudaStream_t s, i
 #define SB_ROWS_CASE(TT, SS)                                                                              \
   if (T == TT && SPW == SS) {                                                                             \
     constexpr int dsm = RowRing<SS, OP, REF>::BYTES + 1024;                                               \
-    static int occ = 0;                                                                                   \
-    if (occ == 0) {                                                                                       \
-      cudaFuncSetAttribute(k_rows<TT, SS, OP, REF>, cudaFuncAttributeMaxDynamicSharedMemorySize, dsm);    \
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_rows<TT, SS, OP, REF>, kRowWarps * 32, dsm); \
-      if (occ <= 0) occ = 1;                                                                              \
-    }                                                                                                     \
+    static std::atomic<uint64_t> attr{0}; /* one bit per device */                                      \
+    const cudaError_t ae = smem_attr_once(k_rows<TT, SS, OP, REF>, dsm, attr);                            \
+    if (ae != cudaSuccess) return ae;                                                                     \
+    int occ = 0;                                                                                          \
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_rows<TT, SS, OP, REF>, kRowWarps * 32, dsm);   \
+    if (occ <= 0) occ = 1;                                                                                \
     const int64_t cap = (int64_t)sms * occ; /* persistent: one wave of resident CTAs */                   \
     const unsigned grid = (unsigned)(ngroups < cap ? ngroups : cap);                                      \
     k_rows<TT, SS, OP, REF><<<grid, kRowWarps * 32, dsm, s>>>(a, mp);                                     \

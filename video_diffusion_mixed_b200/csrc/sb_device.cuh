@@ -21,12 +21,13 @@ namespace sb {
 // Workspace layout (caller-owned memory; see sb_workspace_size)
 // ---------------------------------------------------------------------------------------------
 
-// One slot per aligned group of 32 rows: FP64 pairwise partial sums of the group, maxima.
+// One slot per aligned group of kGroupRows (16) rows: FP64 pairwise partial sums of the group,
+// maxima.
 struct GroupSlot {
   double s[3];       // per-statistic group sum (pre-pass: |x|, (x-r)^2, r^2; TDC: |a-b|, |b|)
   float max_abs;     // max |x| of the group (raw)
   float amax_rot;    // max |Hx| of the group (rotated)
-  int32_t nonfinite; // a row sum was Inf/NaN
+  int32_t nonfinite; // a row held Inf/NaN: its max |x| is Inf or its sum |x| NaN
   int32_t pad[3];
 };
 static_assert(sizeof(GroupSlot) == 48, "GroupSlot layout");

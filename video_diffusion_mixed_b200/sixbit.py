@@ -61,7 +61,7 @@ STATE_BYTES = 64
 STATS_BYTES = 96
 STATE_FIELDS = ("prev_d", "acc", "delta", "have_d", "n_out", "last_skipped", "skip", "steps")
 STATS_FIELDS = ("sum_abs", "sum_d2", "sum_ref2", "max_abs", "amax_rot", "ratio", "d", "numel", "has_ref",
-                "prec_in", "prec_out", "nonfinite")
+                "prec_in", "prec_out", "nonfinite", "error")
 
 _lib = None
 
@@ -202,6 +202,11 @@ def alloc_state(device="cuda", stream=None) -> torch.Tensor:
     return st
 
 
+def state_init(state: torch.Tensor, stream=None):
+    """Reset an existing module state (sb_state_init)."""
+    _ck(lib().sb_state_init(_p(state), _stream(stream)))
+
+
 def alloc_stats(device="cuda") -> torch.Tensor:
     return torch.zeros(STATS_BYTES, dtype=torch.uint8, device=device)
 
@@ -216,7 +221,7 @@ def decode_state(buf: torch.Tensor) -> dict:
 def decode_stats(buf: torch.Tensor) -> dict:
     h = buf.detach().cpu()
     d = h[:64].view(torch.float64).tolist()
-    i = h[64:80].view(torch.int32).tolist()
+    i = h[64:84].view(torch.int32).tolist()
     return dict(zip(STATS_FIELDS, d + i))
 
 
