@@ -195,12 +195,14 @@ class FfnStep:
 
     def _mark(self, ev, name):
         if ev is not None:
-            e = self.torch.cuda.Event(enable_timing=True)
+            # external: inside a graph capture the record becomes an event node of the graph, so
+            # the kernels between two marks are timed as the graph runs them
+            e = self.torch.cuda.Event(enable_timing=True, external=True)
             e.record()
             ev.append((name, e))
 
-    def step(self, ev=None):
-        for prec in (self.sb.NVFP4, self.sb.INT8):
+    def step(self, ev=None, precs=None):
+        for prec in precs or (self.sb.NVFP4, self.sb.INT8):
             sub = [] if ev is not None else None
             self.one_pass(prec, sub)
             if ev is not None:
@@ -208,6 +210,121 @@ class FfnStep:
 
 
 LAUNCHES_PER_PASS = 9  # decide, prepass(2), gemm, prepass(2), gemm, stats prepass, tdc record
+
+
+class L2Flush:
+    """Empties L2 between timed steps: a 512 MiB memset (larger than the 126 MB L2), then a read
+    of a 256 MiB buffer, which writes the memset's dirty lines back and leaves L2 holding clean
+    lines. Without the read the first kernel of a step would pay for writing back about 126 MB of
+    zeros, a cost no real step has. Both run outside the timed events."""
+
+    def __init__(self, torch, device):
+        self.w = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+    def zero_(self):  # the write alone (where the flush sits inside a timed span)
+        self.w.zero_()
+
+
+class ShardedFfnStep:
+    """The FFN step with the token axis split over the ranks (sequence parallelism): each rank
+    holds S.M rows of a tensor of world * S.M rows and does the row work of its rows (rotation,
+    quantization, GEMMs, cache refresh); the whole-tensor statistics -- the pre-pass of X and of
+    the hidden tensor (PDR ratio, NVFP4 tensor amax), the d statistic and the TDC delta -- are
+    assembled from every rank's group slots by one int64 all-reduce SUM each (`gather`), after
+    which every rank runs the same final reduction and gets the same statistics, decisions and
+    module state as one GPU holding all rows. `gather` is sixbit.gather_slots under torchrun and
+    the identity on one rank. Every rank issues the same calls in the same order."""
+
+    def __init__(self, sb, S, rank, world, gather):
+        self.sb, self.S, self.gather = sb, S, gather
+        self.row0, self.Mt = rank * S.M, world * S.M
+        dev = S.X.device
+        self.slots = [sb.alloc_slots(self.Mt, device=dev) for _ in range(4)]
+
+    def one_pass(self, prec):
+        sb, S, g = self.sb, self.S, self.gather
+        cfg = sb.config(rho=64.0, tdc_thresh=-1.0, block=128, force_prec=prec)
+        for sl in self.slots:
+            sl.zero_()  # every rank's copy starts zero-filled; each rank writes only its groups
+        sb.module_decide(S.state, cfg, [S.rule, S.rule], [S.p1, S.p2])
+        sb.prepass_partial(S.X, None, self.row0, self.Mt, cfg, sb.PREPASS_QUANT, S.p1, S.ax8, self.slots[0], S.ws)
+        g(self.slots[0])
+        sb.prepass_finish(self.slots[0], self.Mt, S.K1, False, cfg, sb.PREPASS_QUANT, S.p1, S.sx, S.ws)
+        sb.nvfp4_encode(S.X, cfg, S.p1, S.sx, S.ax4, S.ws)
+        sb.linear(S.X, S.ax4, S.ax8, S.p1, S.w1, S.H, epilogue=sb.EPI_GELU, ws=S.ws)
+        sb.prepass_partial(S.H, None, self.row0, self.Mt, cfg, sb.PREPASS_QUANT, S.p2, S.ah8, self.slots[1], S.ws)
+        g(self.slots[1])
+        sb.prepass_finish(self.slots[1], self.Mt, S.K2, False, cfg, sb.PREPASS_QUANT, S.p2, S.sh, S.ws)
+        sb.nvfp4_encode(S.H, cfg, S.p2, S.sh, S.ah4, S.ws)
+        sb.linear(S.H, S.ah4, S.ah8, S.p2, S.w2, S.Y, ws=S.ws)
+        sb.prepass_partial(S.Y, S.X, self.row0, self.Mt, cfg, sb.PREPASS_STATS, S.p2, None, self.slots[2], S.ws)
+        g(self.slots[2])
+        sb.prepass_finish(self.slots[2], self.Mt, S.N2, True, cfg, sb.PREPASS_STATS, S.p2, S.sy, S.ws)
+        sb.tdc_record_partial(S.Y, S.cache, self.row0, self.Mt, S.state, self.slots[3], S.ws)
+        g(self.slots[3])
+        sb.tdc_finish(self.slots[3], self.Mt, S.N2, S.sy, S.state, S.ws)
+
+    def step(self):
+        for prec in (self.sb.NVFP4, self.sb.INT8):
+            self.one_pass(prec)
+
+
+def run_sharded(args, torch, dist, sb, S, flush, world, rank, device):
+    """Times `args.steps` token-sharded steps (eager launches; the four slot gathers per pass are
+    NCCL all-reduces under torchrun). Returns ms per step, the slowest rank's."""
+    gather = (lambda t: sb.gather_slots(t)) if world > 1 else (lambda t: t)
+    T = ShardedFfnStep(sb, S, rank, world, gather)
+    for _ in range(args.warmup):
+        T.step()
+    torch.cuda.synchronize()
+    sb.check(S.ws)
+    tot = 0.0
+    for _ in range(args.steps):
+        flush()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        T.step()
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    sb.check(S.ws)
+    return max_over_ranks(tot, world, dist, device) / args.steps
+
+
+KERNEL_SPANS = (("prepass_x", "pre1_0", "pre1_1"), ("gemm_w1", "pre1_1", "gemm1_1"), ("prepass_h", "pre2_0", "pre2_1"),
+                ("gemm_w2", "pre2_1", "gemm2_1"), ("stats_d", "gemm2_1", "d_1"), ("tdc_record", "d_1", "tdc_1"))
+
+
+def graph_kernel_times(torch, S, flush, reps, precs):
+    """Per-kernel device times inside a CUDA graph of the step: the step is captured with timing
+    events between its calls (event nodes of the graph), replayed `reps` times after an L2 flush
+    each, and every span's median taken. The spans tile the pass, so their sum is the graph's own
+    time for the pass, with no host gaps."""
+    holder = {}
+
+    def fn():
+        ev = []
+        S.step(ev, precs)
+        holder["ev"] = ev
+    g = capture(torch, fn)
+    kern = {}
+    for _ in range(reps):
+        flush()
+        g.replay()
+        torch.cuda.synchronize()
+        for prec, sub in holder["ev"]:
+            d = dict(sub)
+            for name, a, z in KERNEL_SPANS:
+                kern.setdefault(f"{name}_{S.sb.PREC_NAMES[prec]}", []).append(d[a].elapsed_time(d[z]))
+    del g
+    return {k: statistics.median(v) for k, v in kern.items()}
 
 
 def capture(torch, fn):
@@ -224,6 +341,92 @@ def capture(torch, fn):
         fn()
     torch.cuda.synchronize()
     return g
+
+
+class TrajectoryStep:
+    """One block-step of the decision-driven trajectory (the 30-block DiT walk at full size): the
+    TDC check and both layers' precision from the rule, the pre-pass of the block input (PDR may
+    switch a layer to BF16), the FFN's two GEMMs in whatever precision the device flags hold, the
+    difference statistic and TDC record of the block's module output, and the residual cache:
+    refreshed on a computed step, reused on a skipped one. Every call reads the decisions on the
+    device, so one CUDA graph serves every step; a skipped step's kernels exit at once. The
+    decisions follow the trajectory's own module output y_t (as in the parity test of the decision
+    log); the FFN output is computed on x_t at every computed step."""
+
+    def __init__(self, sb, torch, S):
+        self.sb, self.torch, self.S = sb, torch, S
+        dev = S.X.device
+        self.Xb = torch.empty_like(S.X)
+        self.Yb = torch.empty_like(S.X)  # the block's module output y_t (synthetic walk)
+        self.cache = torch.zeros_like(S.X)
+        self.D = torch.zeros_like(S.X)
+        self.Yout = torch.empty_like(S.X)
+        self.state = sb.alloc_state()
+        self.sx, self.sh, self.sy = sb.alloc_stats(), sb.alloc_stats(), sb.alloc_stats()
+        self.p1 = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.p2 = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.cfg = sb.config(rho=64.0, tdc_thresh=0.1, block=128, force_prec=-1)
+        self.rule = sb.Rule(1.0, 0.0, 0.1)
+
+    def __call__(self):
+        sb, S = self.sb, self.S
+        sb.module_decide(self.state, self.cfg, [self.rule, self.rule], [self.p1, self.p2])
+        sb.prepass(self.Xb, None, self.cfg, sb.PREPASS_QUANT, self.p1, S.ax4, S.ax8, self.sx, S.ws)
+        sb.linear(self.Xb, S.ax4, S.ax8, self.p1, S.w1, S.H, epilogue=sb.EPI_GELU, ws=S.ws)
+        sb.prepass(S.H, None, self.cfg, sb.PREPASS_QUANT, self.p2, S.ah4, S.ah8, self.sh, S.ws)
+        sb.linear(S.H, S.ah4, S.ah8, self.p2, S.w2, S.Y, ws=S.ws)
+        sb.prepass(self.Yb, self.Xb, self.cfg, sb.PREPASS_STATS, self.p2, None, None, self.sy, S.ws)
+        sb.tdc_record(self.Yb, self.cache, self.sy, self.state, S.ws)
+        sb.tdc_refresh(self.Xb, self.Yb, self.D, self.state)
+        sb.tdc_reuse(self.Xb, self.D, self.Yout, self.state)
+
+
+def run_trajectory(torch, sb, synth, S, flush, blocks, steps=50):
+    """Times the decision-driven path: `blocks` of the 30-block trajectory, `steps` steps each, at
+    the module's full token count. Inputs are drawn outside the timed events; each block-step is
+    one graph replay after an L2 flush."""
+    T = TrajectoryStep(sb, torch, S)
+    g = capture(torch, T)
+    names = {sb.NVFP4: "nvfp4", sb.INT8: "int8", sb.BF16: "bf16", sb.SKIP: "skip"}
+    counts = {f"w{i}_{n}": 0 for i in (1, 2) for n in names.values()}
+    by_kind, total, flops = {}, 0.0, 0.0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for k in blocks:
+        traj = synth.Trajectory(S.M, S.K1, k, blocks=30, steps=steps, seed=0, device=S.X.device)
+        sb.state_init(T.state)
+        T.cache.zero_()
+        for t in range(steps):
+            x, y = traj.current()
+            T.Xb.copy_(x)
+            T.Yb.copy_(y)
+            flush()
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            p1, p2 = int(T.p1.item()), int(T.p2.item())
+            counts[f"w1_{names[p1]}"] += 1
+            counts[f"w2_{names[p2]}"] += 1
+            key = names[p1] if p1 == p2 else f"{names[p1]}+{names[p2]}"
+            by_kind.setdefault(key, []).append(ms)
+            total += ms
+            flops += (0.0 if p1 == sb.SKIP else 2.0 * S.M * S.N1 * S.K1) + \
+                     (0.0 if p2 == sb.SKIP else 2.0 * S.M * S.N2 * S.K2)
+            if t + 1 < steps:
+                traj.advance()
+    sb.check(S.ws)
+    del g
+    n = len(blocks) * steps
+    return {"what": "decision-driven FFN block-steps of the 30-block trajectory (hidden 3072, FFN 12288, "
+                    f"{S.M} tokens, rho 64, rule 1*d+0 > 0.1 -> INT8, TDC threshold 0.1): TDC check + rule, "
+                    "pre-passes, GEMMs of the chosen kind, difference and TDC record, residual-cache "
+                    "refresh / reuse; one graph replay per block-step, L2 flushed before each",
+            "blocks": list(blocks), "steps": steps, "block_steps": n, "ms_total": round(total, 3),
+            "ms_per_block_step": round(total / n, 4), "gemm_tflops_effective": round(flops / (total * 1e-3) / 1e12, 1),
+            "decisions": counts,
+            "ms_per_block_step_by_decision": {k: round(statistics.mean(v), 4) for k, v in sorted(by_kind.items())},
+            "block_steps_by_decision": {k: len(v) for k, v in sorted(by_kind.items())}}
 
 
 def run_ours(args):
@@ -244,7 +447,7 @@ def run_ours(args):
     from video_diffusion_mixed_b200 import synth
 
     S = FfnStep(sb, synth, torch, args.workload, seed=rank, device=device, tokens=args.tokens)
-    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)  # > 126 MB L2
+    flush = L2Flush(torch, device)
 
     def barrier():
         if world > 1:
@@ -267,7 +470,7 @@ def run_ours(args):
     barrier()
     t_wall0 = time.perf_counter()
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         starts[i].record()
         g_step.replay()
         ends[i].record()
@@ -281,22 +484,26 @@ def run_ours(args):
     flops = 2 * S.gemm_flops()  # both precision passes
     value = whole_job_tflops(world, flops, ms_per_step)
 
-    # ---- per-kernel breakdown (a separate, untimed-for-value pass with events between calls)
-    kern = {}
-    reps = max(3, min(args.steps, 10))
-    for _ in range(reps):
-        flush.zero_()
-        ev = []
-        S.step(ev)
-        torch.cuda.synchronize()
-        for prec, sub in ev:
-            tag = sb.PREC_NAMES[prec]
-            d = dict(sub)
-            for name, a, z in (("prepass_x", "pre1_0", "pre1_1"), ("gemm_w1", "pre1_1", "gemm1_1"),
-                               ("prepass_h", "pre2_0", "pre2_1"), ("gemm_w2", "pre2_1", "gemm2_1"),
-                               ("stats_d", "gemm2_1", "d_1"), ("tdc_record", "d_1", "tdc_1")):
-                kern.setdefault(f"{name}_{tag}", []).append(d[a].elapsed_time(d[z]))
-    kern_ms = {k: statistics.median(v) for k, v in kern.items()}
+    # ---- per-kernel breakdown: a graph of the same step with timing events between its calls
+    reps = max(5, min(args.steps, 20))
+    kern_ms = graph_kernel_times(torch, S, flush, reps, None)
+    # ---- the BF16 fallback (the Purified Delta Refresh path) forced on the same module, reported
+    # beside the headline step (not part of it)
+    bf16_ms = graph_kernel_times(torch, S, flush, reps, (sb.BF16,))
+    sb.check(S.ws)
+
+    # ---- the token-sharded step (the tensor's rows split over the ranks; statistics gathered)
+    sharded = None
+    if args.shard == "tokens":
+        sms = run_sharded(args, torch, dist, sb, S, flush, world, rank, device)
+        sharded = {"what": f"token-sharded step: {world} ranks x {S.M} rows of one {world * S.M}-row tensor per "
+                           "layer; row work local, whole-tensor statistics from one int64 all-reduce SUM of group "
+                           "slots each (4 per pass); eager launches",
+                   "ms_per_step": round(sms, 4), "value": round(whole_job_tflops(world, 2 * S.gemm_flops(), sms), 2),
+                   "unit": "TFLOPS", "scaling": "weak"}
+
+    # ---- the decision-driven path (rule, restart, PDR and skips live) on the trajectory
+    traj = run_trajectory(torch, sb, synth, S, flush, args.traj_blocks) if args.traj_blocks else None
 
     # ---- end to end through the public API with host buffers: every step uploads its X from
     # pinned host memory and downloads both passes' outputs. A deployment pipelines the transfers:
@@ -358,34 +565,40 @@ def run_ours(args):
 
     # ---- roofline of the dominant kernel and of the fused pre-pass
     pk = peaks()
-    ratio = {"nvfp4": 4.0, "int8": 2.0}  # nominal dense ratio to bf16 (9 / 4.5 / 2.25 PFLOP/s)
+    ratio = {"nvfp4": 4.0, "int8": 2.0, "bf16": 1.0}  # nominal dense ratio to bf16 (9 / 4.5 / 2.25 PFLOP/s)
     # The burst bf16 figure applies while the SM clock stays near its maximum during the timed
     # region; the sustained (power-capped) one otherwise.
     burst = bool(clocks.get("sm_mhz") and clocks.get("sm_max_mhz") and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"])
     tensor_peak = pk["bf16_tflops"] if burst else pk["bf16_tflops_sustained"]
     M, K1, N1, K2, N2 = S.M, S.K1, S.N1, S.K2, S.N2
     gemm_flops = {"gemm_w1": 2.0 * M * N1 * K1, "gemm_w2": 2.0 * M * N2 * K2}
-    rows = []
-    for k, ms in kern_ms.items():
-        base, tag = k.rsplit("_", 1)
-        if base in gemm_flops:
-            ach = gemm_flops[base] / (ms * 1e-3) / 1e12
-            peak = tensor_peak * ratio[tag]
-            rows.append({"kernel": k, "bound": "tensor", "ms": ms, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                         "frac": ach / peak})
-        else:
-            Kx = {"prepass_x": K1, "prepass_h": K2, "stats_d": N2, "tdc_record": N2}[base]
-            el = M * Kx
-            if base in ("prepass_x", "prepass_h"):
-                # algorithmic bytes: read bf16 X, write the quantized form of the chosen precision
-                byt = el * 2 + (el * 1 + M * 4 if tag == "int8" else el * (0.5 + 1 / 16) + 4)
-            elif base == "stats_d":
-                byt = el * 4  # read y and x
+    def roof_rows(kms):
+        out = []
+        for k, ms in kms.items():
+            base, tag = k.rsplit("_", 1)
+            if base in gemm_flops:
+                ach = gemm_flops[base] / (ms * 1e-3) / 1e12
+                peak = tensor_peak * ratio[tag]
+                out.append({"kernel": k, "bound": "tensor", "ms": ms, "achieved": ach, "peak": peak,
+                            "unit": "TFLOP/s", "frac": ach / peak})
             else:
-                byt = el * 6  # read y_new and the cache, refresh the cache
-            ach = byt / (ms * 1e-3) / 1e9
-            rows.append({"kernel": k, "bound": "hbm", "ms": ms, "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": ach / pk["hbm_gbs"]})
+                Kx = {"prepass_x": K1, "prepass_h": K2, "stats_d": N2, "tdc_record": N2}[base]
+                el = M * Kx
+                if base in ("prepass_x", "prepass_h"):
+                    # algorithmic bytes: read bf16 X, write the quantized form of the chosen precision
+                    # (nothing under BF16: the pre-pass then only gathers the statistics)
+                    byt = el * 2 + {"int8": el * 1 + M * 4, "nvfp4": el * (0.5 + 1 / 16) + 4, "bf16": 0}[tag]
+                elif base == "stats_d":
+                    byt = el * 4  # read y and x
+                else:
+                    byt = el * 6  # read y_new and the cache, refresh the cache
+                ach = byt / (ms * 1e-3) / 1e9
+                out.append({"kernel": k, "bound": "hbm", "ms": ms, "achieved": ach, "peak": pk["hbm_gbs"],
+                            "unit": "GB/s", "frac": ach / pk["hbm_gbs"]})
+        return out
+
+    rows = roof_rows(kern_ms)
+    rows_bf16 = roof_rows(bf16_ms)
     dom = max(rows, key=lambda r: r["ms"])
     tr = TRAFFIC.get(dom["kernel"])
     valid = tr is not None and args.workload == "ffn5b" and M == TRAFFIC_TOKENS and src_sha(tr["files"]) == tr["sha"]
@@ -403,13 +616,23 @@ def run_ours(args):
         "config": {"workload": f"{args.workload}: CogVideoX-5B FFN, X [{M} x {K1}] bf16 (0.5% outlier channels x50) "
                                f"-> W1 [{N1} x {K1}] (GELU) -> W2 [{N2} x {K2}]; NVFP4 pass + INT8 pass per step",
                    "tokens": M, "hidden": K1, "ffn": N1, "hadamard_block": 128, "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every step (512 MiB memset, outside the per-step events)",
+                   "l2": "flushed before every step (512 MiB memset, then a 256 MiB read that leaves L2 clean; "
+                         "outside the per-step events)",
                    "launch": "each step replays one CUDA graph of its 18 kernels"},
         "roofline": roofline,
         "roofline_prepass": {r["kernel"]: {"achieved_gbs": round(r["achieved"], 1), "frac": round(r["frac"], 4),
                                            "ms": round(r["ms"], 4)} for r in pre},
         "kernels": {r["kernel"]: {"ms": round(r["ms"], 4), "achieved": round(r["achieved"], 1), "unit": r["unit"],
                                   "frac": round(r["frac"], 4)} for r in rows},
+        "kernels_timing": "event nodes inside a CUDA graph of the step (median of the replays, L2 flushed "
+                          "before each); the spans tile the step",
+        "trajectory": traj,
+        "sharded": sharded,
+        "bf16_pass": {"what": "the same module with every layer forced to the BF16 fallback (the Purified Delta "
+                              "Refresh path), timed like the kernels above; not part of the headline step",
+                      "ms": round(sum(bf16_ms.values()), 4),
+                      "kernels": {r["kernel"]: {"ms": round(r["ms"], 4), "achieved": round(r["achieved"], 1),
+                                                "unit": r["unit"], "frac": round(r["frac"], 4)} for r in rows_bf16}},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_PASS * 2 * args.steps,
         "clocks": clocks,
@@ -537,6 +760,11 @@ def main(argv=None):
     ap.add_argument("--cpu-baseline-rows", type=int, default=1024,
                     help="tokens in the cpu_baseline sample of our arm (about 10 s on 16 cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="none", choices=["none", "tokens"],
+                    help="also time the token-sharded step (under torchrun: the rows of every tensor split "
+                         "over the ranks, statistics gathered with NCCL)")
+    ap.add_argument("--traj-blocks", type=lambda v: [int(x) for x in v.split(",") if x != ""], default=[0, 7, 14, 29],
+                    help="blocks of the 30-block trajectory timed on the decision-driven path ('' to skip)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the token count (small profiling case; the bench line is then not the metric)")
     args = ap.parse_args(argv)
