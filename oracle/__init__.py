@@ -56,6 +56,12 @@ def lib():
             "orc_prepass": (None, [vp, vp, i64, i64, i32, vp, vp, vp, vp]),
             "orc_quant_int8": (None, [vp, i64, i64, vp, vp, vp]),
             "orc_chunk_stats": (None, [vp, i64, i64, i32, vp]),
+            "orc_cube_count": (i64, [i64, i64, i64, i64, i64, i64, i64, i64]),
+            "orc_cube_of_token": (i64, [i64, i64, i64, i64, i64, i64, i64, i64]),
+            "orc_cube_tokens": (i64, [i64, i64, i64, i64, i64, i64, i64, i64, vp]),
+            "orc_delta_split": (None, [vp, i64, i64, i64, i64, i64, i64, i64, i64, i64, vp, vp, vp, vp]),
+            "orc_delta_linear": (None, [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, i64, i64, i32,
+                                        vp, i64, vp]),
             "orc_e2m1_decode": (f32, [ctypes.c_uint8]),
             "orc_e2m1_encode": (ctypes.c_uint8, [f32]),
             "orc_e4m3_decode": (f32, [ctypes.c_uint8]),
@@ -393,3 +399,51 @@ def apply_pdr(prec: int, ratio: float, rho: float, force: int = -1) -> int:
 def tdc_record(s: State, delta=None, d=None) -> None:
     lib().orc_tdc_record(ctypes.byref(s), int(delta is not None), float(delta or 0.0),
                          int(d is not None), float(d or 0.0))
+
+
+# ---------------------------------------------------------------------------------------------
+# Delta tokens (the DeltaQuant page, abstract; readings R-DQ-* in sixbit_oracle.c)
+# ---------------------------------------------------------------------------------------------
+
+def cube_count(M: int, grid) -> int:
+    """Number of cubes of M tokens; grid = (T, F, H, W, ct, ch, cw); -1 if M != T + F H W."""
+    return int(lib().orc_cube_count(M, *grid))
+
+
+def cube_of_token(t: int, grid) -> int:
+    return int(lib().orc_cube_of_token(t, *grid))
+
+
+def cube_tokens(k: int, grid) -> list:
+    T, F, H, W, ct, ch, cw = grid
+    buf = np.zeros(ct * ch * cw, dtype=np.int64)
+    n = lib().orc_cube_tokens(k, T, F, H, W, ct, ch, cw, _P(buf))
+    return buf[:n].tolist()
+
+
+def delta_split(x_bf16, grid):
+    """R-DQ-MEAN / FP8 / DELTA: core codes [ncube][K] (E4M3), scales [ncube], dequantized cores
+    [ncube][K] FP32 and the delta tokens [M][K] (bf16 bits)."""
+    x = _u16(x_bf16)
+    M, K = x.shape
+    n = cube_count(M, grid)
+    assert n > 0, "grid does not match the token count"
+    codes = np.zeros((n, K), dtype=np.uint8)
+    scale = np.zeros(n, dtype=np.float32)
+    dec = np.zeros((n, K), dtype=np.float32)
+    delta = np.zeros((M, K), dtype=np.uint16)
+    lib().orc_delta_split(_P(x), M, K, *grid, _P(codes), _P(scale), _P(dec), _P(delta))
+    return codes, scale, dec, delta
+
+
+def delta_linear(Yd, dec, w_bf16, bias, M, grid, gelu=False, rows=None):
+    """R-DQ-GEMM: the delta GEMM's rows Yd (FP64, no bias) plus the core products, bias, GELU."""
+    w = _u16(w_bf16)
+    N, K = w.shape
+    rows = _rows(M, rows)
+    Yd = np.ascontiguousarray(Yd, dtype=np.float64)
+    Y = np.empty((rows.size, N), dtype=np.float64)
+    b = _u16(bias) if bias is not None else None
+    lib().orc_delta_linear(_P(Yd), _P(np.ascontiguousarray(dec, dtype=np.float32)), _P(w), _P(b), M, N, K,
+                           *grid, int(gelu), _P(rows), rows.size, _P(Y))
+    return Y

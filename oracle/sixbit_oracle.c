@@ -640,3 +640,122 @@ void orc_tdc_record(orc_state* s, int have_delta, double delta, int have_d, doub
     s->have_d = 0;
   }
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Delta tokens ("DeltaQuant: 4-bit Video Diffusion Models with Spatiotemporal Delta          */
+/* Smoothing", abstract): the activations of the latent video grid are grouped into local 3D   */
+/* spatiotemporal cubes; each cube's mean token is its core token, kept in FP8; only the      */
+/* differences of the cube's tokens from it (delta tokens) go through the 4-bit path.          */
+/*   R-DQ-CUBE  tokens [0, T) are text tokens, one cube each; token T + (f H + h) W + w is the */
+/*              grid position (f, h, w) of an F x H x W grid, in cube (f / ct, h / ch, w / cw) */
+/*              (edge cubes are smaller). Cubes are numbered text first, then grid cubes in    */
+/*              (f, h, w) order of their first position.                                        */
+/*   R-DQ-MEAN  the core before FP8, per channel: the pairwise FP32 sum over the cube's tokens */
+/*              in index order (zero-padded to a power of two), divided by the token count.    */
+/*   R-DQ-FP8   per core token: a = max |mean| over its channels, inv = 448 / a, s = a / 448   */
+/*              (FP32); codes E4M3(RN(mean * inv)); dec = E4M3 value * s. a = 0 gives s = 0 and */
+/*              zero codes; when 448 / a overflows, nonzero means take +-448 and zeros 0.      */
+/*   R-DQ-DELTA delta token = bf16(x - dec of its cube's core): the FP32 difference of the     */
+/*              bf16 input and the FP32 core, rounded to nearest even, so the delta tensor is  */
+/*              an ordinary bf16 activation for the 4-bit path (rotation, NVFP4, GEMM).        */
+/*   R-DQ-GEMM  Y = GEMM(delta) + dec(core) W^T + bias (then the optional GELU): the core      */
+/*              product is computed once per cube and added to each of its tokens.            */
+/* ------------------------------------------------------------------------------------------ */
+
+static int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+/* Number of cubes, or -1 when M != T + F H W or a size is not positive (T may be 0). */
+int64_t orc_cube_count(int64_t M, int64_t T, int64_t F, int64_t H, int64_t W, int64_t ct, int64_t ch,
+                       int64_t cw) {
+  if (T < 0 || F < 1 || H < 1 || W < 1 || ct < 1 || ch < 1 || cw < 1 || M != T + F * H * W) return -1;
+  return T + cdiv64(F, ct) * cdiv64(H, ch) * cdiv64(W, cw);
+}
+
+/* Cube of token t (R-DQ-CUBE). */
+int64_t orc_cube_of_token(int64_t t, int64_t T, int64_t F, int64_t H, int64_t W, int64_t ct,
+                          int64_t ch, int64_t cw) {
+  if (t < T) return t;
+  int64_t g = t - T;
+  int64_t f = g / (H * W), h = (g / W) % H, w = g % W;
+  return T + ((f / ct) * cdiv64(H, ch) + h / ch) * cdiv64(W, cw) + w / cw;
+}
+
+/* The tokens of cube k in index order; returns their count (at most ct ch cw). */
+int64_t orc_cube_tokens(int64_t k, int64_t T, int64_t F, int64_t H, int64_t W, int64_t ct,
+                        int64_t ch, int64_t cw, int64_t* tok) {
+  if (k < T) {
+    tok[0] = k;
+    return 1;
+  }
+  int64_t g = k - T;
+  int64_t nh = cdiv64(H, ch), nw = cdiv64(W, cw);
+  int64_t a = g / (nh * nw), b = (g / nw) % nh, c = g % nw;
+  int64_t n = 0;
+  for (int64_t f = a * ct; f < F && f < (a + 1) * ct; ++f)
+    for (int64_t h = b * ch; h < H && h < (b + 1) * ch; ++h)
+      for (int64_t w = c * cw; w < W && w < (c + 1) * cw; ++w) tok[n++] = T + (f * H + h) * W + w;
+  return n;
+}
+
+/* R-DQ-MEAN, R-DQ-FP8, R-DQ-DELTA for every cube of X [M][K] (bf16):
+ * codes [ncube][K] E4M3, scale [ncube] (s), dec [ncube][K] FP32, delta [M][K] bf16. */
+void orc_delta_split(const uint16_t* X, int64_t M, int64_t K, int64_t T, int64_t F, int64_t H,
+                     int64_t W, int64_t ct, int64_t ch, int64_t cw, uint8_t* codes, float* scale,
+                     float* dec, uint16_t* delta) {
+  int64_t ncube = orc_cube_count(M, T, F, H, W, ct, ch, cw);
+  if (ncube < 0) return;
+#pragma omp parallel
+  {
+    int64_t* tok = (int64_t*)malloc((size_t)(ct * ch * cw) * sizeof(int64_t));
+    float* col = (float*)malloc((size_t)(ct * ch * cw) * sizeof(float));
+    float* mean = (float*)malloc((size_t)K * sizeof(float));
+#pragma omp for schedule(static)
+    for (int64_t k = 0; k < ncube; ++k) {
+      int64_t n = orc_cube_tokens(k, T, F, H, W, ct, ch, cw, tok);
+      float a = 0.0f;
+      for (int64_t c = 0; c < K; ++c) {
+        for (int64_t j = 0; j < n; ++j) col[j] = bf16_to_f32(X[tok[j] * K + c]);
+        mean[c] = orc_pairwise_f32(col, n) / (float)n;
+        float m = fabsf(mean[c]);
+        if (m > a) a = m;
+      }
+      float s = (a == 0.0f) ? 0.0f : a / 448.0f;
+      float inv = (a == 0.0f) ? 0.0f : 448.0f / a;
+      scale[k] = s;
+      for (int64_t c = 0; c < K; ++c) {
+        uint8_t q;
+        if (a == 0.0f) q = 0;
+        else if (!(inv <= FLT_MAX)) q = (mean[c] == 0.0f) ? 0 : (uint8_t)((mean[c] < 0.0f ? 0x80 : 0) | 0x7e);
+        else q = orc_e4m3_encode(mean[c] * inv);
+        codes[k * K + c] = q;
+        dec[k * K + c] = orc_e4m3_decode(q) * s;
+      }
+      for (int64_t j = 0; j < n; ++j)
+        for (int64_t c = 0; c < K; ++c)
+          delta[tok[j] * K + c] = orc_f32_to_bf16(bf16_to_f32(X[tok[j] * K + c]) - dec[k * K + c]);
+    }
+    free(tok);
+    free(col);
+    free(mean);
+  }
+}
+
+/* R-DQ-GEMM for the token rows `rows`: Y[r][n] = Yd[r][n] + sum_k dec[cube(m)][k] w[n][k] +
+ * bias[n] (optional GELU), FP64; Yd: the delta GEMM's rows without bias or GELU (FP64). */
+void orc_delta_linear(const double* Yd, const float* dec, const uint16_t* Wt, const uint16_t* bias,
+                      int64_t M, int64_t N, int64_t K, int64_t T, int64_t F, int64_t H, int64_t W,
+                      int64_t ct, int64_t ch, int64_t cw, int gelu, const int64_t* rows, int64_t nrows,
+                      double* Y) {
+  (void)M;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t cube = orc_cube_of_token(rows[r], T, F, H, W, ct, ch, cw);
+    const float* d = dec + cube * K;
+    for (int64_t n = 0; n < N; ++n) {
+      double s = 0.0;
+      for (int64_t k = 0; k < K; ++k) s += (double)d[k] * (double)bf16_to_f32(Wt[n * K + k]);
+      double v = Yd[r * N + n] + s + bias_at(bias, n);
+      Y[r * N + n] = gelu ? orc_gelu_tanh(v) : v;
+    }
+  }
+}
