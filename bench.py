@@ -356,8 +356,10 @@ class TrajectoryStep:
     def __init__(self, sb, torch, S):
         self.sb, self.torch, self.S = sb, torch, S
         dev = S.X.device
-        self.Xb = torch.empty_like(S.X)
-        self.Yb = torch.empty_like(S.X)  # the block's module output y_t (synthetic walk)
+        # The block input x_t and module output y_t are copied in before every replay; they start
+        # as finite data because the graph capture runs the step once eagerly on them first.
+        self.Xb = S.X.clone()
+        self.Yb = S.X.clone()
         self.cache = torch.zeros_like(S.X)
         self.D = torch.zeros_like(S.X)
         self.Yout = torch.empty_like(S.X)
@@ -367,6 +369,7 @@ class TrajectoryStep:
         self.p2 = torch.zeros(1, dtype=torch.int32, device=dev)
         self.cfg = sb.config(rho=64.0, tdc_thresh=0.1, block=128, force_prec=-1)
         self.rule = sb.Rule(1.0, 0.0, 0.1)
+        sb.state_init(self.state)
 
     def __call__(self):
         sb, S = self.sb, self.S
@@ -381,12 +384,103 @@ class TrajectoryStep:
         sb.tdc_reuse(self.Xb, self.D, self.Yout, self.state)
 
 
+class DeltaTokensLayer:
+    """The CogVideoX-2B attention projection (17776 x 1920 -> 1920) two ways: the plain NVFP4
+    linear (pre-pass + NVFP4 GEMM), and with delta tokens (2 x 2 x 2 cubes of the 13 x 30 x 45
+    latent grid, 226 text tokens one cube each): the split into FP8 core and bf16 delta tokens,
+    the delta tokens' pre-pass and NVFP4 GEMM (FP32 output), the cores' BF16 GEMM, and the
+    combine into bf16 output."""
+
+    def __init__(self, sb, torch, synth, device):
+        self.sb, self.torch = sb, torch
+        X, layers = synth.workload_inputs("attn2b", seed=7, device=device, bias_std=0.02)
+        self.X = X
+        self.M, self.K = X.shape
+        self.N = layers[0]["N"]
+        self.c = sb.cubes(226, 13, 30, 45, 2, 2, 2)
+        self.ws = sb.Workspace(self.M, self.K)
+        self.w_nb = sb.Weight(layers[0]["W"], None, 128, self.ws)
+        self.w_b = sb.Weight(layers[0]["W"], layers[0]["bias"], 128, self.ws)
+        self.core = sb.CoreTokens(self.c, self.M, self.K)
+        self.delta = torch.empty_like(X)
+        self.a4, self.a8, self.st = sb.Fp4Tensor(self.M, self.K), sb.I8Tensor(self.M, self.K), sb.alloc_stats()
+        self.p4 = torch.tensor([sb.NVFP4], dtype=torch.int32, device=device)
+        self.pb = torch.tensor([sb.BF16], dtype=torch.int32, device=device)
+        self.Yd = torch.empty((self.M, self.N), dtype=torch.float32, device=device)
+        self.Yc = torch.empty((self.core.n, self.N), dtype=torch.float32, device=device)
+        self.Y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=device)
+        self.cfg = sb.config(force_prec=sb.NVFP4)
+
+    def _mark(self, ev, name):
+        e = self.torch.cuda.Event(enable_timing=True, external=True)
+        e.record()
+        ev.append((name, e))
+
+    def plain(self, ev):
+        sb = self.sb
+        self._mark(ev, "p0")
+        sb.prepass(self.X, None, self.cfg, sb.PREPASS_QUANT, self.p4, self.a4, self.a8, self.st, self.ws)
+        self._mark(ev, "p1")
+        sb.linear(self.X, self.a4, self.a8, self.p4, self.w_b, self.Y, ws=self.ws)
+        self._mark(ev, "p2")
+
+    def delta_tokens(self, ev):
+        sb = self.sb
+        self._mark(ev, "d0")
+        sb.delta_split(self.X, self.c, self.core, self.delta)
+        self._mark(ev, "d1")
+        sb.prepass(self.delta, None, self.cfg, sb.PREPASS_QUANT, self.p4, self.a4, self.a8, self.st, self.ws)
+        self._mark(ev, "d2")
+        sb.linear(self.delta, self.a4, self.a8, self.p4, self.w_nb, self.Yd, out_dtype=sb.OUT_F32, ws=self.ws)
+        self._mark(ev, "d3")
+        sb.linear(self.core.bf16, None, None, self.pb, self.w_b, self.Yc, out_dtype=sb.OUT_F32, ws=self.ws)
+        self._mark(ev, "d4")
+        sb.delta_combine(self.Yd, self.Yc, self.c, self.Y)
+        self._mark(ev, "d5")
+
+
+def run_delta_tokens(torch, sb, synth, flush, device, reps=10):
+    L = DeltaTokensLayer(sb, torch, synth, device)
+    spans = {"plain_prepass": ("p0", "p1"), "plain_gemm_nvfp4": ("p1", "p2"), "split": ("d0", "d1"),
+             "delta_prepass": ("d1", "d2"), "delta_gemm_nvfp4_f32": ("d2", "d3"), "core_gemm_bf16": ("d3", "d4"),
+             "combine": ("d4", "d5")}
+    holder = {}
+
+    def fn():
+        ev = []
+        L.plain(ev)
+        L.delta_tokens(ev)
+        holder["ev"] = ev
+    g = capture(torch, fn)
+    times = {}
+    for _ in range(reps):
+        flush()
+        g.replay()
+        torch.cuda.synchronize()
+        d = dict(holder["ev"])
+        for k, (a, z) in spans.items():
+            times.setdefault(k, []).append(d[a].elapsed_time(d[z]))
+    sb.check(L.ws)
+    del g
+    ms = {k: round(statistics.median(v), 4) for k, v in times.items()}
+    plain = ms["plain_prepass"] + ms["plain_gemm_nvfp4"]
+    dq = sum(v for k, v in ms.items() if not k.startswith("plain"))
+    flops = 2.0 * L.M * L.N * L.K
+    return {"what": "CogVideoX-2B attention projection (17776 x 1920 -> 1920): the plain NVFP4 linear against the "
+                    "delta-token linear (2x2x2 cubes of the 13x30x45 latent grid + 226 text tokens: FP8 cores, "
+                    "4-bit deltas), one graph of both, L2 flushed before each replay",
+            "cubes": L.core.n, "ms": ms, "ms_plain": round(plain, 4), "ms_delta_tokens": round(dq, 4),
+            "tflops_plain": round(flops / (plain * 1e-3) / 1e12, 1),
+            "tflops_delta_tokens": round(flops / (dq * 1e-3) / 1e12, 1)}
+
+
 def run_trajectory(torch, sb, synth, S, flush, blocks, steps=50):
     """Times the decision-driven path: `blocks` of the 30-block trajectory, `steps` steps each, at
     the module's full token count. Inputs are drawn outside the timed events; each block-step is
     one graph replay after an L2 flush."""
     T = TrajectoryStep(sb, torch, S)
     g = capture(torch, T)
+    sb.check(S.ws)
     names = {sb.NVFP4: "nvfp4", sb.INT8: "int8", sb.BF16: "bf16", sb.SKIP: "skip"}
     counts = {f"w{i}_{n}": 0 for i in (1, 2) for n in names.values()}
     by_kind, total, flops = {}, 0.0, 0.0
@@ -427,6 +521,70 @@ def run_trajectory(torch, sb, synth, S, flush, blocks, steps=50):
             "decisions": counts,
             "ms_per_block_step_by_decision": {k: round(statistics.mean(v), 4) for k, v in sorted(by_kind.items())},
             "block_steps_by_decision": {k: len(v) for k, v in sorted(by_kind.items())}}
+
+
+def run_e2e(torch, sb, S, flush, steps, barrier, with_outputs):
+    """The end-to-end leg (see run_ours). Returns (ms for `steps` steps, H2D bytes per step, D2H
+    bytes per step)."""
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    Xh = torch.empty(S.X.shape, dtype=S.X.dtype, pin_memory=True)
+    Xh.copy_(S.X.cpu())
+    Xd = [S.X, S.X.clone()]  # finite from the start: capturing a pass runs it once eagerly
+    Yd = [S.Y, torch.empty_like(S.Y)]
+    # per pass: the output tensor (with_outputs) or the statistics records and module state
+    recs = [S.sx, S.sh, S.sy, S.state]
+    Rh = [[torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in recs] for _ in range(2)]
+    Yh = [torch.empty(S.Y.shape, dtype=S.Y.dtype, pin_memory=True) for _ in range(2)] if with_outputs else None
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    x_free = [None, None]      # compute finished with Xd[b]
+    y_free = [None, None]      # download finished with pass p's results
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # one graph per (pass, input buffer); pass p always writes Yd[p]
+    g_pass = {(p, b): capture(torch, lambda prec=prec, b=b, p=p: S.one_pass(prec, X=Xd[b], Y=Yd[p]))
+              for p, prec in enumerate((sb.NVFP4, sb.INT8)) for b in range(2)}
+    sb.check(S.ws)
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(steps):
+        b = i % 2
+        with torch.cuda.stream(up):
+            if i == 0:
+                t0.record()
+            if x_free[b] is not None:
+                up.wait_event(x_free[b])
+            Xd[b].copy_(Xh, non_blocking=True)
+            x_ready = ev()
+            x_ready.record()
+        comp.wait_event(x_ready)
+        flush.zero_()
+        for p, prec in enumerate((sb.NVFP4, sb.INT8)):
+            if y_free[p] is not None:
+                comp.wait_event(y_free[p])
+            g_pass[(p, b)].replay()
+            y_ready = ev()
+            y_ready.record()
+            with torch.cuda.stream(down):
+                down.wait_event(y_ready)
+                if with_outputs:
+                    Yh[p].copy_(Yd[p], non_blocking=True)
+                for r, h in zip(recs, Rh[p]):
+                    h.copy_(r, non_blocking=True)
+                y_free[p] = ev()
+                y_free[p].record()
+        x_free[b] = ev()
+        x_free[b].record()
+    with torch.cuda.stream(down):
+        down.wait_event(x_free[(steps - 1) % 2])
+        t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    del g_pass
+    h2d = S.X.numel() * S.X.element_size()
+    d2h = 2 * sum(r.numel() * r.element_size() for r in recs)
+    if with_outputs:
+        d2h += 2 * S.Y.numel() * S.Y.element_size()
+    return t0.elapsed_time(t1), h2d, d2h
 
 
 def run_ours(args):
@@ -502,66 +660,27 @@ def run_ours(args):
                    "ms_per_step": round(sms, 4), "value": round(whole_job_tflops(world, 2 * S.gemm_flops(), sms), 2),
                    "unit": "TFLOPS", "scaling": "weak"}
 
+    # ---- delta tokens on the attention projection, beside the plain NVFP4 linear
+    delta_tok = run_delta_tokens(torch, sb, synth, flush, device) if not args.no_delta_tokens else None
+
     # ---- the decision-driven path (rule, restart, PDR and skips live) on the trajectory
     traj = run_trajectory(torch, sb, synth, S, flush, args.traj_blocks) if args.traj_blocks else None
 
     # ---- end to end through the public API with host buffers: every step uploads its X from
-    # pinned host memory and downloads both passes' outputs. A deployment pipelines the transfers:
-    # the upload of step i + 1 (copy stream U) and the download of each pass's output (copy
-    # stream D) overlap the compute of the neighbouring passes on the compute stream, through
-    # double-buffered device inputs and outputs ordered by events. The timed span runs from the
-    # first upload to the last download; the L2 flush stays inside it on the compute stream.
-    comp = torch.cuda.current_stream()
-    up, down = torch.cuda.Stream(), torch.cuda.Stream()
-    Xh = torch.empty(S.X.shape, dtype=S.X.dtype, pin_memory=True)
-    Xh.copy_(S.X.cpu())
-    Yh = [torch.empty(S.Y.shape, dtype=S.Y.dtype, pin_memory=True) for _ in range(2)]
-    Xd = [S.X, torch.empty_like(S.X)]
-    Yd = [S.Y, torch.empty_like(S.Y)]
-    ev = lambda: torch.cuda.Event(enable_timing=False)
-    x_free = [None, None]      # compute finished with Xd[b]
-    y_free = [None, None]      # download finished with Yd[p]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # one graph per (pass, input buffer); pass p always writes Yd[p]
-    g_pass = {(p, b): capture(torch, lambda prec=prec, b=b, p=p: S.one_pass(prec, X=Xd[b], Y=Yd[p]))
-              for p, prec in enumerate((sb.NVFP4, sb.INT8)) for b in range(2)}
-    sb.check(S.ws)
-    torch.cuda.synchronize()
-    barrier()
-    for i in range(args.steps):
-        b = i % 2
-        with torch.cuda.stream(up):
-            if i == 0:
-                t0.record()
-            if x_free[b] is not None:
-                up.wait_event(x_free[b])
-            Xd[b].copy_(Xh, non_blocking=True)
-            x_ready = ev()
-            x_ready.record()
-        comp.wait_event(x_ready)
-        flush.zero_()
-        for p, prec in enumerate((sb.NVFP4, sb.INT8)):
-            if y_free[p] is not None:
-                comp.wait_event(y_free[p])
-            g_pass[(p, b)].replay()
-            y_ready = ev()
-            y_ready.record()
-            with torch.cuda.stream(down):
-                down.wait_event(y_ready)
-                Yh[p].copy_(Yd[p], non_blocking=True)
-                y_free[p] = ev()
-                y_free[p].record()
-        x_free[b] = ev()
-        x_free[b].record()
-    with torch.cuda.stream(down):
-        down.wait_event(x_free[(args.steps - 1) % 2])
-        t1.record()
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, dist, device)
+    # pinned host memory and reads back, per pass, the step's result: the module's statistics
+    # records and decision state (what the host sees of a module step; its output tensor feeds the
+    # next module on the device). A second leg also downloads both passes' output tensors (218 MB
+    # a step at full size, bound by the host link). A deployment pipelines the transfers: the
+    # upload of step i + 1 (copy stream U) and each pass's download (copy stream D) overlap the
+    # compute of the neighbouring passes on the compute stream, through double-buffered device
+    # inputs (and outputs) ordered by events. The timed span runs from the first upload to the last
+    # download; the L2 flush stays inside it on the compute stream.
+    e2e_ms, h2d, d2h = run_e2e(torch, sb, S, flush, args.steps, barrier, with_outputs=False)
+    e2e_ms = max_over_ranks(e2e_ms, world, dist, device)
     e2e_value = whole_job_tflops(world, flops, e2e_ms / args.steps)
-    h2d = S.X.numel() * S.X.element_size()
-    d2h = 2 * S.Y.numel() * S.Y.element_size()
+    e2eo_ms, _, d2ho = run_e2e(torch, sb, S, flush, args.steps, barrier, with_outputs=True)
+    e2eo_ms = max_over_ranks(e2eo_ms, world, dist, device)
+    e2eo_value = whole_job_tflops(world, flops, e2eo_ms / args.steps)
 
     # ---- roofline of the dominant kernel and of the fused pre-pass
     pk = peaks()
@@ -628,19 +747,24 @@ def run_ours(args):
                           "before each); the spans tile the step",
         "trajectory": traj,
         "sharded": sharded,
+        "delta_tokens": delta_tok,
         "bf16_pass": {"what": "the same module with every layer forced to the BF16 fallback (the Purified Delta "
                               "Refresh path), timed like the kernels above; not part of the headline step",
                       "ms": round(sum(bf16_ms.values()), 4),
                       "kernels": {r["kernel"]: {"ms": round(r["ms"], 4), "achieved": round(r["achieved"], 1),
                                                 "unit": r["unit"], "frac": round(r["frac"], 4)} for r in rows_bf16}},
-        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "result": "per pass the statistics records (pre-pass of X, of the hidden tensor, d of the output) and "
+                          "the module state"},
+        "e2e_with_outputs": {"value": round(e2eo_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+                             "d2h_bytes_per_step": d2ho, "result": "also both passes' output tensors"},
         "gpu_launches": LAUNCHES_PER_PASS * 2 * args.steps,
         "clocks": clocks,
         "wall_s_timed": round(t_wall, 3),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args, S.X, S.w1.W, S.w2.W)
-    del g_step, g_pass  # the graphs hold no collectives; released before the process group anyway
+    del g_step  # the graphs hold no collectives; released before the process group anyway
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -760,6 +884,7 @@ def main(argv=None):
     ap.add_argument("--cpu-baseline-rows", type=int, default=1024,
                     help="tokens in the cpu_baseline sample of our arm (about 10 s on 16 cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-delta-tokens", action="store_true", help="skip the delta-token layer timing")
     ap.add_argument("--shard", default="none", choices=["none", "tokens"],
                     help="also time the token-sharded step (under torchrun: the rows of every tensor split "
                          "over the ranks, statistics gathered with NCCL)")

@@ -324,6 +324,44 @@ sb_status sb_tdc_record_partial(const void* y_new, void* y_cache, int64_t M, int
 sb_status sb_tdc_finish(const void* slots, int64_t M_total, int64_t C, const sb_stats* d_src,
                         sb_module_state* state, void* ws, sb_stream stream);
 
+/* ---- Delta tokens ("DeltaQuant: 4-bit Video Diffusion Models with Spatiotemporal Delta
+ * Smoothing", abstract): the activations of the latent video grid are grouped into local 3D
+ * spatiotemporal cubes; each cube's mean token (its core token) is kept in FP8 and only the
+ * differences of the cube's tokens from it (delta tokens) take the 4-bit path. A linear layer is
+ * then Y = GEMM(delta) + core W^T (+ bias), the core product computed once per cube and added to
+ * each of its tokens. With these calls the caller runs: sb_delta_split; sb_prepass and sb_linear
+ * on the delta tokens (SB_OUT_F32, no bias, no epilogue); sb_linear in BF16 on the core tokens
+ * (SB_OUT_F32, with the bias); sb_delta_combine (adds them, optional GELU, bf16 output). */
+
+/* Token layout: tokens [0, text) are text tokens, one cube each; token text + (f*height + h)*width
+ * + w is position (f, h, w) of the frames x height x width latent grid, in cube (f/ct, h/ch, w/cw)
+ * (edge cubes are smaller). Cubes are numbered text first, then grid cubes in (f, h, w) order. */
+typedef struct {
+  int64_t text, frames, height, width;
+  int32_t ct, ch, cw; /* cube extent; ct*ch*cw <= 32 */
+} sb_cubes;
+
+/* Number of cubes of M tokens, or -1 when M != text + frames*height*width or a size is invalid. */
+int64_t sb_cube_count(const sb_cubes* cubes /* host */, int64_t M);
+
+/* Split X [M][K] bf16 into core and delta tokens. Per cube and channel: the pairwise FP32 sum of
+ * the cube's tokens (token order, zero-padded to a power of two) divided by the token count; per
+ * core token a = max |mean|, scale s = a / 448, codes E4M3(RN(mean * (448 / a))) (satfinite;
+ * a = 0: s = 0, zero codes; if 448 / a overflows, nonzero means take +-448), dequantized core
+ * dec = E4M3 value * s. Writes core_codes [ncube][K] (E4M3 bytes), core_scale [ncube] (FP32),
+ * core_bf16 [ncube][K] (bf16(dec), the operand of the core GEMM) and delta [M][K] (bf16 of the
+ * FP32 difference x - dec). K % 64 == 0, K <= 16384 (SB_EUNSUPPORTED); pointers 16-byte aligned
+ * (SB_EALIGN); the cube layout must cover M tokens (SB_ESHAPE). */
+sb_status sb_delta_split(const void* X, int64_t M, int64_t K, const sb_cubes* cubes /* host */,
+                         uint8_t* core_codes, float* core_scale, void* core_bf16, void* delta,
+                         sb_stream stream);
+
+/* Y [M][N] bf16 = act(Y_delta[t] + Y_core[cube(t)]) with Y_delta FP32 [M][N] and Y_core FP32
+ * [ncube][N] (the core GEMM's output, which carries the bias); epilogue SB_EPI_NONE or
+ * SB_EPI_GELU_TANH (tanh GELU with the hardware tanh approximation). N % 8 == 0. */
+sb_status sb_delta_combine(const float* y_delta, const float* y_core, int64_t M, int64_t N,
+                           const sb_cubes* cubes /* host */, int32_t epilogue, void* Y, sb_stream stream);
+
 /* Bounded device-side wait, the library's failure-detection primitive (the pages have no
  * counterpart). Enqueues on `stream` a one-thread kernel that polls the device int32 at `flag`
  * (acquire loads, ~1 us apart) until it equals `value`. If `limit_ns` nanoseconds of device time
@@ -334,6 +372,19 @@ sb_status sb_tdc_finish(const void* slots, int64_t M_total, int64_t C, const sb_
  * a kernel launched later on the same GPU. flag: 4-byte aligned device pointer (SB_EALIGN);
  * limit_ns in [1, 1e10] (SB_EINVAL otherwise). */
 sb_status sb_wait_flag(const int32_t* flag, int32_t value, uint64_t limit_ns, void* ws, sb_stream stream);
+
+/* Stall drill of the quantized linear layer (testing only; the pages have no counterpart). Arms
+ * the next sb_linear launch of this process, on any stream or host thread, as follows: in every
+ * CTA pair of the GEMM the leader CTA's TMA producer skips the copies of its `withhold_stage`-th
+ * K-block stage (counted from 0 over all the pair's tiles) but still announces their bytes, so that
+ * stage never completes. The MMA issuer's wait for it gives up after `limit_ns` of device time
+ * (%globaltimer); the abort flag and the same limit end every other wait of both CTAs, in-flight
+ * copies and MMAs are drained, tensor memory is freed, and the launch records SB_ETIMEOUT in its
+ * workspace (read by sb_check). Its output is undefined; the stream and context stay usable. The
+ * launch that takes the drill disarms it; a stage index past the pair's last K-block leaves that
+ * launch unaffected. A layer whose precision flag reads SB_SKIP also takes (and drops) the drill.
+ * withhold_stage >= 0 and limit_ns in [1e5, 1e10], else SB_EINVAL. */
+sb_status sb_drill_gemm_stall(int64_t withhold_stage, uint64_t limit_ns);
 
 /* Synchronise `stream`, read and clear the device error word of `ws`. Returns SB_OK,
  * SB_ETIMEOUT, SB_ENONFINITE, SB_EINVAL or SB_ECUDA. */

@@ -437,7 +437,8 @@ def delta_split(x_bf16, grid):
 
 
 def delta_linear(Yd, dec, w_bf16, bias, M, grid, gelu=False, rows=None):
-    """R-DQ-GEMM: the delta GEMM's rows Yd (FP64, no bias) plus the core products, bias, GELU."""
+    """R-DQ-GEMM: the delta GEMM's rows Yd (FP64, no bias) plus the products of the bf16-rounded
+    cores, the bias and the optional GELU."""
     w = _u16(w_bf16)
     N, K = w.shape
     rows = _rows(M, rows)

@@ -658,8 +658,10 @@ void orc_tdc_record(orc_state* s, int have_delta, double delta, int have_d, doub
 /*   R-DQ-DELTA delta token = bf16(x - dec of its cube's core): the FP32 difference of the     */
 /*              bf16 input and the FP32 core, rounded to nearest even, so the delta tensor is  */
 /*              an ordinary bf16 activation for the 4-bit path (rotation, NVFP4, GEMM).        */
-/*   R-DQ-GEMM  Y = GEMM(delta) + dec(core) W^T + bias (then the optional GELU): the core      */
-/*              product is computed once per cube and added to each of its tokens.            */
+/*   R-DQ-GEMM  Y = GEMM(delta) + bf16(dec) W^T + bias (then the optional GELU): the core      */
+/*              product is computed once per cube, on the dequantized core rounded to bf16 (the */
+/*              operand format of the full-precision tensor path; the page keeps cores in FP8   */
+/*              but names no FP8 weight format), and added to each of the cube's tokens.        */
 /* ------------------------------------------------------------------------------------------ */
 
 static int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -740,8 +742,8 @@ void orc_delta_split(const uint16_t* X, int64_t M, int64_t K, int64_t T, int64_t
   }
 }
 
-/* R-DQ-GEMM for the token rows `rows`: Y[r][n] = Yd[r][n] + sum_k dec[cube(m)][k] w[n][k] +
- * bias[n] (optional GELU), FP64; Yd: the delta GEMM's rows without bias or GELU (FP64). */
+/* R-DQ-GEMM for the token rows `rows`: Y[r][n] = Yd[r][n] + sum_k bf16(dec[cube(m)][k]) w[n][k]
+ * + bias[n] (optional GELU), FP64; Yd: the delta GEMM's rows without bias or GELU (FP64). */
 void orc_delta_linear(const double* Yd, const float* dec, const uint16_t* Wt, const uint16_t* bias,
                       int64_t M, int64_t N, int64_t K, int64_t T, int64_t F, int64_t H, int64_t W,
                       int64_t ct, int64_t ch, int64_t cw, int gelu, const int64_t* rows, int64_t nrows,
@@ -753,7 +755,8 @@ void orc_delta_linear(const double* Yd, const float* dec, const uint16_t* Wt, co
     const float* d = dec + cube * K;
     for (int64_t n = 0; n < N; ++n) {
       double s = 0.0;
-      for (int64_t k = 0; k < K; ++k) s += (double)d[k] * (double)bf16_to_f32(Wt[n * K + k]);
+      for (int64_t k = 0; k < K; ++k)
+        s += (double)bf16_to_f32(orc_f32_to_bf16(d[k])) * (double)bf16_to_f32(Wt[n * K + k]);
       double v = Yd[r * N + n] + s + bias_at(bias, n);
       Y[r * N + n] = gelu ? orc_gelu_tanh(v) : v;
     }

@@ -73,6 +73,9 @@ def test_wait_flag_validation_without_gpu(sb):
     assert L.sb_wait_flag(_fake(0x1002), 1, 1000, _fake(0x100), None) == sb.SB_EALIGN
     assert L.sb_wait_flag(_fake(0x1000), 1, 0, _fake(0x100), None) == sb.SB_EINVAL
     assert L.sb_wait_flag(_fake(0x1000), 1, 10_000_000_001, _fake(0x100), None) == sb.SB_EINVAL
+    assert L.sb_drill_gemm_stall(-1, 1_000_000) == sb.SB_EINVAL
+    assert L.sb_drill_gemm_stall(0, 99_999) == sb.SB_EINVAL
+    assert L.sb_drill_gemm_stall(0, 10_000_000_001) == sb.SB_EINVAL
     assert "limit_ns" in L.sb_last_error().decode()
 
 
@@ -194,3 +197,25 @@ def test_prepass_chunks_validation_without_gpu(sb):
     assert "128" in L.sb_last_error().decode()
     assert L.sb_prepass_chunks(X, chunks, 64, 1024, ctypes.byref(cfg), 0, prec, None, None, stats, ws,
                                None) == sb.SB_EINVAL
+
+
+def test_delta_token_validation_without_gpu(sb):
+    L = sb.lib()
+    c = sb.cubes(226, 13, 30, 45)  # the CogVideoX token layout: 226 text tokens, 13 x 30 x 45 grid
+    M = 226 + 13 * 30 * 45
+    assert M == 17776
+    assert L.sb_cube_count(ctypes.byref(c), M) == 226 + 7 * 15 * 23
+    assert L.sb_cube_count(ctypes.byref(c), M + 1) == -1  # the grid must cover the tokens exactly
+    big = sb.cubes(0, 4, 4, 4, 4, 4, 4)  # 64 tokens per cube: above the 32-token limit
+    assert L.sb_cube_count(ctypes.byref(big), 64) == -1
+    X, codes, scale, core, delta = (_fake(0x10000), _fake(0x20000), _fake(0x30000), _fake(0x40000),
+                                    _fake(0x50000))
+    assert L.sb_delta_split(None, M, 3072, ctypes.byref(c), codes, scale, core, delta, None) == sb.SB_EINVAL
+    assert L.sb_delta_split(_fake(0x10008), M, 3072, ctypes.byref(c), codes, scale, core, delta,
+                            None) == sb.SB_EALIGN
+    assert L.sb_delta_split(X, M, 3000, ctypes.byref(c), codes, scale, core, delta, None) == sb.SB_EUNSUPPORTED
+    assert L.sb_delta_split(X, M - 1, 3072, ctypes.byref(c), codes, scale, core, delta, None) == sb.SB_ESHAPE
+    Yd, Yc, Y = _fake(0x60000), _fake(0x70000), _fake(0x80000)
+    assert L.sb_delta_combine(Yd, Yc, M, 1924, ctypes.byref(c), 0, Y, None) == sb.SB_EUNSUPPORTED
+    assert L.sb_delta_combine(Yd, Yc, M, 1920, ctypes.byref(c), 5, Y, None) == sb.SB_EINVAL
+    assert L.sb_delta_combine(Yd, Yc, M - 2, 1920, ctypes.byref(c), 0, Y, None) == sb.SB_ESHAPE

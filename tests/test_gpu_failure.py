@@ -85,3 +85,42 @@ def test_wait_ends_when_the_host_sets_the_flag(sbg):
     finally:
         torch.cuda.synchronize()
         cudart.cudaFreeHost(hptr)
+
+
+@pytest.mark.parametrize("M,N,stage", [(512, 512, 2), (4096, 2560, 6)])
+@pytest.mark.parametrize("prec", [0, 1, 2])
+def test_gemm_stall_drill_times_out_and_the_next_gemm_is_exact(sbg, prec, M, N, stage):
+    """The GEMM's pipeline waits give up on a withheld stage: the leader CTA of every pair skips the
+    copies of one K-block stage, the MMA issuer's bounded wait for it runs out (20 ms), every other
+    role ends by the abort flag or its own limit, and the launch reports SB_ETIMEOUT. The next,
+    unarmed launch in the same context gives the same outputs bit for bit as one before the drill.
+    (512 x 512: one tile per pair; 4096 x 2560: 160 tiles, so pairs stall with tiles still queued.)"""
+    K = 1024
+    X = synth.activations(M, K, n_outlier=4, scale=20.0, seed=9, device="cuda")
+    W = synth.weight(N, K, seed=9, device="cuda")
+    ws = sbg.Workspace(max(M, N), K)
+    w = sbg.Weight(W, None, 128, ws)
+    a4, a8, st = sbg.Fp4Tensor(M, K), sbg.I8Tensor(M, K), sbg.alloc_stats()
+    p = torch.tensor([prec], dtype=torch.int32, device="cuda")
+    sbg.prepass(X, None, sbg.config(force_prec=prec), sbg.PREPASS_QUANT, p, a4, a8, st, ws)
+    sbg.check(ws)
+    out = sbg.OUT_RAW if prec == sbg.INT8 else sbg.OUT_F32
+    dt = torch.int32 if prec == sbg.INT8 else torch.float32
+
+    def run():
+        Y = torch.full((M, N), 7, dtype=dt, device="cuda")
+        sbg.linear(X, a4, a8, p, w, Y, out_dtype=out, ws=ws)
+        return Y
+
+    before = run()
+    sbg.check(ws)
+    t0 = time.monotonic()
+    sbg.drill_gemm_stall(stage, 20_000_000)
+    run()
+    with pytest.raises(sbg.SixbitError) as e:
+        sbg.check(ws)
+    assert e.value.status == sbg.SB_ETIMEOUT
+    assert time.monotonic() - t0 < 5.0
+    after = run()
+    sbg.check(ws)
+    assert torch.equal(before.view(torch.int32), after.view(torch.int32))

@@ -169,3 +169,59 @@ def test_trajectory_decisions_bitexact(sbg, M, ks):
     assert np.array_equal(log_gpu, log_ref)
     # the workload exercises every branch of the decision logic
     assert {0, 1, 2, 3} <= set(np.unique(log_ref).tolist())
+
+
+def test_trajectory_resumes_from_a_checkpoint(sbg):
+    """Checkpoint and resume: the decision state of a module is the 64-byte state record plus its
+    cached last output (and, for the reuse path, the kept residual), all caller-owned device
+    buffers. Saving them to host memory at step 25 of a 50-step trajectory, restoring them into
+    fresh buffers and running steps 25..49 must give the decision log, every state field and the
+    cache of the uninterrupted run, bit for bit."""
+    M, C, steps, k = 256, 3072, 50, 3  # block 3 carries the outlier channels (PDR fires)
+    cfg = sbg.config(rho=64.0, tdc_thresh=0.1)
+    rule = sbg.Rule(1.0, 0.0, 0.1)
+    ws = sbg.Workspace(M, C)
+    a4, a8 = sbg.Fp4Tensor(M, C), sbg.I8Tensor(M, C)
+    sx, sy = sbg.alloc_stats(), sbg.alloc_stats()
+    prec = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def run(traj, st, cache, D, t0, t1, log):
+        for t in range(t0, t1):
+            x, y = traj.current()
+            sbg.tdc_step(st, cfg)
+            sbg.select_precision(st, rule, cfg, prec)
+            sbg.prepass(x, None, cfg, sbg.PREPASS_QUANT, prec, a4, a8, sx, ws)
+            sbg.prepass(y, x, cfg, sbg.PREPASS_STATS, prec, None, None, sy, ws)
+            sbg.tdc_record(y, cache, sy, st, ws)
+            sbg.tdc_refresh(x, y, D, st)
+            sbg.check(ws)
+            log.append(int(prec.item()))
+            if t + 1 < steps:
+                traj.advance()
+
+    # uninterrupted
+    traj = synth.Trajectory(M, C, k, steps=steps, seed=0, device="cuda")
+    st = sbg.alloc_state()
+    cache = torch.zeros((M, C), dtype=torch.bfloat16, device="cuda")
+    D = torch.zeros_like(cache)
+    full = []
+    run(traj, st, cache, D, 0, steps, full)
+    # interrupted at step 25: checkpoint to host, fresh buffers, restore, continue
+    traj2 = synth.Trajectory(M, C, k, steps=steps, seed=0, device="cuda")
+    st2 = sbg.alloc_state()
+    cache2 = torch.zeros_like(cache)
+    D2 = torch.zeros_like(cache)
+    part = []
+    run(traj2, st2, cache2, D2, 0, 25, part)
+    ckpt = {"state": st2.cpu().clone(), "cache": cache2.cpu().clone(), "D": D2.cpu().clone()}
+    del st2, cache2, D2
+    st3 = sbg.alloc_state()
+    cache3 = torch.zeros_like(cache)
+    D3 = torch.zeros_like(cache)
+    st3.copy_(ckpt["state"])
+    cache3.copy_(ckpt["cache"])
+    D3.copy_(ckpt["D"])
+    run(traj2, st3, cache3, D3, 25, steps, part)
+    assert part == full
+    assert sbg.SKIP in full and any(p != sbg.SKIP for p in full)  # skipped and computed steps
+    assert torch.equal(st3, st) and torch.equal(cache3, cache) and torch.equal(D3, D)

@@ -20,7 +20,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsixbit.so")
-SOURCES = ["api.cu", "prepass.cu", "decide.cu", "gemm.cu", "prepass_static.cu", "reuse.cu", "chunks.cu"]
+SOURCES = ["api.cu", "prepass.cu", "decide.cu", "gemm.cu", "prepass_static.cu", "reuse.cu", "chunks.cu", "delta.cu"]
 HEADERS = ["sb_device.cuh", "sb_kernels.h", "rows.cuh", "prepass_blk.cuh", "tmap.h", "launch_util.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -42,7 +42,7 @@ def _deps_mtime() -> float:
 
 # Per-file flags. The streaming kernels must round every multiply and add separately (their
 # codes and statistics are compared bit for bit), so no multiply-add contraction there.
-FILE_FLAGS = {"prepass.cu": ["-fmad=false"], "chunks.cu": ["-fmad=false"]}
+FILE_FLAGS = {"prepass.cu": ["-fmad=false"], "chunks.cu": ["-fmad=false"], "delta.cu": ["-fmad=false"]}
 
 
 def _compile(src: str, verbose: bool, extra=()) -> str:

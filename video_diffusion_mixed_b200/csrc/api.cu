@@ -640,6 +640,78 @@ sb_status sb_wait_flag(const int32_t* flag, int32_t value, uint64_t limit_ns, vo
   return ok();
 }
 
+sb_status sb_drill_gemm_stall(int64_t withhold_stage, uint64_t limit_ns) {
+  SB_REQUIRE(withhold_stage >= 0, SB_EINVAL, "withhold_stage must be >= 0 (got %lld)", (long long)withhold_stage);
+  SB_REQUIRE(limit_ns >= 100000ull && limit_ns <= 10000000000ull, SB_EINVAL,
+             "limit_ns must be in [1e5, 1e10] (got %llu)", (unsigned long long)limit_ns);
+  sb::arm_gemm_stall_drill(withhold_stage, limit_ns);
+  return ok();
+}
+
+static bool cubes_geom(const sb_cubes* c, int64_t M, sb::DeltaCubes* g, int64_t* ncube) {
+  if (!c || c->text < 0 || c->frames < 1 || c->height < 1 || c->width < 1 || c->ct < 1 || c->ch < 1 || c->cw < 1)
+    return false;
+  if ((int64_t)c->ct * c->ch * c->cw > sb::kDeltaMaxCube) return false;
+  if (c->frames > ((int64_t)1 << 30) / c->height / c->width) return false;
+  if (M != c->text + c->frames * c->height * c->width) return false;
+  g->T = c->text;
+  g->F = c->frames;
+  g->H = c->height;
+  g->W = c->width;
+  g->ct = c->ct;
+  g->ch = c->ch;
+  g->cw = c->cw;
+  *ncube = c->text + sb::ceil_div(c->frames, c->ct) * sb::ceil_div(c->height, c->ch) * sb::ceil_div(c->width, c->cw);
+  return true;
+}
+
+int64_t sb_cube_count(const sb_cubes* cubes, int64_t M) {
+  sb::DeltaCubes g;
+  int64_t n = -1;
+  if (!cubes_geom(cubes, M, &g, &n)) return -1;
+  return n;
+}
+
+sb_status sb_delta_split(const void* X, int64_t M, int64_t K, const sb_cubes* cubes, uint8_t* core_codes,
+                         float* core_scale, void* core_bf16, void* delta, sb_stream stream) {
+  SB_REQUIRE(X && cubes && core_codes && core_scale && core_bf16 && delta, SB_EINVAL,
+             "X, cubes, core_codes, core_scale, core_bf16 and delta are required");
+  SB_ALIGNED(X, "X");
+  SB_ALIGNED(core_codes, "core_codes");
+  SB_ALIGNED(core_scale, "core_scale");
+  SB_ALIGNED(core_bf16, "core_bf16");
+  SB_ALIGNED(delta, "delta");
+  SB_REQUIRE(K >= 64 && K % 64 == 0 && K <= sb::kMaxK, SB_EUNSUPPORTED, "K must be a multiple of 64 in [64, %d]",
+             sb::kMaxK);
+  sb::DeltaCubes g;
+  int64_t ncube = 0;
+  SB_REQUIRE(M >= 1 && cubes_geom(cubes, M, &g, &ncube), SB_ESHAPE,
+             "the cube layout must cover the M = %lld tokens (text + frames*height*width) with cubes of at most %d "
+             "tokens",
+             (long long)M, sb::kDeltaMaxCube);
+  cudaError_t e = sb::launch_delta_split(X, K, g, ncube, core_codes, core_scale, core_bf16, delta, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_delta_split");
+  return ok();
+}
+
+sb_status sb_delta_combine(const float* y_delta, const float* y_core, int64_t M, int64_t N, const sb_cubes* cubes,
+                           int32_t epilogue, void* Y, sb_stream stream) {
+  SB_REQUIRE(y_delta && y_core && cubes && Y, SB_EINVAL, "y_delta, y_core, cubes and Y are required");
+  SB_ALIGNED(y_delta, "y_delta");
+  SB_ALIGNED(y_core, "y_core");
+  SB_ALIGNED(Y, "Y");
+  SB_REQUIRE(epilogue == SB_EPI_NONE || epilogue == SB_EPI_GELU_TANH, SB_EINVAL, "bad epilogue");
+  SB_REQUIRE(N >= 8 && N % 8 == 0 && N <= (int64_t)1 << 20, SB_EUNSUPPORTED, "N must be a multiple of 8");
+  sb::DeltaCubes g;
+  int64_t ncube = 0;
+  SB_REQUIRE(M >= 1 && cubes_geom(cubes, M, &g, &ncube), SB_ESHAPE,
+             "the cube layout must cover the M = %lld tokens", (long long)M);
+  cudaError_t e = sb::launch_delta_combine(y_delta, y_core, M, N, g, epilogue == SB_EPI_GELU_TANH ? 1 : 0, Y,
+                                           (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_delta_combine");
+  return ok();
+}
+
 sb_status sb_check(void* ws, sb_stream stream) {
   SB_REQUIRE(ws != nullptr, SB_EINVAL, "ws is NULL");
   cudaStream_t s = (cudaStream_t)stream;

@@ -62,7 +62,7 @@ constexpr uint32_t kRegsEpi = 216;  // epilogue warpgroups
 constexpr int kRegsNeeded = (int)(kRegsCtl * 128 + kRegsEpi * 256);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCols = 48;             // NVFP4: 16 SFA + 32 SFB columns per K-block
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait (the default limit)
 constexpr uint64_t kDrainNs = 20000000ull;   // 20 ms to let in-flight copies land after an abort
 // After the stages: 1 KB of barriers, then the epilogue's output staging (bf16 output): two
 // 32 x 32 bf16 boxes (2 KB each, 64B swizzle) per epilogue warp.
@@ -105,6 +105,8 @@ struct GemmParams {
   int epilogue;
   int tma_store;  // bf16 output through shared memory and TMA stores
   int group_m;    // M-tiles per raster group (tile_coords)
+  uint64_t wait_ns;  // limit of the pipeline waits (kWaitNs unless a stall drill is armed)
+  int64_t withhold;  // stall drill: the leader's producer skips the loads of this stage (-1: none)
   WsHeader* hdr;
 };
 
@@ -282,6 +284,7 @@ struct EpiCtx {
   volatile int* abort;
   uint32_t tmem;
   int unit, tiles, nunits, m_tiles, n_tiles, group_m, nacc, BN, M, N, row_off, q, half, lane;
+  uint64_t wait_ns;
   uint32_t out_box;  // this warp's two staging boxes
   uint32_t bias_s;   // NVFP4: this warp's bias slice in shared memory
   float alpha;
@@ -334,7 +337,7 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
     } else {
       if (tma) load_colops<KIND>(p, n0, ops);
     }
-    if (!mbar_wait_bounded(&e.tfull[b], tph, e.abort, kWaitNs)) {
+    if (!mbar_wait_bounded(&e.tfull[b], tph, e.abort, e.wait_ns)) {
       set_error(p.hdr, SB_ETIMEOUT);
       *e.abort = 1;
       break;
@@ -416,6 +419,7 @@ struct Issuer {
   uint32_t smem;      // shared address of stage 0
   uint32_t stage16;   // stage size in 16-byte units
   int stages, nkb, tail_nk, tiles, unit, nunits, BN, nacc, m_tiles, n_tiles, group_m;
+  uint64_t wait_ns;
   uint32_t tmem, sfa, sfb, idesc;  // TMEM base, scale columns (absolute), instruction descriptor
 };
 
@@ -475,7 +479,7 @@ __device__ __noinline__ bool issue_all(const Issuer c) {
   for (int tile = c.unit; tile < c.tiles; tile += c.nunits, ++it) {
     const int b = (c.nacc == 1) ? 0 : (it & 1);
     const uint32_t tph = (uint32_t)(((c.nacc == 1) ? it : (it >> 1)) & 1);
-    if (!mbar_wait_bounded(&c.tempty[b], tph ^ 1u, c.abort, kWaitNs)) return false;
+    if (!mbar_wait_bounded(&c.tempty[b], tph ^ 1u, c.abort, c.wait_ns)) return false;
     tc_fence_after();
     const uint32_t d = c.tmem + (uint32_t)(b * c.BN);
     uint32_t shift = 0;
@@ -485,7 +489,7 @@ __device__ __noinline__ bool issue_all(const Issuer c) {
       shift = (uint32_t)(((nt * c.BN) & 127) >> 5);
     }
     for (int kb = 0; kb < c.nkb; ++kb) {
-      if (!mbar_wait_bounded(&c.full[s], ph, c.abort, kWaitNs)) return false;
+      if (!mbar_wait_bounded(&c.full[s], ph, c.abort, c.wait_ns)) return false;
       tc_fence_after();
       const uint32_t so = (uint32_t)s * c.stage16;
       const uint64_t ad = dsw + so;
@@ -589,7 +593,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tile_coords(tile, m_tiles, n_tiles, p.group_m, &mt, &nt);
           const int m0 = mt * 256 + row_off, n0 = nt * BN;
           for (int kb = 0; kb < nkb; ++kb) {
-            if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitNs)) {
+            if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -597,6 +601,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t fb = full_leader + 8u * s;
             if (leader) mbar_arrive_expect_tx(&full[s], stage_tx);
             const int x = (kind == KIND_BF16) ? kb * 64 : kb * 128;  // 128-byte column slab
+            if (leader && issued == p.withhold) {  // stall drill: announced bytes that never come
+              ++issued;
+              if (++s == stages) {
+                s = 0;
+                ph ^= 1u;
+              }
+              continue;
+            }
             tma_load_2d_pair(st, &tm.a[kind], fb, x, m0);
             tma_load_2d_pair(st + kOffB, &tm.b[kind], fb, x, n0 + (BN / 2) * (int)rank);
             if (fp4) {
@@ -645,6 +657,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         c.m_tiles = m_tiles;
         c.n_tiles = n_tiles;
         c.group_m = p.group_m;
+        c.wait_ns = p.wait_ns;
         c.nacc = nacc;
         c.tmem = tmem_base;
         c.sfa = tmem_base + sfa_col;
@@ -681,6 +694,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     e.m_tiles = m_tiles;
     e.n_tiles = n_tiles;
     e.group_m = p.group_m;
+    e.wait_ns = p.wait_ns;
     e.nacc = nacc;
     e.BN = BN;
     e.M = M;
@@ -755,6 +769,15 @@ static int pick_group_m(int64_t m_tiles, int64_t n_tiles, int64_t units) {
   return 8;
 }
 
+// Stall drill (sb_drill_gemm_stall): armed by the host, taken by the next launch.
+static std::atomic<int64_t> g_drill_withhold{-1};
+static std::atomic<uint64_t> g_drill_wait_ns{0};
+
+void arm_gemm_stall_drill(int64_t withhold_stage, uint64_t wait_ns) {
+  g_drill_wait_ns.store(wait_ns);
+  g_drill_withhold.store(withhold_stage);
+}
+
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   static std::atomic<uint64_t> attr{0};  // one bit per device
   const cudaError_t attr_err = smem_attr_once(k_gemm, kSmemBytes, attr);
@@ -802,6 +825,9 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   p.out_dtype = L.out_dtype;
   p.epilogue = L.epilogue;
   p.hdr = reinterpret_cast<WsHeader*>(L.hdr);
+  p.withhold = g_drill_withhold.exchange(-1);
+  const uint64_t drill_ns = g_drill_wait_ns.exchange(0);
+  p.wait_ns = (p.withhold >= 0 && drill_ns != 0) ? drill_ns : kWaitNs;
   // bf16 output through TMA stores when the output satisfies their alignment (else direct stores)
   if (L.out_dtype == SB_OUT_BF16 && (reinterpret_cast<uintptr_t>(L.Y) & 15) == 0) {
     auto fn = encode_fn();

@@ -287,8 +287,18 @@ __device__ __forceinline__ void build_scale_tables(float s_g, float* inv, float*
       v = __uint_as_float(0x7fc00000u);  // unreachable code: NaN, never <= amax
     } else {
       // smallest non-negative float bit pattern b with sb(b) >= c (non-negative floats order
-      // like their bit patterns, and sb is monotone): invariant sb(lo) < c <= sb(hi)
-      uint32_t lo = 0u, hi = 0x7f800000u;
+      // like their bit patterns, and sb is monotone): invariant sb(lo) < c <= sb(hi). The search
+      // starts from a bracket of +-2^-14 around the estimate 6 s_g m (m: the E4M3 rounding
+      // midpoint below code c) and falls back to the whole range when the bracket misses.
+      const float m = 0.5f * (e4m3_to_f32(c - 1u) + e4m3_to_f32(c < 127u ? c : 126u));
+      const float est = __fmul_rn(__fmul_rn(m, 6.0f), s_g);
+      uint32_t lo = __float_as_uint(__fmul_rn(est, 1.0f - 0x1p-14f));
+      uint32_t hi = __float_as_uint(__fmul_rn(est, 1.0f + 0x1p-14f));
+      if (!(hi <= 0x7f800000u && block_scale_code(__uint_as_float(lo), s_g) < c &&
+            block_scale_code(__uint_as_float(hi), s_g) >= c)) {
+        lo = 0u;
+        hi = 0x7f800000u;
+      }
       if (block_scale_code(0.0f, s_g) >= c) hi = 0u;
       while (lo + 1u < hi) {
         const uint32_t mid = lo + ((hi - lo) >> 1);

@@ -176,7 +176,10 @@ __device__ __forceinline__ float pb_stages_rest(float2 (&P)[64], float cx) {  //
 // Per-token INT8 codes of the lane's rotated block, q = rne(RN(y * inv)) with inv = RN(127 / a_m),
 // clamped to +-127, stored at dst (128 bytes). When 127 / a_m overflows (a_m below 127 / FLT_MAX)
 // the product is +-inf for every nonzero y and the clamp gives +-127; y = 0 gives 0. The codes go
-// out in two halves (pairs P[0..31], then P[32..63]) so that few words are live at a time.
+// out in two halves (pairs P[0..31], then P[32..63]) so that few words are live at a time. The
+// rounding stays a float-to-integer conversion: the cheaper RN(v + 1.5 2^23) needs the product
+// and the addition rounded apart, and the compiler fuses an FP32x2 multiply with the FP32x2 add
+// that consumes it (measured: codes off by one against the oracle).
 __device__ __forceinline__ uint32_t pb_pack4(float a, float b, float c, float d) {
   const uint32_t q0 = (uint32_t)__float2int_rn(a), q1 = (uint32_t)__float2int_rn(b);
   const uint32_t q2 = (uint32_t)__float2int_rn(c), q3 = (uint32_t)__float2int_rn(d);

@@ -142,8 +142,10 @@ __device__ __forceinline__ void unpack_pairs(const Raw32& r, float2 (&p)[16]) {
 
 // FP32x2 arithmetic in PTX. Each half is rounded exactly like the scalar operation, with one
 // caveat measured on this toolchain: an FP32x2 multiply whose result feeds an FP32x2 add can be
-// fused into one rounding even with .rn. So mul2 is only used where its product goes to a
-// conversion; products that are summed are formed with scalar mul.rn (sq2).
+// fused into one rounding even with .rn (an INT8 rounding through RN(RN(y * inv) + 1.5 2^23),
+// written with the CUDA 12.9 paired-FP32 built-ins, also came out off by one against the oracle).
+// So mul2 is only used where its product goes to a conversion; products that are summed are
+// formed with scalar mul.rn (sq2).
 __device__ __forceinline__ uint64_t f2_bits(float2 a) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));

@@ -110,6 +110,8 @@ struct DecideLayers {
 };
 cudaError_t launch_decide(sb_module_state* st, double thr, int force, const DecideLayers& L, cudaStream_t s);
 cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t s, const char** why);
+// Arms the stall drill for the next launch_gemm (sb_drill_gemm_stall).
+void arm_gemm_stall_drill(int64_t withhold_stage, uint64_t wait_ns);
 
 cudaError_t launch_state_init(sb_module_state* st, cudaStream_t s);
 cudaError_t launch_tdc_step(sb_module_state* st, double thr, cudaStream_t s);
@@ -122,6 +124,17 @@ cudaError_t launch_tdc_refresh(const void* x, const void* y, void* d, int64_t n,
 cudaError_t launch_tdc_reuse(const void* x, const void* d, void* y, int64_t n, const sb_module_state* st,
                              cudaStream_t s);
 cudaError_t launch_ws_init(void* ws, size_t bytes, cudaStream_t s);
+
+// Delta tokens: the cube geometry (text tokens, grid F x H x W, cube ct x ch x cw).
+struct DeltaCubes {
+  int64_t T, F, H, W;
+  int ct, ch, cw;
+};
+constexpr int kDeltaMaxCube = 32;  // tokens per cube
+cudaError_t launch_delta_split(const void* X, int64_t K, const DeltaCubes& c, int64_t ncube, uint8_t* codes,
+                               float* scale, void* core16, void* delta, cudaStream_t s);
+cudaError_t launch_delta_combine(const float* Yd, const float* Yc, int64_t M, int64_t N, const DeltaCubes& c,
+                                 int gelu, void* Y, cudaStream_t s);
 
 sb_status report_error(sb_status st, const char* msg);
 

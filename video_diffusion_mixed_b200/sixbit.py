@@ -57,6 +57,12 @@ class Config(ctypes.Structure):
                 ("force_prec", ctypes.c_int32)]
 
 
+class Cubes(ctypes.Structure):
+    """sb_cubes: text tokens, the frames x height x width latent grid and the cube extent."""
+    _fields_ = [("text", ctypes.c_int64), ("frames", ctypes.c_int64), ("height", ctypes.c_int64),
+                ("width", ctypes.c_int64), ("ct", ctypes.c_int32), ("ch", ctypes.c_int32), ("cw", ctypes.c_int32)]
+
+
 STATE_BYTES = 64
 STATS_BYTES = 96
 STATE_FIELDS = ("prev_d", "acc", "delta", "have_d", "n_out", "last_skipped", "skip", "steps")
@@ -91,6 +97,7 @@ def lib():
             "sb_check": (st, [vp, vp]),
             "sb_prepass_static": (st, [vp, vp, i64, i64, P(Config), i32, vp, P(Fp4), P(I8), vp, vp]),
             "sb_wait_flag": (st, [vp, i32, ctypes.c_uint64, vp, vp]),
+            "sb_drill_gemm_stall": (st, [i64, ctypes.c_uint64]),
             "sb_tdc_refresh": (st, [vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_reuse": (st, [vp, vp, vp, i64, i64, vp, vp]),
             "sb_group_slots_bytes": (i64, [i64]),
@@ -101,6 +108,9 @@ def lib():
             "sb_tdc_finish": (st, [vp, i64, i64, vp, vp, vp, vp]),
             "sb_module_decide": (st, [vp, P(Config), i32, vp, vp, vp]),
             "sb_prepass_chunks": (st, [vp, vp, i64, i64, P(Config), i32, vp, P(Fp4), P(I8), vp, vp, vp]),
+            "sb_cube_count": (i64, [P(Cubes), i64]),
+            "sb_delta_split": (st, [vp, i64, i64, P(Cubes), vp, vp, vp, vp, vp]),
+            "sb_delta_combine": (st, [vp, vp, i64, i64, P(Cubes), i32, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -114,7 +124,8 @@ EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_in
             "sb_state_init", "sb_rotate", "sb_prepare_weight", "sb_tdc_step", "sb_select_precision", "sb_prepass",
             "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static", "sb_wait_flag", "sb_tdc_refresh",
             "sb_tdc_reuse", "sb_group_slots_bytes", "sb_prepass_partial", "sb_prepass_finish", "sb_nvfp4_encode",
-            "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide", "sb_prepass_chunks")
+            "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide", "sb_prepass_chunks", "sb_cube_count",
+            "sb_delta_split", "sb_delta_combine", "sb_drill_gemm_stall")
 
 
 def _ck(status: int):
@@ -372,3 +383,42 @@ def wait_flag(flag, value: int, limit_ns: int, ws: Workspace, stream=None):
     """Enqueue a bounded device-side wait until flag[0] == value (see sb_wait_flag)."""
     assert flag.dtype == torch.int32
     _ck(lib().sb_wait_flag(_p(flag), int(value), int(limit_ns), ws.ptr, _stream(stream)))
+
+
+def drill_gemm_stall(withhold_stage: int, limit_ns: int):
+    """Arm the next linear() launch to stall on a withheld stage (see sb_drill_gemm_stall)."""
+    _ck(lib().sb_drill_gemm_stall(int(withhold_stage), int(limit_ns)))
+
+
+# ---- delta tokens (include/sixbit.h: sb_cubes, sb_delta_split, sb_delta_combine) ----
+
+def cubes(text: int, frames: int, height: int, width: int, ct: int = 2, ch: int = 2, cw: int = 2) -> Cubes:
+    return Cubes(text, frames, height, width, ct, ch, cw)
+
+
+def cube_count(c: Cubes, M: int) -> int:
+    return int(lib().sb_cube_count(ctypes.byref(c), M))
+
+
+class CoreTokens:
+    """Caller-owned outputs of sb_delta_split for M tokens of K channels."""
+
+    def __init__(self, c: Cubes, M: int, K: int, device="cuda"):
+        n = cube_count(c, M)
+        if n < 1:
+            raise SixbitError(SB_ESHAPE, "the cube layout does not cover the tokens")
+        self.n = n
+        self.codes = torch.empty((n, K), dtype=torch.uint8, device=device)
+        self.scale = torch.empty(n, dtype=torch.float32, device=device)
+        self.bf16 = torch.empty((n, K), dtype=torch.bfloat16, device=device)
+
+
+def delta_split(X, c: Cubes, core: CoreTokens, delta, stream=None):
+    M, K = X.shape
+    _ck(lib().sb_delta_split(_p(X), M, K, ctypes.byref(c), _p(core.codes), _p(core.scale), _p(core.bf16), _p(delta),
+                             _stream(stream)))
+
+
+def delta_combine(y_delta, y_core, c: Cubes, Y, epilogue: int = EPI_NONE, stream=None):
+    M, N = Y.shape
+    _ck(lib().sb_delta_combine(_p(y_delta), _p(y_core), M, N, ctypes.byref(c), epilogue, _p(Y), _stream(stream)))
