@@ -77,6 +77,8 @@ def lib():
             "orc_tdc_delta": (f64, [vp, vp, i64, i64, vp]),
             "orc_tdc_refresh": (None, [vp, vp, i64, vp]),
             "orc_tdc_reuse": (None, [vp, vp, i64, vp]),
+            "orc_tdc_refresh_fp8": (None, [vp, vp, i64, i64, vp, vp]),
+            "orc_tdc_reuse_fp8": (None, [vp, vp, vp, i64, i64, vp]),
             "orc_state_init": (None, [vp]),
             "orc_tdc_step": (None, [vp, f64]),
             "orc_select_precision": (i32, [vp, f64, f64, f64, i32]),
@@ -367,6 +369,30 @@ def tdc_reuse(x_bf16, d_bf16):
     assert x.shape == d.shape
     y = np.empty_like(x)
     lib().orc_tdc_reuse(_P(x), _P(d), x.size, _P(y))
+    return y
+
+
+def tdc_refresh_fp8(x_bf16, y_bf16):
+    """R-REUSE-FP8: the residual kept in FP8, E4M3 codes [M][C] and one FP32 scale per row."""
+    x = _u16(x_bf16)
+    y = _u16(y_bf16)
+    assert x.shape == y.shape and x.ndim == 2
+    M, C = x.shape
+    codes = np.zeros((M, C), dtype=np.uint8)
+    scale = np.zeros(M, dtype=np.float32)
+    lib().orc_tdc_refresh_fp8(_P(x), _P(y), M, C, _P(codes), _P(scale))
+    return codes, scale
+
+
+def tdc_reuse_fp8(x_bf16, codes, scale):
+    """R-REUSE-FP8: the output of a skipped step, y = bf16(x + E4M3(code) * s) (bf16 bits)."""
+    x = _u16(x_bf16)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    M, C = x.shape
+    assert codes.shape == (M, C) and scale.shape == (M,)
+    y = np.empty_like(x)
+    lib().orc_tdc_reuse_fp8(_P(x), _P(codes), _P(scale), M, C, _P(y))
     return y
 
 

@@ -29,6 +29,8 @@
  *   R-REUSE the cache keeps the module's residual D = y - x of its last computed step (bf16: the
  *           FP32 difference of the bf16 values, rounded to nearest even); a skipped step
  *           returns y = x + D (FP32 sum of the bf16 values, rounded to nearest even).
+ *   R-REUSE-FP8 the same residual kept in FP8: E4M3 codes with one FP32 scale per token
+ *           (s = max|d| / 448, the recipe of R-DQ-FP8); a skipped step returns bf16(x + E4M3 * s).
  * Parity of R-RULE constants, R-TDC accumulator semantics and R-PDR granularity is pinned only
  * to these definitions ("parity unpinned" against the pages, which print no constants).
  *
@@ -575,6 +577,49 @@ void orc_tdc_refresh(const uint16_t* x, const uint16_t* y, int64_t n, uint16_t* 
 
 void orc_tdc_reuse(const uint16_t* x, const uint16_t* d, int64_t n, uint16_t* y) {
   for (int64_t i = 0; i < n; ++i) y[i] = orc_f32_to_bf16(bf16_to_f32(x[i]) + bf16_to_f32(d[i]));
+}
+
+/* R-REUSE-FP8 ([VU] 七: the cache's historical results may be kept in low-precision formats):
+ * the residual of a computed step kept in FP8, one E4M3 code per element and one FP32 scale per
+ * row (token), with the per-token recipe of R-DQ-FP8: d = RN(y - x) in FP32 from the bf16 values,
+ * a = max |d| over the row, s = a / 448, codes E4M3(RN(d * (448 / a))) (round to nearest even,
+ * saturating); a = 0 gives s = 0 and zero codes; 448 / a overflowing gives +-448 (0x7e) for every
+ * nonzero d and 0 for zeros. At a skipped step y = bf16(x + dec) with dec = RN(E4M3(code) * s).
+ * x, y: bf16 [M][C]; codes [M][C]; scale [M]. */
+void orc_tdc_refresh_fp8(const uint16_t* x, const uint16_t* y, int64_t M, int64_t C, uint8_t* codes,
+                         float* scale) {
+#pragma omp parallel
+  {
+    float* d = (float*)malloc((size_t)C * sizeof(float));
+#pragma omp for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+      float a = 0.0f;
+      for (int64_t c = 0; c < C; ++c) {
+        d[c] = bf16_to_f32(y[m * C + c]) - bf16_to_f32(x[m * C + c]);
+        if (fabsf(d[c]) > a) a = fabsf(d[c]);
+      }
+      const float s = (a == 0.0f) ? 0.0f : a / 448.0f;
+      const float inv = (a == 0.0f) ? 0.0f : 448.0f / a;
+      scale[m] = s;
+      for (int64_t c = 0; c < C; ++c) {
+        uint8_t q;
+        if (a == 0.0f) q = 0;
+        else if (!(inv <= FLT_MAX)) q = (d[c] == 0.0f) ? 0 : (uint8_t)((d[c] < 0.0f ? 0x80 : 0) | 0x7e);
+        else q = orc_e4m3_encode(d[c] * inv);
+        codes[m * C + c] = q;
+      }
+    }
+    free(d);
+  }
+}
+
+void orc_tdc_reuse_fp8(const uint16_t* x, const uint8_t* codes, const float* scale, int64_t M, int64_t C,
+                       uint16_t* y) {
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t c = 0; c < C; ++c) {
+      const float dec = orc_e4m3_decode(codes[m * C + c]) * scale[m];
+      y[m * C + c] = orc_f32_to_bf16(bf16_to_f32(x[m * C + c]) + dec);
+    }
 }
 
 /* Per-module state of the Temporal Delta Cache and of the precision rule. */

@@ -467,6 +467,68 @@ def test_tdc_reuse_closed_form(orc):
     assert np.array_equal(orc.tdc_refresh(xb, xb), np.zeros_like(xb))  # +0, not -0
 
 
+def test_tdc_fp8_residual_closed_form(orc):
+    """R-REUSE-FP8 on rows whose residuals are integers with row maximum 7: s = 7 / 448 = 2^-6 is
+    exact, every d / s = 64 d is an E4M3 value, so codes decode exactly and a reuse with the same
+    input returns the output bit for bit. A zero row keeps s = 0, zero codes and returns x."""
+    rng = np.random.default_rng(12)
+    M, C = 6, 40
+    x = rng.integers(-50, 50, (M, C)).astype(np.float64)
+    d = rng.integers(-7, 8, (M, C)).astype(np.float64)
+    d[:, 0] = np.where(np.arange(M) % 2 == 0, 7, -7)  # row max |d| = 7, either sign
+    d[M - 1] = 0.0
+    xb = _bf16(x).view(torch.int16).numpy().view(np.uint16)
+    yb = _bf16(x + d).view(torch.int16).numpy().view(np.uint16)
+    codes, scale = orc.tdc_refresh_fp8(xb, yb)
+    assert np.array_equal(scale[:M - 1], np.full(M - 1, 2.0 ** -6, dtype=np.float32))
+    assert scale[M - 1] == 0.0 and not codes[M - 1].any()
+    # 64 d: 0 -> 0x00, 64 -> 0x60 (2^6), 448 -> 0x7e, and the sign bit for negative d
+    assert codes[0, 0] == 0x7E and codes[1, 0] == 0xFE
+    dec = np.array([orc.e4m3_decode(int(c)) for c in codes.ravel()], dtype=np.float64).reshape(M, C)
+    assert np.array_equal(dec * 2.0 ** -6, d)
+    assert np.array_equal(orc.tdc_reuse_fp8(xb, codes, scale), yb)
+
+
+def test_tdc_fp8_residual_matches_ml_dtypes_and_error_bound(orc):
+    """R-REUSE-FP8 through independent implementations: the codes are ml_dtypes' E4M3 cast of the
+    FP32 residual times 448 / a, the output is ml_dtypes' bf16 cast of x + dec; the decoded residual
+    is within half an E4M3 step of d (2^-4 relative for normals, 2^-10 s absolute for subnormals)."""
+    ml = pytest.importorskip("ml_dtypes")
+    rng = np.random.default_rng(13)
+    M, C = 24, 96
+    xs = np.exp2(rng.integers(-8, 8, (M, 1)))
+    x = (rng.standard_normal((M, C)) * xs).astype(np.float32).astype(ml.bfloat16)
+    y = (x.astype(np.float32) + rng.standard_normal((M, C)).astype(np.float32) * 0.1 * xs.astype(np.float32)
+         * np.exp2(rng.integers(-12, 1, (M, C))).astype(np.float32)).astype(ml.bfloat16)
+    xb, yb = x.view(np.uint16), y.view(np.uint16)
+    codes, scale = orc.tdc_refresh_fp8(xb, yb)
+    d = y.astype(np.float32) - x.astype(np.float32)
+    a = np.max(np.abs(d), axis=1)
+    assert np.all(a > 0)
+    ref = (d * (np.float32(448.0) / a)[:, None]).astype(np.float32).astype(ml.float8_e4m3fn)
+    assert np.array_equal(codes, ref.view(np.uint8))
+    dec = ref.astype(np.float32) * scale[:, None]
+    err = np.abs(dec.astype(np.float64) - d.astype(np.float64))
+    bound = np.maximum(2.0 ** -4 * np.abs(d), 2.0 ** -10 * scale[:, None]) * (1 + 2.0 ** -20) + 1e-44
+    assert np.all(err <= bound)
+    out = (x.astype(np.float32) + dec).astype(ml.bfloat16)
+    assert np.array_equal(orc.tdc_reuse_fp8(xb, codes, scale), out.view(np.uint16))
+
+
+def test_tdc_fp8_residual_overflow_row(orc):
+    """A row whose largest residual is so small that 448 / a overflows FP32 codes every nonzero
+    residual as +-448 (0x7e, 0xfe) and zeros as 0; s = a / 448 stays a positive subnormal."""
+    x = np.zeros((1, 16), dtype=np.uint16)
+    y = np.zeros((1, 16), dtype=np.uint16)
+    y[0, 3] = 0x0001   # +2^-133 (the smallest bf16 subnormal)
+    y[0, 9] = 0x8001   # -2^-133
+    codes, scale = orc.tdc_refresh_fp8(x, y)
+    assert 0.0 < scale[0] < 2.0 ** -133
+    want = np.zeros(16, dtype=np.uint8)
+    want[3], want[9] = 0x7E, 0xFE
+    assert np.array_equal(codes[0], want)
+
+
 def test_tdc_schedule_dyadic(orc):
     """delta = 1/32, threshold 1/8: after the two warm-up outputs, four skips then a compute."""
     s = orc.State()
