@@ -33,22 +33,23 @@ if ROOT not in sys.path:
 
 METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT shapes"
 
-# ncu DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the kernels that
-# can be the dominant one, from the 8192-token captures summarised under profiles/ scaled to 17776
-# tokens (every term grows with the token count), for the ffn5b workload at full size only. An
-# entry is valid only for the sources it was measured on (sha over the listed files of csrc/).
+# ncu DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum, one capture of the
+# step's 18 launches at full size, 17776 tokens; ncu flushes the caches before each launch, so
+# these are cold-cache figures) of the kernels that can be the dominant one, summarised under
+# profiles/, for the ffn5b workload at full size only. An entry is valid only for the sources it
+# was measured on (sha over the listed files of csrc/).
 _GEMM_SRC = ("gemm.cu", "sb_device.cuh")
 _ROWS_SRC = ("prepass.cu", "rows.cuh", "prepass_blk.cuh", "sb_device.cuh", "tmap.h")
 TRAFFIC = {
-    "gemm_w1_int8": {"bytes": 743.7e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
-    "gemm_w2_int8": {"bytes": 801.8e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
-    "gemm_w1_nvfp4": {"bytes": 487.6e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
-    "gemm_w2_nvfp4": {"bytes": 269.0e6, "files": _GEMM_SRC, "sha": "a922a472af6d1013"},
+    "gemm_w1_int8": {"bytes": 764.7e6, "files": _GEMM_SRC, "sha": "7f299b94f250d919"},
+    "gemm_w2_int8": {"bytes": 773.0e6, "files": _GEMM_SRC, "sha": "7f299b94f250d919"},
+    "gemm_w1_nvfp4": {"bytes": 509.4e6, "files": _GEMM_SRC, "sha": "7f299b94f250d919"},
+    "gemm_w2_nvfp4": {"bytes": 256.2e6, "files": _GEMM_SRC, "sha": "7f299b94f250d919"},
     # k_prepass_blk + k_nvfp4_blk (the encode exits at once in the INT8 pass)
-    "prepass_h_nvfp4": {"bytes": 941.1e6, "files": _ROWS_SRC, "sha": "3f4b80ad2d9b6473"},
-    "prepass_h_int8": {"bytes": 577.2e6, "files": _ROWS_SRC, "sha": "3f4b80ad2d9b6473"},
-    "prepass_x_nvfp4": {"bytes": 218.8e6, "files": _ROWS_SRC, "sha": "3f4b80ad2d9b6473"},
-    "prepass_x_int8": {"bytes": 111.7e6, "files": _ROWS_SRC, "sha": "3f4b80ad2d9b6473"},
+    "prepass_h_nvfp4": {"bytes": 971.6e6, "files": _ROWS_SRC, "sha": "f0590a17a64890f5"},
+    "prepass_h_int8": {"bytes": 630.1e6, "files": _ROWS_SRC, "sha": "f0590a17a64890f5"},
+    "prepass_x_nvfp4": {"bytes": 224.7e6, "files": _ROWS_SRC, "sha": "f0590a17a64890f5"},
+    "prepass_x_int8": {"bytes": 127.6e6, "files": _ROWS_SRC, "sha": "f0590a17a64890f5"},
 }
 TRAFFIC_TOKENS = 17776
 
@@ -188,10 +189,9 @@ class FfnStep:
         self._mark(ev, "pre2_1")
         sb.linear(self.H, self.ah4, self.ah8, self.p2, self.w2, Y, ws=self.ws)
         self._mark(ev, "gemm2_1")
-        sb.prepass(Y, X, cfg, sb.PREPASS_STATS, self.p2, None, None, self.sy, self.ws)
-        self._mark(ev, "d_1")
-        sb.tdc_record(Y, self.cache, self.sy, self.state, self.ws)
-        self._mark(ev, "tdc_1")
+        # the difference statistic of Y against X and the TDC record of Y, one pass over Y
+        sb.module_record(Y, X, self.cache, self.p2, self.sy, self.state, self.ws)
+        self._mark(ev, "rec_1")
 
     def _mark(self, ev, name):
         if ev is not None:
@@ -209,7 +209,7 @@ class FfnStep:
                 ev.append((prec, sub))
 
 
-LAUNCHES_PER_PASS = 9  # decide, prepass(2), gemm, prepass(2), gemm, stats prepass, tdc record
+LAUNCHES_PER_PASS = 8  # decide, prepass(2), gemm, prepass(2), gemm, module record
 
 
 class L2Flush:
@@ -299,7 +299,7 @@ def run_sharded(args, torch, dist, sb, S, flush, world, rank, device):
 
 
 KERNEL_SPANS = (("prepass_x", "pre1_0", "pre1_1"), ("gemm_w1", "pre1_1", "gemm1_1"), ("prepass_h", "pre2_0", "pre2_1"),
-                ("gemm_w2", "pre2_1", "gemm2_1"), ("stats_d", "gemm2_1", "d_1"), ("tdc_record", "d_1", "tdc_1"))
+                ("gemm_w2", "pre2_1", "gemm2_1"), ("record", "gemm2_1", "rec_1"))
 
 
 def graph_kernel_times(torch, S, flush, reps, precs):
@@ -378,8 +378,7 @@ class TrajectoryStep:
         sb.linear(self.Xb, S.ax4, S.ax8, self.p1, S.w1, S.H, epilogue=sb.EPI_GELU, ws=S.ws)
         sb.prepass(S.H, None, self.cfg, sb.PREPASS_QUANT, self.p2, S.ah4, S.ah8, self.sh, S.ws)
         sb.linear(S.H, S.ah4, S.ah8, self.p2, S.w2, S.Y, ws=S.ws)
-        sb.prepass(self.Yb, self.Xb, self.cfg, sb.PREPASS_STATS, self.p2, None, None, self.sy, S.ws)
-        sb.tdc_record(self.Yb, self.cache, self.sy, self.state, S.ws)
+        sb.module_record(self.Yb, self.Xb, self.cache, self.p2, self.sy, self.state, S.ws)
         sb.tdc_refresh(self.Xb, self.Yb, self.D, self.state)
         sb.tdc_reuse(self.Xb, self.D, self.Yout, self.state)
 
@@ -472,6 +471,43 @@ def run_delta_tokens(torch, sb, synth, flush, device, reps=10):
             "cubes": L.core.n, "ms": ms, "ms_plain": round(plain, 4), "ms_delta_tokens": round(dq, 4),
             "tflops_plain": round(flops / (plain * 1e-3) / 1e12, 1),
             "tflops_delta_tokens": round(flops / (dq * 1e-3) / 1e12, 1)}
+
+
+def run_residual_cache(torch, sb, S, flush, reps=10):
+    """The Temporal Delta Cache's residual on the module's block (17776 x 3072 at full size): the
+    refresh of a computed step and the reuse of a skipped one, with the residual in bf16 and in
+    FP8 (E4M3 codes + one FP32 scale per token). Each call is timed alone after an L2 flush."""
+    M, C = S.X.shape
+    x = S.X
+    y = S.X.clone()
+    y.add_(0.125)
+    out = torch.empty_like(x)
+    d16 = torch.empty_like(x)
+    d8 = sb.Fp8Residual(M, C)
+    st_c, st_s = sb.alloc_state(), sb.alloc_state()
+    sb.state_init(st_c)
+    sb.state_init(st_s)
+    st_s.view(torch.int32)[9] = 1  # sb_module_state.skip (bytes 36..39): the reuse calls run
+    calls = {"refresh_bf16": lambda: sb.tdc_refresh(x, y, d16, st_c), "reuse_bf16": lambda: sb.tdc_reuse(x, d16, out, st_s),
+             "refresh_fp8": lambda: sb.tdc_refresh_fp8(x, y, d8, st_c), "reuse_fp8": lambda: sb.tdc_reuse_fp8(x, d8, out, st_s)}
+    nbytes = {"refresh_bf16": 6 * M * C, "reuse_bf16": 6 * M * C, "refresh_fp8": 5 * M * C + 4 * M, "reuse_fp8": 5 * M * C + 4 * M}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    res = {}
+    for k, fn in calls.items():
+        fn()
+        ts = []
+        for _ in range(reps):
+            flush()
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        res[k] = {"ms": round(ms, 4), "achieved_gbs": round(nbytes[k] / (ms * 1e-3) / 1e9, 1)}
+    return {"what": f"TDC residual cache on the block input ({M} x {C}): refresh (computed step) and reuse (skipped "
+                    "step), residual in bf16 or FP8 (E4M3 + FP32 scale per token); algorithmic bytes: bf16 6 B/el, "
+                    "FP8 5 B/el + 4 B/token; one call per L2 flush", **res}
 
 
 def run_trajectory(torch, sb, synth, S, flush, blocks, steps=50):
@@ -663,6 +699,9 @@ def run_ours(args):
     # ---- delta tokens on the attention projection, beside the plain NVFP4 linear
     delta_tok = run_delta_tokens(torch, sb, synth, flush, device) if not args.no_delta_tokens else None
 
+    # ---- the residual cache of the reuse path, bf16 and FP8
+    resid = run_residual_cache(torch, sb, S, flush)
+
     # ---- the decision-driven path (rule, restart, PDR and skips live) on the trajectory
     traj = run_trajectory(torch, sb, synth, S, flush, args.traj_blocks) if args.traj_blocks else None
 
@@ -701,16 +740,14 @@ def run_ours(args):
                 out.append({"kernel": k, "bound": "tensor", "ms": ms, "achieved": ach, "peak": peak,
                             "unit": "TFLOP/s", "frac": ach / peak})
             else:
-                Kx = {"prepass_x": K1, "prepass_h": K2, "stats_d": N2, "tdc_record": N2}[base]
+                Kx = {"prepass_x": K1, "prepass_h": K2, "record": N2}[base]
                 el = M * Kx
                 if base in ("prepass_x", "prepass_h"):
                     # algorithmic bytes: read bf16 X, write the quantized form of the chosen precision
                     # (nothing under BF16: the pre-pass then only gathers the statistics)
                     byt = el * 2 + {"int8": el * 1 + M * 4, "nvfp4": el * (0.5 + 1 / 16) + 4, "bf16": 0}[tag]
-                elif base == "stats_d":
-                    byt = el * 4  # read y and x
                 else:
-                    byt = el * 6  # read y_new and the cache, refresh the cache
+                    byt = el * 8  # record: read y, x and the cache, refresh the cache
                 ach = byt / (ms * 1e-3) / 1e9
                 out.append({"kernel": k, "bound": "hbm", "ms": ms, "achieved": ach, "peak": pk["hbm_gbs"],
                             "unit": "GB/s", "frac": ach / pk["hbm_gbs"]})
@@ -719,9 +756,13 @@ def run_ours(args):
     rows = roof_rows(kern_ms)
     rows_bf16 = roof_rows(bf16_ms)
     dom = max(rows, key=lambda r: r["ms"])
-    tr = TRAFFIC.get(dom["kernel"])
-    valid = tr is not None and args.workload == "ffn5b" and M == TRAFFIC_TOKENS and src_sha(tr["files"]) == tr["sha"]
-    traffic = int(tr["bytes"]) if valid else None  # bytes per launch
+
+    def traffic_of(kernel):  # measured DRAM bytes per launch, while the sources are the measured ones
+        tr = TRAFFIC.get(kernel)
+        ok = tr is not None and args.workload == "ffn5b" and M == TRAFFIC_TOKENS and src_sha(tr["files"]) == tr["sha"]
+        return int(tr["bytes"]) if ok else None
+
+    traffic = traffic_of(dom["kernel"])
     roofline = {"bound": dom["bound"], "achieved": round(dom["achieved"], 1), "peak": round(dom["peak"], 1),
                 "unit": dom["unit"], "frac": round(dom["frac"], 4), "traffic": traffic, "kernel": dom["kernel"],
                 "peak_src": f"{pk['src']} bf16 {'burst' if burst else 'sustained'} x nominal dtype ratio"
@@ -740,7 +781,7 @@ def run_ours(args):
                    "launch": "each step replays one CUDA graph of its 18 kernels"},
         "roofline": roofline,
         "roofline_prepass": {r["kernel"]: {"achieved_gbs": round(r["achieved"], 1), "frac": round(r["frac"], 4),
-                                           "ms": round(r["ms"], 4)} for r in pre},
+                                           "ms": round(r["ms"], 4), "traffic": traffic_of(r["kernel"])} for r in pre},
         "kernels": {r["kernel"]: {"ms": round(r["ms"], 4), "achieved": round(r["achieved"], 1), "unit": r["unit"],
                                   "frac": round(r["frac"], 4)} for r in rows},
         "kernels_timing": "event nodes inside a CUDA graph of the step (median of the replays, L2 flushed "
@@ -748,6 +789,7 @@ def run_ours(args):
         "trajectory": traj,
         "sharded": sharded,
         "delta_tokens": delta_tok,
+        "residual_cache": resid,
         "bf16_pass": {"what": "the same module with every layer forced to the BF16 fallback (the Purified Delta "
                               "Refresh path), timed like the kernels above; not part of the headline step",
                       "ms": round(sum(bf16_ms.values()), 4),

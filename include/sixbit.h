@@ -137,7 +137,8 @@ const char* sb_version(void);
 const char* sb_last_error(void);
 
 /* Bytes of workspace needed by calls with at most max_M rows (tokens or weight rows N) of at most
- * max_K columns. `bytes` is a host pointer. */
+ * max_K columns: a 256-byte header and two arrays of one 48-byte slot per 16 rows. `bytes` is a
+ * host pointer. */
 sb_status sb_workspace_size(int64_t max_M, int64_t max_K, size_t* bytes);
 
 /* Zero a workspace (counters and error word) before its first use. */
@@ -235,6 +236,21 @@ sb_status sb_linear(const void* X, const sb_fp4* a4 /* host */, const sb_i8* a8 
 sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C,
                         const sb_stats* d_src, int32_t update_cache, sb_module_state* state,
                         void* ws, sb_stream stream);
+
+/* The module's output record in one pass ("write-up" sections 一 and 二): the difference statistic
+ * of the module output y against its input x, then the TDC record of y against the cached last
+ * output, reading y once. Bit for bit the same results (stats, state, cache) as
+ *   sb_prepass(y, x, M, C, cfg, SB_PREPASS_STATS, prec, NULL, NULL, stats, ws) followed by
+ *   sb_tdc_record(y, cache, M, C, stats, update_cache, state, ws),
+ * each part with its own gate: the statistics are skipped when *prec == SB_SKIP (prec may be
+ * NULL: never skipped; *prec is not modified), the record when state->skip; the record takes its d
+ * from the stats this call writes. y, x, cache: bf16 [M][C] row-major, 16-byte aligned
+ * (SB_EALIGN); stats: device sb_stats; state: device sb_module_state; C a multiple of 64 in
+ * [64, 16384] (SB_EUNSUPPORTED); M in [1, 2^30] (SB_ESHAPE). The call uses two group-slot arrays
+ * of ws, so ws must come from sb_workspace_size with max_M >= M. */
+sb_status sb_module_record(const void* y, const void* x, void* cache, int64_t M, int64_t C, int32_t* prec,
+                           int32_t update_cache, sb_stats* stats, sb_module_state* state, void* ws,
+                           sb_stream stream);
 
 /* sb_prepass without a caller workspace. The paper has no counterpart: this exists for callers
  * that cannot allocate device memory -- e.g. a plugin inside a host program that owns the whole
@@ -361,6 +377,22 @@ sb_status sb_delta_split(const void* X, int64_t M, int64_t K, const sb_cubes* cu
  * SB_EPI_GELU_TANH (tanh GELU with the hardware tanh approximation). N % 8 == 0. */
 sb_status sb_delta_combine(const float* y_delta, const float* y_core, int64_t M, int64_t N,
                            const sb_cubes* cubes /* host */, int32_t epilogue, void* Y, sb_stream stream);
+
+/* The same reuse path with the residual kept in FP8 ("write-up" section 七: the cache's history
+ * may be stored in low-precision formats): half the bytes of the bf16 residual.
+ *   sb_tdc_refresh_fp8: if the module computed this step (state->skip == 0), per token row m:
+ *     d = RN(y - x) in FP32, a = max |d| over the row, scale[m] = a / 448, codes E4M3(RN(d * (448 /
+ *     a))) with round to nearest even and saturation to +-448; a = 0 gives scale 0 and zero codes;
+ *     448 / a overflowing FP32 gives +-448 (0x7e / 0xfe) for nonzero d and 0 for zeros;
+ *   sb_tdc_reuse_fp8: if the module is skipped this step (state->skip == 1),
+ *     y = bf16(x + RN(E4M3(code) * scale[m])).
+ * The other case writes nothing. x, y: bf16 [M][C]; codes: E4M3 [M][C]; scale: FP32 [M]; all
+ * row-major, caller-owned device memory; x, y, codes 16-byte aligned, scale 4-byte aligned
+ * (SB_EALIGN); C a multiple of 16 (SB_EUNSUPPORTED); M in [1, 2^30] (SB_ESHAPE). */
+sb_status sb_tdc_refresh_fp8(const void* x, const void* y, uint8_t* codes, float* scale, int64_t M, int64_t C,
+                             const sb_module_state* state, sb_stream stream);
+sb_status sb_tdc_reuse_fp8(const void* x, const uint8_t* codes, const float* scale, void* y, int64_t M, int64_t C,
+                           const sb_module_state* state, sb_stream stream);
 
 /* Bounded device-side wait, the library's failure-detection primitive (the pages have no
  * counterpart). Enqueues on `stream` a one-thread kernel that polls the device int32 at `flag`

@@ -67,6 +67,35 @@ def test_tdc_reuse_validation_without_gpu(sb):
     assert L.sb_tdc_refresh(*ok, 0, 64, _fake(0x4000), None) == sb.SB_ESHAPE
 
 
+def test_tdc_fp8_validation_without_gpu(sb):
+    L = sb.lib()
+    x, y, q, s, st = _fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x4000), _fake(0x5000)
+    assert L.sb_tdc_refresh_fp8(None, y, q, s, 4, 64, st, None) == sb.SB_EINVAL
+    assert L.sb_tdc_refresh_fp8(x, y, q, None, 4, 64, st, None) == sb.SB_EINVAL
+    assert L.sb_tdc_refresh_fp8(x, y, _fake(0x3008), s, 4, 64, st, None) == sb.SB_EALIGN
+    assert L.sb_tdc_reuse_fp8(x, q, _fake(0x4002), y, 4, 64, st, None) == sb.SB_EALIGN
+    assert L.sb_tdc_reuse_fp8(x, q, s, y, 4, 72, st, None) == sb.SB_EUNSUPPORTED
+    assert L.sb_tdc_reuse_fp8(x, q, s, y, 0, 64, st, None) == sb.SB_ESHAPE
+
+
+def test_module_record_validation_without_gpu(sb):
+    L = sb.lib()
+    y, x, c, s, st, ws = (_fake(a) for a in (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000))
+    assert L.sb_module_record(None, x, c, 4, 64, None, 1, s, st, ws, None) == sb.SB_EINVAL
+    assert L.sb_module_record(y, x, c, 4, 64, None, 1, s, None, ws, None) == sb.SB_EINVAL
+    assert L.sb_module_record(y, _fake(0x2008), c, 4, 64, None, 1, s, st, ws, None) == sb.SB_EALIGN
+    assert L.sb_module_record(y, x, c, 4, 64, _fake(0x7002), 1, s, st, ws, None) == sb.SB_EALIGN
+    assert L.sb_module_record(y, x, c, 0, 64, None, 1, s, st, ws, None) == sb.SB_ESHAPE
+    assert L.sb_module_record(y, x, c, 4, 96, None, 1, s, st, ws, None) == sb.SB_EUNSUPPORTED
+    assert L.sb_module_record(y, x, c, 4, 16448, None, 1, s, st, ws, None) == sb.SB_EUNSUPPORTED
+
+
+def test_workspace_holds_two_slot_arrays(sb):
+    n = ctypes.c_size_t(0)
+    assert sb.lib().sb_workspace_size(17776, 3072, ctypes.byref(n)) == sb.SB_OK
+    assert n.value >= 256 + 2 * 48 * ((17776 + 15) // 16)
+
+
 def test_wait_flag_validation_without_gpu(sb):
     L = sb.lib()
     assert L.sb_wait_flag(None, 1, 1000, _fake(0x100), None) == sb.SB_EINVAL

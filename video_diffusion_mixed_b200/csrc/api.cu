@@ -4,7 +4,8 @@
 //   [0, 128)    WsHeader (device error word, last-CTA tickets)
 //   [128, 224)  sb_stats scratch (weight preparation)
 //   [224, 228)  int32 precision scratch (weight preparation)
-//   [256, ...)  one 48-byte GroupSlot per aligned group of 16 rows (kGroupRows)
+//   [256, ...)  one 48-byte GroupSlot per aligned group of 16 rows (kGroupRows), then (for
+//               sb_module_record) a second such array right after the call's own groups
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -83,7 +84,7 @@ sb_status sb_workspace_size(int64_t max_M, int64_t max_K, size_t* bytes) {
   SB_REQUIRE(bytes != nullptr, SB_EINVAL, "bytes is NULL");
   SB_REQUIRE(max_M >= 0 && max_K >= 0, SB_ESHAPE, "negative size");
   const size_t groups = (size_t)sb::ceil_div(max_M > 0 ? max_M : 1, sb::kGroupRows);
-  size_t b = kOffGroups + groups * sizeof(sb::GroupSlot);
+  size_t b = kOffGroups + 2 * groups * sizeof(sb::GroupSlot);  // two slot arrays (sb_module_record)
   *bytes = (b + 255) & ~(size_t)255;
   return ok();
 }
@@ -627,6 +628,71 @@ sb_status sb_tdc_reuse(const void* x, const void* delta, void* y, int64_t M, int
   if (st != SB_OK) return st;
   cudaError_t e = sb::launch_tdc_reuse(x, delta, y, M * C, state, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "k_tdc_combine (reuse) launch");
+  return ok();
+}
+
+static sb_status tdc_fp8_args(const void* x, const void* yd, const void* codes, const float* scale, int64_t M,
+                              int64_t C, const sb_module_state* state) {
+  SB_REQUIRE(x && yd && codes && scale && state, SB_EINVAL, "x, y, codes, scale and state are required");
+  SB_ALIGNED(x, "x");
+  SB_ALIGNED(yd, "y");
+  SB_ALIGNED(codes, "codes");
+  SB_REQUIRE((reinterpret_cast<uintptr_t>(scale) & 3u) == 0, SB_EALIGN, "scale misaligned");
+  SB_REQUIRE(M >= 1 && M <= (int64_t)1 << 30, SB_ESHAPE, "M out of range (%lld)", (long long)M);
+  SB_REQUIRE(C >= 16 && C % 16 == 0 && C <= (int64_t)1 << 20, SB_EUNSUPPORTED,
+             "C must be a multiple of 16 (got %lld)", (long long)C);
+  return SB_OK;
+}
+
+sb_status sb_tdc_refresh_fp8(const void* x, const void* y, uint8_t* codes, float* scale, int64_t M, int64_t C,
+                             const sb_module_state* state, sb_stream stream) {
+  const sb_status st = tdc_fp8_args(x, y, codes, scale, M, C, state);
+  if (st != SB_OK) return st;
+  cudaError_t e = sb::launch_tdc_refresh8(x, y, codes, scale, M, C, state, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "k_tdc_refresh8 launch");
+  return ok();
+}
+
+sb_status sb_tdc_reuse_fp8(const void* x, const uint8_t* codes, const float* scale, void* y, int64_t M, int64_t C,
+                           const sb_module_state* state, sb_stream stream) {
+  const sb_status st = tdc_fp8_args(x, y, codes, scale, M, C, state);
+  if (st != SB_OK) return st;
+  cudaError_t e = sb::launch_tdc_reuse8(x, codes, scale, y, M, C, state, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "k_tdc_reuse8 launch");
+  return ok();
+}
+
+sb_status sb_module_record(const void* y, const void* x, void* cache, int64_t M, int64_t C, int32_t* prec,
+                           int32_t update_cache, sb_stats* stats, sb_module_state* state, void* ws,
+                           sb_stream stream) {
+  SB_REQUIRE(y && x && cache && stats && state && ws, SB_EINVAL, "y, x, cache, stats, state and ws are required");
+  SB_ALIGNED(y, "y");
+  SB_ALIGNED(x, "x");
+  SB_ALIGNED(cache, "cache");
+  SB_ALIGNED(stats, "stats");
+  SB_ALIGNED(state, "state");
+  SB_ALIGNED(ws, "ws");
+  if (prec) SB_REQUIRE((reinterpret_cast<uintptr_t>(prec) & 3u) == 0, SB_EALIGN, "prec misaligned");
+  SB_REQUIRE(M >= 1 && M <= (int64_t)1 << 30, SB_ESHAPE, "M out of range (%lld)", (long long)M);
+  SB_REQUIRE(C >= 64 && C % 64 == 0 && C <= sb::kMaxK, SB_EUNSUPPORTED, "C must be a multiple of 64 in [64, %d]",
+             sb::kMaxK);
+  sb::RecordLaunch p{};
+  p.Y = y;
+  p.X = x;
+  p.Cache = cache;
+  p.M = M;
+  p.C = C;
+  p.prec = prec;
+  p.rho = 0.0;
+  p.force = -1;
+  p.update = update_cache ? 1 : 0;
+  p.stats = stats;
+  p.st = state;
+  p.groups = ws_groups(ws);
+  p.groups2 = static_cast<char*>(ws_groups(ws)) + sb::ceil_div(M, sb::kGroupRows) * sizeof(sb::GroupSlot);
+  p.hdr = ws;
+  cudaError_t e = sb::launch_module_record(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sb_module_record");
   return ok();
 }
 

@@ -6,10 +6,11 @@
 // the delta tokens' GEMM plus, once per cube, the core token's product with the weight, added to
 // every token of the cube.
 //
-//  k_delta_split    one CTA per cube: per channel the pairwise FP32 sum over the cube's tokens
-//                   (token order, zero-padded to a power of two), the mean, the core's amax and
-//                   scale, its E4M3 codes, its dequantized value (kept as bf16 for the core GEMM),
-//                   and the cube's delta tokens bf16(x - core).
+//  k_delta_split    one CTA per cube, 8 channels per thread and step: per channel the pairwise
+//                   FP32 sum over the cube's tokens (token order, zero-padded to a power of two),
+//                   the mean, the core's amax and scale, its E4M3 codes, its dequantized value
+//                   (kept as bf16 for the core GEMM), and the cube's delta tokens bf16(x - core).
+//                   Instantiated for cubes of up to 8 tokens and of up to 32.
 //  k_delta_combine  Y[t] = act(Yd[t] + Yc[cube(t)]) in FP32, stored as bf16.
 #include <cfloat>
 
@@ -50,62 +51,74 @@ __device__ __forceinline__ int cube_tokens(const CubeGeom& g, int64_t k, int64_t
   return n;
 }
 
-// Pairwise FP32 tree over v[0 .. N) (N a power of two), in place.
-template <int N>
-__device__ __forceinline__ float2 tree_pair2(float2 (&v)[kDqMaxCube]) {
+// Sum of the leaves v[0 .. n2) by the canonical pairwise tree (n2 a power of two <= NMAX; the
+// leaves in [n, n2) are +0). The levels are formed for all NMAX leaves and the level of n2 is
+// returned, so every index is a compile-time constant and the leaves stay in registers.
+template <int NMAX>
+__device__ __forceinline__ float tree_sum(float (&v)[NMAX], int n2) {
+  float r = v[0];
 #pragma unroll
-  for (int len = N; len > 1; len >>= 1) {
+  for (int len = 2; len <= NMAX; len <<= 1) {
 #pragma unroll
-    for (int i = 0; i < len / 2; ++i) v[i] = make_float2(__fadd_rn(v[2 * i].x, v[2 * i + 1].x), __fadd_rn(v[2 * i].y, v[2 * i + 1].y));
+    for (int i = 0; i < NMAX / len; ++i) v[i] = __fadd_rn(v[2 * i], v[2 * i + 1]);
+    if (n2 == len) r = v[0];
   }
-  return v[0];
+  return r;
 }
 
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&f)[8]) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(u[i] << 16);
+    f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+  }
+}
+
+// One CTA per cube; each thread takes groups of 8 channels (16-byte loads of every token of the
+// cube). Pass 1: the channel means (into shared memory) and the core's amax; pass 2: codes, the
+// bf16 core, and the delta tokens from a second read of the cube's rows (L1-resident by then).
+template <int NMAX>
 __global__ void __launch_bounds__(kDqThreads) k_delta_split(const __nv_bfloat16* X, int K, CubeGeom g,
                                                            uint8_t* codes, float* scale, __nv_bfloat16* core16,
                                                            __nv_bfloat16* delta) {
   extern __shared__ float s_mean[];  // K means of this cube
   __shared__ float s_wmax[kDqThreads / 32];
-  __shared__ int64_t tok[kDqMaxCube];  // the cube's tokens, index order
+  __shared__ int64_t s_tok[kDqMaxCube];  // the cube's tokens, index order
   __shared__ int s_n;
   const int64_t k = blockIdx.x;
-  if (threadIdx.x == 0) {
-    int64_t t[kDqMaxCube];
-    const int nn = cube_tokens(g, k, t);
-    for (int j = 0; j < nn; ++j) tok[j] = t[j];
-    s_n = nn;
-  }
+  if (threadIdx.x == 0) s_n = cube_tokens(g, k, s_tok);
   __syncthreads();
   const int n = s_n;
   int n2 = 1;
   while (n2 < n) n2 <<= 1;
   const float fn = (float)n;
-  // ---- pass 1: means of channel pairs (one 32-bit word of bf16 per token)
-  float am = 0.0f;
-  for (int c2 = threadIdx.x; c2 < K / 2; c2 += kDqThreads) {
-    float2 v[kDqMaxCube];
+  const int G = K / 8;  // 8-channel groups per token
+  const uint4* rows[NMAX];
 #pragma unroll
-    for (int j = 0; j < kDqMaxCube; ++j) {
-      if (j < n) {
-        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(X + tok[j] * K) + c2);
-        v[j] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-      } else {
-        v[j] = make_float2(0.0f, 0.0f);
+  for (int j = 0; j < NMAX; ++j) rows[j] = reinterpret_cast<const uint4*>(X + (j < n ? s_tok[j] : s_tok[0]) * K);
+  // ---- pass 1: means and amax
+  float am = 0.0f;
+  for (int gi = threadIdx.x; gi < G; gi += kDqThreads) {
+    uint4 raw[NMAX];
+#pragma unroll
+    for (int j = 0; j < NMAX; ++j) raw[j] = (j < n) ? __ldg(rows[j] + gi) : make_uint4(0u, 0u, 0u, 0u);
+    float m[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float v[NMAX];
+#pragma unroll
+      for (int j = 0; j < NMAX; ++j) {
+        float f[8];
+        bf16x8_to_f32(raw[j], f);
+        v[j] = f[c];
       }
+      m[c] = __fdiv_rn(tree_sum<NMAX>(v, n2), fn);
+      am = fmaxf(am, fabsf(m[c]));
     }
-    float2 s;
-    switch (n2) {  // the canonical tree over exactly n2 leaves (padding with +0 beyond n)
-      case 1: s = v[0]; break;
-      case 2: s = tree_pair2<2>(v); break;
-      case 4: s = tree_pair2<4>(v); break;
-      case 8: s = tree_pair2<8>(v); break;
-      case 16: s = tree_pair2<16>(v); break;
-      default: s = tree_pair2<32>(v); break;
-    }
-    const float m0 = __fdiv_rn(s.x, fn), m1 = __fdiv_rn(s.y, fn);
-    s_mean[2 * c2] = m0;
-    s_mean[2 * c2 + 1] = m1;
-    am = fmaxf(am, fmaxf(fabsf(m0), fabsf(m1)));
+    float4* sm = reinterpret_cast<float4*>(s_mean + 8 * gi);
+    sm[0] = make_float4(m[0], m[1], m[2], m[3]);
+    sm[1] = make_float4(m[4], m[5], m[6], m[7]);
   }
   am = warp_max_f32(am);
   if ((threadIdx.x & 31) == 0) s_wmax[threadIdx.x >> 5] = am;
@@ -118,28 +131,52 @@ __global__ void __launch_bounds__(kDqThreads) k_delta_split(const __nv_bfloat16*
   const float inv = (a == 0.0f) ? 0.0f : __fdiv_rn(448.0f, a);
   const bool finite = inv <= FLT_MAX;
   if (threadIdx.x == 0) scale[k] = s;
-  for (int c2 = threadIdx.x; c2 < K / 2; c2 += kDqThreads) {
-    const float m0 = s_mean[2 * c2], m1 = s_mean[2 * c2 + 1];
-    uint32_t q0, q1;
-    if (a == 0.0f) {
-      q0 = q1 = 0u;
-    } else if (!finite) {  // 448 / a overflowed: nonzero means take +-448, zeros 0
-      q0 = (m0 == 0.0f) ? 0u : ((m0 < 0.0f ? 0x80u : 0u) | 0x7eu);
-      q1 = (m1 == 0.0f) ? 0u : ((m1 < 0.0f ? 0x80u : 0u) | 0x7eu);
-    } else {
-      uint16_t c16;
-      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c16) : "f"(__fmul_rn(m1, inv)), "f"(__fmul_rn(m0, inv)));
-      q0 = c16 & 0xffu;
-      q1 = c16 >> 8;
+  for (int gi = threadIdx.x; gi < G; gi += kDqThreads) {
+    const float4* sm = reinterpret_cast<const float4*>(s_mean + 8 * gi);
+    const float4 m0 = sm[0], m1 = sm[1];
+    const float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+    uint32_t q[8];
+#pragma unroll
+    for (int c = 0; c < 8; c += 2) {
+      if (a == 0.0f) {
+        q[c] = q[c + 1] = 0u;
+      } else if (!finite) {  // 448 / a overflowed: nonzero means take +-448, zeros 0
+        q[c] = (m[c] == 0.0f) ? 0u : ((m[c] < 0.0f ? 0x80u : 0u) | 0x7eu);
+        q[c + 1] = (m[c + 1] == 0.0f) ? 0u : ((m[c + 1] < 0.0f ? 0x80u : 0u) | 0x7eu);
+      } else {
+        uint16_t c16;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(c16)
+            : "f"(__fmul_rn(m[c + 1], inv)), "f"(__fmul_rn(m[c], inv)));
+        q[c] = c16 & 0xffu;
+        q[c + 1] = c16 >> 8;
+      }
     }
-    reinterpret_cast<uint16_t*>(codes + k * K)[c2] = (uint16_t)(q0 | (q1 << 8));
-    const float d0 = __fmul_rn(e4m3_to_f32(q0), s), d1 = __fmul_rn(e4m3_to_f32(q1), s);
-    reinterpret_cast<__nv_bfloat162*>(core16 + k * K)[c2] = __floats2bfloat162_rn(d0, d1);
-    for (int j = 0; j < n; ++j) {
-      const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(X + tok[j] * K) + c2);
-      const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
-      reinterpret_cast<__nv_bfloat162*>(delta + tok[j] * K)[c2] =
-          __floats2bfloat162_rn(__fsub_rn(x0, d0), __fsub_rn(x1, d1));
+    reinterpret_cast<uint2*>(codes + k * K)[gi] =
+        make_uint2(q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24), q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24));
+    float d[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) d[c] = __fmul_rn(e4m3_to_f32(q[c]), s);
+    uint32_t cw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(d[2 * i], d[2 * i + 1]);
+      cw[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    reinterpret_cast<uint4*>(core16 + k * K)[gi] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+#pragma unroll
+    for (int j = 0; j < NMAX; ++j) {
+      if (j < n) {
+        float x[8];
+        bf16x8_to_f32(__ldg(rows[j] + gi), x);
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(__fsub_rn(x[2 * i], d[2 * i]), __fsub_rn(x[2 * i + 1], d[2 * i + 1]));
+          o[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        reinterpret_cast<uint4*>(delta + s_tok[j] * K)[gi] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
   }
 }
@@ -204,15 +241,21 @@ static CubeGeom geom_from(const DeltaCubes& c) {
 cudaError_t launch_delta_split(const void* X, int64_t K, const DeltaCubes& c, int64_t ncube, uint8_t* codes,
                                float* scale, void* core16, void* delta, cudaStream_t s) {
   const int dsm = (int)(K * sizeof(float));
-  static std::atomic<uint64_t> attr{0};
+  const bool small = (int64_t)c.ct * c.ch * c.cw <= 8;
+  static std::atomic<uint64_t> attr8{0}, attr32{0};
   if (dsm > 48 * 1024) {
-    const cudaError_t e = smem_attr_once(k_delta_split, 64 * 1024, attr);
+    const cudaError_t e = small ? smem_attr_once(k_delta_split<8>, 64 * 1024, attr8)
+                                : smem_attr_once(k_delta_split<kDqMaxCube>, 64 * 1024, attr32);
     if (e != cudaSuccess) return e;
   }
-  k_delta_split<<<(unsigned)ncube, kDqThreads, dsm, s>>>(reinterpret_cast<const __nv_bfloat16*>(X), (int)K,
-                                                         geom_from(c), codes, scale,
-                                                         reinterpret_cast<__nv_bfloat16*>(core16),
-                                                         reinterpret_cast<__nv_bfloat16*>(delta));
+  const CubeGeom g = geom_from(c);
+  const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(X);
+  __nv_bfloat16* c16 = reinterpret_cast<__nv_bfloat16*>(core16);
+  __nv_bfloat16* d16 = reinterpret_cast<__nv_bfloat16*>(delta);
+  if (small)
+    k_delta_split<8><<<(unsigned)ncube, kDqThreads, dsm, s>>>(x, (int)K, g, codes, scale, c16, d16);
+  else
+    k_delta_split<kDqMaxCube><<<(unsigned)ncube, kDqThreads, dsm, s>>>(x, (int)K, g, codes, scale, c16, d16);
   return cudaGetLastError();
 }
 

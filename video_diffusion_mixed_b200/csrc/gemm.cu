@@ -807,11 +807,13 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   p.M = (int)L.M;
   p.N = (int)L.N;
   p.K = (int)L.K;
-  // Tile width per precision: 256, or 128 when N is not a multiple of 256; the kernel also takes
-  // 192-wide NVFP4 tiles (two accumulators next to the scale columns), which measured slower than
-  // one 256-wide accumulator on the FFN shapes.
+  // Tile width per precision: 256, or 128 when N is not a multiple of 256. NVFP4 takes 192-wide
+  // tiles (two accumulators next to the scale columns) when N is a multiple of 192 but not of 256:
+  // measured on B200, 16% and 10% faster than 128-wide tiles on 1920-wide layers, while on the FFN
+  // shapes one 256-wide accumulator beats two 192-wide ones by 5-12% (the narrower tile reads more
+  // shared memory per MMA flop).
   const int bn_q = (L.N % 256 == 0) ? 256 : 128;
-  const int bn_f = bn_q;
+  const int bn_f = (L.N % 256 != 0 && L.N % 192 == 0) ? 192 : bn_q;
   p.bn[KIND_FP4] = bn_f;
   p.bn[KIND_I8] = p.bn[KIND_BF16] = bn_q;
   p.invB = 1.0f / (float)L.B;

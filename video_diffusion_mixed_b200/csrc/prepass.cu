@@ -10,6 +10,8 @@
 //  k_rows<.., OP_TDC>      relative L1 change between a module's new output and its cached last
 //                 output, cache refresh in the same pass, module-state update by the last CTA.
 //                 ("write-up" section 二; explainer section 3.)
+//  k_rows<.., OP_REC>      OP_STATS (with the module input as x_ref) and OP_TDC over one read of
+//                 the module output: both statistics records, the cache refresh, the state.
 //  k_nvfp4        re-reads X once the tensor amax is known, rotates again and writes E2M1 codes,
 //                 E4M3 block scales in the tensor-core layout and the FP32 tensor scale.
 //  k_rotate       rotation only (test hook).
@@ -109,6 +111,34 @@ cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s) {
   RowMaps mp;
   row_maps(a, mp, p.Y, p.Cache);
   return launch_rows_t<OP_TDC, true>(a, mp, s, sm_count());
+}
+
+cudaError_t launch_module_record(const RecordLaunch& p, cudaStream_t s) {
+  RowArgs a{};
+  a.X = reinterpret_cast<const __nv_bfloat16*>(p.Y);
+  a.R = const_cast<__nv_bfloat16*>(reinterpret_cast<const __nv_bfloat16*>(p.X));
+  a.C3 = reinterpret_cast<__nv_bfloat16*>(p.Cache);
+  a.M = p.M;
+  a.K = (int)p.C;
+  a.B = 0;
+  a.mode = SB_PREPASS_STATS;
+  a.prec = p.prec;
+  a.rho = p.rho;
+  a.force = p.force;
+  a.update = p.update;
+  a.st = p.st;
+  a.stats = p.stats;
+  a.groups = reinterpret_cast<GroupSlot*>(p.groups);
+  a.groups2 = reinterpret_cast<GroupSlot*>(p.groups2);
+  a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
+  a.finish = 1;
+  RowMaps mp;
+  memset(&mp, 0, sizeof(mp));
+  a.tma = (make_row_segment_map(&mp.x, p.Y, a.M, a.K) && make_row_segment_map(&mp.r, p.X, a.M, a.K) &&
+           make_row_segment_map(&mp.c, p.Cache, a.M, a.K))
+              ? 1
+              : 0;
+  return launch_rows_rec(a, mp, s, sm_count());
 }
 
 cudaError_t launch_finish(const FinishLaunch& p, cudaStream_t s) {

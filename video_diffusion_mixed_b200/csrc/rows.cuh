@@ -31,11 +31,12 @@ namespace sb {
 constexpr int kRowWarps = 8;  // warps per CTA
 constexpr int kG = kGroupRows;  // rows per FP64 group
 
-enum { OP_PREPASS = 0, OP_STATS = 1, OP_TDC = 2 };
+enum { OP_PREPASS = 0, OP_STATS = 1, OP_TDC = 2, OP_REC = 3 };  // OP_REC: OP_STATS (x_ref) + OP_TDC in one pass
 
 struct RowArgs {
-  const __nv_bfloat16* X;  // PREPASS / STATS: the tensor; TDC: the new module output
-  __nv_bfloat16* R;        // PREPASS / STATS: x_ref (may be null); TDC: the cached last output
+  const __nv_bfloat16* X;  // PREPASS / STATS: the tensor; TDC, REC: the new module output
+  __nv_bfloat16* R;        // PREPASS / STATS: x_ref (may be null); TDC: the cached last output; REC: x_ref
+  __nv_bfloat16* C3;       // REC: the cached last output
   int64_t M;
   int K, B;
   int mode;         // SB_PREPASS_QUANT / SB_PREPASS_STATS
@@ -49,6 +50,7 @@ struct RowArgs {
   const sb_stats* dsrc;   // TDC: where d comes from
   sb_module_state* st;    // TDC: module state
   GroupSlot* groups;
+  GroupSlot* groups2;     // REC: the TDC record's group slots (groups: the statistics')
   WsHeader* hdr;
   sb_stats* stats;
   int tma;  // rows arrive through the TMA rings (the maps below are valid)
@@ -61,6 +63,7 @@ struct RowArgs {
 struct RowMaps {
   CUtensorMap x;
   CUtensorMap r;
+  CUtensorMap c;  // REC: the cache
 };
 
 constexpr uint64_t kRowWaitNs = 2000000000ull;  // 2 s: far above any legitimate wait
@@ -70,11 +73,15 @@ constexpr uint64_t kRowDrainNs = 20000000ull;
 // warp, D slots per warp (2..4, about 200 KB per CTA at most).
 template <int SPW, int OP, bool REF>
 struct RowRing {
-  static constexpr int NT = (OP == OP_TDC || REF) ? 2 : 1;
+  static constexpr int NT = (OP == OP_REC) ? 3 : ((OP == OP_TDC || REF) ? 2 : 1);
   static constexpr int SEG = 2048;
   static constexpr int SLOT = NT * SPW * SEG;
   static constexpr int D0 = (200 * 1024) / (kRowWarps * SLOT);
-  static constexpr int D = D0 < 2 ? 2 : (D0 > 4 ? 4 : D0);
+  // two rows in flight per warp; the fused record (three tensors) may keep one: its slot is read
+  // into registers before the next row is issued into it, so that row's load still overlaps the
+  // current row's arithmetic
+  static constexpr int DMIN = (OP == OP_REC) ? 1 : 2;
+  static constexpr int D = D0 < DMIN ? DMIN : (D0 > 4 ? 4 : D0);
   static constexpr int BYTES = kRowWarps * D * SLOT;
 };
 
@@ -459,7 +466,9 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   constexpr int NTEAM = kRowWarps / T;
   constexpr int NSEG = T * SPW;
   constexpr int NSEG2 = pow2_at_least(NSEG);
-  constexpr int NST = (OP == OP_TDC) ? 2 : 3;  // statistics per row
+  // statistics per row; REC: |y|, (y - x)^2, x^2 of the difference statistic, then |y - c|, |c|
+  constexpr int NST = (OP == OP_TDC) ? 2 : (OP == OP_REC ? 5 : 3);
+  static_assert(RG::BYTES + 1024 <= 227 * 1024, "row ring exceeds shared memory");
   __shared__ float s_seg[NTEAM][2][NST][NSEG];  // team exchange (T > 1), by row parity
   __shared__ float s_wmax[NTEAM][2][T];        // per-warp rotated amax
   __shared__ float s_wraw[NTEAM][2][T];        // per-warp raw max |x|
@@ -480,8 +489,15 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
 
   int prec = -1;
   bool have_prev = true;
+  bool do_stats = OP != OP_TDC, do_tdc = OP == OP_TDC;  // REC: each part keeps its own gate
   if (OP == OP_TDC) {
     if (a.st->skip) return;  // the module reuses its cache at this step
+    have_prev = a.st->n_out >= 1;
+  } else if (OP == OP_REC) {
+    prec = a.prec ? *a.prec : -1;
+    do_stats = prec != SB_SKIP;
+    do_tdc = a.st->skip == 0;
+    if (!do_stats && !do_tdc) return;
     have_prev = a.st->n_out >= 1;
   } else {
     prec = a.force_int8 ? SB_INT8 : (a.prec ? *a.prec : -1);
@@ -492,11 +508,16 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   const int64_t ngroups = ceil_div(a.M, kG);
 
   // A team walks its rows of the CTA's groups in order: row i = team + NTEAM * j (j < RPT) of
-  // group g = blockIdx.x + n * gridDim.x.
+  // group g = blockIdx.x + n * gridDim.x. The difference statistic (OP_STATS) walks the groups from
+  // the end of the tensor instead: its input is usually a GEMM output whose last rows were written
+  // last and are still in L2, and the TDC record that follows it (forward) then finds the first
+  // rows, which this pass read last. Returns false past the last group.
   constexpr int RPT = kG / NTEAM;
-  auto row_of = [&](int64_t it, int64_t* g, int* i) {
-    *g = blockIdx.x + (it / RPT) * (int64_t)gridDim.x;
+  auto row_of = [&](int64_t it, int64_t* g, int* i) -> bool {
+    const int64_t g0 = blockIdx.x + (it / RPT) * (int64_t)gridDim.x;
+    *g = (OP == OP_STATS) ? ngroups - 1 - g0 : g0;
     *i = team + (int)(it % RPT) * NTEAM;
+    return g0 < ngroups;
   };
   // this warp's ring: slot s holds, per tensor t and segment c, the box of segment c*T + wt
   const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * RG::D * RG::SLOT);
@@ -504,8 +525,7 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   auto issue_row = [&](int64_t it) {  // lane 0
     int64_t g;
     int i;
-    row_of(it, &g, &i);
-    if (g >= ngroups) return;
+    if (!row_of(it, &g, &i)) return;
     const int m = (int)(g * kG + i);  // rows past M read as zero
     const int slot = (int)(it % RG::D);
     const uint32_t bar = smem_u32(&s_bar[warp][slot]);
@@ -514,8 +534,8 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
     for (int t = 0; t < RG::NT; ++t) {
 #pragma unroll
       for (int c = 0; c < SPW; ++c)
-        tma_load_3d(ring_w + (uint32_t)(slot * RG::SLOT + (t * SPW + c) * RG::SEG), t == 0 ? &mp.x : &mp.r, bar, 0,
-                    (c * T + wt) * 16, m);
+        tma_load_3d(ring_w + (uint32_t)(slot * RG::SLOT + (t * SPW + c) * RG::SEG),
+                    t == 0 ? &mp.x : (t == 1 ? &mp.r : &mp.c), bar, 0, (c * T + wt) * 16, m);
     }
   };
   int64_t bad_it = -1;  // last row whose wait gave up (its copy may still be in flight)
@@ -532,13 +552,12 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   for (int64_t it = 0;; ++it) {
     int64_t g;
     int i;
-    row_of(it, &g, &i);
-    if (g >= ngroups) break;
+    if (!row_of(it, &g, &i)) break;
     const int gpar = (int)((it / RPT) & 1);
     const int rpar = (int)(it & 1);
     const bool group_end = (it % RPT) == RPT - 1;
     const int64_t m = g * kG + i;
-    Raw32 xr[SPW], rr[SPW];
+    Raw32 xr[SPW], rr[SPW], cr[OP == OP_REC ? SPW : 1];
     if (use_tma) {
       // this row's slot: wait for its boxes, copy the lane's part to registers, refill the slot
       // with the row D steps ahead
@@ -550,9 +569,13 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
       const uint32_t sl = ring_w + (uint32_t)(slot * RG::SLOT);
 #pragma unroll
       for (int c = 0; c < SPW; ++c) read_seg_sw128(xr[c], sl + (uint32_t)(c * RG::SEG), lane);
-      if (RG::NT == 2) {
+      if (RG::NT >= 2) {
 #pragma unroll
         for (int c = 0; c < SPW; ++c) read_seg_sw128(rr[c], sl + (uint32_t)((SPW + c) * RG::SEG), lane);
+      }
+      if (OP == OP_REC) {
+#pragma unroll
+        for (int c = 0; c < SPW; ++c) read_seg_sw128(cr[c], sl + (uint32_t)((2 * SPW + c) * RG::SEG), lane);
       }
       __syncwarp();
       if (lane == 0) issue_row(it + RG::D);
@@ -560,10 +583,15 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
 #pragma unroll
         for (int c = 0; c < SPW; ++c) rr[c].q[0] = rr[c].q[1] = rr[c].q[2] = rr[c].q[3] = make_uint4(0, 0, 0, 0);
       }
+      if (OP == OP_REC && !have_prev) {
+#pragma unroll
+        for (int c = 0; c < SPW; ++c) cr[c].q[0] = cr[c].q[1] = cr[c].q[2] = cr[c].q[3] = make_uint4(0, 0, 0, 0);
+      }
     }
     if (m < a.M) {
       const __nv_bfloat16* xrow = a.X + m * K;
       __nv_bfloat16* rrow = (OP == OP_TDC || REF) ? a.R + m * K : nullptr;
+      __nv_bfloat16* crow = (OP == OP_REC) ? a.C3 + m * K : nullptr;
       if (!use_tma) {
 #pragma unroll
         for (int c = 0; c < SPW; ++c) {
@@ -571,6 +599,7 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
           load_raw(xr[c], xrow, e0, K, true);
           if (OP == OP_TDC) load_raw_coherent(rr[c], rrow, e0, K, have_prev);
           else if (REF) load_raw(rr[c], rrow, e0, K, true);
+          if (OP == OP_REC) load_raw_coherent(cr[c], crow, e0, K, have_prev);
         }
       }
       float seg[NST][SPW];
@@ -622,6 +651,29 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
           } else {
             seg[1][c] = 0.0f;
             seg[2][c] = 0.0f;
+          }
+          if (OP == OP_REC) {  // the TDC record's |y - c| and |c|, and the cache refresh
+            float2 r[16];
+            unpack_pairs(cr[c], r);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) t[k] = abs2(sub2(p[k], r[k]));
+            seg[NST == 5 ? 3 : 0][c] = warp_pairwise_f32(tree_pairs(t));
+#pragma unroll
+            for (int k = 0; k < 16; ++k) t[k] = abs2(r[k]);
+            seg[NST == 5 ? 4 : 0][c] = warp_pairwise_f32(tree_pairs(t));
+            const int e0 = (c * T + wt) * 1024 + lane * 32;
+            if (do_tdc && a.update) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int e = e0 + 16 * h;
+                if (e + 16 <= K && aligned32(crow + e)) {
+                  stg_v8(crow + e, xr[c].q[2 * h], xr[c].q[2 * h + 1]);
+                } else {
+                  if (e < K) *reinterpret_cast<uint4*>(crow + e) = xr[c].q[2 * h];
+                  if (e + 8 < K) *reinterpret_cast<uint4*>(crow + e + 8) = xr[c].q[2 * h + 1];
+                }
+              }
+            }
           }
           if (OP == OP_PREPASS) {
             fwht_pairs(p, lane, a.B);
@@ -738,10 +790,19 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
       if (lane == 0) {
         GroupSlot* slot = a.groups + g;
 #pragma unroll
-        for (int s = 0; s < NST; ++s) slot->s[s] = gs[s];
+        for (int s = 0; s < (NST < 3 ? NST : 3); ++s) slot->s[s] = gs[s];
         slot->max_abs = gmx;
         slot->amax_rot = gam;
         slot->nonfinite = gnf;
+        if (OP == OP_REC) {
+          GroupSlot* slot2 = a.groups2 + g;
+          slot2->s[0] = gs[NST == 5 ? 3 : 0];
+          slot2->s[1] = gs[NST == 5 ? 4 : 0];
+          slot2->s[2] = 0.0;
+          slot2->max_abs = 0.0f;
+          slot2->amax_rot = 0.0f;
+          slot2->nonfinite = 0;
+        }
       }
     }
   }
@@ -749,7 +810,19 @@ __global__ void __launch_bounds__(256) k_rows(RowArgs a, const __grid_constant__
   // ring is reused or the CTA exits
   if (use_tma && bad_it >= 0 && lane == 0)
     mbar_wait_bounded(&s_bar[warp][bad_it % RG::D], (uint32_t)((bad_it / RG::D) & 1), nullptr, kRowDrainNs);
-  if (a.finish) rows_finish<OP, REF>(a, ngroups, prec, have_prev, s_fin);
+  if (OP == OP_REC) {
+    // the statistics record first: the TDC record takes its d (the last CTA of the second ticket
+    // runs after every CTA has passed the first finish, which wrote the record)
+    if (a.finish && do_stats) rows_finish<OP_STATS, true>(a, ngroups, prec, true, s_fin);
+    if (a.finish && do_tdc) {
+      RowArgs t = a;
+      t.groups = a.groups2;
+      t.dsrc = a.stats;
+      rows_finish<OP_TDC, true>(t, ngroups, prec, have_prev, s_fin);
+    }
+  } else if (a.finish) {
+    rows_finish<OP, REF>(a, ngroups, prec, have_prev, s_fin);
+  }
 }
 
 // The final reduction alone, over group slots written by earlier launches (the shards of a
@@ -806,6 +879,40 @@ cudaError_t launch_rows_t(const RowArgs& a, const RowMaps& mp, cudaStream_t s, i
   SB_ROWS_CASE(4, 3)
   SB_ROWS_CASE(8, 2)
 #undef SB_ROWS_CASE
+  return cudaErrorInvalidValue;
+}
+
+// The fused record (OP_REC) rings three tensors per row; it takes the tiling of the other row
+// kernels (with one row in flight per warp at SPW = 3).
+inline void pick_rec_tiling(int K, int* T, int* SPW) { pick_row_tiling(K, T, SPW); }
+
+inline cudaError_t launch_rows_rec(const RowArgs& a, const RowMaps& mp, cudaStream_t s, int sms) {
+  int T, SPW;
+  pick_rec_tiling(a.K, &T, &SPW);
+  const int64_t ngroups = ceil_div(a.M, kG);
+#define SB_REC_CASE(TT, SS)                                                                               \
+  if (T == TT && SPW == SS) {                                                                             \
+    constexpr int dsm = RowRing<SS, OP_REC, true>::BYTES + 1024;                                          \
+    static std::atomic<uint64_t> attr{0};                                                                 \
+    const cudaError_t ae = smem_attr_once(k_rows<TT, SS, OP_REC, true>, dsm, attr);                       \
+    if (ae != cudaSuccess) return ae;                                                                     \
+    int occ = 0;                                                                                          \
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_rows<TT, SS, OP_REC, true>, kRowWarps * 32, dsm); \
+    if (occ <= 0) occ = 1;                                                                                \
+    const int64_t cap = (int64_t)sms * occ;                                                               \
+    const unsigned grid = (unsigned)(ngroups < cap ? ngroups : cap);                                      \
+    k_rows<TT, SS, OP_REC, true><<<grid, kRowWarps * 32, dsm, s>>>(a, mp);                                \
+    return cudaGetLastError();                                                                            \
+  }
+  SB_REC_CASE(1, 1)
+  SB_REC_CASE(1, 2)
+  SB_REC_CASE(1, 3)
+  SB_REC_CASE(2, 2)
+  SB_REC_CASE(2, 3)
+  SB_REC_CASE(4, 2)
+  SB_REC_CASE(4, 3)
+  SB_REC_CASE(8, 2)
+#undef SB_REC_CASE
   return cudaErrorInvalidValue;
 }
 

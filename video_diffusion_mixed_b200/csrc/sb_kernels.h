@@ -98,6 +98,25 @@ cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s);
 cudaError_t launch_nvfp4(const Nvfp4Launch& p, cudaStream_t s);
 cudaError_t launch_rotate(const void* X, float* Y, int64_t M, int64_t K, int B, cudaStream_t s);
 cudaError_t launch_tdc_record(const TdcLaunch& p, cudaStream_t s);
+
+// The module's output record: the difference statistic of Y against X and the TDC record of Y
+// against the cache, one pass (OP_REC).
+struct RecordLaunch {
+  const void* Y;
+  const void* X;
+  void* Cache;
+  int64_t M, C;
+  int32_t* prec;
+  double rho;
+  int force;
+  int update;
+  sb_stats* stats;
+  sb_module_state* st;
+  void* groups;
+  void* groups2;
+  void* hdr;
+};
+cudaError_t launch_module_record(const RecordLaunch& p, cudaStream_t s);
 cudaError_t launch_finish(const FinishLaunch& p, cudaStream_t s);
 cudaError_t launch_prepass_chunks(const PrepassLaunch& p, float* chunks, cudaStream_t s);
 
@@ -123,6 +142,10 @@ cudaError_t launch_tdc_refresh(const void* x, const void* y, void* d, int64_t n,
                                cudaStream_t s);
 cudaError_t launch_tdc_reuse(const void* x, const void* d, void* y, int64_t n, const sb_module_state* st,
                              cudaStream_t s);
+cudaError_t launch_tdc_refresh8(const void* x, const void* y, uint8_t* codes, float* scale, int64_t M, int64_t C,
+                                const sb_module_state* st, cudaStream_t s);
+cudaError_t launch_tdc_reuse8(const void* x, const uint8_t* codes, const float* scale, void* y, int64_t M, int64_t C,
+                              const sb_module_state* st, cudaStream_t s);
 cudaError_t launch_ws_init(void* ws, size_t bytes, cudaStream_t s);
 
 // Delta tokens: the cube geometry (text tokens, grid F x H x W, cube ct x ch x cw).

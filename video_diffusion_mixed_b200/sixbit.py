@@ -98,6 +98,9 @@ def lib():
             "sb_prepass_static": (st, [vp, vp, i64, i64, P(Config), i32, vp, P(Fp4), P(I8), vp, vp]),
             "sb_wait_flag": (st, [vp, i32, ctypes.c_uint64, vp, vp]),
             "sb_drill_gemm_stall": (st, [i64, ctypes.c_uint64]),
+            "sb_tdc_refresh_fp8": (st, [vp, vp, vp, vp, i64, i64, vp, vp]),
+            "sb_module_record": (st, [vp, vp, vp, i64, i64, vp, i32, vp, vp, vp, vp]),
+            "sb_tdc_reuse_fp8": (st, [vp, vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_refresh": (st, [vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_reuse": (st, [vp, vp, vp, i64, i64, vp, vp]),
             "sb_group_slots_bytes": (i64, [i64]),
@@ -125,7 +128,8 @@ EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_in
             "sb_linear", "sb_tdc_record", "sb_check", "sb_prepass_static", "sb_wait_flag", "sb_tdc_refresh",
             "sb_tdc_reuse", "sb_group_slots_bytes", "sb_prepass_partial", "sb_prepass_finish", "sb_nvfp4_encode",
             "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide", "sb_prepass_chunks", "sb_cube_count",
-            "sb_delta_split", "sb_delta_combine", "sb_drill_gemm_stall")
+            "sb_delta_split", "sb_delta_combine", "sb_drill_gemm_stall", "sb_tdc_refresh_fp8",
+            "sb_tdc_reuse_fp8", "sb_module_record")
 
 
 def _ck(status: int):
@@ -295,6 +299,13 @@ def linear(X, a4: Fp4Tensor | None, a8: I8Tensor | None, prec, w: Weight, Y, epi
                         _stream(stream)))
 
 
+def module_record(y, x, cache, prec, stats, state, ws: Workspace, update_cache: bool = True, stream=None):
+    """The difference statistic of y against x and the TDC record of y in one pass (sb_module_record)."""
+    M, C = y.shape
+    _ck(lib().sb_module_record(_p(y), _p(x), _p(cache), M, C, _p(prec), int(update_cache), _p(stats), _p(state),
+                               ws.ptr, _stream(stream)))
+
+
 def tdc_record(y_new, y_cache, d_src, state, ws: Workspace, update_cache: bool = True, stream=None):
     M, C = y_new.shape
     _ck(lib().sb_tdc_record(_p(y_new), _p(y_cache), M, C, _p(d_src), int(update_cache), _p(state), ws.ptr,
@@ -377,6 +388,24 @@ def tdc_reuse(x, delta, y, state, stream=None):
     """At a skipped step produce the output from the kept residual: y = bf16(x + delta)."""
     M, C = x.shape
     _ck(lib().sb_tdc_reuse(_p(x), _p(delta), _p(y), M, C, _p(state), _stream(stream)))
+
+
+class Fp8Residual:
+    """Caller-owned FP8 residual of M token rows of C channels: E4M3 codes and one scale per row."""
+
+    def __init__(self, M: int, C: int, device="cuda"):
+        self.codes = torch.zeros((M, C), dtype=torch.uint8, device=device)
+        self.scale = torch.zeros(M, dtype=torch.float32, device=device)
+
+
+def tdc_refresh_fp8(x, y, d: Fp8Residual, state, stream=None):
+    M, C = x.shape
+    _ck(lib().sb_tdc_refresh_fp8(_p(x), _p(y), _p(d.codes), _p(d.scale), M, C, _p(state), _stream(stream)))
+
+
+def tdc_reuse_fp8(x, d: Fp8Residual, y, state, stream=None):
+    M, C = x.shape
+    _ck(lib().sb_tdc_reuse_fp8(_p(x), _p(d.codes), _p(d.scale), _p(y), M, C, _p(state), _stream(stream)))
 
 
 def wait_flag(flag, value: int, limit_ns: int, ws: Workspace, stream=None):
