@@ -41,15 +41,17 @@ METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT sh
 _GEMM_SRC = ("gemm.cu", "sb_device.cuh")
 _ROWS_SRC = ("prepass.cu", "rows.cuh", "prepass_blk.cuh", "sb_device.cuh", "tmap.h")
 TRAFFIC = {
-    "gemm_w1_int8": {"bytes": 764.7e6, "files": _GEMM_SRC, "sha": "7f299b94f250d919"},
-    "gemm_w2_int8": {"bytes": 773.0e6, "files": _GEMM_SRC, "sha": "7f299b94f250d919"},
-    "gemm_w1_nvfp4": {"bytes": 509.4e6, "files": _GEMM_SRC, "sha": "7f299b94f250d919"},
-    "gemm_w2_nvfp4": {"bytes": 256.2e6, "files": _GEMM_SRC, "sha": "7f299b94f250d919"},
+    "gemm_w1_int8": {"bytes": 744.3e6, "files": _GEMM_SRC, "sha": "ead2d2d5eba64b00"},
+    "gemm_w2_int8": {"bytes": 744.3e6, "files": _GEMM_SRC, "sha": "ead2d2d5eba64b00"},
+    "gemm_w1_nvfp4": {"bytes": 501.4e6, "files": _GEMM_SRC, "sha": "ead2d2d5eba64b00"},
+    "gemm_w2_nvfp4": {"bytes": 256.3e6, "files": _GEMM_SRC, "sha": "ead2d2d5eba64b00"},
     # k_prepass_blk + k_nvfp4_blk (the encode exits at once in the INT8 pass)
-    "prepass_h_nvfp4": {"bytes": 971.6e6, "files": _ROWS_SRC, "sha": "f0590a17a64890f5"},
-    "prepass_h_int8": {"bytes": 630.1e6, "files": _ROWS_SRC, "sha": "f0590a17a64890f5"},
-    "prepass_x_nvfp4": {"bytes": 224.7e6, "files": _ROWS_SRC, "sha": "f0590a17a64890f5"},
-    "prepass_x_int8": {"bytes": 127.6e6, "files": _ROWS_SRC, "sha": "f0590a17a64890f5"},
+    "prepass_h_nvfp4": {"bytes": 971.4e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
+    "prepass_h_int8": {"bytes": 630.3e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
+    "prepass_x_nvfp4": {"bytes": 224.6e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
+    "prepass_x_int8": {"bytes": 127.9e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
+    "record_nvfp4": {"bytes": 401.8e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
+    "record_int8": {"bytes": 402.2e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
 }
 TRAFFIC_TOKENS = 17776
 
@@ -387,8 +389,8 @@ class DeltaTokensLayer:
     """The CogVideoX-2B attention projection (17776 x 1920 -> 1920) two ways: the plain NVFP4
     linear (pre-pass + NVFP4 GEMM), and with delta tokens (2 x 2 x 2 cubes of the 13 x 30 x 45
     latent grid, 226 text tokens one cube each): the split into FP8 core and bf16 delta tokens,
-    the delta tokens' pre-pass and NVFP4 GEMM (FP32 output), the cores' BF16 GEMM, and the
-    combine into bf16 output."""
+    the delta tokens' pre-pass, the cores' BF16 GEMM (FP32, no bias), and the delta tokens' NVFP4
+    GEMM whose epilogue adds each token's core row and the bias (bf16 output)."""
 
     def __init__(self, sb, torch, synth, device):
         self.sb, self.torch = sb, torch
@@ -405,7 +407,6 @@ class DeltaTokensLayer:
         self.a4, self.a8, self.st = sb.Fp4Tensor(self.M, self.K), sb.I8Tensor(self.M, self.K), sb.alloc_stats()
         self.p4 = torch.tensor([sb.NVFP4], dtype=torch.int32, device=device)
         self.pb = torch.tensor([sb.BF16], dtype=torch.int32, device=device)
-        self.Yd = torch.empty((self.M, self.N), dtype=torch.float32, device=device)
         self.Yc = torch.empty((self.core.n, self.N), dtype=torch.float32, device=device)
         self.Y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=device)
         self.cfg = sb.config(force_prec=sb.NVFP4)
@@ -430,19 +431,16 @@ class DeltaTokensLayer:
         self._mark(ev, "d1")
         sb.prepass(self.delta, None, self.cfg, sb.PREPASS_QUANT, self.p4, self.a4, self.a8, self.st, self.ws)
         self._mark(ev, "d2")
-        sb.linear(self.delta, self.a4, self.a8, self.p4, self.w_nb, self.Yd, out_dtype=sb.OUT_F32, ws=self.ws)
+        sb.linear(self.core.bf16, None, None, self.pb, self.w_nb, self.Yc, out_dtype=sb.OUT_F32, ws=self.ws)
         self._mark(ev, "d3")
-        sb.linear(self.core.bf16, None, None, self.pb, self.w_b, self.Yc, out_dtype=sb.OUT_F32, ws=self.ws)
+        sb.delta_linear(self.delta, self.a4, self.a8, self.p4, self.w_b, self.Yc, self.c, self.Y, ws=self.ws)
         self._mark(ev, "d4")
-        sb.delta_combine(self.Yd, self.Yc, self.c, self.Y)
-        self._mark(ev, "d5")
 
 
 def run_delta_tokens(torch, sb, synth, flush, device, reps=10):
     L = DeltaTokensLayer(sb, torch, synth, device)
     spans = {"plain_prepass": ("p0", "p1"), "plain_gemm_nvfp4": ("p1", "p2"), "split": ("d0", "d1"),
-             "delta_prepass": ("d1", "d2"), "delta_gemm_nvfp4_f32": ("d2", "d3"), "core_gemm_bf16": ("d3", "d4"),
-             "combine": ("d4", "d5")}
+             "delta_prepass": ("d1", "d2"), "core_gemm_bf16": ("d2", "d3"), "delta_gemm_nvfp4_core_added": ("d3", "d4")}
     holder = {}
 
     def fn():
@@ -783,7 +781,7 @@ def run_ours(args):
         "roofline_prepass": {r["kernel"]: {"achieved_gbs": round(r["achieved"], 1), "frac": round(r["frac"], 4),
                                            "ms": round(r["ms"], 4), "traffic": traffic_of(r["kernel"])} for r in pre},
         "kernels": {r["kernel"]: {"ms": round(r["ms"], 4), "achieved": round(r["achieved"], 1), "unit": r["unit"],
-                                  "frac": round(r["frac"], 4)} for r in rows},
+                                  "frac": round(r["frac"], 4), "traffic": traffic_of(r["kernel"])} for r in rows},
         "kernels_timing": "event nodes inside a CUDA graph of the step (median of the replays, L2 flushed "
                           "before each); the spans tile the step",
         "trajectory": traj,

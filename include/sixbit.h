@@ -378,6 +378,20 @@ sb_status sb_delta_split(const void* X, int64_t M, int64_t K, const sb_cubes* cu
 sb_status sb_delta_combine(const float* y_delta, const float* y_core, int64_t M, int64_t N,
                            const sb_cubes* cubes /* host */, int32_t epilogue, void* Y, sb_stream stream);
 
+/* The delta tokens' linear layer with the combine fused into the GEMM epilogue: as sb_linear on
+ * the delta tokens (delta, a4, a8, prec, w, epilogue, out_dtype, Y, M, ws as there), except that
+ * every output row t adds, before the activation, row cube(t) of y_core (FP32 [cubes][N], the
+ * cores' product with W without bias, e.g. from sb_linear on the cores with SB_OUT_F32):
+ *   Y[t] = act(linear(delta)[t] + bias + y_core[cube(t)]).
+ * The same result as sb_linear with SB_OUT_F32 and no bias followed by sb_delta_combine, within
+ * FP32 rounding (the bias enters the sum at another place), without the FP32 round trip. y_core:
+ * 16-byte aligned (SB_EALIGN); cubes: as for sb_delta_split, covering the M tokens (SB_ESHAPE);
+ * out_dtype SB_OUT_BF16 or SB_OUT_F32 (SB_EINVAL otherwise). */
+sb_status sb_delta_linear(const void* delta, const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */,
+                          const int32_t* prec, const sb_weight* w /* host */, const float* y_core,
+                          const sb_cubes* cubes /* host */, int32_t epilogue, int32_t out_dtype, void* Y, int64_t M,
+                          void* ws, sb_stream stream);
+
 /* The same reuse path with the residual kept in FP8 ("write-up" section 七: the cache's history
  * may be stored in low-precision formats): half the bytes of the bf16 residual.
  *   sb_tdc_refresh_fp8: if the module computed this step (state->skip == 0), per token row m:

@@ -248,3 +248,13 @@ def test_delta_token_validation_without_gpu(sb):
     assert L.sb_delta_combine(Yd, Yc, M, 1924, ctypes.byref(c), 0, Y, None) == sb.SB_EUNSUPPORTED
     assert L.sb_delta_combine(Yd, Yc, M, 1920, ctypes.byref(c), 5, Y, None) == sb.SB_EINVAL
     assert L.sb_delta_combine(Yd, Yc, M - 2, 1920, ctypes.byref(c), 0, Y, None) == sb.SB_ESHAPE
+    # the fused form: y_core and the cubes first, then sb_linear's own checks
+    p, w, ws = _fake(0x90000), sb.WeightC(), _fake(0xA0000)
+    assert L.sb_delta_linear(delta, None, None, p, ctypes.byref(w), None, ctypes.byref(c), 0, 0, Y, M, ws,
+                             None) == sb.SB_EINVAL
+    assert L.sb_delta_linear(delta, None, None, p, ctypes.byref(w), _fake(0x70004), ctypes.byref(c), 0, 0, Y, M,
+                             ws, None) == sb.SB_EALIGN
+    assert L.sb_delta_linear(delta, None, None, p, ctypes.byref(w), Yc, ctypes.byref(c), 0, 2, Y, M, ws,
+                             None) == sb.SB_EINVAL  # raw accumulators are not an output of this form
+    assert L.sb_delta_linear(delta, None, None, p, ctypes.byref(w), Yc, ctypes.byref(c), 0, 0, Y, M - 1, ws,
+                             None) == sb.SB_ESHAPE

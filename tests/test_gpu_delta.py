@@ -148,3 +148,76 @@ def test_delta_linear_full_size_sampled(sbg):
     cube_of = np.array([oracle.cube_of_token(t, g) for t in rows])
     y32 = npy(Yd)[rows] + npy(Yc)[cube_of]
     assert_close(y32, ref, 1e-3)
+
+
+def _fused_delta_linear(sbg, X, c, W, bias, gelu, prec, out_dtype):
+    """sb_delta_linear: the cores' product without bias (BF16 GEMM, FP32), then the delta tokens'
+    GEMM with the bias and the per-token core row added in its epilogue."""
+    M, K = X.shape
+    N = W.shape[0]
+    ws = sbg.Workspace(max(M, N), K)
+    w_nb = sbg.Weight(W, None, 128, ws)
+    w_b = sbg.Weight(W, bias, 128, ws)
+    core = sbg.CoreTokens(c, M, K)
+    delta = torch.empty_like(X)
+    sbg.delta_split(X, c, core, delta)
+    a4, a8, st = sbg.Fp4Tensor(M, K), sbg.I8Tensor(M, K), sbg.alloc_stats()
+    p = torch.tensor([prec], dtype=torch.int32, device="cuda")
+    sbg.prepass(delta, None, sbg.config(force_prec=prec), sbg.PREPASS_QUANT, p, a4, a8, st, ws)
+    pb = torch.tensor([sbg.BF16], dtype=torch.int32, device="cuda")
+    Yc = torch.empty((core.n, N), dtype=torch.float32, device="cuda")
+    sbg.linear(core.bf16, None, None, pb, w_nb, Yc, out_dtype=sbg.OUT_F32, ws=ws)
+    Y = torch.full((M, N), 7.0, dtype=torch.float32 if out_dtype == sbg.OUT_F32 else torch.bfloat16, device="cuda")
+    sbg.delta_linear(delta, a4, a8, p, w_b, Yc, c, Y, epilogue=sbg.EPI_GELU if gelu else sbg.EPI_NONE,
+                     out_dtype=out_dtype, ws=ws)
+    sbg.check(ws)
+    return Y, delta
+
+
+# N = 768 and 1920: 128- and 192-wide tiles (two accumulators, chunked epilogue); 3072: 256-wide
+# NVFP4 tiles (one accumulator, the epilogue drains every column first); BF16: the raw delta tokens
+@pytest.mark.parametrize("N,gelu,prec", [(768, False, 0), (768, True, 0), (1920, True, 0), (3072, False, 0),
+                                         (1920, False, 2)], ids=["768", "768_gelu", "1920_gelu", "3072", "1920_bf16"])
+def test_fused_delta_linear_against_oracle(sbg, N, gelu, prec):
+    text, F, H, W_, cube = 7, 4, 6, 10, (2, 2, 2)
+    M, K = text + F * H * W_, 1920
+    X = synth.activations(M, K, n_outlier=19, scale=30.0, student=True, seed=5, device="cuda")
+    Wt = synth.weight(N, K, seed=5, device="cuda")
+    bias = synth.bias(N, std=0.02, seed=5, device="cuda")
+    c = sbg.cubes(text, F, H, W_, *cube)
+    Y32, delta = _fused_delta_linear(sbg, X, c, Wt, bias, gelu, prec, sbg.OUT_F32)
+    Y16, _ = _fused_delta_linear(sbg, X, c, Wt, bias, gelu, prec, sbg.OUT_BF16)
+    g = _grid(text, F, H, W_, cube)
+    _, _, dec, dref = oracle.delta_split(u16(X), g)
+    if prec == 0:
+        dp = oracle.prepass(dref, None, 128)
+        c4, sfl, _, sg = oracle.quant_nvfp4(dp["y"], dp["amax_rot"])
+        wp = oracle.prepare_weight(u16(Wt), 128)
+        yd_ref = oracle.gemm_nvfp4(c4, sfl, sg, wp["c4"], wp["sf4"], wp["sg4"], None, K, 128)
+    else:
+        yd_ref = oracle.gemm_bf16(dref, u16(Wt), None)
+    ref = oracle.delta_linear(yd_ref, dec, u16(Wt), u16(bias), M, g, gelu=gelu)
+    assert_close(npy(Y32).astype(np.float64), ref, 1e-3)
+    # the bf16 output is the same epilogue value rounded to bf16
+    assert np.array_equal(u16(Y16), oracle.f32_to_bf16(npy(Y32).astype(np.float32)))
+
+
+def test_fused_delta_linear_full_size_sampled(sbg):
+    """The CogVideoX-2B attention projection with the CogVideoX token layout (17776 tokens),
+    sampled rows against the oracle."""
+    text, F, H, W_, cube = 226, 13, 30, 45, (2, 2, 2)
+    M, K, N = 17776, 1920, 1920
+    X = synth.activations(M, K, n_outlier=19, scale=30.0, student=True, seed=6, device="cuda")
+    Wt = synth.weight(N, K, seed=6, device="cuda")
+    bias = synth.bias(N, std=0.02, seed=6, device="cuda")
+    c = sbg.cubes(text, F, H, W_, *cube)
+    Y32, delta = _fused_delta_linear(sbg, X, c, Wt, bias, False, 0, sbg.OUT_F32)
+    g = _grid(text, F, H, W_, cube)
+    _, _, dec, dref = oracle.delta_split(u16(X), g)
+    rows = sample_rows(M)
+    dp = oracle.prepass(dref, None, 128)
+    c4, sfl, _, sg = oracle.quant_nvfp4(dp["y"], dp["amax_rot"])
+    wp = oracle.prepare_weight(u16(Wt), 128)
+    yd_ref = oracle.gemm_nvfp4(c4, sfl, sg, wp["c4"], wp["sf4"], wp["sg4"], None, K, 128, rows=rows)
+    ref = oracle.delta_linear(yd_ref, dec, u16(Wt), u16(bias), M, g, rows=rows)
+    assert_close(npy(Y32)[rows].astype(np.float64), ref, 1e-3)

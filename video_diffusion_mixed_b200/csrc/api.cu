@@ -345,8 +345,10 @@ sb_status sb_prepass(const void* X, const void* X_ref, int64_t M, int64_t K, con
   return ok();
 }
 
-sb_status sb_linear(const void* X, const sb_fp4* a4, const sb_i8* a8, const int32_t* prec, const sb_weight* w,
-                    int32_t epilogue, int32_t out_dtype, void* Y, int64_t M, void* ws, sb_stream stream) {
+// sb_linear's validation and launch; `row` (may be NULL) adds a gathered row to each output row.
+static sb_status linear_impl(const void* X, const sb_fp4* a4, const sb_i8* a8, const int32_t* prec,
+                             const sb_weight* w, int32_t epilogue, int32_t out_dtype, void* Y, int64_t M, void* ws,
+                             sb_stream stream, const sb::GemmLaunch* row) {
   SB_REQUIRE(prec && w && Y && ws, SB_EINVAL, "prec, w, Y and ws are required");
   SB_ALIGNED(Y, "Y");
   SB_ALIGNED(ws, "ws");
@@ -398,10 +400,24 @@ sb_status sb_linear(const void* X, const sb_fp4* a4, const sb_i8* a8, const int3
   L.out_dtype = out_dtype;
   L.Y = Y;
   L.hdr = ws;
+  if (row) {
+    L.rowadd = row->rowadd;
+    L.ra_T = row->ra_T;
+    L.ra_H = row->ra_H;
+    L.ra_W = row->ra_W;
+    L.ra_ct = row->ra_ct;
+    L.ra_ch = row->ra_ch;
+    L.ra_cw = row->ra_cw;
+  }
   const char* why = "kernel launch";
   cudaError_t e = sb::launch_gemm(L, (cudaStream_t)stream, &why);
   if (e != cudaSuccess) return cuda_fail(e, why);
   return ok();
+}
+
+sb_status sb_linear(const void* X, const sb_fp4* a4, const sb_i8* a8, const int32_t* prec, const sb_weight* w,
+                    int32_t epilogue, int32_t out_dtype, void* Y, int64_t M, void* ws, sb_stream stream) {
+  return linear_impl(X, a4, a8, prec, w, epilogue, out_dtype, Y, M, ws, stream, nullptr);
 }
 
 sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C, const sb_stats* d_src,
@@ -736,6 +752,27 @@ int64_t sb_cube_count(const sb_cubes* cubes, int64_t M) {
   int64_t n = -1;
   if (!cubes_geom(cubes, M, &g, &n)) return -1;
   return n;
+}
+
+sb_status sb_delta_linear(const void* delta, const sb_fp4* a4, const sb_i8* a8, const int32_t* prec,
+                          const sb_weight* w, const float* y_core, const sb_cubes* cubes, int32_t epilogue,
+                          int32_t out_dtype, void* Y, int64_t M, void* ws, sb_stream stream) {
+  SB_REQUIRE(y_core && cubes, SB_EINVAL, "y_core and cubes are required");
+  SB_ALIGNED(y_core, "y_core");
+  SB_REQUIRE(out_dtype == SB_OUT_BF16 || out_dtype == SB_OUT_F32, SB_EINVAL, "out_dtype must be BF16 or F32");
+  sb::DeltaCubes g;
+  int64_t ncube = 0;
+  SB_REQUIRE(cubes_geom(cubes, M, &g, &ncube), SB_ESHAPE, "the cube layout does not cover the %lld tokens",
+             (long long)M);
+  sb::GemmLaunch row{};
+  row.rowadd = y_core;
+  row.ra_T = g.T;
+  row.ra_H = g.H;
+  row.ra_W = g.W;
+  row.ra_ct = g.ct;
+  row.ra_ch = g.ch;
+  row.ra_cw = g.cw;
+  return linear_impl(delta, a4, a8, prec, w, epilogue, out_dtype, Y, M, ws, stream, &row);
 }
 
 sb_status sb_delta_split(const void* X, int64_t M, int64_t K, const sb_cubes* cubes, uint8_t* core_codes,

@@ -107,8 +107,21 @@ struct GemmParams {
   int group_m;    // M-tiles per raster group (tile_coords)
   uint64_t wait_ns;  // limit of the pipeline waits (kWaitNs unless a stall drill is armed)
   int64_t withhold;  // stall drill: the leader's producer skips the loads of this stage (-1: none)
+  // Row addend (delta tokens, k_gemm<true> only): output row t adds the FP32 row ra_row(t) of
+  // rowadd ([cubes][N]) before the activation; rows map to the cubes of a T + F x H x W token grid.
+  const float* rowadd;
+  int64_t ra_T, ra_H, ra_W, ra_nh, ra_nw;
+  int ra_ct, ra_ch, ra_cw;
   WsHeader* hdr;
 };
+
+// The cube of token t (text tokens first, one cube each; then the grid in (f, h, w) order).
+__device__ __forceinline__ int64_t ra_row(const GemmParams& p, int64_t t) {
+  if (t < p.ra_T) return t;
+  const int64_t q = t - p.ra_T;
+  const int64_t f = q / (p.ra_H * p.ra_W), h = (q / p.ra_W) % p.ra_H, w = q % p.ra_W;
+  return p.ra_T + ((f / p.ra_ct) * p.ra_nh + h / p.ra_ch) * p.ra_nw + w / p.ra_cw;
+}
 
 __device__ __forceinline__ uint32_t idesc_for(int kind, int BM, int BN) {
   const uint32_t n = (uint32_t)(BN >> 3) << 17;
@@ -207,10 +220,16 @@ __device__ __forceinline__ void load_colops(const GemmParams& p, int n, ColOps<K
 // Epilogue arithmetic of 32 accumulator columns of one row, in place: the accumulator words become
 // the FP32 outputs. Dequant scale and bias are one FMA, then the optional GELU; columns go in
 // pairs through FP32x2 arithmetic.
-template <int KIND>
+template <int KIND, bool ROWADD = false>
 __device__ __forceinline__ void epilogue_math(const GemmParams& p, const ColOps<KIND>& o, float sxb, float alpha,
-                                              uint32_t (&r)[32]) {
+                                              uint32_t (&r)[32], const float* rowp = nullptr) {
   const bool has_bias = p.bias != nullptr, gelu = p.epilogue == SB_EPI_GELU_TANH;
+  float4 ra[ROWADD ? 8 : 1];  // the row addend's 32 columns (zero for rows past M)
+  if constexpr (ROWADD) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      ra[i] = rowp ? __ldg(reinterpret_cast<const float4*>(rowp) + i) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
 #pragma unroll
   for (int j = 0; j < 16; ++j) {  // columns 2j, 2j + 1
     const uint4 bq = o.b[j >> 2];
@@ -229,6 +248,10 @@ __device__ __forceinline__ void epilogue_math(const GemmParams& p, const ColOps<
     } else {
       y = make_float2(__uint_as_float(r[2 * j]) + bias.x, __uint_as_float(r[2 * j + 1]) + bias.y);
     }
+    if constexpr (ROWADD) {
+      const float4 q = ra[j >> 1];
+      y = make_float2(y.x + ((j & 1) ? q.z : q.x), y.y + ((j & 1) ? q.w : q.y));
+    }
     if (gelu) y = gelu_tanh2(y);
     r[2 * j] = __float_as_uint(y.x);
     r[2 * j + 1] = __float_as_uint(y.y);
@@ -236,9 +259,9 @@ __device__ __forceinline__ void epilogue_math(const GemmParams& p, const ColOps<
 }
 
 // Direct global stores of one row's 32 columns (FP32 / raw outputs, or bf16 without TMA).
-template <int KIND>
+template <int KIND, bool ROWADD = false>
 __device__ __forceinline__ void store_direct(const GemmParams& p, int m, int n, float sxb, float alpha,
-                                             uint32_t (&r)[32]) {
+                                             uint32_t (&r)[32], const float* rowp = nullptr) {
   if (p.out_dtype == SB_OUT_RAW) {
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint32_t*>(p.Y) + (int64_t)m * p.N + n);
 #pragma unroll
@@ -247,7 +270,7 @@ __device__ __forceinline__ void store_direct(const GemmParams& p, int m, int n, 
   }
   ColOps<KIND> o;
   load_colops<KIND>(p, n, o);
-  epilogue_math<KIND>(p, o, sxb, alpha, r);
+  epilogue_math<KIND, ROWADD>(p, o, sxb, alpha, r, rowp);
   if (p.out_dtype == SB_OUT_F32) {
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.Y) + (int64_t)m * p.N + n);
 #pragma unroll
@@ -312,7 +335,7 @@ __device__ __forceinline__ void store_chunk_tma(const CUtensorMap* ty, const Epi
 // are moved to registers and the buffer released before any arithmetic, so the next tile's MMAs
 // can start. Otherwise (two buffers) 32-column chunks are loaded as they are processed and the
 // buffer is released after the last load.
-template <int KIND, bool DRAIN_ALL>
+template <int KIND, bool DRAIN_ALL, bool ROWADD>
 __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtensorMap* ty, const EpiCtx& e) {
   const int nch = e.BN / 64;  // 32-column chunks per warp: 2 or 4
   const int row = 32 * e.q + e.lane;
@@ -329,6 +352,7 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
     const bool tma = p.tma_store && m_warp < e.M;
     // operands that do not depend on the accumulator are loaded before waiting for it
     const float sxb = (KIND == KIND_I8 && m < e.M) ? __fmul_rn(__ldg(p.sA8 + m), p.invB) : 0.0f;
+    const float* rrow = (ROWADD && m < e.M) ? p.rowadd + ra_row(p, m) * (int64_t)e.N : nullptr;
     ColOps<KIND> ops;
     if constexpr (DRAIN_ALL) {
       // the warp's bias slice (128 columns, 256 bytes) goes to shared memory asynchronously
@@ -364,10 +388,10 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
 #pragma unroll
               for (int i = 0; i < 4; ++i) ops.b[i] = ld_shared_v4(e.bias_s + 64u * c + 16u * i);
             }
-            epilogue_math<KIND>(p, ops, sxb, e.alpha, r[c]);
+            epilogue_math<KIND, ROWADD>(p, ops, sxb, e.alpha, r[c], rrow ? rrow + n : nullptr);
             store_chunk_tma(ty, e, r[c], n, m_warp, oc);
           } else if (m < e.M) {
-            store_direct<KIND>(p, m, n, sxb, e.alpha, r[c]);
+            store_direct<KIND, ROWADD>(p, m, n, sxb, e.alpha, r[c], rrow ? rrow + n : nullptr);
           }
         }
       }
@@ -388,11 +412,11 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
             if (tma) {
               ColOps<KIND> next;
               if (c + 1 < nch && n + 32 < e.N) load_colops<KIND>(p, n + 32, next);
-              epilogue_math<KIND>(p, ops, sxb, e.alpha, r);
+              epilogue_math<KIND, ROWADD>(p, ops, sxb, e.alpha, r, rrow ? rrow + n : nullptr);
               store_chunk_tma(ty, e, r, n, m_warp, oc);
               ops = next;
             } else if (m < e.M) {
-              store_direct<KIND>(p, m, n, sxb, e.alpha, r);
+              store_direct<KIND, ROWADD>(p, m, n, sxb, e.alpha, r, rrow ? rrow + n : nullptr);
             }
           }
         }
@@ -506,6 +530,9 @@ __device__ __noinline__ bool issue_all(const Issuer c) {
   return true;
 }
 
+// ROWADD: the delta-token form, whose epilogue adds each output row's cube row of p.rowadd (a
+// separate instantiation, so the plain kernel's code and registers do not change).
+template <bool ROWADD>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ TMaps tm, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -706,12 +733,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     e.out_box = smem_u32(smem + kOutOff) + (uint32_t)(2 * (warp - kEpiWarp0) * kOutBox);
     e.bias_s = smem_u32(smem + kBiasOffF) + 256u * (uint32_t)(warp - kEpiWarp0);
     e.alpha = fp4 ? __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB) : 1.0f;
-    if (fp4)
-      epilogue_loop<KIND_FP4, true>(p, &tm.y, e);
-    else if (kind == KIND_I8)
-      epilogue_loop<KIND_I8, false>(p, &tm.y, e);
-    else
-      epilogue_loop<KIND_BF16, false>(p, &tm.y, e);
+    if (fp4) {
+      // with two accumulators the row-addend form streams its chunks (one chunk of accumulators
+      // and addends live at a time); the plain form drains every column first
+      if (ROWADD && nacc == 2)
+        epilogue_loop<KIND_FP4, false, ROWADD>(p, &tm.y, e);
+      else
+        epilogue_loop<KIND_FP4, true, ROWADD>(p, &tm.y, e);
+    } else if (kind == KIND_I8) {
+      epilogue_loop<KIND_I8, false, ROWADD>(p, &tm.y, e);
+    } else {
+      epilogue_loop<KIND_BF16, false, ROWADD>(p, &tm.y, e);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -778,28 +811,37 @@ void arm_gemm_stall_drill(int64_t withhold_stage, uint64_t wait_ns) {
   g_drill_withhold.store(withhold_stage);
 }
 
-cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
+// Shared-memory attribute and register-split check of one k_gemm instantiation.
+template <bool ROWADD>
+static cudaError_t gemm_ready(const char** why) {
   static std::atomic<uint64_t> attr{0};  // one bit per device
-  const cudaError_t attr_err = smem_attr_once(k_gemm, kSmemBytes, attr);
+  const cudaError_t attr_err = smem_attr_once(k_gemm<ROWADD>, kSmemBytes, attr);
   if (attr_err != cudaSuccess) {
     *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
     return attr_err;
   }
   // The register split of the kernel must fit what a CTA is launched with, or the epilogue's
   // setmaxnreg.inc would wait for registers that never come free.
-  static int regs = -1;
-  if (regs < 0) {
+  static std::atomic<int> regs{-1};
+  if (regs.load() < 0) {
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, k_gemm) != cudaSuccess) {
+    if (cudaFuncGetAttributes(&fa, k_gemm<ROWADD>) != cudaSuccess) {
       *why = "cudaFuncGetAttributes(k_gemm) failed";
       return cudaErrorInvalidValue;
     }
-    regs = fa.numRegs;
+    regs.store(fa.numRegs);
   }
-  if (regs * kThreads < kRegsNeeded) {
+  if (regs.load() * kThreads < kRegsNeeded) {
     *why = "k_gemm was compiled with fewer registers per thread than its warpgroup split needs";
     return cudaErrorInvalidConfiguration;
   }
+  return cudaSuccess;
+}
+
+cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
+  const bool rowadd = L.rowadd != nullptr;
+  const cudaError_t ready = rowadd ? gemm_ready<true>(why) : gemm_ready<false>(why);
+  if (ready != cudaSuccess) return ready;
   TMaps tm;
   memset(&tm, 0, sizeof(tm));
   GemmParams p;
@@ -827,6 +869,17 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   p.out_dtype = L.out_dtype;
   p.epilogue = L.epilogue;
   p.hdr = reinterpret_cast<WsHeader*>(L.hdr);
+  p.rowadd = L.rowadd;
+  if (rowadd) {
+    p.ra_T = L.ra_T;
+    p.ra_H = L.ra_H;
+    p.ra_W = L.ra_W;
+    p.ra_ct = L.ra_ct;
+    p.ra_ch = L.ra_ch;
+    p.ra_cw = L.ra_cw;
+    p.ra_nh = ceil_div(L.ra_H, L.ra_ch > 0 ? L.ra_ch : 1);
+    p.ra_nw = ceil_div(L.ra_W, L.ra_cw > 0 ? L.ra_cw : 1);
+  }
   p.withhold = g_drill_withhold.exchange(-1);
   const uint64_t drill_ns = g_drill_wait_ns.exchange(0);
   p.wait_ns = (p.withhold >= 0 && drill_ns != 0) ? drill_ns : kWaitNs;
@@ -873,7 +926,10 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   const int sms = device_sms() & ~1;
   const unsigned grid = (unsigned)(want < sms ? want : sms);
   p.group_m = pick_group_m(ceil_div(L.M, 256), ceil_div(L.N, bn_q), grid / 2);
-  k_gemm<<<grid, kThreads, kSmemBytes, s>>>(tm, p);
+  if (rowadd)
+    k_gemm<true><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
+  else
+    k_gemm<false><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
   return cudaGetLastError();
 }
 

@@ -92,6 +92,10 @@ struct GemmLaunch {
   int out_dtype;
   void* Y;
   void* hdr;
+  // delta tokens: output row t adds row cube(t) of rowadd (FP32 [cubes][N]) before the activation
+  const float* rowadd;
+  int64_t ra_T, ra_H, ra_W;
+  int ra_ct, ra_ch, ra_cw;
 };
 
 cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s);

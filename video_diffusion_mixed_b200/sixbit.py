@@ -100,6 +100,7 @@ def lib():
             "sb_drill_gemm_stall": (st, [i64, ctypes.c_uint64]),
             "sb_tdc_refresh_fp8": (st, [vp, vp, vp, vp, i64, i64, vp, vp]),
             "sb_module_record": (st, [vp, vp, vp, i64, i64, vp, i32, vp, vp, vp, vp]),
+            "sb_delta_linear": (st, [vp, P(Fp4), P(I8), vp, P(WeightC), vp, P(Cubes), i32, i32, vp, i64, vp, vp]),
             "sb_tdc_reuse_fp8": (st, [vp, vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_refresh": (st, [vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_reuse": (st, [vp, vp, vp, i64, i64, vp, vp]),
@@ -129,7 +130,7 @@ EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_in
             "sb_tdc_reuse", "sb_group_slots_bytes", "sb_prepass_partial", "sb_prepass_finish", "sb_nvfp4_encode",
             "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide", "sb_prepass_chunks", "sb_cube_count",
             "sb_delta_split", "sb_delta_combine", "sb_drill_gemm_stall", "sb_tdc_refresh_fp8",
-            "sb_tdc_reuse_fp8", "sb_module_record")
+            "sb_tdc_reuse_fp8", "sb_module_record", "sb_delta_linear")
 
 
 def _ck(status: int):
@@ -446,6 +447,16 @@ def delta_split(X, c: Cubes, core: CoreTokens, delta, stream=None):
     M, K = X.shape
     _ck(lib().sb_delta_split(_p(X), M, K, ctypes.byref(c), _p(core.codes), _p(core.scale), _p(core.bf16), _p(delta),
                              _stream(stream)))
+
+
+def delta_linear(delta, a4, a8, prec, w: "Weight", y_core, c: Cubes, Y, epilogue: int = EPI_NONE,
+                 out_dtype: int = OUT_BF16, ws: "Workspace" = None, stream=None):
+    """Y = act(linear(delta) + y_core[cube(t)]) with the combine in the GEMM epilogue (sb_delta_linear)."""
+    M = Y.shape[0]
+    c4 = ctypes.byref(a4.c()) if a4 is not None else None
+    c8 = ctypes.byref(a8.c()) if a8 is not None else None
+    _ck(lib().sb_delta_linear(_p(delta), c4, c8, _p(prec), ctypes.byref(w.c()), _p(y_core), ctypes.byref(c), epilogue,
+                              out_dtype, _p(Y), M, ws.ptr, _stream(stream)))
 
 
 def delta_combine(y_delta, y_core, c: Cubes, Y, epilogue: int = EPI_NONE, stream=None):
