@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT shapes"
 
 # ncu DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum, one capture of the
-# step's 18 launches at full size, 17776 tokens; ncu flushes the caches before each launch, so
+# step's 16 launches at full size, 17776 tokens; ncu flushes the caches before each launch, so
 # these are cold-cache figures) of the kernels that can be the dominant one, summarised under
 # profiles/, for the ffn5b workload at full size only. An entry is valid only for the sources it
 # was measured on (sha over the listed files of csrc/).
@@ -776,7 +776,7 @@ def run_ours(args):
                    "tokens": M, "hidden": K1, "ffn": N1, "hadamard_block": 128, "parallelism": f"replicas x{world}",
                    "l2": "flushed before every step (512 MiB memset, then a 256 MiB read that leaves L2 clean; "
                          "outside the per-step events)",
-                   "launch": "each step replays one CUDA graph of its 18 kernels"},
+                   "launch": f"each step replays one CUDA graph of its {2 * LAUNCHES_PER_PASS} kernels"},
         "roofline": roofline,
         "roofline_prepass": {r["kernel"]: {"achieved_gbs": round(r["achieved"], 1), "frac": round(r["frac"], 4),
                                            "ms": round(r["ms"], 4), "traffic": traffic_of(r["kernel"])} for r in pre},
