@@ -177,7 +177,8 @@ def _fused_delta_linear(sbg, X, c, W, bias, gelu, prec, out_dtype):
 # N = 768 and 1920: 128- and 192-wide tiles (two accumulators, chunked epilogue); 3072: 256-wide
 # NVFP4 tiles (one accumulator, the epilogue drains every column first); BF16: the raw delta tokens
 @pytest.mark.parametrize("N,gelu,prec", [(768, False, 0), (768, True, 0), (1920, True, 0), (3072, False, 0),
-                                         (1920, False, 2)], ids=["768", "768_gelu", "1920_gelu", "3072", "1920_bf16"])
+                                         (1920, False, 1), (1920, False, 2)],
+                         ids=["768", "768_gelu", "1920_gelu", "3072", "1920_int8", "1920_bf16"])
 def test_fused_delta_linear_against_oracle(sbg, N, gelu, prec):
     text, F, H, W_, cube = 7, 4, 6, 10, (2, 2, 2)
     M, K = text + F * H * W_, 1920
@@ -194,6 +195,11 @@ def test_fused_delta_linear_against_oracle(sbg, N, gelu, prec):
         c4, sfl, _, sg = oracle.quant_nvfp4(dp["y"], dp["amax_rot"])
         wp = oracle.prepare_weight(u16(Wt), 128)
         yd_ref = oracle.gemm_nvfp4(c4, sfl, sg, wp["c4"], wp["sf4"], wp["sg4"], None, K, 128)
+    elif prec == 1:
+        dp = oracle.prepass(dref, None, 128)
+        q8, s8 = oracle.quant_int8(dp["y"], dp["row_amax"])
+        wp = oracle.prepare_weight(u16(Wt), 128)
+        yd_ref = oracle.gemm_int8(q8, s8, wp["q8"], wp["s8"], None, 128)
     else:
         yd_ref = oracle.gemm_bf16(dref, u16(Wt), None)
     ref = oracle.delta_linear(yd_ref, dec, u16(Wt), u16(bias), M, g, gelu=gelu)
