@@ -41,9 +41,11 @@ def two_steps(sb, M, C, fused, prec_value=0, update=True):
     return x, ys, out
 
 
-# (1, 64) one segment; 1920 and 3072 two- and four-segment rows of warp teams; 12288 the widest
-# team; 70001 rows more than 4096 groups, so the last CTA folds the group sums in chunks
-@pytest.mark.parametrize("M,C", [(1, 64), (33, 1920), (256, 3072), (17776, 3072), (100, 12288), (70001, 64)])
+# Row tilings (warps per row x 1024-element segments per warp): (1, 64) 1 x 1; 1920 1 x 2;
+# 3072 1 x 3; 4096 2 x 2; 6144 2 x 3; 8192 4 x 2; 12288 4 x 3; 16384 8 x 2. 70001 rows: more than
+# 4096 groups, so the last CTA folds the group sums in chunks.
+@pytest.mark.parametrize("M,C", [(1, 64), (33, 1920), (256, 3072), (17776, 3072), (64, 4096), (48, 6144), (16, 8192),
+                                 (100, 12288), (24, 16384), (70001, 64)])
 def test_module_record_equals_the_two_calls(sbg, M, C):
     x, ys, sep = two_steps(sbg, M, C, fused=False)
     _, _, fus = two_steps(sbg, M, C, fused=True)
