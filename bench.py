@@ -437,6 +437,30 @@ class DeltaTokensLayer:
         self._mark(ev, "d4")
 
 
+def delta_accuracy(torch, sb, synth, L):
+    """Output error of the 4-bit linear with and without delta tokens against the BF16 linear (our
+    BF16 GEMM, FP32 output), relative Frobenius, on the timed input (independent tokens with outlier
+    channels) and on tokens with a video latent's local redundancy (synth.smooth_video_tokens)."""
+    out = {}
+    f32 = lambda: torch.empty((L.M, L.N), dtype=torch.float32, device=L.X.device)
+    Yref, Yp, Yd = f32(), f32(), f32()
+    inputs = {"independent_tokens": L.X,
+              "smooth_video_tokens": synth.smooth_video_tokens(226, 13, 30, 45, L.K, seed=8, device=L.X.device)}
+    for name, X in inputs.items():
+        sb.linear(X, None, None, L.pb, L.w_b, Yref, out_dtype=sb.OUT_F32, ws=L.ws)
+        sb.prepass(X, None, L.cfg, sb.PREPASS_QUANT, L.p4, L.a4, L.a8, L.st, L.ws)
+        sb.linear(X, L.a4, L.a8, L.p4, L.w_b, Yp, out_dtype=sb.OUT_F32, ws=L.ws)
+        sb.delta_split(X, L.c, L.core, L.delta)
+        sb.prepass(L.delta, None, L.cfg, sb.PREPASS_QUANT, L.p4, L.a4, L.a8, L.st, L.ws)
+        sb.linear(L.core.bf16, None, None, L.pb, L.w_nb, L.Yc, out_dtype=sb.OUT_F32, ws=L.ws)
+        sb.delta_linear(L.delta, L.a4, L.a8, L.p4, L.w_b, L.Yc, L.c, Yd, out_dtype=sb.OUT_F32, ws=L.ws)
+        sb.check(L.ws)
+        nref = float(torch.linalg.vector_norm(Yref.double()))
+        out[name] = {"rel_err_nvfp4": round(float(torch.linalg.vector_norm((Yp - Yref).double())) / nref, 5),
+                     "rel_err_delta_tokens": round(float(torch.linalg.vector_norm((Yd - Yref).double())) / nref, 5)}
+    return out
+
+
 def run_delta_tokens(torch, sb, synth, flush, device, reps=10):
     L = DeltaTokensLayer(sb, torch, synth, device)
     spans = {"plain_prepass": ("p0", "p1"), "plain_gemm_nvfp4": ("p1", "p2"), "split": ("d0", "d1"),
@@ -468,7 +492,8 @@ def run_delta_tokens(torch, sb, synth, flush, device, reps=10):
                     "4-bit deltas), one graph of both, L2 flushed before each replay",
             "cubes": L.core.n, "ms": ms, "ms_plain": round(plain, 4), "ms_delta_tokens": round(dq, 4),
             "tflops_plain": round(flops / (plain * 1e-3) / 1e12, 1),
-            "tflops_delta_tokens": round(flops / (dq * 1e-3) / 1e12, 1)}
+            "tflops_delta_tokens": round(flops / (dq * 1e-3) / 1e12, 1),
+            "accuracy_vs_bf16": delta_accuracy(torch, sb, synth, L)}
 
 
 def run_residual_cache(torch, sb, S, flush, reps=10):

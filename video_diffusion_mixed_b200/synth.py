@@ -101,6 +101,29 @@ WORKLOADS = {
 }
 
 
+def smooth_video_tokens(text: int, F: int, H: int, W: int, K: int, *, noise: float = 0.1, waves: int = 4,
+                        seed: int = 0, tensor_id: int = 500, device="cpu") -> torch.Tensor:
+    """Tokens with the local redundancy of a video latent, bf16 [text + F H W, K]: `text` tokens
+    N(0, 1), then the F x H x W grid in (f, h, w) order, each channel a sum of `waves` sinusoids of
+    low frequency (up to one period along each axis, random phase), scaled to unit variance, plus
+    N(0, noise^2): neighbouring grid tokens differ by a small fraction of their magnitude."""
+    g = _gen(device, sub_seed(seed, tensor_id))
+    n = F * H * W
+    f = torch.arange(F, device=device, dtype=torch.float32).repeat_interleave(H * W) / F
+    h = torch.arange(H, device=device, dtype=torch.float32).repeat_interleave(W).repeat(F) / H
+    w = torch.arange(W, device=device, dtype=torch.float32).repeat(F * H) / W
+    coords = torch.stack([f, h, w], dim=1)  # [n, 3]
+    field = torch.zeros((n, K), device=device, dtype=torch.float32)
+    for _ in range(waves):
+        freq = torch.rand((3, K), generator=g, device=device)  # up to one period along each axis
+        phase = torch.rand((1, K), generator=g, device=device) * (2 * math.pi)
+        field += torch.cos(2 * math.pi * (coords @ freq) + phase)
+    field *= math.sqrt(2.0 / waves)
+    field += noise * torch.randn((n, K), generator=g, device=device)
+    txt = torch.randn((text, K), generator=g, device=device)
+    return torch.cat([txt, field], dim=0).to(torch.bfloat16)
+
+
 def workload_inputs(name: str, *, seed: int = 0, device="cpu", tokens: int | None = None, bias_std: float = 0.0):
     """Activations, weights and biases of one named workload."""
     w = WORKLOADS[name]
