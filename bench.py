@@ -708,6 +708,17 @@ def run_ours(args):
     # beside the headline step (not part of it)
     bf16_ms = graph_kernel_times(torch, S, flush, reps, (sb.BF16,))
     sb.check(S.ws)
+    # ---- what the quantized passes cost in accuracy: the module output of each pass against the
+    # BF16 pass on the same input (relative Frobenius; bf16 outputs)
+    outs = {}
+    for prec in (sb.BF16, sb.NVFP4, sb.INT8):
+        S.one_pass(prec)
+        outs[prec] = S.Y.double()
+    sb.check(S.ws)
+    ref_norm = float(torch.linalg.vector_norm(outs[sb.BF16]))
+    accuracy = {sb.PREC_NAMES[p]: round(float(torch.linalg.vector_norm(outs[p] - outs[sb.BF16])) / ref_norm, 5)
+                for p in (sb.NVFP4, sb.INT8)}
+    del outs
 
     # ---- the token-sharded step (the tensor's rows split over the ranks; statistics gathered)
     sharded = None
@@ -813,6 +824,8 @@ def run_ours(args):
         "sharded": sharded,
         "delta_tokens": delta_tok,
         "residual_cache": resid,
+        "accuracy_vs_bf16": {"what": "relative Frobenius error of the module output of each pass against the "
+                                     "BF16 pass on the same input (block Hadamard B = 128, bf16 outputs)", **accuracy},
         "bf16_pass": {"what": "the same module with every layer forced to the BF16 fallback (the Purified Delta "
                               "Refresh path), timed like the kernels above; not part of the headline step",
                       "ms": round(sum(bf16_ms.values()), 4),
