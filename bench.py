@@ -718,6 +718,24 @@ def run_ours(args):
     ref_norm = float(torch.linalg.vector_norm(outs[sb.BF16]))
     accuracy = {sb.PREC_NAMES[p]: round(float(torch.linalg.vector_norm(outs[p] - outs[sb.BF16])) / ref_norm, 5)
                 for p in (sb.NVFP4, sb.INT8)}
+    # the same passes with weights and activations rotated by smaller or larger Hadamard blocks
+    by_block = {"nvfp4": {}, "int8": {}}
+    for B in (16, 64, 128, 256):
+        w1 = sb.Weight(S.w1.W, S.w1.bias, B, S.ws)
+        w2 = sb.Weight(S.w2.W, S.w2.bias, B, S.ws)
+        for prec in (sb.NVFP4, sb.INT8):
+            cfg = sb.config(rho=64.0, tdc_thresh=-1.0, block=B, force_prec=prec)  # no PDR switch
+            S.p1.fill_(prec)
+            S.p2.fill_(prec)
+            sb.prepass(S.X, None, cfg, sb.PREPASS_QUANT, S.p1, S.ax4, S.ax8, S.sx, S.ws)
+            sb.linear(S.X, S.ax4, S.ax8, S.p1, w1, S.H, epilogue=sb.EPI_GELU, ws=S.ws)
+            sb.prepass(S.H, None, cfg, sb.PREPASS_QUANT, S.p2, S.ah4, S.ah8, S.sh, S.ws)
+            sb.linear(S.H, S.ah4, S.ah8, S.p2, w2, S.Y, ws=S.ws)
+            sb.check(S.ws)
+            by_block[sb.PREC_NAMES[prec]][B] = round(
+                float(torch.linalg.vector_norm(S.Y.double() - outs[sb.BF16])) / ref_norm, 5)
+        del w1, w2
+    accuracy["by_hadamard_block"] = by_block
     del outs
 
     # ---- the token-sharded step (the tensor's rows split over the ranks; statistics gathered)
