@@ -150,8 +150,11 @@ def whole_job_tflops(world, flops_per_rank_step, ms_per_step):
 class FfnStep:
     """All buffers of one FFN module step, allocated once (the library allocates nothing)."""
 
-    def __init__(self, sb, synth, torch, wl, seed, device, tokens=None):
+    def __init__(self, sb, synth, torch, wl, seed, device, tokens=None, records_for=()):
         self.sb, self.torch = sb, torch
+        # precisions whose W1 GEMM also writes the hidden tensor's chunk records, which then stand
+        # in for the hidden tensor's statistics pass (FFN-pair fusion)
+        self.records_for = tuple(records_for)
         X, layers = synth.workload_inputs(wl, seed=seed, device=device, bias_std=0.0, tokens=tokens)
         self.X = X
         self.M, self.C = X.shape
@@ -162,6 +165,8 @@ class FfnStep:
         self.ax4, self.ax8 = sb.Fp4Tensor(self.M, self.K1), sb.I8Tensor(self.M, self.K1)
         self.ah4, self.ah8 = sb.Fp4Tensor(self.M, self.K2), sb.I8Tensor(self.M, self.K2)
         self.H = torch.empty((self.M, self.N1), dtype=torch.bfloat16, device=device)
+        self.hrec = (torch.empty((self.M, self.N1 // 128, 4), dtype=torch.float32, device=device)
+                     if self.records_for else None)
         self.Y = torch.empty((self.M, self.N2), dtype=torch.bfloat16, device=device)
         self.cache = torch.zeros_like(self.Y)
         self.state = sb.alloc_state()
@@ -184,10 +189,18 @@ class FfnStep:
         self._mark(ev, "pre1_0")
         sb.prepass(X, None, cfg, sb.PREPASS_QUANT, self.p1, self.ax4, self.ax8, self.sx, self.ws)
         self._mark(ev, "pre1_1")
-        sb.linear(X, self.ax4, self.ax8, self.p1, self.w1, self.H, epilogue=sb.EPI_GELU, ws=self.ws)
+        fused = prec in self.records_for
+        if fused:
+            sb.linear_records(X, self.ax4, self.ax8, self.p1, self.w1, self.H, self.hrec, epilogue=sb.EPI_GELU,
+                              block=128, ws=self.ws)
+        else:
+            sb.linear(X, self.ax4, self.ax8, self.p1, self.w1, self.H, epilogue=sb.EPI_GELU, ws=self.ws)
         self._mark(ev, "gemm1_1")
         self._mark(ev, "pre2_0")
-        sb.prepass(self.H, None, cfg, sb.PREPASS_QUANT, self.p2, self.ah4, self.ah8, self.sh, self.ws)
+        if fused:
+            sb.prepass_chunks(self.H, self.hrec, cfg, sb.PREPASS_QUANT, self.p2, self.ah4, self.ah8, self.sh, self.ws)
+        else:
+            sb.prepass(self.H, None, cfg, sb.PREPASS_QUANT, self.p2, self.ah4, self.ah8, self.sh, self.ws)
         self._mark(ev, "pre2_1")
         sb.linear(self.H, self.ah4, self.ah8, self.p2, self.w2, Y, ws=self.ws)
         self._mark(ev, "gemm2_1")
@@ -212,6 +225,7 @@ class FfnStep:
 
 
 LAUNCHES_PER_PASS = 8  # decide, prepass(2), gemm, prepass(2), gemm, module record
+# with the hidden tensor's chunk records, its pre-pass is 3 launches: fold, INT8 codes, NVFP4 encode
 
 
 class L2Flush:
@@ -663,7 +677,9 @@ def run_ours(args):
     from video_diffusion_mixed_b200 import sixbit as sb
     from video_diffusion_mixed_b200 import synth
 
-    S = FfnStep(sb, synth, torch, args.workload, seed=rank, device=device, tokens=args.tokens)
+    records_for = {"none": (), "nvfp4": (sb.NVFP4,), "both": (sb.NVFP4, sb.INT8)}[args.ffn_records]
+    S = FfnStep(sb, synth, torch, args.workload, seed=rank, device=device, tokens=args.tokens,
+                records_for=records_for)
     flush = L2Flush(torch, device)
 
     def barrier():
@@ -821,6 +837,7 @@ def run_ours(args):
                 if dom["bound"] == "tensor"
                 else f"{pk['src']} HBM copy"}
     pre = [r for r in rows if r["kernel"].startswith("prepass")]
+    launches_per_step = 2 * LAUNCHES_PER_PASS + len(S.records_for)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -830,7 +847,8 @@ def run_ours(args):
                    "tokens": M, "hidden": K1, "ffn": N1, "hadamard_block": 128, "parallelism": f"replicas x{world}",
                    "l2": "flushed before every step (512 MiB memset, then a 256 MiB read that leaves L2 clean; "
                          "outside the per-step events)",
-                   "launch": f"each step replays one CUDA graph of its {2 * LAUNCHES_PER_PASS} kernels"},
+                   "ffn_records": args.ffn_records,
+                   "launch": f"each step replays one CUDA graph of its {launches_per_step} kernels"},
         "roofline": roofline,
         "roofline_prepass": {r["kernel"]: {"achieved_gbs": round(r["achieved"], 1), "frac": round(r["frac"], 4),
                                            "ms": round(r["ms"], 4), "traffic": traffic_of(r["kernel"])} for r in pre},
@@ -854,7 +872,7 @@ def run_ours(args):
                           "the module state"},
         "e2e_with_outputs": {"value": round(e2eo_value, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                              "d2h_bytes_per_step": d2ho, "result": "also both passes' output tensors"},
-        "gpu_launches": LAUNCHES_PER_PASS * 2 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "wall_s_timed": round(t_wall, 3),
     }
@@ -981,6 +999,8 @@ def main(argv=None):
                     help="tokens in the cpu_baseline sample of our arm (about 10 s on 16 cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-delta-tokens", action="store_true", help="skip the delta-token layer timing")
+    ap.add_argument("--ffn-records", default="none", choices=["none", "nvfp4", "both"],
+                    help="passes whose W1 GEMM writes the hidden tensor's chunk records for its pre-pass")
     ap.add_argument("--shard", default="none", choices=["none", "tokens"],
                     help="also time the token-sharded step (under torchrun: the rows of every tensor split "
                          "over the ranks, statistics gathered with NCCL)")

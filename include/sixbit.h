@@ -212,6 +212,25 @@ sb_status sb_prepass_chunks(const void* X, float* chunks, int64_t M, int64_t K,
                             const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */, sb_stats* stats,
                             void* ws, sb_stream stream);
 
+/* The producer of those records (FFN-pair fusion, "write-up" section 四): sb_linear with bf16
+ * output Y [M][N] that also writes, from its epilogue, the chunk records of Y as it stores it
+ * (float4 [M][N/128]; x = max |H_B y| over the chunk, y = the canonical pairwise sum of |y|,
+ * z = max |y|, w = 0), for a next pre-pass whose cfg->block is `block`, which must be 128 here
+ * (SB_EUNSUPPORTED otherwise; sb_chunk_records covers the smaller blocks). The records describe
+ * the bf16 values Y holds, whatever precision *prec
+ * selects; under SB_SKIP neither Y nor the records are written. records: 16-byte aligned device
+ * memory (SB_EALIGN), owned by the caller; requires N % 256 == 0 (SB_EUNSUPPORTED), else as
+ * sb_linear (whose out_dtype is SB_OUT_BF16 here). */
+sb_status sb_linear_records(const void* X, const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */,
+                            const int32_t* prec, const sb_weight* w /* host */, int32_t epilogue, void* Y,
+                            int64_t M, int32_t block, float* records, void* ws, sb_stream stream);
+
+/* The same chunk records computed from a bf16 tensor X [M][K] in device memory (K % 128 == 0,
+ * K <= 16384, block in {16, 32, 64, 128}, else SB_EUNSUPPORTED; M >= 1, else SB_ESHAPE; X and
+ * records 16-byte aligned, else SB_EALIGN), with the arithmetic of sb_linear_records' epilogue:
+ * a stand-alone producer for tensors that no GEMM of this library wrote. */
+sb_status sb_chunk_records(const void* X, int64_t M, int64_t K, int32_t block, float* records, sb_stream stream);
+
 /* Quantized linear layer Y = X W^T + bias ("write-up" section 四; tcgen05 tensor cores):
  *   NVFP4: Y = acc * s_gx * s_gw / B + bias, acc = sum of block-scaled E2M1 products
  *          (tcgen05.mma kind::mxf4nvf4, UE4M3 scales per 16);

@@ -258,3 +258,23 @@ def test_delta_token_validation_without_gpu(sb):
                              None) == sb.SB_EINVAL  # raw accumulators are not an output of this form
     assert L.sb_delta_linear(delta, None, None, p, ctypes.byref(w), Yc, ctypes.byref(c), 0, 0, Y, M - 1, ws,
                              None) == sb.SB_ESHAPE
+
+
+def test_chunk_record_validation_without_gpu(sb):
+    L = sb.lib()
+    X, rec, Y, p, ws = _fake(0x10000), _fake(0x20000), _fake(0x30000), _fake(0x100), _fake(0x300)
+    assert L.sb_chunk_records(None, 4, 256, 128, rec, None) == sb.SB_EINVAL
+    assert L.sb_chunk_records(X, 4, 256, 128, _fake(0x20008), None) == sb.SB_EALIGN
+    assert L.sb_chunk_records(X, 0, 256, 128, rec, None) == sb.SB_ESHAPE
+    assert L.sb_chunk_records(X, 4, 320, 128, rec, None) == sb.SB_EUNSUPPORTED
+    assert L.sb_chunk_records(X, 4, 256, 256, rec, None) == sb.SB_EUNSUPPORTED
+    assert L.sb_chunk_records(X, 4, 256, 8, rec, None) == sb.SB_EUNSUPPORTED
+    w = sb.WeightC()
+    w.N, w.K, w.block = 512, 256, 128
+    assert L.sb_linear_records(X, None, None, p, ctypes.byref(w), 0, Y, 4, 128, None, ws, None) == sb.SB_EINVAL
+    assert L.sb_linear_records(X, None, None, p, ctypes.byref(w), 0, Y, 4, 128, _fake(0x20004), ws,
+                               None) == sb.SB_EALIGN
+    assert L.sb_linear_records(X, None, None, p, ctypes.byref(w), 0, Y, 4, 64, rec, ws, None) == sb.SB_EUNSUPPORTED
+    w.N = 384  # records need 256-wide output tiles
+    assert L.sb_linear_records(X, None, None, p, ctypes.byref(w), 0, Y, 4, 128, rec, ws, None) == sb.SB_EUNSUPPORTED
+    assert "256" in L.sb_last_error().decode()

@@ -401,6 +401,7 @@ static sb_status linear_impl(const void* X, const sb_fp4* a4, const sb_i8* a8, c
   L.Y = Y;
   L.hdr = ws;
   if (row) {
+    L.records = row->records;
     L.rowadd = row->rowadd;
     L.ra_T = row->ra_T;
     L.ra_H = row->ra_H;
@@ -418,6 +419,32 @@ static sb_status linear_impl(const void* X, const sb_fp4* a4, const sb_i8* a8, c
 sb_status sb_linear(const void* X, const sb_fp4* a4, const sb_i8* a8, const int32_t* prec, const sb_weight* w,
                     int32_t epilogue, int32_t out_dtype, void* Y, int64_t M, void* ws, sb_stream stream) {
   return linear_impl(X, a4, a8, prec, w, epilogue, out_dtype, Y, M, ws, stream, nullptr);
+}
+
+sb_status sb_linear_records(const void* X, const sb_fp4* a4, const sb_i8* a8, const int32_t* prec,
+                            const sb_weight* w, int32_t epilogue, void* Y, int64_t M, int32_t block, float* records,
+                            void* ws, sb_stream stream) {
+  SB_REQUIRE(records && w, SB_EINVAL, "records and w are required");
+  SB_ALIGNED(records, "records");
+  SB_REQUIRE(block == 128, SB_EUNSUPPORTED, "the GEMM's chunk records are for block 128 (got %d)", (int)block);
+  SB_REQUIRE(w->N % 256 == 0, SB_EUNSUPPORTED, "chunk records need N a multiple of 256 (got %lld)", (long long)w->N);
+  sb::GemmLaunch rec{};
+  rec.records = records;
+  return linear_impl(X, a4, a8, prec, w, epilogue, SB_OUT_BF16, Y, M, ws, stream, &rec);
+}
+
+sb_status sb_chunk_records(const void* X, int64_t M, int64_t K, int32_t block, float* records, sb_stream stream) {
+  SB_REQUIRE(X && records, SB_EINVAL, "X and records are required");
+  SB_ALIGNED(X, "X");
+  SB_ALIGNED(records, "records");
+  SB_REQUIRE(M >= 1 && M <= (int64_t)1 << 30, SB_ESHAPE, "M out of range (%lld)", (long long)M);
+  SB_REQUIRE(K >= 128 && K % 128 == 0 && K <= sb::kMaxK, SB_EUNSUPPORTED, "K must be a multiple of 128 in [128, %d]",
+             sb::kMaxK);
+  SB_REQUIRE(block == 16 || block == 32 || block == 64 || block == 128, SB_EUNSUPPORTED,
+             "chunk records need block in {16, 32, 64, 128} (got %d)", (int)block);
+  cudaError_t e = sb::launch_chunk_records(X, M, K, block, records, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "k_chunk_records launch");
+  return ok();
 }
 
 sb_status sb_tdc_record(const void* y_new, void* y_cache, int64_t M, int64_t C, const sb_stats* d_src,

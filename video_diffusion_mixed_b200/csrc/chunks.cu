@@ -201,4 +201,36 @@ cudaError_t launch_prepass_chunks(const PrepassLaunch& p, float* chunks, cudaStr
   }
 }
 
+// Chunk records of a bf16 tensor [M][K] (K % 128 == 0) with the same arithmetic the GEMM's
+// record epilogue uses: one thread per (row, 128-channel chunk).
+__global__ void __launch_bounds__(128) k_chunk_records(const __nv_bfloat16* X, int64_t M, int K, int B,
+                                                        float4* out) {
+  const int nc = K / 128;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M * nc) return;
+  const int64_t m = i / nc;
+  const int c = (int)(i - m * nc);
+  const uint4* src = reinterpret_cast<const uint4*>(X + m * K + 128 * c);
+  uint32_t v[4][32];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const uint4 w = src[q];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int k = 8 * q + 2 * t;
+      v[k >> 5][k & 31] = ws[t] << 16;
+      v[(k + 1) >> 5][(k + 1) & 31] = ws[t] & 0xffff0000u;
+    }
+  }
+  out[i] = chunk_record(v, B);
+}
+
+cudaError_t launch_chunk_records(const void* X, int64_t M, int64_t K, int B, float* out, cudaStream_t s) {
+  const int64_t n = M * (K / 128);
+  k_chunk_records<<<(unsigned)ceil_div(n, 128), 128, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(X), M, (int)K,
+                                                             B, reinterpret_cast<float4*>(out));
+  return cudaGetLastError();
+}
+
 }  // namespace sb

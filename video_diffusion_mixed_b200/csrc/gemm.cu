@@ -107,13 +107,21 @@ struct GemmParams {
   int group_m;    // M-tiles per raster group (tile_coords)
   uint64_t wait_ns;  // limit of the pipeline waits (kWaitNs unless a stall drill is armed)
   int64_t withhold;  // stall drill: the leader's producer skips the loads of this stage (-1: none)
-  // Row addend (delta tokens, k_gemm<true> only): output row t adds the FP32 row ra_row(t) of
-  // rowadd ([cubes][N]) before the activation; rows map to the cubes of a T + F x H x W token grid.
+  // Row addend (delta tokens, k_gemm<kEpiRowAdd> only): output row t adds the FP32 row ra_row(t)
+  // of rowadd ([cubes][N]) before the activation; rows map to the cubes of a T + F x H x W grid.
   const float* rowadd;
   int64_t ra_T, ra_H, ra_W, ra_nh, ra_nw;
   int ra_ct, ra_ch, ra_cw;
+  // Chunk records (k_gemm<kEpiRecord> only): per row and aligned 128-column chunk of the bf16
+  // output, {max |H_128 y|, canonical pairwise sum |y|, max |y|, 0}, float4 [M][N / 128].
+  float4* records;
+  int rec_nc;  // chunks per row
   WsHeader* hdr;
 };
+
+// Epilogue forms, one k_gemm instantiation each (the plain one is what every ordinary launch runs).
+enum { kEpiPlain = 0, kEpiRowAdd = 1, kEpiRecord = 2 };
+
 
 // The cube of token t (text tokens first, one cube each; then the grid in (f, h, w) order).
 __device__ __forceinline__ int64_t ra_row(const GemmParams& p, int64_t t) {
@@ -309,7 +317,7 @@ struct EpiCtx {
   int unit, tiles, nunits, m_tiles, n_tiles, group_m, nacc, BN, M, N, row_off, q, half, lane;
   uint64_t wait_ns;
   uint32_t out_box;  // this warp's two staging boxes
-  uint32_t bias_s;   // NVFP4: this warp's bias slice in shared memory
+  uint32_t bias_s;   // NVFP4: this warp's bias slice in shared memory (past the NVFP4 stages)
   float alpha;
 };
 
@@ -331,12 +339,13 @@ __device__ __forceinline__ void store_chunk_tma(const CUtensorMap* ty, const Epi
   ++oc;
 }
 
-// The epilogue of every tile of this CTA. DRAIN_ALL (one accumulator buffer): the warp's columns
-// are moved to registers and the buffer released before any arithmetic, so the next tile's MMAs
-// can start. Otherwise (two buffers) 32-column chunks are loaded as they are processed and the
-// buffer is released after the last load.
-template <int KIND, bool DRAIN_ALL, bool ROWADD>
+// The epilogue of every tile of this CTA. DRAIN_ALL (one accumulator buffer, and the record form
+// in every precision): the warp's columns are moved to registers and the buffer released before
+// any arithmetic, so the next tile's MMAs can start. Otherwise (two buffers) 32-column chunks are
+// loaded as they are processed and the buffer is released after the last load.
+template <int KIND, bool DRAIN_ALL, int EPI>
 __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtensorMap* ty, const EpiCtx& e) {
+  constexpr bool ROWADD = EPI == kEpiRowAdd, RECORD = EPI == kEpiRecord;
   const int nch = e.BN / 64;  // 32-column chunks per warp: 2 or 4
   const int row = 32 * e.q + e.lane;
   uint32_t oc = 0;
@@ -355,8 +364,11 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
     const float* rrow = (ROWADD && m < e.M) ? p.rowadd + ra_row(p, m) * (int64_t)e.N : nullptr;
     ColOps<KIND> ops;
     if constexpr (DRAIN_ALL) {
-      // the warp's bias slice (128 columns, 256 bytes) goes to shared memory asynchronously
-      if (tma && p.bias && e.lane < 16) cp_async16(e.bias_s + 16u * (uint32_t)e.lane, p.bias + n0 + 8 * e.lane);
+      // NVFP4: the warp's bias slice (128 columns, 256 bytes) goes to shared memory asynchronously
+      // (the INT8 / BF16 stages fill the whole stage area, so their drained form reads it per chunk)
+      if constexpr (KIND == KIND_FP4) {
+        if (tma && p.bias && e.lane < 16) cp_async16(e.bias_s + 16u * (uint32_t)e.lane, p.bias + n0 + 8 * e.lane);
+      }
       cp_async_commit();
     } else {
       if (tma) load_colops<KIND>(p, n0, ops);
@@ -384,15 +396,33 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
         const int n = n0 + 32 * c;
         if (c < nch && n < e.N) {
           if (tma) {
-            if (p.bias) {
+            if constexpr (KIND == KIND_FP4) {
+              if (p.bias) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) ops.b[i] = ld_shared_v4(e.bias_s + 64u * c + 16u * i);
+                for (int i = 0; i < 4; ++i) ops.b[i] = ld_shared_v4(e.bias_s + 64u * c + 16u * i);
+              }
+            } else {  // the record form drains INT8 / BF16 tiles too: bias (and scales) from L1
+              load_colops<KIND>(p, n, ops);
             }
             epilogue_math<KIND, ROWADD>(p, ops, sxb, e.alpha, r[c], rrow ? rrow + n : nullptr);
             store_chunk_tma(ty, e, r[c], n, m_warp, oc);
           } else if (m < e.M) {
             store_direct<KIND, ROWADD>(p, m, n, sxb, e.alpha, r[c], rrow ? rrow + n : nullptr);
           }
+        }
+      }
+      if constexpr (RECORD) {  // 256-wide tiles: the warp's 128 columns are one aligned chunk
+        if (m < e.M) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {  // the values the bf16 output holds
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint32_t w = pack_bf16(__uint_as_float(r[c][2 * i]), __uint_as_float(r[c][2 * i + 1]));
+              r[c][2 * i] = w << 16;
+              r[c][2 * i + 1] = w & 0xffff0000u;
+            }
+          }
+          p.records[(int64_t)m * p.rec_nc + (n0 >> 7)] = chunk_record<128>(r);
         }
       }
     } else {
@@ -530,9 +560,10 @@ __device__ __noinline__ bool issue_all(const Issuer c) {
   return true;
 }
 
-// ROWADD: the delta-token form, whose epilogue adds each output row's cube row of p.rowadd (a
-// separate instantiation, so the plain kernel's code and registers do not change).
-template <bool ROWADD>
+// EPI: kEpiPlain; kEpiRowAdd, the delta-token form, whose epilogue adds each output row's cube row
+// of p.rowadd; kEpiRecord, which also writes the output's chunk records. Separate instantiations,
+// so the plain kernel's code and registers do not change.
+template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ TMaps tm, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -736,14 +767,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (fp4) {
       // with two accumulators the row-addend form streams its chunks (one chunk of accumulators
       // and addends live at a time); the plain form drains every column first
-      if (ROWADD && nacc == 2)
-        epilogue_loop<KIND_FP4, false, ROWADD>(p, &tm.y, e);
+      if (EPI == kEpiRowAdd && nacc == 2)
+        epilogue_loop<KIND_FP4, false, EPI>(p, &tm.y, e);
       else
-        epilogue_loop<KIND_FP4, true, ROWADD>(p, &tm.y, e);
-    } else if (kind == KIND_I8) {
-      epilogue_loop<KIND_I8, false, ROWADD>(p, &tm.y, e);
+        epilogue_loop<KIND_FP4, true, EPI>(p, &tm.y, e);
+    } else if (kind == KIND_I8) {  // the record form drains every column first in all precisions
+      epilogue_loop<KIND_I8, EPI == kEpiRecord, EPI>(p, &tm.y, e);
     } else {
-      epilogue_loop<KIND_BF16, false, ROWADD>(p, &tm.y, e);
+      epilogue_loop<KIND_BF16, EPI == kEpiRecord, EPI>(p, &tm.y, e);
     }
   }
   tc_fence_before();
@@ -812,10 +843,10 @@ void arm_gemm_stall_drill(int64_t withhold_stage, uint64_t wait_ns) {
 }
 
 // Shared-memory attribute and register-split check of one k_gemm instantiation.
-template <bool ROWADD>
+template <int EPI>
 static cudaError_t gemm_ready(const char** why) {
   static std::atomic<uint64_t> attr{0};  // one bit per device
-  const cudaError_t attr_err = smem_attr_once(k_gemm<ROWADD>, kSmemBytes, attr);
+  const cudaError_t attr_err = smem_attr_once(k_gemm<EPI>, kSmemBytes, attr);
   if (attr_err != cudaSuccess) {
     *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
     return attr_err;
@@ -825,7 +856,7 @@ static cudaError_t gemm_ready(const char** why) {
   static std::atomic<int> regs{-1};
   if (regs.load() < 0) {
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, k_gemm<ROWADD>) != cudaSuccess) {
+    if (cudaFuncGetAttributes(&fa, k_gemm<EPI>) != cudaSuccess) {
       *why = "cudaFuncGetAttributes(k_gemm) failed";
       return cudaErrorInvalidValue;
     }
@@ -839,8 +870,9 @@ static cudaError_t gemm_ready(const char** why) {
 }
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
-  const bool rowadd = L.rowadd != nullptr;
-  const cudaError_t ready = rowadd ? gemm_ready<true>(why) : gemm_ready<false>(why);
+  const bool rowadd = L.rowadd != nullptr, record = L.records != nullptr;
+  const cudaError_t ready = record ? gemm_ready<kEpiRecord>(why) : (rowadd ? gemm_ready<kEpiRowAdd>(why)
+                                                                            : gemm_ready<kEpiPlain>(why));
   if (ready != cudaSuccess) return ready;
   TMaps tm;
   memset(&tm, 0, sizeof(tm));
@@ -880,6 +912,8 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
     p.ra_nh = ceil_div(L.ra_H, L.ra_ch > 0 ? L.ra_ch : 1);
     p.ra_nw = ceil_div(L.ra_W, L.ra_cw > 0 ? L.ra_cw : 1);
   }
+  p.records = reinterpret_cast<float4*>(L.records);
+  p.rec_nc = (int)(L.N / 128);
   p.withhold = g_drill_withhold.exchange(-1);
   const uint64_t drill_ns = g_drill_wait_ns.exchange(0);
   p.wait_ns = (p.withhold >= 0 && drill_ns != 0) ? drill_ns : kWaitNs;
@@ -926,10 +960,12 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   const int sms = device_sms() & ~1;
   const unsigned grid = (unsigned)(want < sms ? want : sms);
   p.group_m = pick_group_m(ceil_div(L.M, 256), ceil_div(L.N, bn_q), grid / 2);
-  if (rowadd)
-    k_gemm<true><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
+  if (record)
+    k_gemm<kEpiRecord><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
+  else if (rowadd)
+    k_gemm<kEpiRowAdd><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
   else
-    k_gemm<false><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
+    k_gemm<kEpiPlain><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
   return cudaGetLastError();
 }
 

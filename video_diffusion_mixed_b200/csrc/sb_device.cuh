@@ -584,4 +584,93 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Chunk records (FFN-pair fusion)
+// ---------------------------------------------------------------------------------------------
+
+// FP32x2 butterfly of two adjacent pairs: (a0, a1) <- (a0 + b0, a1 + b1), (b0, b1) <- (a0 - b0,
+// a1 - b1), every lane rounded to nearest as the scalar sum and difference are.
+__device__ __forceinline__ void bfly2(uint32_t& a0, uint32_t& a1, uint32_t& b0, uint32_t& b1) {
+  uint64_t a, b, s, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "r"(a0), "r"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "r"(b0), "r"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(s) : "l"(a), "l"(b));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a0), "=r"(a1) : "l"(s));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(b0), "=r"(b1) : "l"(d));
+}
+
+// max(a, b, c) with fmaxf's rule for NaN (a NaN input is ignored unless all are NaN).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+
+// The chunk record of one row's 128 output columns, in place on v[c][j] = column 32 c + j (FP32
+// bit patterns of the values the bf16 output holds), B the Hadamard block (16, 32, 64 or 128):
+//  - max |v|;
+//  - the canonical pairwise sum of |v|, whose first level RN(|a| + |b|) = max(|a + b|, |a - b|)
+//    comes out of the first butterfly;
+//  - the unnormalised FWHT stages h = 1 .. B/4 in ascending order (a + b, a - b rounded to
+//    nearest), one transform per aligned block of B columns; the last stage h = B/2 is not
+//    formed: its outputs' largest magnitude is max(|RN(a + b)|, |RN(a - b)|) = RN(|a| + |b|);
+//  - the rotated amax.
+template <int B>
+__device__ __forceinline__ float4 chunk_record(uint32_t (&v)[4][32]) {
+#define SB_V(k) v[(k) >> 5][(k) & 31]
+  float mx = 0.0f, part[16];  // part[g]: the tree sum of elements 8 g .. 8 g + 7
+#pragma unroll
+  for (int g = 0; g < 16; ++g) {
+    float l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int k = 8 * g + 2 * u;
+      const float a = __uint_as_float(SB_V(k)), b = __uint_as_float(SB_V(k + 1));
+      mx = fmax3(mx, fabsf(a), fabsf(b));
+      const float s = __fadd_rn(a, b), d = __fsub_rn(a, b);
+      SB_V(k) = __float_as_uint(s);
+      SB_V(k + 1) = __float_as_uint(d);
+      l[u] = fmaxf(fabsf(s), fabsf(d));
+    }
+    part[g] = __fadd_rn(__fadd_rn(l[0], l[1]), __fadd_rn(l[2], l[3]));
+  }
+#pragma unroll
+  for (int len = 16; len > 1; len >>= 1) {
+#pragma unroll
+    for (int i = 0; i < len / 2; ++i) part[i] = __fadd_rn(part[2 * i], part[2 * i + 1]);
+  }
+  float am = 0.0f;
+#pragma unroll
+  for (int h = 2; h <= B / 2; h <<= 1) {
+    if (2 * h < B) {
+#pragma unroll
+      for (int k = 0; k < 128; k += 2) {
+        if ((k & h) == 0) bfly2(SB_V(k), SB_V(k + 1), SB_V(k + h), SB_V(k + h + 1));
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 128; k += 2) {
+        if ((k & h) == 0) {
+          const float t0 = __fadd_rn(fabsf(__uint_as_float(SB_V(k))), fabsf(__uint_as_float(SB_V(k + h))));
+          const float t1 = __fadd_rn(fabsf(__uint_as_float(SB_V(k + 1))), fabsf(__uint_as_float(SB_V(k + h + 1))));
+          am = fmax3(am, t0, t1);
+        }
+      }
+    }
+  }
+#undef SB_V
+  return make_float4(am, part[0], mx, 0.0f);
+}
+
+// chunk_record for a block size known at run time (one instantiation per supported block).
+__device__ __forceinline__ float4 chunk_record(uint32_t (&v)[4][32], int B) {
+  switch (B) {
+    case 16: return chunk_record<16>(v);
+    case 32: return chunk_record<32>(v);
+    case 64: return chunk_record<64>(v);
+    default: return chunk_record<128>(v);
+  }
+}
+
 }  // namespace sb

@@ -96,6 +96,9 @@ struct GemmLaunch {
   const float* rowadd;
   int64_t ra_T, ra_H, ra_W;
   int ra_ct, ra_ch, ra_cw;
+  // FFN-pair fusion: the output's chunk records (float4 [M][N/128], rotated amax over Hadamard
+  // blocks of 128 columns; needs 256-wide tiles)
+  float* records;
 };
 
 cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s);
@@ -133,6 +136,8 @@ struct DecideLayers {
 };
 cudaError_t launch_decide(sb_module_state* st, double thr, int force, const DecideLayers& L, cudaStream_t s);
 cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t s, const char** why);
+// Chunk records of a bf16 tensor (sb_chunk_records).
+cudaError_t launch_chunk_records(const void* X, int64_t M, int64_t K, int B, float* out, cudaStream_t s);
 // Arms the stall drill for the next launch_gemm (sb_drill_gemm_stall).
 void arm_gemm_stall_drill(int64_t withhold_stage, uint64_t wait_ns);
 

@@ -101,6 +101,8 @@ def lib():
             "sb_tdc_refresh_fp8": (st, [vp, vp, vp, vp, i64, i64, vp, vp]),
             "sb_module_record": (st, [vp, vp, vp, i64, i64, vp, i32, vp, vp, vp, vp]),
             "sb_delta_linear": (st, [vp, P(Fp4), P(I8), vp, P(WeightC), vp, P(Cubes), i32, i32, vp, i64, vp, vp]),
+            "sb_linear_records": (st, [vp, P(Fp4), P(I8), vp, P(WeightC), i32, vp, i64, i32, vp, vp, vp]),
+            "sb_chunk_records": (st, [vp, i64, i64, i32, vp, vp]),
             "sb_tdc_reuse_fp8": (st, [vp, vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_refresh": (st, [vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_reuse": (st, [vp, vp, vp, i64, i64, vp, vp]),
@@ -130,7 +132,8 @@ EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_in
             "sb_tdc_reuse", "sb_group_slots_bytes", "sb_prepass_partial", "sb_prepass_finish", "sb_nvfp4_encode",
             "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide", "sb_prepass_chunks", "sb_cube_count",
             "sb_delta_split", "sb_delta_combine", "sb_drill_gemm_stall", "sb_tdc_refresh_fp8",
-            "sb_tdc_reuse_fp8", "sb_module_record", "sb_delta_linear")
+            "sb_tdc_reuse_fp8", "sb_module_record", "sb_delta_linear", "sb_linear_records",
+            "sb_chunk_records")
 
 
 def _ck(status: int):
@@ -305,6 +308,23 @@ def module_record(y, x, cache, prec, stats, state, ws: Workspace, update_cache: 
     M, C = y.shape
     _ck(lib().sb_module_record(_p(y), _p(x), _p(cache), M, C, _p(prec), int(update_cache), _p(stats), _p(state),
                                ws.ptr, _stream(stream)))
+
+
+def linear_records(X, a4, a8, prec, w: Weight, Y, records, epilogue: int = EPI_NONE, block: int = 128,
+                   ws: Workspace = None, stream=None):
+    """sb_linear (bf16 output) that also writes Y's chunk records (float32 [M][N/128][4]) for a
+    next pre-pass with Hadamard block `block`."""
+    M = Y.shape[0]
+    c4 = ctypes.byref(a4.c()) if a4 is not None else None
+    c8 = ctypes.byref(a8.c()) if a8 is not None else None
+    _ck(lib().sb_linear_records(_p(X), c4, c8, _p(prec), ctypes.byref(w.c()), epilogue, _p(Y), M, block,
+                                _p(records), ws.ptr, _stream(stream)))
+
+
+def chunk_records(X, records, block: int = 128, stream=None):
+    """The chunk records of a bf16 tensor (sb_chunk_records)."""
+    M, K = X.shape
+    _ck(lib().sb_chunk_records(_p(X), M, K, block, _p(records), _stream(stream)))
 
 
 def tdc_record(y_new, y_cache, d_src, state, ws: Workspace, update_cache: bool = True, stream=None):
