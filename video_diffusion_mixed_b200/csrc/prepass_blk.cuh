@@ -142,7 +142,10 @@ __device__ __forceinline__ float pb_stage1_raw(float2 (&P)[64], float* rmax) {
 // join and spill. The stage h = 64 adds and subtracts the halves of each pair as one fused
 // multiply-add by +-1 each (exact product, one rounding): (x + y, x - y) for a pair (lower, upper)
 // and (y - x, y + x) for a swapped pair (upper, lower) -- the same two results in swapped places.
-template <int B>
+// Without Y (the rotated values are not needed, only their amax) that stage is not formed: the
+// larger magnitude of RN(x + y) and RN(x - y) is RN(|x| + |y|) (rounding is monotone and
+// symmetric), NaN and infinities included, so a pair costs one add.
+template <int B, bool Y = true>
 __device__ __forceinline__ float pb_stages_rest(float2 (&P)[64], float cx) {  // cx = -1: swapped pairs
 #pragma unroll
   for (int h = 2; h <= 32; h <<= 1) {
@@ -158,7 +161,13 @@ __device__ __forceinline__ float pb_stages_rest(float2 (&P)[64], float cx) {  //
     }
   }
   float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent chains
-  if (64 < B) {
+  if (64 < B && !Y) {
+#pragma unroll
+    for (int k = 0; k < 64; k += 2) {
+      const float t0 = __fadd_rn(fabsf(P[k].x), fabsf(P[k].y)), t1 = __fadd_rn(fabsf(P[k + 1].x), fabsf(P[k + 1].y));
+      am[(k >> 1) & 3] = max3(am[(k >> 1) & 3], t0, t1);
+    }
+  } else if (64 < B) {
     const float cy = -cx;
 #pragma unroll
     for (int k = 0; k < 64; ++k) {
@@ -339,7 +348,7 @@ __global__ void __launch_bounds__(kPbThreads, 1) k_prepass_blk(RowArgs a, PbGeom
 
       float rmax;
       const float bsum = pb_stage1_raw(P, &rmax);
-      const float am = pb_stages_rest<B>(P, pb_swap(lane) ? -1.0f : 1.0f);
+      const float am = pb_stages_rest<B, Q>(P, pb_swap(lane) ? -1.0f : 1.0f);  // Q: the codes need y
 
       // ---- row maxima and sums of aligned runs of SUB blocks, then the team meets
       if (!Q && it >= 2) bounded(&s_empty[team][pb], (uint32_t)(((it >> 1) & 1) ^ 1), it);

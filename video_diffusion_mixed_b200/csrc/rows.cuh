@@ -184,11 +184,6 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {  // a - b = fma(b, 
   return fma2(b, make_float2(-1.0f, -1.0f), a);
 }
 __device__ __forceinline__ float sign127(float v) { return v > 0.0f ? 127.0f : (v < 0.0f ? -127.0f : 0.0f); }
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
 
 // Pairwise tree over the lane's 32 terms t (packed like p): levels 1..4 pair indices differing in
 // bits 0..3 (one FP32x2 add each), the last level adds the two halves. Destroys t.

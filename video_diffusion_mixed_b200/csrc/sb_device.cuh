@@ -584,6 +584,14 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// max(a, b, c) in one instruction, with fmaxf's rule for NaN (a NaN input is ignored unless all
+// three are NaN).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // ---------------------------------------------------------------------------------------------
 // Chunk records (FFN-pair fusion)
 // ---------------------------------------------------------------------------------------------
@@ -600,12 +608,6 @@ __device__ __forceinline__ void bfly2(uint32_t& a0, uint32_t& a1, uint32_t& b0, 
   asm("mov.b64 {%0, %1}, %2;" : "=r"(b0), "=r"(b1) : "l"(d));
 }
 
-// max(a, b, c) with fmaxf's rule for NaN (a NaN input is ignored unless all are NaN).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float m;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
-  return m;
-}
 
 // The chunk record of one row's 128 output columns, in place on v[c][j] = column 32 c + j (FP32
 // bit patterns of the values the bf16 output holds), B the Hadamard block (16, 32, 64 or 128):
@@ -627,7 +629,7 @@ __device__ __forceinline__ float4 chunk_record(uint32_t (&v)[4][32]) {
     for (int u = 0; u < 4; ++u) {
       const int k = 8 * g + 2 * u;
       const float a = __uint_as_float(SB_V(k)), b = __uint_as_float(SB_V(k + 1));
-      mx = fmax3(mx, fabsf(a), fabsf(b));
+      mx = max3(mx, fabsf(a), fabsf(b));
       const float s = __fadd_rn(a, b), d = __fsub_rn(a, b);
       SB_V(k) = __float_as_uint(s);
       SB_V(k + 1) = __float_as_uint(d);
@@ -654,7 +656,7 @@ __device__ __forceinline__ float4 chunk_record(uint32_t (&v)[4][32]) {
         if ((k & h) == 0) {
           const float t0 = __fadd_rn(fabsf(__uint_as_float(SB_V(k))), fabsf(__uint_as_float(SB_V(k + h))));
           const float t1 = __fadd_rn(fabsf(__uint_as_float(SB_V(k + 1))), fabsf(__uint_as_float(SB_V(k + h + 1))));
-          am = fmax3(am, t0, t1);
+          am = max3(am, t0, t1);
         }
       }
     }
