@@ -38,12 +38,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool valid_block(int b) { return b == 16 || b == 32 || b == 64 || b == 128 || b == 256; }
 
 constexpr size_t kOffStats = 128;
-constexpr size_t kOffPrec = 224;
 constexpr size_t kOffGroups = 256;
 
 void* ws_groups(void* ws) { return static_cast<char*>(ws) + kOffGroups; }
 sb_stats* ws_stats(void* ws) { return reinterpret_cast<sb_stats*>(static_cast<char*>(ws) + kOffStats); }
-int32_t* ws_prec(void* ws) { return reinterpret_cast<int32_t*>(static_cast<char*>(ws) + kOffPrec); }
 
 sb_status cuda_fail(cudaError_t e, const char* what) {
   return fail(SB_ECUDA, "%s: %s", what, cudaGetErrorString(e));
