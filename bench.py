@@ -41,17 +41,17 @@ METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT sh
 _GEMM_SRC = ("gemm.cu", "sb_device.cuh")
 _ROWS_SRC = ("prepass.cu", "rows.cuh", "prepass_blk.cuh", "sb_device.cuh", "tmap.h")
 TRAFFIC = {
-    "gemm_w1_int8": {"bytes": 744.3e6, "files": _GEMM_SRC, "sha": "ead2d2d5eba64b00"},
-    "gemm_w2_int8": {"bytes": 744.3e6, "files": _GEMM_SRC, "sha": "ead2d2d5eba64b00"},
-    "gemm_w1_nvfp4": {"bytes": 501.4e6, "files": _GEMM_SRC, "sha": "ead2d2d5eba64b00"},
-    "gemm_w2_nvfp4": {"bytes": 256.3e6, "files": _GEMM_SRC, "sha": "ead2d2d5eba64b00"},
+    "gemm_w1_int8": {"bytes": 766.5e6, "files": _GEMM_SRC, "sha": "d37b28c09870f7a8"},
+    "gemm_w2_int8": {"bytes": 792.5e6, "files": _GEMM_SRC, "sha": "d37b28c09870f7a8"},
+    "gemm_w1_nvfp4": {"bytes": 505.3e6, "files": _GEMM_SRC, "sha": "d37b28c09870f7a8"},
+    "gemm_w2_nvfp4": {"bytes": 257.3e6, "files": _GEMM_SRC, "sha": "d37b28c09870f7a8"},
     # k_prepass_blk + k_nvfp4_blk (the encode exits at once in the INT8 pass)
-    "prepass_h_nvfp4": {"bytes": 971.4e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
-    "prepass_h_int8": {"bytes": 630.3e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
-    "prepass_x_nvfp4": {"bytes": 224.6e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
-    "prepass_x_int8": {"bytes": 127.9e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
-    "record_nvfp4": {"bytes": 401.8e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
-    "record_int8": {"bytes": 402.2e6, "files": _ROWS_SRC, "sha": "8a0c345f640e1ea2"},
+    "prepass_h_nvfp4": {"bytes": 970.7e6, "files": _ROWS_SRC, "sha": "e95fb4fcaa331876"},
+    "prepass_h_int8": {"bytes": 630.0e6, "files": _ROWS_SRC, "sha": "e95fb4fcaa331876"},
+    "prepass_x_nvfp4": {"bytes": 225.6e6, "files": _ROWS_SRC, "sha": "e95fb4fcaa331876"},
+    "prepass_x_int8": {"bytes": 127.3e6, "files": _ROWS_SRC, "sha": "e95fb4fcaa331876"},
+    "record_nvfp4": {"bytes": 401.2e6, "files": _ROWS_SRC, "sha": "e95fb4fcaa331876"},
+    "record_int8": {"bytes": 401.4e6, "files": _ROWS_SRC, "sha": "e95fb4fcaa331876"},
 }
 TRAFFIC_TOKENS = 17776
 
