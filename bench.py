@@ -150,7 +150,7 @@ def whole_job_tflops(world, flops_per_rank_step, ms_per_step):
 class FfnStep:
     """All buffers of one FFN module step, allocated once (the library allocates nothing)."""
 
-    def __init__(self, sb, synth, torch, wl, seed, device, tokens=None, records_for=()):
+    def __init__(self, sb, synth, torch, wl, seed, device, tokens=None, records_for=(), fused_record=False):
         self.sb, self.torch = sb, torch
         # precisions whose W1 GEMM also writes the hidden tensor's chunk records, which then stand
         # in for the hidden tensor's statistics pass (FFN-pair fusion)
@@ -169,6 +169,12 @@ class FfnStep:
                      if self.records_for else None)
         self.Y = torch.empty((self.M, self.N2), dtype=torch.bfloat16, device=device)
         self.cache = torch.zeros_like(self.Y)
+        # the module record computed by the W2 GEMM's epilogue (partial sums per row and 128-column
+        # chunk) and folded by one more kernel, instead of a pass over the output
+        self.fused_record = fused_record
+        self.mrec = (torch.empty(self.M * (self.N2 // 128) * 8, dtype=torch.float32, device=device)
+                     if fused_record else None)
+        self.spans = KERNEL_SPANS if not fused_record else KERNEL_SPANS[:-1]
         self.state = sb.alloc_state()
         self.sx, self.sh, self.sy = sb.alloc_stats(), sb.alloc_stats(), sb.alloc_stats()
         self.p1 = torch.zeros(1, dtype=torch.int32, device=device)
@@ -202,10 +208,15 @@ class FfnStep:
         else:
             sb.prepass(self.H, None, cfg, sb.PREPASS_QUANT, self.p2, self.ah4, self.ah8, self.sh, self.ws)
         self._mark(ev, "pre2_1")
-        sb.linear(self.H, self.ah4, self.ah8, self.p2, self.w2, Y, ws=self.ws)
-        self._mark(ev, "gemm2_1")
-        # the difference statistic of Y against X and the TDC record of Y, one pass over Y
-        sb.module_record(Y, X, self.cache, self.p2, self.sy, self.state, self.ws)
+        if self.fused_record:  # the W2 GEMM and the module record of its output, one span
+            sb.linear_module_record(self.H, self.ah4, self.ah8, self.p2, self.w2, Y, X, self.cache, self.mrec,
+                                    self.sy, self.state, self.ws)
+            self._mark(ev, "gemm2_1")
+        else:
+            sb.linear(self.H, self.ah4, self.ah8, self.p2, self.w2, Y, ws=self.ws)
+            self._mark(ev, "gemm2_1")
+            # the difference statistic of Y against X and the TDC record of Y, one pass over Y
+            sb.module_record(Y, X, self.cache, self.p2, self.sy, self.state, self.ws)
         self._mark(ev, "rec_1")
 
     def _mark(self, ev, name):
@@ -337,7 +348,7 @@ def graph_kernel_times(torch, S, flush, reps, precs):
         torch.cuda.synchronize()
         for prec, sub in holder["ev"]:
             d = dict(sub)
-            for name, a, z in KERNEL_SPANS:
+            for name, a, z in S.spans:
                 kern.setdefault(f"{name}_{S.sb.PREC_NAMES[prec]}", []).append(d[a].elapsed_time(d[z]))
     del g
     return {k: statistics.median(v) for k, v in kern.items()}
@@ -679,7 +690,7 @@ def run_ours(args):
 
     records_for = {"none": (), "nvfp4": (sb.NVFP4,), "both": (sb.NVFP4, sb.INT8)}[args.ffn_records]
     S = FfnStep(sb, synth, torch, args.workload, seed=rank, device=device, tokens=args.tokens,
-                records_for=records_for)
+                records_for=records_for, fused_record=(args.module_record == "fused"))
     flush = L2Flush(torch, device)
 
     def barrier():
@@ -848,6 +859,7 @@ def run_ours(args):
                    "l2": "flushed before every step (512 MiB memset, then a 256 MiB read that leaves L2 clean; "
                          "outside the per-step events)",
                    "ffn_records": args.ffn_records,
+                   "module_record": args.module_record,
                    "launch": f"each step replays one CUDA graph of its {launches_per_step} kernels"},
         "roofline": roofline,
         "roofline_prepass": {r["kernel"]: {"achieved_gbs": round(r["achieved"], 1), "frac": round(r["frac"], 4),
@@ -999,6 +1011,8 @@ def main(argv=None):
                     help="tokens in the cpu_baseline sample of our arm (about 10 s on 16 cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-delta-tokens", action="store_true", help="skip the delta-token layer timing")
+    ap.add_argument("--module-record", default="separate", choices=["fused", "separate"],
+                    help="the module record in the W2 GEMM's epilogue + a fold kernel, or its own pass")
     ap.add_argument("--ffn-records", default="none", choices=["none", "nvfp4", "both"],
                     help="passes whose W1 GEMM writes the hidden tensor's chunk records for its pre-pass")
     ap.add_argument("--shard", default="none", choices=["none", "tokens"],

@@ -271,6 +271,24 @@ sb_status sb_module_record(const void* y, const void* x, void* cache, int64_t M,
                            int32_t update_cache, sb_stats* stats, sb_module_state* state, void* ws,
                            sb_stream stream);
 
+/* sb_linear (bf16 output, the module's output Y [M][N]) fused with sb_module_record(Y, x, cache,
+ * M, N, prec, update_cache, stats, state, ws): the GEMM's epilogue computes, for every row and
+ * aligned 128-column chunk of the bf16 values it stores, the partial sums of the difference
+ * statistic (sum |y|, sum (y - x)^2, sum x^2, max |y|) and of the TDC record (sum |y - c|, sum |c|;
+ * c, the cached output, reads as zero while state->n_out == 0), and stores the output to the cache
+ * as well when update_cache is set and state->skip == 0; a second kernel folds the partial sums into
+ * the rows' canonical sums, the group slots and both finishes ("write-up" sections 三 and 四). Stats,
+ * state and cache come out bit for bit as from the two separate calls whenever *prec != SB_SKIP;
+ * under SB_SKIP nothing runs (the separate record would still record the stale Y when the module's
+ * own skip flag is clear, which sb_module_decide never leaves so). records: caller-owned device
+ * scratch of M * (N / 128) * 8 floats, 16-byte aligned. x, cache: bf16 [M][N], 16-byte aligned.
+ * Requires N % 256 == 0 and N <= 16384 (SB_EUNSUPPORTED), else as sb_linear. ws holds two slot
+ * arrays for M rows (sb_workspace_size). */
+sb_status sb_linear_module_record(const void* X, const sb_fp4* a4 /* host */, const sb_i8* a8 /* host */,
+                                  int32_t* prec, const sb_weight* w /* host */, int32_t epilogue, void* Y, int64_t M,
+                                  const void* x, void* cache, int32_t update_cache, float* records, sb_stats* stats,
+                                  sb_module_state* state, void* ws, sb_stream stream);
+
 /* sb_prepass without a caller workspace. The paper has no counterpart: this exists for callers
  * that cannot allocate device memory -- e.g. a plugin inside a host program that owns the whole
  * device-memory pool and forbids other allocations, or a latency-critical loop that must never

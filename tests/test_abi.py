@@ -278,3 +278,25 @@ def test_chunk_record_validation_without_gpu(sb):
     w.N = 384  # records need 256-wide output tiles
     assert L.sb_linear_records(X, None, None, p, ctypes.byref(w), 0, Y, 4, 128, rec, ws, None) == sb.SB_EUNSUPPORTED
     assert "256" in L.sb_last_error().decode()
+
+
+def test_fused_module_record_validation_without_gpu(sb):
+    L = sb.lib()
+    X, Y, x, c, rec, stats, st, ws, p = (_fake(0x10000), _fake(0x20000), _fake(0x30000), _fake(0x40000),
+                                         _fake(0x50000), _fake(0x60000), _fake(0x70000), _fake(0x80000),
+                                         _fake(0x100))
+    w = sb.WeightC()
+    w.N, w.K, w.block = 512, 256, 128
+    args = lambda **o: [o.get("X", X), None, None, p, ctypes.byref(o.get("w", w)), 0, Y, o.get("M", 4),
+                        o.get("x", x), o.get("c", c), 1, o.get("rec", rec), o.get("stats", stats), o.get("st", st),
+                        ws, None]
+    assert L.sb_linear_module_record(*args(x=None)) == sb.SB_EINVAL
+    assert L.sb_linear_module_record(*args(rec=None)) == sb.SB_EINVAL
+    assert L.sb_linear_module_record(*args(st=None)) == sb.SB_EINVAL
+    assert L.sb_linear_module_record(*args(c=_fake(0x40008))) == sb.SB_EALIGN
+    assert L.sb_linear_module_record(*args(rec=_fake(0x50004))) == sb.SB_EALIGN
+    assert L.sb_linear_module_record(*args(M=0)) == sb.SB_ESHAPE
+    w2 = sb.WeightC()
+    w2.N, w2.K, w2.block = 384, 256, 128  # the record's chunks need 256-wide output tiles
+    assert L.sb_linear_module_record(*args(w=w2)) == sb.SB_EUNSUPPORTED
+    assert "256" in L.sb_last_error().decode()

@@ -400,6 +400,11 @@ static sb_status linear_impl(const void* X, const sb_fp4* a4, const sb_i8* a8, c
   L.hdr = ws;
   if (row) {
     L.records = row->records;
+    L.mr_x = row->mr_x;
+    L.mr_c = row->mr_c;
+    L.mr_rec = row->mr_rec;
+    L.mr_st = row->mr_st;
+    L.mr_update = row->mr_update;
     L.rowadd = row->rowadd;
     L.ra_T = row->ra_T;
     L.ra_H = row->ra_H;
@@ -429,6 +434,48 @@ sb_status sb_linear_records(const void* X, const sb_fp4* a4, const sb_i8* a8, co
   sb::GemmLaunch rec{};
   rec.records = records;
   return linear_impl(X, a4, a8, prec, w, epilogue, SB_OUT_BF16, Y, M, ws, stream, &rec);
+}
+
+sb_status sb_linear_module_record(const void* X, const sb_fp4* a4, const sb_i8* a8, int32_t* prec,
+                                  const sb_weight* w, int32_t epilogue, void* Y, int64_t M, const void* x, void* cache,
+                                  int32_t update_cache, float* records, sb_stats* stats, sb_module_state* state,
+                                  void* ws, sb_stream stream) {
+  SB_REQUIRE(w && x && cache && records && stats && state && ws, SB_EINVAL,
+             "w, x, cache, records, stats, state and ws are required");
+  SB_ALIGNED(x, "x");
+  SB_ALIGNED(cache, "cache");
+  SB_ALIGNED(records, "records");
+  SB_ALIGNED(stats, "stats");
+  SB_ALIGNED(state, "state");
+  SB_REQUIRE(w->N % 256 == 0 && w->N <= sb::kMaxK, SB_EUNSUPPORTED,
+             "the fused module record needs N a multiple of 256 up to %d (got %lld)", sb::kMaxK, (long long)w->N);
+  SB_REQUIRE(M >= 1 && M <= (int64_t)1 << 30, SB_ESHAPE, "M out of range (%lld)", (long long)M);
+  sb::GemmLaunch rec{};
+  rec.mr_x = x;
+  rec.mr_c = cache;
+  rec.mr_rec = records;
+  rec.mr_st = state;
+  rec.mr_update = update_cache ? 1 : 0;
+  const sb_status st = linear_impl(X, a4, a8, prec, w, epilogue, SB_OUT_BF16, Y, M, ws, stream, &rec);
+  if (st != SB_OK) return st;
+  sb::RecordLaunch p{};
+  p.Y = Y;
+  p.X = x;
+  p.Cache = cache;
+  p.M = M;
+  p.C = w->N;
+  p.prec = prec;
+  p.rho = 0.0;
+  p.force = -1;
+  p.update = update_cache ? 1 : 0;
+  p.stats = stats;
+  p.st = state;
+  p.groups = ws_groups(ws);
+  p.groups2 = static_cast<char*>(ws_groups(ws)) + sb::ceil_div(M, sb::kGroupRows) * sizeof(sb::GroupSlot);
+  p.hdr = ws;
+  cudaError_t e = sb::launch_fold_modrec(p, records, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "k_fold_modrec launch");
+  return ok();
 }
 
 sb_status sb_chunk_records(const void* X, int64_t M, int64_t K, int32_t block, float* records, sb_stream stream) {

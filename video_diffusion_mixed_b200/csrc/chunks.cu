@@ -201,6 +201,109 @@ cudaError_t launch_prepass_chunks(const PrepassLaunch& p, float* chunks, cudaStr
   }
 }
 
+// The fused module record from the GEMM's per-chunk partial sums (two float4 per row and
+// 128-column chunk: {sum |y|, sum (y - x)^2, sum x^2, sum |y - c|}, {sum |c|, max |y|, 0, 0}). A
+// chunk's sums are aligned subtrees of the row's canonical tree, so one warp per 16-row group
+// rebuilds each row's five sums as the row engine does (the chunks zero-padded to a power of two),
+// then writes the group's two FP64 slots; the last CTA runs the record's two finishes: the
+// difference statistic into *stats, then the TDC record with d from it, as k_rows<.., OP_REC>.
+__global__ void __launch_bounds__(kFoldWarps * 32) k_fold_modrec(RowArgs a, const float4* rec, int NB) {
+  __shared__ double s_fin[kFinChunk];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int prec = a.prec ? *a.prec : -1;
+  if (prec == SB_SKIP) return;  // the GEMM did not run: no output to record
+  const bool do_tdc = a.st->skip == 0;
+  const bool have_prev = a.st->n_out >= 1;
+  const int64_t G = ceil_div(a.M, kG);
+  int NB2 = 1;
+  while (NB2 < NB) NB2 <<= 1;
+  const int c = NB2 >= 32 ? NB2 / 32 : 1;  // chunks per lane (a power of two <= 16)
+  const int span = NB2 / c;                // lanes covering one row
+  for (int64_t g = (int64_t)blockIdx.x * kFoldWarps + warp; g < G; g += (int64_t)gridDim.x * kFoldWarps) {
+    float rs[5] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f}, rmx = 0.0f;  // lane i < kG: row i of the group
+    for (int i = 0; i < kG; ++i) {
+      const int64_t m = g * kG + i;
+      float v[5], mx = 0.0f;
+#pragma unroll
+      for (int st = 0; st < 5; ++st) {
+        float t[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int idx = lane * c + u;
+          t[u] = 0.0f;
+          if (m < a.M && u < c && idx < NB) {
+            const float4* r = rec + 2 * (m * NB + idx);
+            t[u] = st == 0 ? r[0].x : st == 1 ? r[0].y : st == 2 ? r[0].z : st == 3 ? r[0].w : r[1].x;
+            if (st == 0) mx = fmaxf(mx, r[1].y);
+          }
+        }
+        float w = tree16(t);
+        for (int s2 = 1; s2 < span; s2 <<= 1) w = __fadd_rn(w, __shfl_xor_sync(0xffffffffu, w, s2));
+        v[st] = __shfl_sync(0xffffffffu, w, 0);  // lanes 0 .. span-1 hold the row; past them only zeros
+      }
+      mx = warp_max_f32(mx);
+      if (lane == i) {
+#pragma unroll
+        for (int st = 0; st < 5; ++st) rs[st] = v[st];
+        rmx = mx;
+      }
+    }
+    const bool in = lane < kG;
+    double gs[5];
+#pragma unroll
+    for (int st = 0; st < 5; ++st) gs[st] = warp_pairwise_f64(in ? (double)rs[st] : 0.0);
+    const float gmx = warp_max_f32(in ? rmx : 0.0f);
+    const int gnf = __any_sync(0xffffffffu, in && (isnan(rs[0]) || isinf(rmx)));  // Inf or NaN in a row
+    if (lane == 0) {
+      GroupSlot* slot = a.groups + g;
+      slot->s[0] = gs[0];
+      slot->s[1] = gs[1];
+      slot->s[2] = gs[2];
+      slot->max_abs = gmx;
+      slot->amax_rot = 0.0f;
+      slot->nonfinite = gnf;
+      GroupSlot* slot2 = a.groups2 + g;
+      slot2->s[0] = gs[3];
+      slot2->s[1] = gs[4];
+      slot2->s[2] = 0.0;
+      slot2->max_abs = 0.0f;
+      slot2->amax_rot = 0.0f;
+      slot2->nonfinite = 0;
+    }
+  }
+  rows_finish<OP_STATS, true>(a, G, prec, true, s_fin);
+  if (do_tdc) {
+    RowArgs t = a;
+    t.groups = a.groups2;
+    t.dsrc = a.stats;
+    rows_finish<OP_TDC, true>(t, G, prec, have_prev, s_fin);
+  }
+}
+
+cudaError_t launch_fold_modrec(const RecordLaunch& p, const float* rec, cudaStream_t s) {
+  RowArgs a{};
+  a.M = p.M;
+  a.K = (int)p.C;
+  a.mode = SB_PREPASS_STATS;
+  a.prec = p.prec;
+  a.rho = p.rho;
+  a.force = p.force;
+  a.update = p.update;
+  a.st = p.st;
+  a.stats = p.stats;
+  a.groups = reinterpret_cast<GroupSlot*>(p.groups);
+  a.groups2 = reinterpret_cast<GroupSlot*>(p.groups2);
+  a.hdr = reinterpret_cast<WsHeader*>(p.hdr);
+  a.finish = 1;
+  const int NB = (int)(p.C / 128);
+  const int64_t G = ceil_div(p.M, kG);
+  const int64_t want = ceil_div(G, kFoldWarps);
+  const int sms = chunks_sms();
+  k_fold_modrec<<<(unsigned)(want < sms ? want : sms), kFoldWarps * 32, 0, s>>>(a, reinterpret_cast<const float4*>(rec),
+                                                                                  NB);
+  return cudaGetLastError();
+}
+
 // Chunk records of a bf16 tensor [M][K] (K % 128 == 0) with the same arithmetic the GEMM's
 // record epilogue uses: one thread per (row, 128-channel chunk).
 __global__ void __launch_bounds__(128) k_chunk_records(const __nv_bfloat16* X, int64_t M, int K, int B,

@@ -87,6 +87,7 @@ struct TMaps {
   CUtensorMap sfa;  // NVFP4 scales of A, 3-D: 128 words x K/64 atoms x 128-row tiles
   CUtensorMap sfb;  // NVFP4 scales of B, same shape over the N rows of the weight
   CUtensorMap y;    // bf16 output, box 32 columns x 32 rows, 64B swizzle
+  CUtensorMap yc;   // k_gemm<kEpiModRec>: the module's cached output, same boxes (c := y is stored there)
 };
 
 struct GemmParams {
@@ -116,11 +117,22 @@ struct GemmParams {
   // output, {max |H_128 y|, canonical pairwise sum |y|, max |y|, 0}, float4 [M][N / 128].
   float4* records;
   int rec_nc;  // chunks per row
+  // Module record (k_gemm<kEpiModRec> only; the output y is the module's output): per row and
+  // aligned 128-column chunk, from the bf16 values y holds, the module input x (mr_x) and the cached
+  // output c (mr_c, read as zero while the module has no cached output), the partial sums
+  // {sum |y|, sum (y - x)^2, sum x^2, sum |y - c|} and {sum |c|, max |y|, 0, 0} (two float4 per
+  // chunk, mr_rec [M][N / 128][2]); each sum is the balanced tree over the chunk's columns. When
+  // the module's TDC record runs and mr_update is set, the staged output is stored to the cache too.
+  const __nv_bfloat16* mr_x;
+  const __nv_bfloat16* mr_c;
+  float4* mr_rec;
+  const sb_module_state* mr_st;
+  int mr_update;
   WsHeader* hdr;
 };
 
 // Epilogue forms, one k_gemm instantiation each (the plain one is what every ordinary launch runs).
-enum { kEpiPlain = 0, kEpiRowAdd = 1, kEpiRecord = 2 };
+enum { kEpiPlain = 0, kEpiRowAdd = 1, kEpiRecord = 2, kEpiModRec = 3 };
 
 
 // The cube of token t (text tokens first, one cube each; then the grid in (f, h, w) order).
@@ -170,6 +182,11 @@ __device__ __forceinline__ float2 ep_mul2(float2 a, float2 b) {
 __device__ __forceinline__ float2 ep_fma2(float2 a, float2 b, float2 c) {
   uint64_t r;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(ep_bits(a)), "l"(ep_bits(b)), "l"(ep_bits(c)));
+  return ep_f2(r);
+}
+__device__ __forceinline__ float2 ep_add2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ep_bits(a)), "l"(ep_bits(b)));
   return ep_f2(r);
 }
 
@@ -308,6 +325,14 @@ __device__ __forceinline__ void stage_bf16_row(uint32_t box, int lane, const uin
   }
 }
 
+// stage_bf16_row for columns already packed as bf16 pairs (word i: columns 2i, 2i + 1).
+__device__ __forceinline__ void stage_packed_row(uint32_t box, int lane, const uint32_t (&w)[16]) {
+  const uint32_t row = box + 64u * (uint32_t)lane;
+  const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) st_shared_v4(row + 16u * ((uint32_t)g ^ sw), w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+}
+
 // What the epilogue warps of one CTA share.
 struct EpiCtx {
   uint64_t* tfull;
@@ -319,24 +344,132 @@ struct EpiCtx {
   uint32_t out_box;  // this warp's two staging boxes
   uint32_t bias_s;   // NVFP4: this warp's bias slice in shared memory (past the NVFP4 stages)
   float alpha;
+  const CUtensorMap* tyc;  // kEpiModRec: where the refreshed cache goes (null: no refresh)
+  bool have_prev;          // kEpiModRec: the module has a cached output (else c reads as zero)
+  uint64_t pol;            // kEpiModRec: L2 evict-first policy of the record's streams
 };
+
+// The module record's streams (x and the old cache read once, the new cache written once) go
+// through L2 as evict-first lines, so they do not push out the GEMM's operands, which the tile
+// order keeps in L2 for reuse.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// 16-byte read-only load with an L2 policy, kept in program order (volatile): the record's loads of
+// one chunk must not be hoisted above the previous chunk's stores, or their registers pile up.
+__device__ __forceinline__ uint4 ld_nc_hint(const uint4* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.b32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void tma_store_2d_hint(const void* tmap, uint32_t smem_src, int x, int y, uint64_t pol) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(tmap),
+               "r"(x), "r"(y), "r"(smem_src), "l"(pol)
+               : "memory");
+}
 
 // One 32 x 32 bf16 chunk (a row per lane) through a staging box and one TMA store; rows past M
 // are clipped by the store. Lane kStoreLane issues the stores and owns their bulk groups, so lane
 // 0's release-arrive on the accumulator barrier never waits for them.
-__device__ __forceinline__ void store_chunk_tma(const CUtensorMap* ty, const EpiCtx& e, const uint32_t (&r)[32],
+template <bool MR = false, int NW = 32>
+__device__ __forceinline__ void store_chunk_tma(const CUtensorMap* ty, const EpiCtx& e, const uint32_t (&r)[NW],
                                                 int n, int m_warp, uint32_t& oc) {
   const uint32_t box = e.out_box + (oc & 1u) * (uint32_t)kOutBox;
   if (e.lane == kStoreLane) bulk_wait_read<1>();  // the store issued from this box before has read it
   __syncwarp();
-  stage_bf16_row(box, e.lane, r);
+  if constexpr (NW == 32)
+    stage_bf16_row(box, e.lane, r);  // FP32 values, packed here
+  else
+    stage_packed_row(box, e.lane, r);  // bf16 pairs
   fence_proxy_async_smem();
   __syncwarp();
   if (e.lane == kStoreLane) {
     tma_store_2d(ty, box, n, m_warp);
+    if (MR && e.tyc) tma_store_2d_hint(e.tyc, box, n, m_warp, e.pol);  // the module's cache refresh, same group
     bulk_commit();
   }
   ++oc;
+}
+
+
+// bf16 pair k of 32 packed columns (16 words; word i holds columns 2i and 2i + 1): columns k and
+// k + 16 as FP32, the pairing of the row engine's statistics.
+__device__ __forceinline__ float2 mr_pair(const uint32_t (&w)[16], int k) {
+  const uint32_t lo = w[k >> 1], hi = w[8 + (k >> 1)];
+  return (k & 1) ? make_float2(__uint_as_float(lo & 0xffff0000u), __uint_as_float(hi & 0xffff0000u))
+                 : make_float2(__uint_as_float(lo << 16), __uint_as_float(hi << 16));
+}
+
+// Balanced tree over the 32 columns held as 16 pairs (column k, column k + 16): adjacent columns
+// first, as the row engine sums a lane's run.
+__device__ __forceinline__ float mr_tree(float2 (&t)[16]) {
+#pragma unroll
+  for (int len = 16; len > 1; len >>= 1) {
+#pragma unroll
+    for (int i = 0; i < len / 2; ++i) t[i] = ep_add2(t[2 * i], t[2 * i + 1]);
+  }
+  return __fadd_rn(t[0].x, t[0].y);
+}
+
+// Module record of one row's 32 output columns n .. n + 31 (kEpiModRec), yw the bf16 outputs: the
+// terms are those of the row engine's fused record, on the bf16 values the output holds
+// (|y|; (y - x)^2 and x^2 with the difference and the squares each rounded once; |y - c|; |c|),
+// q[s] the balanced tree of term s over the 32 columns, rmx the running max |y|.
+__device__ __forceinline__ void modrec_chunk(const GemmParams& p, const EpiCtx& e, int m, int n,
+                                             const uint32_t (&yw)[16], float (&q)[5], float& rmx) {
+  uint32_t xw[16], cw[16];
+  const uint4* xp = reinterpret_cast<const uint4*>(p.mr_x + (int64_t)m * e.N + n);
+  const uint4* cp = reinterpret_cast<const uint4*>(p.mr_c + (int64_t)m * e.N + n);
+  // x and c together, so that one memory round trip serves both; each element of c is read here
+  // before this thread's own chunk is stored to the cache, so the read-only path never serves a
+  // value this kernel has overwritten
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = ld_nc_hint(xp + i, e.pol);
+    xw[4 * i] = v.x, xw[4 * i + 1] = v.y, xw[4 * i + 2] = v.z, xw[4 * i + 3] = v.w;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = e.have_prev ? ld_nc_hint(cp + i, e.pol) : make_uint4(0u, 0u, 0u, 0u);
+    cw[4 * i] = v.x, cw[4 * i + 1] = v.y, cw[4 * i + 2] = v.z, cw[4 * i + 3] = v.w;
+  }
+  float2 t[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float2 y = mr_pair(yw, k);
+    t[k] = make_float2(fabsf(y.x), fabsf(y.y));
+    rmx = max3(rmx, t[k].x, t[k].y);
+  }
+  q[0] = mr_tree(t);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float2 y = mr_pair(yw, k), x = mr_pair(xw, k);
+    const float dx = __fsub_rn(y.x, x.x), dy = __fsub_rn(y.y, x.y);
+    t[k] = make_float2(__fmul_rn(dx, dx), __fmul_rn(dy, dy));
+  }
+  q[1] = mr_tree(t);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float2 x = mr_pair(xw, k);
+    t[k] = make_float2(__fmul_rn(x.x, x.x), __fmul_rn(x.y, x.y));
+  }
+  q[2] = mr_tree(t);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float2 y = mr_pair(yw, k), c = mr_pair(cw, k);
+    t[k] = make_float2(fabsf(__fsub_rn(y.x, c.x)), fabsf(__fsub_rn(y.y, c.y)));
+  }
+  q[3] = mr_tree(t);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float2 c = mr_pair(cw, k);
+    t[k] = make_float2(fabsf(c.x), fabsf(c.y));
+  }
+  q[4] = mr_tree(t);
 }
 
 // The epilogue of every tile of this CTA. DRAIN_ALL (one accumulator buffer, and the record form
@@ -345,7 +478,7 @@ __device__ __forceinline__ void store_chunk_tma(const CUtensorMap* ty, const Epi
 // loaded as they are processed and the buffer is released after the last load.
 template <int KIND, bool DRAIN_ALL, int EPI>
 __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtensorMap* ty, const EpiCtx& e) {
-  constexpr bool ROWADD = EPI == kEpiRowAdd, RECORD = EPI == kEpiRecord;
+  constexpr bool ROWADD = EPI == kEpiRowAdd, RECORD = EPI == kEpiRecord, MODREC = EPI == kEpiModRec;
   const int nch = e.BN / 64;  // 32-column chunks per warp: 2 or 4
   const int row = 32 * e.q + e.lane;
   uint32_t oc = 0;
@@ -363,6 +496,7 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
     const float sxb = (KIND == KIND_I8 && m < e.M) ? __fmul_rn(__ldg(p.sA8 + m), p.invB) : 0.0f;
     const float* rrow = (ROWADD && m < e.M) ? p.rowadd + ra_row(p, m) * (int64_t)e.N : nullptr;
     ColOps<KIND> ops;
+    float mq[MODREC ? 4 : 1][5], mrx = 0.0f;  // MODREC: per 32-column chunk partial sums, max |y|
     if constexpr (DRAIN_ALL) {
       // NVFP4: the warp's bias slice (128 columns, 256 bytes) goes to shared memory asynchronously
       // (the INT8 / BF16 stages fill the whole stage area, so their drained form reads it per chunk)
@@ -405,9 +539,27 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
               load_colops<KIND>(p, n, ops);
             }
             epilogue_math<KIND, ROWADD>(p, ops, sxb, e.alpha, r[c], rrow ? rrow + n : nullptr);
-            store_chunk_tma(ty, e, r[c], n, m_warp, oc);
+            if constexpr (MODREC) {  // packed now; recorded and stored below, once every chunk is
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                r[c][i] = pack_bf16(__uint_as_float(r[c][2 * i]), __uint_as_float(r[c][2 * i + 1]));
+            } else {
+              store_chunk_tma(ty, e, r[c], n, m_warp, oc);
+            }
           } else if (m < e.M) {
             store_direct<KIND, ROWADD>(p, m, n, sxb, e.alpha, r[c], rrow ? rrow + n : nullptr);
+          }
+        }
+      }
+      if constexpr (MODREC) {  // each chunk's record reads the old cache before the chunk is stored there
+        if (tma) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t yw[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) yw[i] = r[c][i];
+            if (m < e.M) modrec_chunk(p, e, m, n0 + 32 * c, yw, mq[c], mrx);
+            store_chunk_tma<true, 16>(ty, e, yw, n0 + 32 * c, m_warp, oc);
           }
         }
       }
@@ -443,13 +595,31 @@ __device__ __forceinline__ void epilogue_loop(const GemmParams& p, const CUtenso
               ColOps<KIND> next;
               if (c + 1 < nch && n + 32 < e.N) load_colops<KIND>(p, n + 32, next);
               epilogue_math<KIND, ROWADD>(p, ops, sxb, e.alpha, r, rrow ? rrow + n : nullptr);
-              store_chunk_tma(ty, e, r, n, m_warp, oc);
+              if constexpr (MODREC) {
+                uint32_t yw[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) yw[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                if (m < e.M) modrec_chunk(p, e, m, n, yw, mq[c], mrx);
+                store_chunk_tma<true, 16>(ty, e, yw, n, m_warp, oc);
+              } else {
+                store_chunk_tma(ty, e, r, n, m_warp, oc);
+              }
               ops = next;
             } else if (m < e.M) {
               store_direct<KIND, ROWADD>(p, m, n, sxb, e.alpha, r, rrow ? rrow + n : nullptr);
             }
           }
         }
+      }
+    }
+    if constexpr (MODREC) {  // 256-wide tiles: the warp's 128 columns are one aligned chunk
+      if (tma && m < e.M) {
+        float q[5];
+#pragma unroll
+        for (int k = 0; k < 5; ++k) q[k] = __fadd_rn(__fadd_rn(mq[0][k], mq[1][k]), __fadd_rn(mq[2][k], mq[3][k]));
+        float4* dst = p.mr_rec + 2 * ((int64_t)m * p.rec_nc + (n0 >> 7));
+        dst[0] = make_float4(q[0], q[1], q[2], q[3]);
+        dst[1] = make_float4(q[4], mrx, 0.0f, 0.0f);
       }
     }
   }
@@ -764,6 +934,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     e.out_box = smem_u32(smem + kOutOff) + (uint32_t)(2 * (warp - kEpiWarp0) * kOutBox);
     e.bias_s = smem_u32(smem + kBiasOffF) + 256u * (uint32_t)(warp - kEpiWarp0);
     e.alpha = fp4 ? __fmul_rn(__fmul_rn(*p.gA4, *p.gB4), p.invB) : 1.0f;
+    e.tyc = nullptr;
+    e.have_prev = false;
+    e.pol = 0;
+    if (EPI == kEpiModRec) {  // the module state decides the cache's part: read as zero, refreshed
+      e.have_prev = p.mr_st->n_out >= 1;
+      e.pol = l2_evict_first_policy();
+      if (p.mr_update && p.mr_st->skip == 0) e.tyc = &tm.yc;
+    }
     if (fp4) {
       // with two accumulators the row-addend form streams its chunks (one chunk of accumulators
       // and addends live at a time); the plain form drains every column first
@@ -870,9 +1048,10 @@ static cudaError_t gemm_ready(const char** why) {
 }
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
-  const bool rowadd = L.rowadd != nullptr, record = L.records != nullptr;
-  const cudaError_t ready = record ? gemm_ready<kEpiRecord>(why) : (rowadd ? gemm_ready<kEpiRowAdd>(why)
-                                                                            : gemm_ready<kEpiPlain>(why));
+  const bool rowadd = L.rowadd != nullptr, record = L.records != nullptr, modrec = L.mr_rec != nullptr;
+  const cudaError_t ready = modrec ? gemm_ready<kEpiModRec>(why)
+                                   : (record ? gemm_ready<kEpiRecord>(why)
+                                             : (rowadd ? gemm_ready<kEpiRowAdd>(why) : gemm_ready<kEpiPlain>(why)));
   if (ready != cudaSuccess) return ready;
   TMaps tm;
   memset(&tm, 0, sizeof(tm));
@@ -914,6 +1093,11 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   }
   p.records = reinterpret_cast<float4*>(L.records);
   p.rec_nc = (int)(L.N / 128);
+  p.mr_x = reinterpret_cast<const __nv_bfloat16*>(L.mr_x);
+  p.mr_c = reinterpret_cast<const __nv_bfloat16*>(L.mr_c);
+  p.mr_rec = reinterpret_cast<float4*>(L.mr_rec);
+  p.mr_st = L.mr_st;
+  p.mr_update = L.mr_update;
   p.withhold = g_drill_withhold.exchange(-1);
   const uint64_t drill_ns = g_drill_wait_ns.exchange(0);
   p.wait_ns = (p.withhold >= 0 && drill_ns != 0) ? drill_ns : kWaitNs;
@@ -927,6 +1111,14 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
     p.tma_store = fn && fn(&tm.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L.Y, dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (modrec && p.tma_store)
+      p.tma_store = fn(&tm.yc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L.mr_c, dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  if (modrec && !p.tma_store) {  // the record form stores the output and the cache through TMA only
+    *why = "cuTensorMapEncodeTiled failed (output or cache of the module record)";
+    return cudaErrorInvalidValue;
   }
   const uint64_t M = (uint64_t)L.M, N = (uint64_t)L.N, K = (uint64_t)L.K;
   const uint32_t half = (uint32_t)bn_q / 2;  // B rows each CTA of the pair loads (INT8 / BF16)
@@ -960,7 +1152,9 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, const char** why) {
   const int sms = device_sms() & ~1;
   const unsigned grid = (unsigned)(want < sms ? want : sms);
   p.group_m = pick_group_m(ceil_div(L.M, 256), ceil_div(L.N, bn_q), grid / 2);
-  if (record)
+  if (modrec)
+    k_gemm<kEpiModRec><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
+  else if (record)
     k_gemm<kEpiRecord><<<grid, kThreads, kSmemBytes, s>>>(tm, p);
   else if (rowadd)
     k_gemm<kEpiRowAdd><<<grid, kThreads, kSmemBytes, s>>>(tm, p);

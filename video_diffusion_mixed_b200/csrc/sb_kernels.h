@@ -99,6 +99,14 @@ struct GemmLaunch {
   // FFN-pair fusion: the output's chunk records (float4 [M][N/128], rotated amax over Hadamard
   // blocks of 128 columns; needs 256-wide tiles)
   float* records;
+  // Module record fused into the GEMM (the output is the module's output; needs 256-wide tiles):
+  // the module input, the cached output (read, then refreshed), the per-chunk partial sums
+  // (float4 [M][N/128][2]) and the module state that gates the cache's part
+  const void* mr_x;
+  void* mr_c;
+  float* mr_rec;
+  const sb_module_state* mr_st;
+  int mr_update;
 };
 
 cudaError_t launch_prepass(const PrepassLaunch& p, cudaStream_t s);
@@ -137,6 +145,9 @@ struct DecideLayers {
 cudaError_t launch_decide(sb_module_state* st, double thr, int force, const DecideLayers& L, cudaStream_t s);
 cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t s, const char** why);
 // Chunk records of a bf16 tensor (sb_chunk_records).
+// The module record from the GEMM's per-chunk partial sums (sb_linear_module_record): the rows'
+// sums, the group slots and both finishes of the fused record.
+cudaError_t launch_fold_modrec(const RecordLaunch& p, const float* rec, cudaStream_t s);
 cudaError_t launch_chunk_records(const void* X, int64_t M, int64_t K, int B, float* out, cudaStream_t s);
 // Arms the stall drill for the next launch_gemm (sb_drill_gemm_stall).
 void arm_gemm_stall_drill(int64_t withhold_stage, uint64_t wait_ns);

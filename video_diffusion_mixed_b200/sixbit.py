@@ -103,6 +103,8 @@ def lib():
             "sb_delta_linear": (st, [vp, P(Fp4), P(I8), vp, P(WeightC), vp, P(Cubes), i32, i32, vp, i64, vp, vp]),
             "sb_linear_records": (st, [vp, P(Fp4), P(I8), vp, P(WeightC), i32, vp, i64, i32, vp, vp, vp]),
             "sb_chunk_records": (st, [vp, i64, i64, i32, vp, vp]),
+            "sb_linear_module_record": (st, [vp, P(Fp4), P(I8), vp, P(WeightC), i32, vp, i64, vp, vp, i32, vp, vp, vp,
+                                             vp, vp]),
             "sb_tdc_reuse_fp8": (st, [vp, vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_refresh": (st, [vp, vp, vp, i64, i64, vp, vp]),
             "sb_tdc_reuse": (st, [vp, vp, vp, i64, i64, vp, vp]),
@@ -133,7 +135,7 @@ EXPORTED = ("sb_version", "sb_last_error", "sb_workspace_size", "sb_workspace_in
             "sb_tdc_record_partial", "sb_tdc_finish", "sb_module_decide", "sb_prepass_chunks", "sb_cube_count",
             "sb_delta_split", "sb_delta_combine", "sb_drill_gemm_stall", "sb_tdc_refresh_fp8",
             "sb_tdc_reuse_fp8", "sb_module_record", "sb_delta_linear", "sb_linear_records",
-            "sb_chunk_records")
+            "sb_chunk_records", "sb_linear_module_record")
 
 
 def _ck(status: int):
@@ -319,6 +321,18 @@ def linear_records(X, a4, a8, prec, w: Weight, Y, records, epilogue: int = EPI_N
     c8 = ctypes.byref(a8.c()) if a8 is not None else None
     _ck(lib().sb_linear_records(_p(X), c4, c8, _p(prec), ctypes.byref(w.c()), epilogue, _p(Y), M, block,
                                 _p(records), ws.ptr, _stream(stream)))
+
+
+def linear_module_record(X, a4, a8, prec, w: Weight, Y, x, cache, records, stats, state, ws: Workspace,
+                         epilogue: int = EPI_NONE, update_cache: bool = True, stream=None):
+    """sb_linear (bf16 output) fused with sb_module_record of that output (sb_linear_module_record);
+    records: float32 scratch of M * (N / 128) * 8 values."""
+    M = Y.shape[0]
+    c4 = ctypes.byref(a4.c()) if a4 is not None else None
+    c8 = ctypes.byref(a8.c()) if a8 is not None else None
+    _ck(lib().sb_linear_module_record(_p(X), c4, c8, _p(prec), ctypes.byref(w.c()), epilogue, _p(Y), M, _p(x),
+                                      _p(cache), int(update_cache), _p(records), _p(stats), _p(state), ws.ptr,
+                                      _stream(stream)))
 
 
 def chunk_records(X, records, block: int = 128, stream=None):
