@@ -41,10 +41,10 @@ METRIC = "quantized-linear TFLOPS & fused quant GB/s (frac of B200 peak), DiT sh
 _GEMM_SRC = ("gemm.cu", "sb_device.cuh")
 _ROWS_SRC = ("prepass.cu", "rows.cuh", "prepass_blk.cuh", "sb_device.cuh", "tmap.h")
 TRAFFIC = {
-    "gemm_w1_int8": {"bytes": 766.5e6, "files": _GEMM_SRC, "sha": "d37b28c09870f7a8"},
-    "gemm_w2_int8": {"bytes": 792.5e6, "files": _GEMM_SRC, "sha": "d37b28c09870f7a8"},
-    "gemm_w1_nvfp4": {"bytes": 505.3e6, "files": _GEMM_SRC, "sha": "d37b28c09870f7a8"},
-    "gemm_w2_nvfp4": {"bytes": 257.3e6, "files": _GEMM_SRC, "sha": "d37b28c09870f7a8"},
+    "gemm_w1_int8": {"bytes": 773.8e6, "files": _GEMM_SRC, "sha": "18b7efe3b2cd2be6"},
+    "gemm_w2_int8": {"bytes": 809.3e6, "files": _GEMM_SRC, "sha": "18b7efe3b2cd2be6"},
+    "gemm_w1_nvfp4": {"bytes": 516.4e6, "files": _GEMM_SRC, "sha": "18b7efe3b2cd2be6"},
+    "gemm_w2_nvfp4": {"bytes": 262.4e6, "files": _GEMM_SRC, "sha": "18b7efe3b2cd2be6"},
     # k_prepass_blk + k_nvfp4_blk (the encode exits at once in the INT8 pass)
     "prepass_h_nvfp4": {"bytes": 970.7e6, "files": _ROWS_SRC, "sha": "e95fb4fcaa331876"},
     "prepass_h_int8": {"bytes": 630.0e6, "files": _ROWS_SRC, "sha": "e95fb4fcaa331876"},
