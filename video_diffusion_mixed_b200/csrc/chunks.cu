@@ -9,8 +9,8 @@
 // quantization pass reads the tensor: the NVFP4 encode as in sb_prepass, or a streaming INT8
 // pass that knows every row's amax in advance and so needs no team of warps per row.
 //
-//  k_fold_chunks   one warp per 16-row group: per row, the tree over the chunk sums and the
-//                  chunk maxima; INT8 scales; the group's FP64 slot; rows_finish in the last CTA.
+//  k_fold_chunks   one warp per 16-row group, a lane per row: the tree over the chunk sums and
+//                  the chunk maxima; INT8 scales; the group's FP64 slot; rows_finish in the last CTA.
 //                  The row's rotated amax is left in the fourth float of its first record.
 //  k_int8_blk      INT8 codes, one 128-channel block per lane (as the NVFP4 encode).
 #include "launch_util.h"
@@ -21,7 +21,7 @@ namespace sb {
 
 constexpr int kFoldWarps = 8;
 
-// Canonical pairwise tree over 16 values whose tail is zero (the run of a lane).
+// Canonical pairwise tree over 16 values whose tail is zero.
 __device__ __forceinline__ float tree16(float (&t)[16]) {
 #pragma unroll
   for (int len = 16; len > 1; len >>= 1) {
@@ -31,6 +31,7 @@ __device__ __forceinline__ float tree16(float (&t)[16]) {
   return t[0];
 }
 
+
 __global__ void __launch_bounds__(kFoldWarps * 32) k_fold_chunks(RowArgs a, float4* chunks, int NB) {
   __shared__ double s_fin[kFinChunk];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -38,41 +39,41 @@ __global__ void __launch_bounds__(kFoldWarps * 32) k_fold_chunks(RowArgs a, floa
   if (prec == SB_SKIP) return;
   const bool do_int8 = a.mode == SB_PREPASS_QUANT && prec == SB_INT8;
   const int64_t G = ceil_div(a.M, kG);
-  int NB2 = 1;
-  while (NB2 < NB) NB2 <<= 1;
-  const int c = NB2 >= 32 ? NB2 / 32 : 1;  // chunk sums per lane (a power of two <= 16)
-  const int span = NB2 / c;                // lanes covering one row
   for (int64_t g = (int64_t)blockIdx.x * kFoldWarps + warp; g < G; g += (int64_t)gridDim.x * kFoldWarps) {
-    float rs = 0.0f, ram = 0.0f, rmx = 0.0f;  // lane i < kG: row i of the group
-    for (int i = 0; i < kG; ++i) {
-      const int64_t m = g * kG + i;
-      float t[16];
-      float am = 0.0f, mx = 0.0f;
+    // lane i < kG: row i of the group, its chunks read in order
+    const int64_t m = g * kG + lane;
+    const bool row = lane < kG && m < a.M;
+    const float4* rc = chunks + (row ? m : 0) * NB;
+    // the row's tree in two levels: aligned runs of 8 chunks in registers, then the 16 run sums
+    float runs[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int idx = lane * c + u;
-        t[u] = 0.0f;
-        if (m < a.M && u < c && idx < NB) {
-          const float4 r = chunks[m * NB + idx];
-          t[u] = r.y;
-          am = fmaxf(am, r.x);
-          mx = fmaxf(mx, r.z);
+    for (int k = 0; k < 16; ++k) runs[k] = 0.0f;
+    float ram = 0.0f, rmx = 0.0f;
+    if (row) {
+#pragma unroll 4
+      for (int b0 = 0; b0 < NB; b0 += 8) {  // several runs' loads in flight at once
+        float t[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          t[u] = 0.0f;
+          if (b0 + u < NB) {
+            const float4 r = rc[b0 + u];
+            t[u] = r.y;
+            ram = fmaxf(ram, r.x);
+            rmx = fmaxf(rmx, r.z);
+          }
         }
+        const float s8 = __fadd_rn(__fadd_rn(__fadd_rn(t[0], t[1]), __fadd_rn(t[2], t[3])),
+                                   __fadd_rn(__fadd_rn(t[4], t[5]), __fadd_rn(t[6], t[7])));
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          if (k == (b0 >> 3)) runs[k] = s8;  // a register per run: no indexed local array
       }
-      float v = tree16(t);
-      for (int s = 1; s < span; s <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
-      v = __shfl_sync(0xffffffffu, v, 0);  // lanes 0 .. span-1 hold the row; past them only zeros
-      am = warp_max_f32(am);
-      mx = warp_max_f32(mx);
-      if (lane == i) {
-        rs = v;
-        ram = am;
-        rmx = mx;
-      }
-      if (lane == 0 && m < a.M) {
-        chunks[m * NB].w = am;
-        if (do_int8) a.s8[m] = (am == 0.0f) ? 0.0f : __fdiv_rn(am, 127.0f);
-      }
+    }
+    const float rs = tree16(runs);
+    if (row) {
+      chunks[m * NB].w = ram;
+      if (do_int8) a.s8[m] = (ram == 0.0f) ? 0.0f : __fdiv_rn(ram, 127.0f);
     }
     const bool in = lane < kG;
     const double gs = warp_pairwise_f64(in ? (double)rs : 0.0);
@@ -203,8 +204,8 @@ cudaError_t launch_prepass_chunks(const PrepassLaunch& p, float* chunks, cudaStr
 
 // The fused module record from the GEMM's per-chunk partial sums (two float4 per row and
 // 128-column chunk: {sum |y|, sum (y - x)^2, sum x^2, sum |y - c|}, {sum |c|, max |y|, 0, 0}). A
-// chunk's sums are aligned subtrees of the row's canonical tree, so one warp per 16-row group
-// rebuilds each row's five sums as the row engine does (the chunks zero-padded to a power of two),
+// chunk's sums are aligned subtrees of the row's canonical tree, so one warp per 16-row group (a
+// lane per row) rebuilds each row's five sums as the row engine does (the chunks zero-padded),
 // then writes the group's two FP64 slots; the last CTA runs the record's two finishes: the
 // difference statistic into *stats, then the TDC record with d from it, as k_rows<.., OP_REC>.
 __global__ void __launch_bounds__(kFoldWarps * 32) k_fold_modrec(RowArgs a, const float4* rec, int NB) {
@@ -220,34 +221,48 @@ __global__ void __launch_bounds__(kFoldWarps * 32) k_fold_modrec(RowArgs a, cons
   const int c = NB2 >= 32 ? NB2 / 32 : 1;  // chunks per lane (a power of two <= 16)
   const int span = NB2 / c;                // lanes covering one row
   for (int64_t g = (int64_t)blockIdx.x * kFoldWarps + warp; g < G; g += (int64_t)gridDim.x * kFoldWarps) {
-    float rs[5] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f}, rmx = 0.0f;  // lane i < kG: row i of the group
-    for (int i = 0; i < kG; ++i) {
-      const int64_t m = g * kG + i;
-      float v[5], mx = 0.0f;
+    // lane i < kG: row i of the group, its chunks read in order
+    const int64_t m = g * kG + lane;
+    const bool row = lane < kG && m < a.M;
+    const float4* rc = rec + 2 * (row ? m : 0) * NB;
+    // each row's trees in two levels: aligned runs of 8 chunks in registers, then the 16 run sums
+    float runs[5][16];
 #pragma unroll
-      for (int st = 0; st < 5; ++st) {
-        float t[16];
+    for (int st = 0; st < 5; ++st)
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int idx = lane * c + u;
-          t[u] = 0.0f;
-          if (m < a.M && u < c && idx < NB) {
-            const float4* r = rec + 2 * (m * NB + idx);
-            t[u] = st == 0 ? r[0].x : st == 1 ? r[0].y : st == 2 ? r[0].z : st == 3 ? r[0].w : r[1].x;
-            if (st == 0) mx = fmaxf(mx, r[1].y);
+      for (int k = 0; k < 16; ++k) runs[st][k] = 0.0f;
+    float rmx = 0.0f;
+    if (row) {
+#pragma unroll 2
+      for (int b0 = 0; b0 < NB; b0 += 8) {  // two runs' loads in flight at once
+        float t[5][8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+#pragma unroll
+          for (int st = 0; st < 5; ++st) t[st][u] = 0.0f;
+          if (b0 + u < NB) {
+            const float4 r0 = rc[2 * (b0 + u)], r1 = rc[2 * (b0 + u) + 1];
+            t[0][u] = r0.x;
+            t[1][u] = r0.y;
+            t[2][u] = r0.z;
+            t[3][u] = r0.w;
+            t[4][u] = r1.x;
+            rmx = fmaxf(rmx, r1.y);
           }
         }
-        float w = tree16(t);
-        for (int s2 = 1; s2 < span; s2 <<= 1) w = __fadd_rn(w, __shfl_xor_sync(0xffffffffu, w, s2));
-        v[st] = __shfl_sync(0xffffffffu, w, 0);  // lanes 0 .. span-1 hold the row; past them only zeros
-      }
-      mx = warp_max_f32(mx);
-      if (lane == i) {
 #pragma unroll
-        for (int st = 0; st < 5; ++st) rs[st] = v[st];
-        rmx = mx;
+        for (int st = 0; st < 5; ++st) {
+          const float s8 = __fadd_rn(__fadd_rn(__fadd_rn(t[st][0], t[st][1]), __fadd_rn(t[st][2], t[st][3])),
+                                     __fadd_rn(__fadd_rn(t[st][4], t[st][5]), __fadd_rn(t[st][6], t[st][7])));
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            if (k == (b0 >> 3)) runs[st][k] = s8;  // a register per run: no indexed local array
+        }
       }
     }
+    float rs[5];
+#pragma unroll
+    for (int st = 0; st < 5; ++st) rs[st] = tree16(runs[st]);
     const bool in = lane < kG;
     double gs[5];
 #pragma unroll
